@@ -1,0 +1,395 @@
+#!/usr/bin/env python
+"""Benchmark of the speculative MoE decode step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--k 3] [--impl ours|reference]
+
+Workload (default): the full decoder (12 layers, d = 1280, 64 routed + 2 shared
+experts, top-6, vocabulary 129,280) with the FastMTP draft at k = 3, batch 1,
+context 256 visual embeddings + 32 prompt tokens, synthetic bf16 weights
+N(0, 0.02) seed 1.  Proposals come from the forced acceptance model
+(0.83 / 0.69 / 0.58 per depth, reference = this library's own k = 0 greedy
+output) after the draft has run, so the draft's compute is inside every step.
+
+One step = draft (k recursions) + forced override + verifier pass over k+1
+rows + acceptance, replayed as one CUDA graph.  The metric is accepted
+(committed) tokens per second over the K timed steps.  Multi-GPU runs are
+independent replicas (one sequence per GPU, no collective on the data path):
+value = tokens of all ranks / max over ranks of the timed region.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from speculative_moe_decoding_b200 import metrics, synth  # noqa: E402
+
+# ---- byte model of one spec step (bf16 weights) ------------------------------
+
+
+def step_bytes(dims: synth.ModelDims, k: int, touched_routed_per_layer: float, kv_len: float):
+    d, V, L = dims.d_model, dims.vocab, dims.n_layers
+    attn = L * 4 * d * d * 2
+    dense0 = dims.n_dense_first * 3 * d * dims.dense_ffn * 2
+    n_moe = L - dims.n_dense_first
+    shared = n_moe * dims.n_shared * 3 * d * dims.shared_ffn * 2
+    routers = n_moe * dims.n_experts * d * 2
+    lm = V * d * 2
+    expert = 3 * d * dims.expert_ffn * 2
+    routed = n_moe * touched_routed_per_layer * expert
+    kv = kv_len * L * 2 * d * 2
+    draft = (d * 2 * d + 4 * d * d + 3 * d * dims.draft_ffn) * 2 if k > 0 else 0
+    draft_kv = kv_len * 2 * d * 2 if k > 0 else 0
+    union = attn + dense0 + shared + routers + lm + routed + kv + draft + draft_kv
+    dep = union + k * lm + max(0, k - 1) * draft + max(0, k - 1) * draft_kv
+    return union, dep
+
+
+# ---- clocks ---------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = "index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---- the reference arm: the CPU oracle -------------------------------------------
+
+ORACLE_SAMPLE = dict(n_visual=32, n_prompt=8, n_ref=16)
+
+
+def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.0):
+    """Times the oracle's speculative decode (forced acceptance, draft running)
+    on a bounded sample; returns (tokens/s, description, threads)."""
+    from oracle import decoder as O
+    w = synth.WORKLOADS["full_spec"]
+    orc = O.Oracle(dims.as_dict(), bits)
+    inp = synth.make_inputs(dims, w.input_seed, ORACLE_SAMPLE["n_visual"], ORACLE_SAMPLE["n_prompt"])
+    C = ORACLE_SAMPLE["n_visual"] + ORACLE_SAMPLE["n_prompt"]
+    st = O.prefill(orc, inp.visual, inp.prompt)
+    ref_list = O.decode(orc, st, 0, ORACLE_SAMPLE["n_ref"])
+    ref = {C + i: t for i, t in enumerate(ref_list)}
+    tab = synth.make_forced_tables(w.stream_seed, C + 4096, dims.vocab, 3, w.accept_p)
+
+    def proposer(s):
+        return O.forced_proposals({p: ref.get(p, 0) for p in range(s.kv_len, s.kv_len + k + 1)}, s.kv_len, k,
+                                  tab.u, tab.r, tab.p, dims.vocab)
+
+    st = O.prefill(orc, inp.visual, inp.prompt)
+    t0 = time.perf_counter()
+    steps = toks = 0
+    while time.perf_counter() - t0 < budget_s and st.n_generated < ORACLE_SAMPLE["n_ref"] - k - 1:
+        before = st.n_generated
+        props = O.draft_propose(orc, st, k)
+        props = proposer(st)
+        O.verify_commit(orc, st, props)
+        toks += st.n_generated - before
+        steps += 1
+    dt = time.perf_counter() - t0
+    try:
+        import threadpoolctl
+        threads = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+    except Exception:
+        threads = 1
+    desc = (f"oracle spec decode k={k}, forced acceptance, draft running; context {C} rows "
+            f"({ORACLE_SAMPLE['n_visual']} visual + {ORACLE_SAMPLE['n_prompt']} prompt) instead of 288; "
+            f"{steps} steps, {toks} tokens in {dt:.1f} s")
+    return toks / dt, desc, threads, steps, dt
+
+
+def reference_arm(args, dims):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    bits, _ = synth.make_weights(dims, synth.WORKLOADS["full_spec"].weight_seed)
+    tps, desc, threads, steps, dt = run_oracle_sample(dims, args.k, bits, budget_s=20.0 * max(1, args.steps) / 50)
+    line = {"impl": "reference", "metric": "accepted tokens/sec (speculative decode step, batch 1)",
+            "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": 0,
+            "ms_per_step": 1000 * dt / max(1, steps), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": "full_spec", "k": args.k, "batch": 1, "sample": desc},
+            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc},
+            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- our arm --------------------------------------------------------------------
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=390)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--k", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-only", action="store_true", help="skip e2e and the CPU baseline (for ncu)")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    dims = synth.FULL
+    if args.impl == "reference":
+        return reference_arm(args, dims)
+
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    dev = torch.cuda.current_device()
+
+    from speculative_moe_decoding_b200 import build
+    build.build()
+    from speculative_moe_decoding_b200 import ocrdec
+
+    wl = synth.WORKLOADS["full_spec"]
+    k = args.k
+    bits, _ = synth.make_weights(dims, wl.weight_seed)
+    names = [n for n, _ in synth.manifest(dims)]
+    n_steps_total = args.warmup + args.steps
+    C = wl.n_visual + wl.n_prompt
+    n_ref = n_steps_total * (k + 1) + 16
+    cap = C + n_ref + 16
+    dec = ocrdec.Decoder(dims.as_dict(), bits, names, max_k=3, max_batch=1, kv_capacity=cap)
+    inp = synth.make_inputs(dims, wl.input_seed, wl.n_visual, wl.n_prompt, index=rank)
+    vis = torch.from_numpy(inp.visual).cuda()
+    prm = torch.from_numpy(inp.prompt).cuda()
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    def max_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    def sum_over_ranks(v: float) -> float:
+        if world == 1:
+            return v
+        t = torch.tensor([v], dtype=torch.float64, device="cuda")
+        torch.distributed.all_reduce(t)
+        return float(t.item())
+
+    # ---- k = 0 reference run (also the plain greedy baseline) ----
+    dec.set_forced_acceptance(None, None, None, ())
+    dec.prefill(0, vis, prm)
+    n0_steps = n_ref - 1
+    for _ in range(args.warmup):
+        dec.step(1, 0)
+    torch.cuda.synchronize()
+    g0 = dec.stats(0).n_generated
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n0_steps - args.warmup):
+        dec.step(1, 0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    k0_ms = e0.elapsed_time(e1)
+    k0_tokens = dec.stats(0).n_generated - g0
+    assert dec.status() == 0, dec.status()
+    ref_hist = dec.history(0, 0, C + n_ref).clone()
+
+    # ---- speculative run with forced acceptance ----
+    tab = synth.make_forced_tables(wl.stream_seed, C + n_ref, dims.vocab, 3, wl.accept_p, index=rank)
+    u_t = torch.from_numpy(tab.u).cuda()
+    r_t = torch.from_numpy(tab.r).cuda()
+    dec.set_forced_acceptance(ref_hist, u_t, r_t, tab.p)
+    dec.prefill(0, vis, prm)
+    for _ in range(args.warmup):
+        dec.step(1, k)
+    torch.cuda.synchronize()
+    dec.reset_counters()
+    st0 = dec.stats(0)
+    clocks = ClockSampler(dev)
+    clocks.start()
+    time.sleep(0.3)
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.steps):
+        dec.step(1, k)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    clk = clocks.stop()
+    ms = e0.elapsed_time(e1)
+    st1 = dec.stats(0)
+    assert dec.status() == 0, dec.status()
+    tokens = st1.n_generated - st0.n_generated
+    steps = st1.steps - st0.steps
+    touched, passes = dec.counters()
+    spec_hist = dec.history(0, C, st1.n_generated).cpu().numpy()
+    lossless = bool(np.array_equal(spec_hist, ref_hist[C:C + st1.n_generated].cpu().numpy()))
+    kernels = dec.step_kernel_count(1, k)
+
+    ms_max = max_over_ranks(ms)
+    tok_all = sum_over_ranks(tokens)
+    value = tok_all / (ms_max / 1000.0)
+    tau = tokens / max(1, steps)
+    step_ms = ms_max / args.steps
+    U = touched / max(1, passes)
+    kv_mid = C + (st0.n_generated + st1.n_generated) / 2
+    union_b, dep_b = step_bytes(dims, k, U, kv_mid)
+
+    # ---- dominant kernel: LM head + argmax over k+1 rows, timed alone ----
+    import math
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    peak_gbs, peak_src = 6650.0, "fallback"
+    if os.path.exists(peaks_path):
+        peak_gbs, peak_src = float(json.load(open(peaks_path))["hbm_gbs"]), "measured"
+    R = k + 1
+    lm_w = dec.weights[names.index("lm_head")]
+    g_w = dec.weights[names.index("final_norm")]
+    xr = torch.randn((R, dims.d_model), dtype=torch.float32, device="cuda")
+    tok = torch.empty(R, dtype=torch.int32, device="cuda")
+    scratch = ocrdec.op_scratch()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    times = []
+    for i in range(23):
+        flush.fill_(i & 0xff)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= 3:
+            times.append(a.elapsed_time(b))
+    lm_ms = float(np.mean(times))
+    lm_bytes = dims.vocab * dims.d_model * 2 + R * dims.d_model * 4 + dims.d_model * 2
+    lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
+
+    # ---- end to end through host buffers ----
+    e2e = None
+    if not args.profile_only:
+        hc = np.zeros(k + 1, np.int32)
+        hn = np.zeros(1, np.int32)
+        dec.prefill(0, vis, prm)
+        for _ in range(args.warmup):
+            dec.step_host(1, k, hc, hn)
+        g_before = dec.stats(0).n_generated
+        barrier()
+        torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            dec.step_host(1, k, hc, hn)
+        t1 = time.perf_counter()
+        barrier()
+        e2e_tok = dec.stats(0).n_generated - g_before
+        e2e_s = max_over_ranks(t1 - t0)
+        e2e = {"value": sum_over_ranks(e2e_tok) / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+               "d2h_bytes_per_step": 4 * (k + 2),
+               "note": "ocrdec_step_host per step: graph launch, D2H of committed tokens + count, stream sync; "
+                       "the step has no per-step host input (state lives on the device)"}
+
+    # ---- CPU baseline (rank 0, N = 1) ----
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.profile_only:
+        try:
+            tps, desc, threads, _, _ = run_oracle_sample(dims, k, bits, budget_s=20.0)
+            cpu = {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle", "sample": desc,
+                   "host_cpus": os.cpu_count()}
+        except MemoryError as e:
+            cpu = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle", "sample": f"failed: {e}"}
+
+    if rank == 0:
+        line = {
+            "metric": "accepted tokens/sec (speculative decode step, batch 1)",
+            "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "full_spec", "k": k, "batch": 1, "context": f"{wl.n_visual} visual + {wl.n_prompt} prompt",
+                       "model": "12L d1280 64+2 experts top6 V129280 + FastMTP block", "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (each step streams ~3.5 GB of weights, L2 is 126 MB)",
+                       "acceptance_model": list(tab.p), "graph": True},
+            "tau": tau, "acceptance": metrics.acceptance_rate(tau, k) if k else None,
+            "lossless_vs_k0": lossless,
+            "k0": {"tokens_per_s": k0_tokens / (k0_ms / 1000.0), "ms_per_step": k0_ms / max(1, n0_steps - args.warmup)},
+            "speedup_vs_k0": value / world / (k0_tokens / (k0_ms / 1000.0)),
+            "step_roofline": {"union_bytes": union_b, "dependency_aware_bytes": dep_b,
+                              "touched_routed_experts_per_layer": U,
+                              "union_GBps": union_b / (step_ms / 1000) / 1e9,
+                              "frac_of_8TBps": union_b / (step_ms / 1000) / 8e12,
+                              "frac_of_measured_peak": union_b / (step_ms / 1000) / 1e9 / peak_gbs,
+                              "dependency_aware_frac_of_measured_peak": dep_b / (step_ms / 1000) / 1e9 / peak_gbs},
+            "roofline": {"kernel": "lm_head_argmax (final RMSNorm + 129,280 x 1280 GEMV + argmax, k+1 rows)",
+                         "bound": "hbm", "achieved": lm_gbs, "peak": peak_gbs, "unit": "GB/s",
+                         "frac": lm_gbs / peak_gbs, "traffic": None, "peak_source": peak_src,
+                         "launch_ms": lm_ms, "bytes_per_launch": lm_bytes,
+                         "timing": "same kernel instantiation as in the step, launched alone through ocrdec_op_lm_argmax, "
+                                   "L2 flushed before each launch, CUDA events on the launching stream"},
+            "gpu_launches": kernels * args.steps,
+            "kernels_per_step": kernels,
+            "clocks": clk,
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    dec.close()
+    if world > 1:
+        torch.distributed.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -278,8 +278,11 @@ class Oracle:
         dcache.length = max(dcache.length, max(positions) + 1)
         return out
 
-    def draft_token(self, hprime_row: np.ndarray) -> int:
-        return greedy_argmax(self.lm_logits(hprime_row[None, :], "draft.final_norm")[0])
+    def draft_token(self, hprime_row: np.ndarray, margins: Optional[list] = None) -> int:
+        logits = self.lm_logits(hprime_row[None, :], "draft.final_norm")[0]
+        if margins is not None:
+            margins.append(top2_margin(logits))
+        return greedy_argmax(logits)
 
 
 # --------------------------------------------------------------------------
@@ -332,7 +335,7 @@ def prefill(orc: Oracle, visual: np.ndarray, prompt: Sequence[int], with_draft: 
                     accepted_at_depth=[0, 0, 0, 0])
 
 
-def draft_propose(orc: Oracle, st: SeqState, k: int) -> List[int]:
+def draft_propose(orc: Oracle, st: SeqState, k: int, margins: Optional[list] = None) -> List[int]:
     """k recursions of the shared draft block.  Recursion 1 consumes the pending
     pairs (verifier hidden at p, committed token at p+1); recursion j >= 2 feeds
     the block's own output hidden with the previous draft token."""
@@ -341,12 +344,12 @@ def draft_propose(orc: Oracle, st: SeqState, k: int) -> List[int]:
     out = orc.draft_rows(st.pend_h, orc.embed(nxt), st.pend_pos, st.dcache)
     base = st.kv_len  # == pend_pos[-1] + 1
     hprime = out[-1]
-    props = [orc.draft_token(hprime)]
+    props = [orc.draft_token(hprime, margins)]
     for j in range(2, k + 1):
         pos = base + j - 2
         out = orc.draft_rows(hprime[None, :], orc.embed([props[-1]]), [pos], st.dcache)
         hprime = out[-1]
-        props.append(orc.draft_token(hprime))
+        props.append(orc.draft_token(hprime, margins))
     st.dcache.truncate(base)  # recursion rows beyond the committed prefix are discarded
     st.pend_h = st.pend_h[:0]
     st.pend_pos = []

@@ -1,0 +1,201 @@
+// Split-K flash-decoding attention over a contiguous per-slot KV cache.
+//
+// For pass row r (slot b, position pos_r) and head h:
+//   out[r][h] = softmax_j(q_r . k_j / sqrt(Dh)) v_j over positions j = 0..pos_r
+// (causal: rows of one pass see each other's keys up to their own position).
+// The position axis is cut into fixed kAttnChunk-position chunks; CTA (c, h, b)
+// loads chunk c of head h for slot b into shared memory with two bulk copies,
+// computes every row's partial (max m, sum l, unnormalised o) over the
+// positions that row may see, and the last CTA of (b, h) merges the partials
+// of each row in chunk order.  Chunk boundaries depend only on positions, so a
+// row's result does not depend on the other rows of the pass.
+#pragma once
+
+#include "common.cuh"
+
+namespace ocrdec {
+
+constexpr int kAttnChunk = 128;
+constexpr int kAttnThreads = 128;
+constexpr int kAttnRows = 8;  // rows of one slot in a pass
+
+struct AttnParams {
+  const float* q;          // [R][H*Dh]
+  const bf16* kc;          // this layer, slot 0: [H][cap][Dh]
+  const bf16* vc;
+  long long slot_stride;   // elements between slots
+  int cap, H, Dh;
+  float scale;             // 1/sqrt(Dh)
+  const int* slot_row0;    // [B] first pass row of each slot
+  const int* slot_nrows;   // [B] rows of each slot in this pass
+  const int* row_pos;      // [R]
+  float* part;             // [R][H][max_chunks][Dh + 2]: o[Dh], m, l
+  int max_chunks;
+  int* counters;           // [B][H], zero between launches
+  bf16* out;               // [R][H*Dh]
+  int* status;
+};
+
+__global__ void __launch_bounds__(kAttnThreads)
+attention_kernel(const AttnParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_abort;
+  __shared__ float qs[kAttnRows][128];
+  __shared__ float sc[kAttnRows][kAttnChunk];
+  __shared__ float s_m[kAttnRows], s_l[kAttnRows];
+  __shared__ int s_last;
+
+  const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int Dh = p.Dh;
+
+  pdl_wait();
+  if (tid == 0) s_abort = status_bad(p.status);
+  __syncthreads();
+  if (s_abort) return;
+  pdl_trigger();
+
+  const int r0 = p.slot_row0[b];
+  const int nr = min(p.slot_nrows[b], kAttnRows);
+  if (nr <= 0) return;
+  int maxpos = 0;
+  for (int i = 0; i < nr; ++i) maxpos = max(maxpos, p.row_pos[r0 + i]);
+  const int nchunks = maxpos / kAttnChunk + 1;
+  if (c >= nchunks) return;
+  const int p0 = c * kAttnChunk;
+  const int npos = min(kAttnChunk, maxpos + 1 - p0);
+
+  bf16* Ks = reinterpret_cast<bf16*>(smem);
+  bf16* Vs = Ks + kAttnChunk * Dh;
+  const long long base = (long long)b * p.slot_stride + ((long long)h * p.cap + p0) * Dh;
+  if (tid == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    uint32_t bytes = npos * Dh * 2;
+    mbar_arrive_expect_tx(&bar, 2 * bytes);
+    bulk_g2s(Ks, p.kc + base, bytes, &bar);
+    bulk_g2s(Vs, p.vc + base, bytes, &bar);
+  }
+  // queries of this slot's rows
+  for (int i = 0; i < nr; ++i)
+    for (int d = tid; d < Dh; d += kAttnThreads) qs[i][d] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + d];
+  __syncthreads();
+  bool ok = mbar_wait(&bar, 0, p.status);
+  if (!ok) return;  // status recorded; no copy can still be pending after a failed wait of this barrier
+
+  // ---- scores: 4 lanes-groups of 8 per warp, one position per group ----
+  // lane l8 of a group owns the 16-byte dim-chunks l8 and l8 + 8 of a key row
+  const int g = lane >> 3, l8 = lane & 7;
+  const int ndc = Dh / 8;  // 16-byte chunks per key row (8 or 16)
+  for (int rb = 0; rb < nr; rb += 4) {
+    float qr[4][16];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int e = 0; e < 16; ++e) {
+        int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
+        qr[i][e] = (rb + i < nr && (e < 8 || l8 + 8 < ndc)) ? qs[rb + i][d] : 0.f;
+      }
+    for (int j0 = warp * 32; j0 < warp * 32 + 32; j0 += 4) {
+      int j = j0 + g;
+      float kv[16];
+      if (j < npos) {
+        uint4 u0 = *reinterpret_cast<const uint4*>(Ks + j * Dh + l8 * 8);
+        float t[8];
+        unpack8(u0, t);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kv[e] = t[e];
+        if (l8 + 8 < ndc) {
+          uint4 u1 = *reinterpret_cast<const uint4*>(Ks + j * Dh + (l8 + 8) * 8);
+          unpack8(u1, t);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[8 + e] = t[e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) kv[8 + e] = 0.f;
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 16; ++e) kv[e] = 0.f;
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        float a = 0.f;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) a = __fmaf_rn(qr[i][e], kv[e], a);
+        a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
+        a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
+        a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
+        int r = rb + i;
+        if (l8 == 0 && r < nr && j < kAttnChunk) {
+          bool valid = j < npos && p0 + j <= p.row_pos[r0 + r];
+          sc[r][j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
+        }
+      }
+    }
+  }
+  __syncthreads();
+
+  // ---- per-row chunk max and exp-sum (warp w takes rows w, w+4) ----
+  for (int r = warp; r < nr; r += 4) {
+    int lim = p.row_pos[r0 + r] - p0 + 1;  // visible positions of this row in the chunk
+    lim = min(lim, npos);
+    float m = -INFINITY;
+    for (int j = lane; j < lim; j += 32) m = fmaxf(m, sc[r][j]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float l = 0.f;
+    for (int j = lane; j < kAttnChunk; j += 32) {
+      float e = 0.f;
+      if (j < lim) e = expf(__fsub_rn(sc[r][j], m));
+      if (j < npos) sc[r][j] = e;
+      l = __fadd_rn(l, e);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) l = __fadd_rn(l, __shfl_xor_sync(0xffffffffu, l, o));
+    if (lane == 0) { s_m[r] = m; s_l[r] = l; }
+  }
+  __syncthreads();
+
+  // ---- o = sum_j p_j v_j, thread per dim, positions in order ----
+  const int ld = Dh + 2;
+  for (int r = 0; r < nr; ++r) {
+    int lim = min(p.row_pos[r0 + r] - p0 + 1, npos);
+    if (lim <= 0) continue;
+    float* dst = p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + c) * ld;
+    for (int d = tid; d < Dh; d += kAttnThreads) {
+      float o = 0.f;
+      for (int j = 0; j < lim; ++j) o = __fmaf_rn(sc[r][j], bf2f(Vs[j * Dh + d]), o);
+      dst[d] = o;
+    }
+    if (tid == 0) { dst[Dh] = s_m[r]; dst[Dh + 1] = s_l[r]; }
+  }
+
+  // ---- last CTA of (slot, head) merges the chunks of every row ----
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_last = (atomicAdd(&p.counters[b * p.H + h], 1) == nchunks - 1);
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int r = 0; r < nr; ++r) {
+    int pos = p.row_pos[r0 + r];
+    int nc = pos / kAttnChunk + 1;
+    const volatile float* pr = p.part + ((long long)(r0 + r) * p.H + h) * p.max_chunks * ld;
+    float M = -INFINITY;
+    for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, pr[cc * ld + Dh]);
+    for (int d = tid; d < Dh; d += kAttnThreads) {
+      float L = 0.f, O = 0.f;
+      for (int cc = 0; cc < nc; ++cc) {
+        float f = expf(__fsub_rn(pr[cc * ld + Dh], M));
+        L = __fmaf_rn(pr[cc * ld + Dh + 1], f, L);
+        O = __fmaf_rn(pr[cc * ld + d], f, O);
+      }
+      p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, L));
+    }
+  }
+  if (tid == 0) p.counters[b * p.H + h] = 0;
+}
+
+}  // namespace ocrdec

@@ -1,0 +1,990 @@
+// The decode-step engine behind the C ABI of include/ocrdec.h.
+//
+// Host side only orders launches; every step of the decode path runs in the
+// kernels of gemv.cuh, attention.cuh and step_kernels.cuh.  One verifier pass
+// per layer is: Q/K/V GEMV (+RoPE, KV append) -> split-K attention -> O-proj
+// GEMV (+residual) -> [dense SwiGLU up/down | router GEMV -> softmax/top-k and
+// bucketing -> expert gate/up GEMV over the touched experts -> expert down
+// GEMV -> combine].  Then final norm + LM head + argmax, then acceptance.
+#include <cmath>
+#include <cstring>
+#include <map>
+#include <new>
+#include <tuple>
+#include <vector>
+
+#include "attention.cuh"
+#include "launch.cuh"
+#include "step_kernels.cuh"
+
+using namespace ocrdec;
+
+namespace {
+
+constexpr int kPrefillChunk = kRmax;  // context rows per prefill pass
+
+struct LayerW {
+  const bf16 *attn_norm, *wqkv, *wo, *ffn_norm;
+  const bf16 *w_gu, *w_down;                                  // dense layers
+  const bf16 *router, *exp_gu, *exp_down, *sh_gu, *sh_down;   // MoE layers
+  bool dense;
+};
+
+struct DraftW {
+  const bf16 *norm_h, *norm_e, *fc, *attn_norm, *wqkv, *wo, *ffn_norm, *w_gu, *w_down, *final_norm;
+};
+
+void manifest(const ocrdec_config& c, std::vector<std::vector<int64_t>>& m) {
+  const int64_t d = c.d_model, V = c.vocab, E = c.n_experts, S = c.n_shared;
+  m.clear();
+  m.push_back({V, d});
+  for (int l = 0; l < c.n_layers; ++l) {
+    m.push_back({d});
+    m.push_back({3 * d, d});
+    m.push_back({d, d});
+    m.push_back({d});
+    if (l < c.n_dense_first) {
+      m.push_back({2 * (int64_t)c.dense_ffn, d});
+      m.push_back({d, c.dense_ffn});
+    } else {
+      m.push_back({E, d});
+      m.push_back({E, 2 * (int64_t)c.expert_ffn, d});
+      m.push_back({E, d, c.expert_ffn});
+      m.push_back({S, 2 * (int64_t)c.shared_ffn, d});
+      m.push_back({S, d, c.shared_ffn});
+    }
+  }
+  m.push_back({d});
+  m.push_back({V, d});
+  m.push_back({d});
+  m.push_back({d});
+  m.push_back({d, 2 * d});
+  m.push_back({d});
+  m.push_back({3 * d, d});
+  m.push_back({d, d});
+  m.push_back({d});
+  m.push_back({2 * (int64_t)c.draft_ffn, d});
+  m.push_back({d, c.draft_ffn});
+  m.push_back({d});
+}
+
+bool config_ok(const ocrdec_config* c) {
+  if (!c) return false;
+  const int pos[] = {c->d_model, c->n_layers, c->n_heads, c->head_dim, c->n_experts, c->top_k, c->expert_ffn,
+                     c->shared_ffn, c->draft_ffn, c->vocab, c->max_batch, c->kv_capacity};
+  for (int v : pos)
+    if (v <= 0) return false;
+  if (c->n_heads * c->head_dim != c->d_model) return false;
+  if (c->head_dim % 16 || c->head_dim > 128) return false;
+  if (c->d_model % 8 || c->expert_ffn % 8 || c->draft_ffn % 8 || c->vocab % kTR) return false;
+  if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
+  if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % 8)) return false;
+  if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
+  if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > 256 || c->top_k + c->n_shared > 127) return false;
+  if (c->max_k < 0 || c->max_k > 3) return false;
+  if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
+  if (c->d_model * 2 > 4096) return false;  // shared-memory copy of the normalised rows
+  if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
+  return true;
+}
+
+size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
+
+struct Layout {
+  size_t status, counters, slots, rows, hist, rope, kvk, kvv, dkvk, dkvv, x, xd, q, part, attn_out, rlogits,
+      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, ybuf, hdense, fcin, am_part, gtok, props,
+      committed, ncommitted, hpend, total;
+  int hist_ld, max_chunks, am_blocks;
+};
+
+Layout make_layout(const ocrdec_config& c, int am_blocks) {
+  Layout L{};
+  const size_t R = kRmax, B = c.max_batch, cap = c.kv_capacity, d = c.d_model, H = c.n_heads, Dh = c.head_dim;
+  const size_t E = c.n_experts, K = c.top_k, S = c.n_shared, f = c.expert_ffn;
+  const size_t F = std::max(c.dense_ffn, c.draft_ffn);
+  const size_t nslot = K + S;
+  L.hist_ld = c.kv_capacity + 8;
+  L.max_chunks = (c.kv_capacity + kAttnChunk - 1) / kAttnChunk;
+  L.am_blocks = am_blocks;
+  size_t o = 0;
+  auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
+  L.status = take(64);
+  L.counters = take(sizeof(int) * (2 * B * H + 16));
+  L.slots = take(sizeof(SlotState) * B);
+  L.rows = take(sizeof(PassRows));
+  L.hist = take(sizeof(int) * B * L.hist_ld);
+  L.rope = take(sizeof(float2) * cap * (Dh / 2));
+  L.kvk = take(2 * B * c.n_layers * H * cap * Dh);
+  L.kvv = take(2 * B * c.n_layers * H * cap * Dh);
+  L.dkvk = take(2 * B * H * cap * Dh);
+  L.dkvv = take(2 * B * H * cap * Dh);
+  L.x = take(4 * R * d);
+  L.xd = take(4 * R * d);
+  L.q = take(4 * R * d);
+  L.part = take(4 * R * H * L.max_chunks * (Dh + 2));
+  L.attn_out = take(2 * R * d);
+  L.rlogits = take(4 * R * E);
+  L.topk_ids = take(4 * R * K);
+  L.topk_gates = take(4 * R * K);
+  L.counts = take(4 * E);
+  L.offsets = take(4 * E);
+  L.rowlist = take(4 * R * K);
+  L.mats = take(4 * (E + S));
+  L.n_mats = take(4);
+  L.hbuf = take(2 * R * nslot * f);
+  L.ybuf = take(4 * R * nslot * d);
+  L.hdense = take(2 * R * F);
+  L.fcin = take(2 * R * 2 * d);
+  L.am_part = take(sizeof(float2) * am_blocks * kRmax);
+  L.gtok = take(4 * R);
+  L.props = take(4 * B * 4);
+  L.committed = take(4 * B * 4);
+  L.ncommitted = take(4 * B);
+  L.hpend = take(4 * B * (c.max_k + 1) * d);
+  L.total = o;
+  return L;
+}
+
+int device_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+cudaError_t prepare_kernels() {
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       2 * kAttnChunk * 128 * 2);
+  if (e != cudaSuccess) return e;
+  return gemv_prepare();
+}
+
+}  // namespace
+
+struct ocrdec_ctx {
+  ocrdec_config cfg;
+  Layout L{};
+  char* ws = nullptr;
+  bool have_weights = false;
+  int num_sms = 0;
+  bool pdl = false;
+  const bf16 *embed = nullptr, *final_norm = nullptr, *lm_head = nullptr;
+  std::vector<LayerW> layers;
+  DraftW dw{};
+  cudaStream_t cap_stream = nullptr;
+  std::map<std::tuple<int, int, void*, void*>, cudaGraphExec_t> graphs;
+  std::map<std::tuple<int, int, void*, void*>, int> graph_kernels;
+  const int* f_ref = nullptr;
+  const float* f_u = nullptr;
+  const int* f_alt = nullptr;
+  int f_npos = 0;
+  float f_p[3] = {0, 0, 0};
+  float* dbg_hidden = nullptr;
+  float* dbg_logits = nullptr;
+
+  template <class T>
+  T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
+  int* status() const { return at<int>(L.status); }
+  int* attn_counters(int which) const { return at<int>(L.counters) + which * cfg.max_batch * cfg.n_heads; }
+  int* am_counter(int which) const { return at<int>(L.counters) + 2 * cfg.max_batch * cfg.n_heads + which; }
+  // misc[0] = routed experts touched by verifier MoE layers, misc[1] = such layer passes
+  int* misc() const { return at<int>(L.counters) + 2 * cfg.max_batch * cfg.n_heads + 8; }
+  SlotState* slots() const { return at<SlotState>(L.slots); }
+  PassRows* rows() const { return at<PassRows>(L.rows); }
+  int* hist() const { return at<int>(L.hist); }
+  LaunchCfg lc(cudaStream_t s) const { return LaunchCfg{s, pdl, num_sms}; }
+
+  void drop_graphs() {
+    for (auto& kv : graphs) cudaGraphExecDestroy(kv.second);
+    graphs.clear();
+    graph_kernels.clear();
+  }
+};
+
+namespace {
+
+#define CK(expr)                                   \
+  do {                                             \
+    cudaError_t e_ = (expr);                       \
+    if (e_ != cudaSuccess) return OCRDEC_ECUDA;    \
+  } while (0)
+
+// ---------------------------------------------------------------------------
+// building blocks
+// ---------------------------------------------------------------------------
+
+struct BlockIO {
+  float* x;            // residual rows of the pass
+  bf16* kc;            // K cache of this block, slot 0 (layer offset applied)
+  bf16* vc;
+  long long slot_stride;
+  int* attn_counters;
+};
+
+int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* attn_norm, const bf16* wqkv,
+                   const bf16* wo, const BlockIO& io) {
+  const ocrdec_config& m = c->cfg;
+  PassRows* rows = c->rows();
+  GemvLaunch g;
+  g.s.W = wqkv;
+  g.s.N = 3 * m.d_model;
+  g.s.K = m.d_model;
+  g.s.pair_half = m.head_dim / 2;
+  g.s.nrows = &rows->n;
+  g.s.status = c->status();
+  gemv_plan(g.s);
+  g.src = SrcKind::Norm;
+  g.norm = SrcNorm::Params{io.x, m.d_model, nullptr, attn_norm, m.rms_eps};
+  g.epi = EpiKind::QKV;
+  g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
+                         m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
+  g.rows_bound = rmax;
+  CK(launch_gemv(g, lc));
+
+  AttnParams a{};
+  a.q = c->at<float>(c->L.q);
+  a.kc = io.kc;
+  a.vc = io.vc;
+  a.slot_stride = io.slot_stride;
+  a.cap = m.kv_capacity;
+  a.H = m.n_heads;
+  a.Dh = m.head_dim;
+  a.scale = 1.0f / std::sqrt((float)m.head_dim);
+  a.slot_row0 = rows->slot_row0;
+  a.slot_nrows = rows->slot_nrows;
+  a.row_pos = rows->pos;
+  a.part = c->at<float>(c->L.part);
+  a.max_chunks = c->L.max_chunks;
+  a.counters = io.attn_counters;
+  a.out = c->at<bf16>(c->L.attn_out);
+  a.status = c->status();
+  CK(launch_ex(attention_kernel, dim3(c->L.max_chunks, m.n_heads, m.max_batch), dim3(kAttnThreads),
+               (size_t)2 * kAttnChunk * m.head_dim * 2, lc, a));
+
+  GemvLaunch o;
+  o.s.W = wo;
+  o.s.N = m.d_model;
+  o.s.K = m.d_model;
+  o.s.nrows = &rows->n;
+  o.s.status = c->status();
+  gemv_plan(o.s);
+  o.src = SrcKind::Bf16;
+  o.bf = SrcBf16::Params{c->at<bf16>(c->L.attn_out), m.d_model, 1, nullptr};
+  o.epi = EpiKind::StoreAdd;
+  o.store = EpiStore<false>::Params{io.x, m.d_model, 1, nullptr};
+  o.rows_bound = rmax;
+  CK(launch_gemv(o, lc));
+  return OCRDEC_OK;
+}
+
+int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16* norm, const bf16* w_gu,
+              const bf16* w_down, int F) {
+  const ocrdec_config& m = c->cfg;
+  PassRows* rows = c->rows();
+  bf16* h = c->at<bf16>(c->L.hdense);
+  GemvLaunch g;
+  g.s.W = w_gu;
+  g.s.N = 2 * F;
+  g.s.K = m.d_model;
+  g.s.pair_half = F;
+  g.s.nrows = &rows->n;
+  g.s.status = c->status();
+  gemv_plan(g.s);
+  g.src = SrcKind::Norm;
+  g.norm = SrcNorm::Params{x, m.d_model, nullptr, norm, m.rms_eps};
+  g.epi = EpiKind::SwiGLU;
+  g.swiglu = EpiSwiGLU::Params{h, F, 1};
+  g.rows_bound = rmax;
+  CK(launch_gemv(g, lc));
+
+  GemvLaunch dn;
+  dn.s.W = w_down;
+  dn.s.N = m.d_model;
+  dn.s.K = F;
+  dn.s.nrows = &rows->n;
+  dn.s.status = c->status();
+  gemv_plan(dn.s);
+  dn.src = SrcKind::Bf16;
+  dn.bf = SrcBf16::Params{h, F, 1, nullptr};
+  dn.epi = EpiKind::StoreAdd;
+  dn.store = EpiStore<false>::Params{x, m.d_model, 1, nullptr};
+  dn.rows_bound = rmax;
+  CK(launch_gemv(dn, lc));
+  return OCRDEC_OK;
+}
+
+int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool count) {
+  const ocrdec_config& m = c->cfg;
+  PassRows* rows = c->rows();
+  float* x = c->at<float>(c->L.x);
+  const int nslot = m.top_k + m.n_shared;
+
+  GemvLaunch r;
+  r.s.W = w.router;
+  r.s.N = m.n_experts;
+  r.s.K = m.d_model;
+  r.s.nrows = &rows->n;
+  r.s.status = c->status();
+  gemv_plan(r.s);
+  r.src = SrcKind::Norm;
+  r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
+  r.epi = EpiKind::Store;
+  r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
+  r.rows_bound = rmax;
+  CK(launch_gemv(r, lc));
+
+  RouteParams rp{};
+  rp.logits = c->at<float>(c->L.rlogits);
+  rp.nrows = &rows->n;
+  rp.E = m.n_experts;
+  rp.top_k = m.top_k;
+  rp.S = m.n_shared;
+  rp.ids = c->at<int>(c->L.topk_ids);
+  rp.gates = c->at<float>(c->L.topk_gates);
+  rp.counts = c->at<int>(c->L.counts);
+  rp.offsets = c->at<int>(c->L.offsets);
+  rp.rowlist = c->at<int>(c->L.rowlist);
+  rp.mats = c->at<int>(c->L.mats);
+  rp.n_mats = c->at<int>(c->L.n_mats);
+  rp.touched = count ? c->misc() : nullptr;
+  rp.status = c->status();
+  CK(launch_ex(route_kernel, dim3(1), dim3(256), 0, lc, rp));
+
+  GemvShape es{};
+  es.n_experts = m.n_experts;
+  es.top_k = m.top_k;
+  es.mats = rp.mats;
+  es.n_mats = rp.n_mats;
+  es.counts = rp.counts;
+  es.offsets = rp.offsets;
+  es.rowlist = rp.rowlist;
+  es.nrows = &rows->n;
+  es.status = c->status();
+
+  GemvLaunch gu;
+  gu.s = es;
+  gu.s.W = w.exp_gu;
+  gu.s.W_sh = w.sh_gu;
+  gu.s.mat_stride = 2LL * m.expert_ffn * m.d_model;
+  gu.s.N = 2 * m.expert_ffn;
+  gu.s.K = m.d_model;
+  gu.s.pair_half = m.expert_ffn;
+  gemv_plan(gu.s);
+  gu.src = SrcKind::Norm;
+  gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
+  gu.epi = EpiKind::SwiGLU;
+  gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot};
+  gu.rows_bound = rmax;
+  CK(launch_gemv(gu, lc));
+
+  GemvLaunch dn;
+  dn.s = es;
+  dn.s.W = w.exp_down;
+  dn.s.W_sh = w.sh_down;
+  dn.s.mat_stride = (long long)m.d_model * m.expert_ffn;
+  dn.s.N = m.d_model;
+  dn.s.K = m.expert_ffn;
+  gemv_plan(dn.s);
+  dn.src = SrcKind::Bf16;
+  dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot, nullptr};
+  dn.epi = EpiKind::Store;
+  dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
+  dn.rows_bound = rmax;
+  CK(launch_gemv(dn, lc));
+
+  CombineParams cp{x, c->at<float>(c->L.ybuf), rp.gates, &rows->n, m.d_model, m.top_k, m.n_shared, c->status()};
+  CK(launch_ex(combine_kernel, dim3((kRmax * m.d_model + 255) / 256), dim3(256), 0, lc, cp));
+  return OCRDEC_OK;
+}
+
+// All verifier layers over the rows prepared in x / rows.
+int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
+  const ocrdec_config& m = c->cfg;
+  const long long layer_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
+  for (int l = 0; l < m.n_layers; ++l) {
+    const LayerW& w = c->layers[l];
+    BlockIO io{c->at<float>(c->L.x), c->at<bf16>(c->L.kvk) + l * layer_elems, c->at<bf16>(c->L.kvv) + l * layer_elems,
+               layer_elems * m.n_layers, c->attn_counters(0)};
+    int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
+    if (st) return st;
+    st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down, m.dense_ffn) : moe_ffn(c, lc, rmax, w, count);
+    if (st) return st;
+    if (c->dbg_hidden)
+      CK(cudaMemcpyAsync(c->dbg_hidden + (size_t)l * kRmax * m.d_model, io.x, sizeof(float) * kRmax * m.d_model,
+                         cudaMemcpyDeviceToDevice, lc.stream));
+  }
+  return OCRDEC_OK;
+}
+
+// final norm + LM head + argmax.  row_src selects x rows (nullptr: rows 0..);
+// nrows / rows_static the row count; tokens to tok[r * tok_stride].
+int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const bf16* norm, const int* row_src,
+            const int* nrows, int rows_static, int* tok, int tok_stride, float* logits, int which_counter) {
+  const ocrdec_config& m = c->cfg;
+  GemvLaunch g;
+  g.s.W = c->lm_head;
+  g.s.N = m.vocab;
+  g.s.K = m.d_model;
+  g.s.nrows = nrows;
+  g.s.rows_static = rows_static;
+  g.s.status = c->status();
+  g.s.counter = c->am_counter(which_counter);
+  gemv_plan(g.s);
+  g.src = SrcKind::Norm;
+  g.norm = SrcNorm::Params{x, m.d_model, row_src, norm, m.rms_eps};
+  g.epi = EpiKind::Argmax;
+  g.argmax = EpiArgmax::Params{tok, tok_stride, logits, c->at<float2>(c->L.am_part), nullptr};
+  g.rows_bound = rmax;
+  g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
+  CK(launch_gemv(g, lc));
+  return OCRDEC_OK;
+}
+
+// The draft block over the rows prepared by draft_setup (fcin, rows).
+// kv_only: stop after the draft KV append (prefill pairs whose outputs are unused).
+int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int* tok, int tok_stride) {
+  const ocrdec_config& m = c->cfg;
+  const DraftW& w = c->dw;
+  PassRows* rows = c->rows();
+  float* xd = c->at<float>(c->L.xd);
+  GemvLaunch fc;
+  fc.s.W = w.fc;
+  fc.s.N = m.d_model;
+  fc.s.K = 2 * m.d_model;
+  fc.s.nrows = &rows->n;
+  fc.s.status = c->status();
+  gemv_plan(fc.s);
+  fc.src = SrcKind::Bf16;
+  fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), 2 * m.d_model, 1, nullptr};
+  fc.epi = EpiKind::Store;
+  fc.store = EpiStore<false>::Params{xd, m.d_model, 1, nullptr};
+  fc.rows_bound = rmax;
+  CK(launch_gemv(fc, lc));
+
+  const long long slot_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
+  BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems, c->attn_counters(1)};
+  if (kv_only) {
+    GemvLaunch g;
+    g.s.W = w.wqkv;
+    g.s.N = 3 * m.d_model;
+    g.s.K = m.d_model;
+    g.s.pair_half = m.head_dim / 2;
+    g.s.nrows = &rows->n;
+    g.s.status = c->status();
+    gemv_plan(g.s);
+    g.src = SrcKind::Norm;
+    g.norm = SrcNorm::Params{xd, m.d_model, nullptr, w.attn_norm, m.rms_eps};
+    g.epi = EpiKind::QKV;
+    g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
+                           m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
+    g.rows_bound = rmax;
+    CK(launch_gemv(g, lc));
+    return OCRDEC_OK;
+  }
+  int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
+  if (st) return st;
+  st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down, m.draft_ffn);
+  if (st) return st;
+  return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, nullptr, 1);
+}
+
+int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) {
+  const ocrdec_config& m = c->cfg;
+  for (int j = 1; j <= k; ++j) {
+    DraftSetupParams dp{};
+    dp.mode = j == 1 ? 0 : 1;
+    dp.B = B;
+    dp.j = j;
+    dp.d = m.d_model;
+    dp.max_k = m.max_k;
+    dp.eps = m.rms_eps;
+    dp.slots = c->slots();
+    dp.hist = c->hist();
+    dp.hist_ld = c->L.hist_ld;
+    dp.hpend = c->at<float>(c->L.hpend);
+    dp.xd = c->at<float>(c->L.xd);
+    dp.dtok = props + (j >= 2 ? j - 2 : 0);
+    dp.dtok_stride = k;
+    dp.embed = c->embed;
+    dp.g_h = c->dw.norm_h;
+    dp.g_e = c->dw.norm_e;
+    dp.fcin = c->at<bf16>(c->L.fcin);
+    dp.rows = c->rows();
+    dp.rows_prev = c->rows();
+    dp.status = c->status();
+    CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
+    int rmax = j == 1 ? std::min(kRmax, B * (m.max_k + 1)) : B;
+    int st = draft_block(c, lc, rmax, false, props + (j - 1), k);
+    if (st) return st;
+  }
+  return OCRDEC_OK;
+}
+
+int enqueue_force(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) {
+  if (!c->f_ref || k == 0) return OCRDEC_OK;
+  ForceParams fp{c->slots(), props, B, k, c->cfg.max_k, c->f_ref, c->f_u, c->f_alt, c->f_npos,
+                 c->f_p[0], c->f_p[1], c->f_p[2], c->status()};
+  CK(launch_ex(force_kernel, dim3(1), dim3(32), 0, lc, fp));
+  return OCRDEC_OK;
+}
+
+int enqueue_verify(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, const int* props, int* committed,
+                   int* ncommitted) {
+  const ocrdec_config& m = c->cfg;
+  const int R = B * (k + 1);
+  VerifySetupParams vp{c->slots(), props, B, k, m.kv_capacity, m.d_model, m.vocab, c->embed,
+                       c->at<float>(c->L.x), c->rows(), c->status()};
+  CK(launch_ex(verify_setup_kernel, dim3(1), dim3(256), 0, lc, vp));
+  int st = verifier_layers(c, lc, R, true);
+  if (st) return st;
+  st = lm_head(c, lc, R, c->at<float>(c->L.x), c->final_norm, nullptr, &c->rows()->n, 0, c->at<int>(c->L.gtok), 1,
+               c->dbg_logits, 0);
+  if (st) return st;
+  AcceptParams ap{c->slots(), c->at<int>(c->L.gtok), props, B, k, m.d_model, m.max_k, c->hist(), c->L.hist_ld,
+                  c->at<float>(c->L.x), c->at<float>(c->L.hpend), committed, ncommitted, c->status()};
+  CK(launch_ex(accept_kernel, dim3(1), dim3(256), 0, lc, ap));
+  return OCRDEC_OK;
+}
+
+int enqueue_step(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* committed, int* ncommitted) {
+  int* props = c->at<int>(c->L.props);
+  int st = OCRDEC_OK;
+  if (k > 0) {
+    st = enqueue_draft(c, lc, B, k, props);
+    if (st) return st;
+    st = enqueue_force(c, lc, B, k, props);
+    if (st) return st;
+  }
+  return enqueue_verify(c, lc, B, k, props, committed, ncommitted);
+}
+
+int check_ready(const ocrdec_ctx* c) {
+  if (!c) return OCRDEC_EINVAL;
+  if (!c->ws || !c->have_weights) return OCRDEC_ESTATE;
+  return OCRDEC_OK;
+}
+
+int check_bk(const ocrdec_ctx* c, int batch, int k) {
+  if (batch < 1 || batch > c->cfg.max_batch || k < 0 || k > c->cfg.max_k) return OCRDEC_EINVAL;
+  if (batch * (k + 1) > kRmax) return OCRDEC_EINVAL;
+  return OCRDEC_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+int ocrdec_create(const ocrdec_config* cfg, ocrdec_ctx** out) {
+  if (!out) return OCRDEC_EINVAL;
+  *out = nullptr;
+  if (!config_ok(cfg)) return OCRDEC_EINVAL;
+  ocrdec_ctx* c = new (std::nothrow) ocrdec_ctx();
+  if (!c) return OCRDEC_ENOMEM;
+  c->cfg = *cfg;
+  c->num_sms = device_sms();
+  if (c->num_sms <= 0) c->num_sms = 148;
+  c->L = make_layout(*cfg, c->num_sms);
+  *out = c;
+  return OCRDEC_OK;
+}
+
+void ocrdec_destroy(ocrdec_ctx* c) {
+  if (!c) return;
+  c->drop_graphs();
+  if (c->cap_stream) cudaStreamDestroy(c->cap_stream);
+  delete c;
+}
+
+int ocrdec_weight_count(const ocrdec_config* cfg) {
+  if (!config_ok(cfg)) return -OCRDEC_EINVAL;
+  std::vector<std::vector<int64_t>> m;
+  manifest(*cfg, m);
+  return (int)m.size();
+}
+
+int ocrdec_weight_info(const ocrdec_config* cfg, int index, int64_t dims[3], int32_t* ndim) {
+  if (!config_ok(cfg) || !dims || !ndim) return OCRDEC_EINVAL;
+  std::vector<std::vector<int64_t>> m;
+  manifest(*cfg, m);
+  if (index < 0 || index >= (int)m.size()) return OCRDEC_EINVAL;
+  *ndim = (int32_t)m[index].size();
+  for (int i = 0; i < 3; ++i) dims[i] = i < *ndim ? m[index][i] : 0;
+  return OCRDEC_OK;
+}
+
+size_t ocrdec_workspace_bytes(const ocrdec_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  int sms = device_sms();
+  return make_layout(*cfg, sms > 0 ? sms : 148).total;
+}
+
+int ocrdec_bind_workspace(ocrdec_ctx* c, void* ws, size_t bytes, ocrdec_stream stream) {
+  if (!c || !ws || (reinterpret_cast<uintptr_t>(ws) & 255)) return OCRDEC_EINVAL;
+  if (bytes < c->L.total) return OCRDEC_ENOMEM;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  c->ws = static_cast<char*>(ws);
+  c->drop_graphs();
+  CK(prepare_kernels());
+  // status, counters, slots, rows and token history start at zero
+  CK(cudaMemsetAsync(c->ws, 0, c->L.rope, s));
+  const ocrdec_config& m = c->cfg;
+  long long n = (long long)m.kv_capacity * (m.head_dim / 2);
+  rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(c->at<float2>(c->L.rope), m.kv_capacity, m.head_dim,
+                                                                  (double)m.rope_theta);
+  CK(cudaGetLastError());
+  if (!c->cap_stream) CK(cudaStreamCreateWithFlags(&c->cap_stream, cudaStreamNonBlocking));
+  return OCRDEC_OK;
+}
+
+int ocrdec_load_weights(ocrdec_ctx* c, const void* const* ptrs, int n) {
+  if (!c || !ptrs) return OCRDEC_EINVAL;
+  const ocrdec_config& m = c->cfg;
+  std::vector<std::vector<int64_t>> man;
+  manifest(m, man);
+  if (n != (int)man.size()) return OCRDEC_EINVAL;
+  for (int i = 0; i < n; ++i)
+    if (!ptrs[i] || (reinterpret_cast<uintptr_t>(ptrs[i]) & 15)) return OCRDEC_EINVAL;
+  auto W = [&](int i) { return static_cast<const bf16*>(ptrs[i]); };
+  int i = 0;
+  c->embed = W(i++);
+  c->layers.assign(m.n_layers, LayerW{});
+  for (int l = 0; l < m.n_layers; ++l) {
+    LayerW& L = c->layers[l];
+    L.attn_norm = W(i++);
+    L.wqkv = W(i++);
+    L.wo = W(i++);
+    L.ffn_norm = W(i++);
+    L.dense = l < m.n_dense_first;
+    if (L.dense) {
+      L.w_gu = W(i++);
+      L.w_down = W(i++);
+    } else {
+      L.router = W(i++);
+      L.exp_gu = W(i++);
+      L.exp_down = W(i++);
+      L.sh_gu = W(i++);
+      L.sh_down = W(i++);
+    }
+  }
+  c->final_norm = W(i++);
+  c->lm_head = W(i++);
+  DraftW& d = c->dw;
+  d.norm_h = W(i++);
+  d.norm_e = W(i++);
+  d.fc = W(i++);
+  d.attn_norm = W(i++);
+  d.wqkv = W(i++);
+  d.wo = W(i++);
+  d.ffn_norm = W(i++);
+  d.w_gu = W(i++);
+  d.w_down = W(i++);
+  d.final_norm = W(i++);
+  c->have_weights = true;
+  c->drop_graphs();
+  return OCRDEC_OK;
+}
+
+int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, const int32_t* prompt, int n_prompt,
+                   int32_t* first_token, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  const ocrdec_config& m = c->cfg;
+  const int C = n_visual + n_prompt;
+  if (slot < 0 || slot >= m.max_batch || n_visual < 0 || n_prompt < 0 || C < 1) return OCRDEC_EINVAL;
+  if ((n_visual > 0 && !visual) || (n_prompt > 0 && !prompt)) return OCRDEC_EINVAL;
+  if (C + m.max_k + 2 > m.kv_capacity) return OCRDEC_ECAPACITY;
+  LaunchCfg lc = c->lc(reinterpret_cast<cudaStream_t>(stream));
+  int last_p0 = 0;
+  for (int p0 = 0; p0 < C; p0 += kPrefillChunk) {
+    const int n = std::min(kPrefillChunk, C - p0);
+    PrefillSetupParams ps{slot, p0, n, n_visual, m.vocab, n_prompt, visual, prompt, c->embed, m.d_model,
+                          c->at<float>(c->L.x), c->rows(), c->status()};
+    CK(launch_ex(prefill_setup_kernel, dim3(1), dim3(256), 0, lc, ps));
+    st = verifier_layers(c, lc, n, false);
+    if (st) return st;
+    if (p0 + n == C) {
+      st = lm_head(c, lc, 1, c->at<float>(c->L.x), c->final_norm, c->rows()->last_row, nullptr, 1,
+                   c->at<int>(c->L.gtok), 1, nullptr, 0);
+      if (st) return st;
+      last_p0 = p0;
+    }
+    const int q1 = std::min(p0 + n, C - 1);
+    if (q1 > p0) {
+      DraftSetupParams dp{};
+      dp.mode = 2;
+      dp.B = 1;
+      dp.d = m.d_model;
+      dp.max_k = m.max_k;
+      dp.eps = m.rms_eps;
+      dp.slots = c->slots();
+      dp.slot = slot;
+      dp.p0 = p0;
+      dp.n = q1 - p0;
+      dp.n_visual = n_visual;
+      dp.xv = c->at<float>(c->L.x);
+      dp.visual = visual;
+      dp.prompt = prompt;
+      dp.embed = c->embed;
+      dp.g_h = c->dw.norm_h;
+      dp.g_e = c->dw.norm_e;
+      dp.fcin = c->at<bf16>(c->L.fcin);
+      dp.rows = c->rows();
+      dp.rows_prev = c->rows();
+      dp.status = c->status();
+      // the verifier rows of this chunk are needed by the draft setup and, on the
+      // last chunk, by the finish step: run the finish first when both apply
+      if (p0 + n == C) {
+        PrefillFinishParams pf{c->slots(), slot, C, C - 1 - p0, m.d_model, m.max_k, c->at<int>(c->L.gtok),
+                               c->at<float>(c->L.x), c->at<float>(c->L.hpend), c->hist(), c->L.hist_ld,
+                               first_token, c->status()};
+        CK(launch_ex(prefill_finish_kernel, dim3(1), dim3(256), 0, lc, pf));
+      }
+      CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
+      st = draft_block(c, lc, q1 - p0, true, nullptr, 0);
+      if (st) return st;
+    } else if (p0 + n == C) {
+      PrefillFinishParams pf{c->slots(), slot, C, C - 1 - p0, m.d_model, m.max_k, c->at<int>(c->L.gtok),
+                             c->at<float>(c->L.x), c->at<float>(c->L.hpend), c->hist(), c->L.hist_ld,
+                             first_token, c->status()};
+      CK(launch_ex(prefill_finish_kernel, dim3(1), dim3(256), 0, lc, pf));
+    }
+  }
+  (void)last_p0;
+  return OCRDEC_OK;
+}
+
+int ocrdec_draft(ocrdec_ctx* c, int batch, int k, int32_t* props, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  if ((st = check_bk(c, batch, k))) return st;
+  if (k < 1 || !props) return OCRDEC_EINVAL;
+  return enqueue_draft(c, c->lc(reinterpret_cast<cudaStream_t>(stream)), batch, k, props);
+}
+
+int ocrdec_verify_commit(ocrdec_ctx* c, int batch, int k, const int32_t* props, int32_t* committed,
+                         int32_t* ncommitted, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  if ((st = check_bk(c, batch, k))) return st;
+  if ((k > 0 && !props) || !committed || !ncommitted) return OCRDEC_EINVAL;
+  return enqueue_verify(c, c->lc(reinterpret_cast<cudaStream_t>(stream)), batch, k, props, committed, ncommitted);
+}
+
+int ocrdec_step(ocrdec_ctx* c, int batch, int k, int32_t* committed, int32_t* ncommitted, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  if ((st = check_bk(c, batch, k))) return st;
+  if (!committed || !ncommitted) return OCRDEC_EINVAL;
+  auto key = std::make_tuple(batch, k, (void*)committed, (void*)ncommitted);
+  auto itg = c->graphs.find(key);
+  cudaGraphExec_t exec = nullptr;
+  if (itg == c->graphs.end()) {
+    cudaGraph_t graph = nullptr;
+    CK(cudaStreamBeginCapture(c->cap_stream, cudaStreamCaptureModeThreadLocal));
+    st = enqueue_step(c, c->lc(c->cap_stream), batch, k, committed, ncommitted);
+    cudaError_t e = cudaStreamEndCapture(c->cap_stream, &graph);
+    if (st) {
+      if (graph) cudaGraphDestroy(graph);
+      return st;
+    }
+    if (e != cudaSuccess) return OCRDEC_ECUDA;
+    size_t nn = 0;
+    int nk = 0;
+    if (cudaGraphGetNodes(graph, nullptr, &nn) == cudaSuccess && nn > 0) {
+      std::vector<cudaGraphNode_t> nodes(nn);
+      if (cudaGraphGetNodes(graph, nodes.data(), &nn) == cudaSuccess)
+        for (auto nd : nodes) {
+          cudaGraphNodeType t;
+          if (cudaGraphNodeGetType(nd, &t) == cudaSuccess && t == cudaGraphNodeTypeKernel) ++nk;
+        }
+    }
+    c->graph_kernels[key] = nk;
+    e = cudaGraphInstantiate(&exec, graph, 0);
+    cudaGraphDestroy(graph);
+    if (e != cudaSuccess) return OCRDEC_ECUDA;
+    c->graphs[key] = exec;
+  } else {
+    exec = itg->second;
+  }
+  CK(cudaGraphLaunch(exec, reinterpret_cast<cudaStream_t>(stream)));
+  return OCRDEC_OK;
+}
+
+int ocrdec_step_host(ocrdec_ctx* c, int batch, int k, int32_t* host_committed, int32_t* host_n, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  if (!host_committed || !host_n) return OCRDEC_EINVAL;
+  int* dc = c->at<int>(c->L.committed);
+  int* dn = c->at<int>(c->L.ncommitted);
+  if ((st = ocrdec_step(c, batch, k, dc, dn, stream))) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(host_committed, dc, sizeof(int) * batch * (k + 1), cudaMemcpyDeviceToHost, s));
+  CK(cudaMemcpyAsync(host_n, dn, sizeof(int) * batch, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return OCRDEC_OK;
+}
+
+int ocrdec_set_forced_acceptance(ocrdec_ctx* c, const int32_t* ref, const float* u, const int32_t* alt, int n_pos,
+                                 const float* host_p) {
+  if (!c) return OCRDEC_EINVAL;
+  c->drop_graphs();
+  if (!ref) {
+    c->f_ref = nullptr;
+    return OCRDEC_OK;
+  }
+  if (!u || !alt || n_pos <= 0 || !host_p) return OCRDEC_EINVAL;
+  c->f_ref = ref;
+  c->f_u = u;
+  c->f_alt = alt;
+  c->f_npos = n_pos;
+  for (int j = 0; j < 3; ++j) c->f_p[j] = j < c->cfg.max_k ? host_p[j] : 0.f;
+  return OCRDEC_OK;
+}
+
+int ocrdec_get_status(ocrdec_ctx* c, int32_t* host_status, ocrdec_stream stream) {
+  if (!c || !host_status) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(host_status, c->status(), sizeof(int), cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return OCRDEC_OK;
+}
+
+int ocrdec_clear_status(ocrdec_ctx* c, ocrdec_stream stream) {
+  if (!c) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  CK(cudaMemsetAsync(c->status(), 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+  return OCRDEC_OK;
+}
+
+int ocrdec_get_slot_stats(ocrdec_ctx* c, int slot, ocrdec_slot_stats* out, ocrdec_stream stream) {
+  if (!c || !out || slot < 0 || slot >= c->cfg.max_batch) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  static_assert(sizeof(ocrdec_slot_stats) == 10 * sizeof(int32_t), "stats layout");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(out, c->slots() + slot, sizeof(ocrdec_slot_stats), cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return OCRDEC_OK;
+}
+
+int ocrdec_token_history(ocrdec_ctx* c, int slot, const int32_t** dev_tokens) {
+  if (!c || !dev_tokens || slot < 0 || slot >= c->cfg.max_batch) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  *dev_tokens = c->hist() + (size_t)slot * c->L.hist_ld;
+  return OCRDEC_OK;
+}
+
+int ocrdec_get_counters(ocrdec_ctx* c, int32_t* host, int n, ocrdec_stream stream) {
+  if (!c || !host || n < 1 || n > 2) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(host, c->misc(), sizeof(int32_t) * n, cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  return OCRDEC_OK;
+}
+
+int ocrdec_reset_counters(ocrdec_ctx* c, ocrdec_stream stream) {
+  if (!c) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  CK(cudaMemsetAsync(c->misc(), 0, 2 * sizeof(int32_t), reinterpret_cast<cudaStream_t>(stream)));
+  return OCRDEC_OK;
+}
+
+int ocrdec_step_kernel_count(ocrdec_ctx* c, int batch, int k, int32_t* dev_committed, int32_t* dev_n_committed,
+                             int32_t* count) {
+  if (!c || !count) return OCRDEC_EINVAL;
+  auto it = c->graph_kernels.find(std::make_tuple(batch, k, (void*)dev_committed, (void*)dev_n_committed));
+  if (it == c->graph_kernels.end()) return OCRDEC_ESTATE;
+  *count = it->second;
+  return OCRDEC_OK;
+}
+
+int ocrdec_set_debug_taps(ocrdec_ctx* c, float* hidden, float* logits) {
+  if (!c) return OCRDEC_EINVAL;
+  c->dbg_hidden = hidden;
+  c->dbg_logits = logits;
+  c->drop_graphs();
+  return OCRDEC_OK;
+}
+
+const char* ocrdec_strerror(int s) {
+  switch (s) {
+    case OCRDEC_OK: return "ok";
+    case OCRDEC_EINVAL: return "invalid argument";
+    case OCRDEC_ENOMEM: return "workspace too small";
+    case OCRDEC_ECUDA: return "CUDA runtime error";
+    case OCRDEC_ECAPACITY: return "KV capacity exceeded";
+    case OCRDEC_ETIMEOUT: return "device wait timed out";
+    case OCRDEC_ESTATE: return "call order violated";
+    default: return "unknown status";
+  }
+}
+
+// ---- single-kernel entry points -------------------------------------------
+
+size_t ocrdec_op_scratch_bytes(void) {
+  int sms = device_sms();
+  return 256 + sizeof(float2) * (size_t)(sms > 0 ? sms : 148) * kRmax;
+}
+
+int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps, int R, int N, int K, float* y,
+                        void* scratch, ocrdec_stream stream) {
+  if (!W || !x || !g || !y || !scratch || R < 1 || R > kRmax || N < kTR || N % kTR || K < 8 || K % 8 ||
+      K * 2 > 4096 * 2)
+    return OCRDEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* st = static_cast<int*>(scratch);
+  CK(prepare_kernels());
+  CK(cudaMemsetAsync(st, 0, 16, s));
+  GemvLaunch gl;
+  gl.s.W = static_cast<const bf16*>(W);
+  gl.s.N = N;
+  gl.s.K = K;
+  gl.s.rows_static = R;
+  gl.s.status = st;
+  gemv_plan(gl.s);
+  gl.src = SrcKind::Norm;
+  gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};
+  gl.epi = EpiKind::Store;
+  gl.store = EpiStore<false>::Params{y, N, 1, nullptr};
+  gl.rows_bound = R;
+  LaunchCfg lc{s, false, device_sms()};
+  CK(launch_gemv(gl, lc));
+  return OCRDEC_OK;
+}
+
+int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps, int R, int N, int K, int32_t* tok,
+                        float* logits, void* scratch, ocrdec_stream stream) {
+  if (!W || !x || !g || !tok || !scratch || R < 1 || R > kRmax || N < kTR || N % kTR || K < 8 || K % 8 ||
+      K > 4096)
+    return OCRDEC_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  int* st = static_cast<int*>(scratch);
+  CK(prepare_kernels());
+  CK(cudaMemsetAsync(st, 0, 16, s));
+  int sms = device_sms();
+  GemvLaunch gl;
+  gl.s.W = static_cast<const bf16*>(W);
+  gl.s.N = N;
+  gl.s.K = K;
+  gl.s.rows_static = R;
+  gl.s.status = st;
+  gl.s.counter = st + 1;
+  gemv_plan(gl.s);
+  gl.src = SrcKind::Norm;
+  gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};
+  gl.epi = EpiKind::Argmax;
+  gl.argmax = EpiArgmax::Params{tok, 1, logits, reinterpret_cast<float2*>(static_cast<char*>(scratch) + 256), nullptr};
+  gl.rows_bound = R;
+  gl.grid = std::min(gl.s.tiles_per_mat, sms);
+  LaunchCfg lc{s, false, sms};
+  CK(launch_gemv(gl, lc));
+  return OCRDEC_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,61 @@
+// Host-side launch helpers shared by the library's translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+
+#include "gemv.cuh"
+
+namespace ocrdec {
+
+struct LaunchCfg {
+  cudaStream_t stream;
+  bool pdl;     // launch with programmatic stream serialization
+  int num_sms;
+};
+
+// cudaLaunchKernelEx with optional programmatic dependent launch.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, const LaunchCfg& lc,
+                      Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = lc.stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = lc.pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+enum class SrcKind { Norm, Bf16 };
+enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax };
+
+// One GEMV launch: shape + the parameters of the chosen source and epilogue.
+struct GemvLaunch {
+  GemvShape s{};
+  SrcKind src = SrcKind::Norm;
+  EpiKind epi = EpiKind::Store;
+  SrcNorm::Params norm{};
+  SrcBf16::Params bf{};
+  EpiStore<false>::Params store{};
+  EpiSwiGLU::Params swiglu{};
+  EpiQKV::Params qkv{};
+  EpiArgmax::Params argmax{};
+  int rows_bound = kRmax;  // static bound on rows of one work item (selects the row-group width)
+  int grid = 0;            // 0: derived from the work and the SM count
+};
+
+// Fills cps/ns/tiles_per_mat for tile height kTR and stage size.
+void gemv_plan(GemvShape& s);
+cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
+// Raises the dynamic shared-memory limit of every GEMV instantiation to the
+// largest size any launch uses (call outside stream capture, once per device).
+cudaError_t gemv_prepare();
+constexpr int kGemvMaxK = 4096;  // largest K of a normalised (shared-memory) source
+
+constexpr int kTR = 8;  // weight rows per tile on every GEMV
+
+}  // namespace ocrdec

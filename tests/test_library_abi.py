@@ -1,0 +1,86 @@
+"""The C-ABI library builds for sm_100a, loads without a GPU and exports every
+entry point declared in include/ocrdec.h.  No compute is called here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from speculative_moe_decoding_b200 import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "ocrdec.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from speculative_moe_decoding_b200 import build
+    build.build(jobs=4)
+    from speculative_moe_decoding_b200 import ocrdec
+    return ocrdec
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = set(re.findall(r"\b(ocrdec_[a-z0-9_]+)\s*\(", text))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 20
+    for n in names:
+        assert hasattr(lib.lib, n), n
+
+
+def test_no_unexpected_exports(lib):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", lib.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {l.split()[-1] for l in out.splitlines() if " T " in l}
+    ours = {n for n in exported if n.startswith("ocrdec_")}
+    assert ours == set(declared_functions())
+
+
+@pytest.mark.parametrize("dims", [synth.TINY, synth.FULL])
+def test_manifest_matches_generator(lib, dims):
+    cfg = lib.make_config(dims.as_dict(), 3, 1, 2048)
+    got = lib.manifest(cfg)
+    want = [shape for _, shape in synth.manifest(dims)]
+    assert got == want
+    assert lib.ocrdec_workspace_bytes(ctypes.byref(cfg)) > 0
+
+
+def test_config_validation(lib):
+    good = synth.TINY.as_dict()
+    ctx = ctypes.c_void_p()
+    cfg = lib.make_config(good, 3, 1, 256)
+    assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.OK
+    lib.ocrdec_destroy(ctx)
+    bad_cases = [
+        dict(good, n_heads=3),             # heads * head_dim != d
+        dict(good, top_k=9),               # top_k > n_experts
+        dict(good, shared_ffn=64),         # shared width must equal expert width
+        dict(good, vocab=4095),            # vocab multiple of 8
+    ]
+    for bad in bad_cases:
+        cfg = lib.make_config(bad, 3, 1, 256)
+        assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
+    cfg = lib.make_config(good, 4, 1, 256)  # max_k > 3
+    assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
+    cfg = lib.make_config(good, 3, 3, 256)  # batch * (k+1) rows beyond one pass
+    assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
+
+
+def test_calls_before_setup_fail_cleanly(lib):
+    ctx = ctypes.c_void_p()
+    cfg = lib.make_config(synth.TINY.as_dict(), 3, 1, 256)
+    assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.OK
+    try:
+        assert lib.ocrdec_step(ctx, 1, 0, None, None, None) in (lib.ESTATE, lib.EINVAL)
+        assert lib.ocrdec_prefill(ctx, 0, None, 0, None, 0, None, None) == lib.ESTATE
+        assert lib.ocrdec_draft(ctx, 1, 1, None, None) == lib.ESTATE
+        assert lib.ocrdec_bind_workspace(ctx, None, 0, None) == lib.EINVAL
+        assert lib.ocrdec_strerror(lib.ECAPACITY) == b"KV capacity exceeded"
+    finally:
+        lib.ocrdec_destroy(ctx)
