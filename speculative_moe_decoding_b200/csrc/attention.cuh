@@ -81,8 +81,7 @@ attention_kernel(const AttnParams p) {
   for (int i = 0; i < nr; ++i)
     for (int d = tid; d < Dh; d += kAttnThreads) qs[i][d] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + d];
   __syncthreads();
-  bool ok = mbar_wait(&bar, 0, p.status);
-  if (!ok) return;  // status recorded; no copy can still be pending after a failed wait of this barrier
+  mbar_wait(&bar, 0, p.status);  // gives up with OCRDEC_ETIMEOUT recorded; control flow stays uniform
 
   // ---- scores: 4 lanes-groups of 8 per warp, one position per group ----
   // lane l8 of a group owns the 16-byte dim-chunks l8 and l8 + 8 of a key row

@@ -459,8 +459,9 @@ gemv_kernel(const GemvShape s, const typename Src::Params sp, const typename Epi
         for (int ps = 0; ps < passes && ok; ++ps) {
           for (int sl = 0; sl < s.ns && ok; ++sl, ++it) {
             int st = it % kStages;
-            if (it >= kStages) ok = mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
-            if (!ok) break;
+            // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
+            // stays uniform so the block always terminates
+            if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
             int c0 = sl * s.cps;
             int cn = min(s.cps, nch - c0);
             uint32_t seg = cn * 16;
@@ -514,7 +515,7 @@ gemv_kernel(const GemvShape s, const typename Src::Params sp, const typename Epi
       float acc[TR][RG];
       for (int sl = 0; sl < s.ns; ++sl, ++it) {
         int st = it % kStages;
-        if (!mbar_wait(&full_bar[st], (it / kStages) & 1, s.status)) { ok = false; break; }
+        mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
         const unsigned char* w_st = stages + st * kStageBytes;
         int c0 = sl * s.cps;
         int cn = min(s.cps, nch - c0);
