@@ -23,16 +23,33 @@ namespace {
 
 constexpr int kPrefillChunk = kRmax;  // context rows per prefill pass
 
+// One weight matrix (or array of E expert matrices) with its tensor map.
+struct Mat {
+  const bf16* p = nullptr;
+  int N = 0, K = 0, E = 1;
+  CUtensorMap map;
+};
+
 struct LayerW {
-  const bf16 *attn_norm, *wqkv, *wo, *ffn_norm;
-  const bf16 *w_gu, *w_down;                                  // dense layers
-  const bf16 *router, *exp_gu, *exp_down, *sh_gu, *sh_down;   // MoE layers
+  const bf16 *attn_norm, *ffn_norm;
+  Mat wqkv, wo;
+  Mat w_gu, w_down;                                 // dense layers
+  Mat router, exp_gu, exp_down, sh_gu, sh_down;     // MoE layers
   bool dense;
 };
 
 struct DraftW {
-  const bf16 *norm_h, *norm_e, *fc, *attn_norm, *wqkv, *wo, *ffn_norm, *w_gu, *w_down, *final_norm;
+  const bf16 *norm_h, *norm_e, *attn_norm, *ffn_norm, *final_norm;
+  Mat fc, wqkv, wo, w_gu, w_down;
 };
+
+bool make_mat(Mat& m, const void* p, int N, int K, int E) {
+  m.p = static_cast<const bf16*>(p);
+  m.N = N;
+  m.K = K;
+  m.E = E;
+  return encode_weight_map(p, K, N, E, &m.map) == cudaSuccess;
+}
 
 void manifest(const ocrdec_config& c, std::vector<std::vector<int64_t>>& m) {
   const int64_t d = c.d_model, V = c.vocab, E = c.n_experts, S = c.n_shared;
@@ -76,7 +93,7 @@ bool config_ok(const ocrdec_config* c) {
     if (v <= 0) return false;
   if (c->n_heads * c->head_dim != c->d_model) return false;
   if (c->head_dim % 16 || c->head_dim > 128) return false;
-  if (c->d_model % 8 || c->expert_ffn % 8 || c->draft_ffn % 8 || c->vocab % kTR) return false;
+  if (c->d_model % 8 || c->expert_ffn % 8 || c->draft_ffn % 8 || c->vocab % 8) return false;
   if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
   if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % 8)) return false;
   if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
@@ -168,7 +185,8 @@ struct ocrdec_ctx {
   bool have_weights = false;
   int num_sms = 0;
   bool pdl = false;
-  const bf16 *embed = nullptr, *final_norm = nullptr, *lm_head = nullptr;
+  const bf16 *embed = nullptr, *final_norm = nullptr;
+  Mat lm_head;
   std::vector<LayerW> layers;
   DraftW dw{};
   cudaStream_t cap_stream = nullptr;
@@ -221,24 +239,32 @@ struct BlockIO {
   int* attn_counters;
 };
 
-int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* attn_norm, const bf16* wqkv,
-                   const bf16* wo, const BlockIO& io) {
+// A GEMV launch over one dense matrix.
+GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* nrows, int rows_static, int rmax) {
+  GemvLaunch g;
+  g.tm_w = m.map;
+  g.tm_sh = m.map;
+  g.s.N = m.N;
+  g.s.K = m.K;
+  g.s.pair_half = pair_half;
+  g.s.nrows = nrows;
+  g.s.rows_static = rows_static;
+  g.s.status = c->status();
+  g.rows_bound = rmax;
+  gemv_plan(g.s);
+  return g;
+}
+
+int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* attn_norm, const Mat& wqkv,
+                   const Mat& wo, const BlockIO& io) {
   const ocrdec_config& m = c->cfg;
   PassRows* rows = c->rows();
-  GemvLaunch g;
-  g.s.W = wqkv;
-  g.s.N = 3 * m.d_model;
-  g.s.K = m.d_model;
-  g.s.pair_half = m.head_dim / 2;
-  g.s.nrows = &rows->n;
-  g.s.status = c->status();
-  gemv_plan(g.s);
+  GemvLaunch g = dense_launch(c, wqkv, m.head_dim / 2, &rows->n, 0, rmax);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{io.x, m.d_model, nullptr, attn_norm, m.rms_eps};
   g.epi = EpiKind::QKV;
   g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
                          m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
-  g.rows_bound = rmax;
   CK(launch_gemv(g, lc));
 
   AttnParams a{};
@@ -261,54 +287,33 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   CK(launch_ex(attention_kernel, dim3(c->L.max_chunks, m.n_heads, m.max_batch), dim3(kAttnThreads),
                (size_t)2 * kAttnChunk * m.head_dim * 2, lc, a));
 
-  GemvLaunch o;
-  o.s.W = wo;
-  o.s.N = m.d_model;
-  o.s.K = m.d_model;
-  o.s.nrows = &rows->n;
-  o.s.status = c->status();
-  gemv_plan(o.s);
+  GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax);
   o.src = SrcKind::Bf16;
   o.bf = SrcBf16::Params{c->at<bf16>(c->L.attn_out), m.d_model, 1, nullptr};
   o.epi = EpiKind::StoreAdd;
   o.store = EpiStore<false>::Params{io.x, m.d_model, 1, nullptr};
-  o.rows_bound = rmax;
   CK(launch_gemv(o, lc));
   return OCRDEC_OK;
 }
 
-int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16* norm, const bf16* w_gu,
-              const bf16* w_down, int F) {
+int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16* norm, const Mat& w_gu,
+              const Mat& w_down) {
   const ocrdec_config& m = c->cfg;
   PassRows* rows = c->rows();
+  const int F = w_down.K;
   bf16* h = c->at<bf16>(c->L.hdense);
-  GemvLaunch g;
-  g.s.W = w_gu;
-  g.s.N = 2 * F;
-  g.s.K = m.d_model;
-  g.s.pair_half = F;
-  g.s.nrows = &rows->n;
-  g.s.status = c->status();
-  gemv_plan(g.s);
+  GemvLaunch g = dense_launch(c, w_gu, F, &rows->n, 0, rmax);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{x, m.d_model, nullptr, norm, m.rms_eps};
   g.epi = EpiKind::SwiGLU;
   g.swiglu = EpiSwiGLU::Params{h, F, 1};
-  g.rows_bound = rmax;
   CK(launch_gemv(g, lc));
 
-  GemvLaunch dn;
-  dn.s.W = w_down;
-  dn.s.N = m.d_model;
-  dn.s.K = F;
-  dn.s.nrows = &rows->n;
-  dn.s.status = c->status();
-  gemv_plan(dn.s);
+  GemvLaunch dn = dense_launch(c, w_down, 0, &rows->n, 0, rmax);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{h, F, 1, nullptr};
   dn.epi = EpiKind::StoreAdd;
   dn.store = EpiStore<false>::Params{x, m.d_model, 1, nullptr};
-  dn.rows_bound = rmax;
   CK(launch_gemv(dn, lc));
   return OCRDEC_OK;
 }
@@ -319,18 +324,11 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   float* x = c->at<float>(c->L.x);
   const int nslot = m.top_k + m.n_shared;
 
-  GemvLaunch r;
-  r.s.W = w.router;
-  r.s.N = m.n_experts;
-  r.s.K = m.d_model;
-  r.s.nrows = &rows->n;
-  r.s.status = c->status();
-  gemv_plan(r.s);
+  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax);
   r.src = SrcKind::Norm;
   r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   r.epi = EpiKind::Store;
   r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
-  r.rows_bound = rmax;
   CK(launch_gemv(r, lc));
 
   RouteParams rp{};
@@ -350,46 +348,31 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   rp.status = c->status();
   CK(launch_ex(route_kernel, dim3(1), dim3(256), 0, lc, rp));
 
-  GemvShape es{};
-  es.n_experts = m.n_experts;
-  es.top_k = m.top_k;
-  es.mats = rp.mats;
-  es.n_mats = rp.n_mats;
-  es.counts = rp.counts;
-  es.offsets = rp.offsets;
-  es.rowlist = rp.rowlist;
-  es.nrows = &rows->n;
-  es.status = c->status();
+  auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half) {
+    GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax);
+    g.tm_sh = shared.map;
+    g.s.n_experts = m.n_experts;
+    g.s.top_k = m.top_k;
+    g.s.mats = rp.mats;
+    g.s.n_mats = rp.n_mats;
+    g.s.counts = rp.counts;
+    g.s.offsets = rp.offsets;
+    g.s.rowlist = rp.rowlist;
+    return g;
+  };
 
-  GemvLaunch gu;
-  gu.s = es;
-  gu.s.W = w.exp_gu;
-  gu.s.W_sh = w.sh_gu;
-  gu.s.mat_stride = 2LL * m.expert_ffn * m.d_model;
-  gu.s.N = 2 * m.expert_ffn;
-  gu.s.K = m.d_model;
-  gu.s.pair_half = m.expert_ffn;
-  gemv_plan(gu.s);
+  GemvLaunch gu = expert_launch(w.exp_gu, w.sh_gu, m.expert_ffn);
   gu.src = SrcKind::Norm;
   gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   gu.epi = EpiKind::SwiGLU;
   gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot};
-  gu.rows_bound = rmax;
   CK(launch_gemv(gu, lc));
 
-  GemvLaunch dn;
-  dn.s = es;
-  dn.s.W = w.exp_down;
-  dn.s.W_sh = w.sh_down;
-  dn.s.mat_stride = (long long)m.d_model * m.expert_ffn;
-  dn.s.N = m.d_model;
-  dn.s.K = m.expert_ffn;
-  gemv_plan(dn.s);
+  GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot, nullptr};
   dn.epi = EpiKind::Store;
   dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
-  dn.rows_bound = rmax;
   CK(launch_gemv(dn, lc));
 
   CombineParams cp{x, c->at<float>(c->L.ybuf), rp.gates, &rows->n, m.d_model, m.top_k, m.n_shared, c->status()};
@@ -407,7 +390,7 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
                layer_elems * m.n_layers, c->attn_counters(0)};
     int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
     if (st) return st;
-    st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down, m.dense_ffn) : moe_ffn(c, lc, rmax, w, count);
+    st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down) : moe_ffn(c, lc, rmax, w, count);
     if (st) return st;
     if (c->dbg_hidden)
       CK(cudaMemcpyAsync(c->dbg_hidden + (size_t)l * kRmax * m.d_model, io.x, sizeof(float) * kRmax * m.d_model,
@@ -421,20 +404,12 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
 int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const bf16* norm, const int* row_src,
             const int* nrows, int rows_static, int* tok, int tok_stride, float* logits, int which_counter) {
   const ocrdec_config& m = c->cfg;
-  GemvLaunch g;
-  g.s.W = c->lm_head;
-  g.s.N = m.vocab;
-  g.s.K = m.d_model;
-  g.s.nrows = nrows;
-  g.s.rows_static = rows_static;
-  g.s.status = c->status();
+  GemvLaunch g = dense_launch(c, c->lm_head, 0, nrows, rows_static, rmax);
   g.s.counter = c->am_counter(which_counter);
-  gemv_plan(g.s);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{x, m.d_model, row_src, norm, m.rms_eps};
   g.epi = EpiKind::Argmax;
   g.argmax = EpiArgmax::Params{tok, tok_stride, logits, c->at<float2>(c->L.am_part), nullptr};
-  g.rows_bound = rmax;
   g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
   CK(launch_gemv(g, lc));
   return OCRDEC_OK;
@@ -447,43 +422,28 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   const DraftW& w = c->dw;
   PassRows* rows = c->rows();
   float* xd = c->at<float>(c->L.xd);
-  GemvLaunch fc;
-  fc.s.W = w.fc;
-  fc.s.N = m.d_model;
-  fc.s.K = 2 * m.d_model;
-  fc.s.nrows = &rows->n;
-  fc.s.status = c->status();
-  gemv_plan(fc.s);
+  GemvLaunch fc = dense_launch(c, w.fc, 0, &rows->n, 0, rmax);
   fc.src = SrcKind::Bf16;
   fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), 2 * m.d_model, 1, nullptr};
   fc.epi = EpiKind::Store;
   fc.store = EpiStore<false>::Params{xd, m.d_model, 1, nullptr};
-  fc.rows_bound = rmax;
   CK(launch_gemv(fc, lc));
 
   const long long slot_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
   BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems, c->attn_counters(1)};
   if (kv_only) {
-    GemvLaunch g;
-    g.s.W = w.wqkv;
-    g.s.N = 3 * m.d_model;
-    g.s.K = m.d_model;
-    g.s.pair_half = m.head_dim / 2;
-    g.s.nrows = &rows->n;
-    g.s.status = c->status();
-    gemv_plan(g.s);
+    GemvLaunch g = dense_launch(c, w.wqkv, m.head_dim / 2, &rows->n, 0, rmax);
     g.src = SrcKind::Norm;
     g.norm = SrcNorm::Params{xd, m.d_model, nullptr, w.attn_norm, m.rms_eps};
     g.epi = EpiKind::QKV;
     g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
                            m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
-    g.rows_bound = rmax;
     CK(launch_gemv(g, lc));
     return OCRDEC_OK;
   }
   int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
   if (st) return st;
-  st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down, m.draft_ffn);
+  st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down);
   if (st) return st;
   return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, nullptr, 1);
 }
@@ -648,40 +608,49 @@ int ocrdec_load_weights(ocrdec_ctx* c, const void* const* ptrs, int n) {
   for (int i = 0; i < n; ++i)
     if (!ptrs[i] || (reinterpret_cast<uintptr_t>(ptrs[i]) & 15)) return OCRDEC_EINVAL;
   auto W = [&](int i) { return static_cast<const bf16*>(ptrs[i]); };
+  const int d = m.d_model;
+  bool ok = true;
   int i = 0;
   c->embed = W(i++);
   c->layers.assign(m.n_layers, LayerW{});
   for (int l = 0; l < m.n_layers; ++l) {
     LayerW& L = c->layers[l];
     L.attn_norm = W(i++);
-    L.wqkv = W(i++);
-    L.wo = W(i++);
+    ok &= make_mat(L.wqkv, W(i++), 3 * d, d, 1);
+    ok &= make_mat(L.wo, W(i++), d, d, 1);
     L.ffn_norm = W(i++);
     L.dense = l < m.n_dense_first;
     if (L.dense) {
-      L.w_gu = W(i++);
-      L.w_down = W(i++);
+      ok &= make_mat(L.w_gu, W(i++), 2 * m.dense_ffn, d, 1);
+      ok &= make_mat(L.w_down, W(i++), d, m.dense_ffn, 1);
     } else {
-      L.router = W(i++);
-      L.exp_gu = W(i++);
-      L.exp_down = W(i++);
-      L.sh_gu = W(i++);
-      L.sh_down = W(i++);
+      ok &= make_mat(L.router, W(i++), m.n_experts, d, 1);
+      ok &= make_mat(L.exp_gu, W(i++), 2 * m.expert_ffn, d, m.n_experts);
+      ok &= make_mat(L.exp_down, W(i++), d, m.expert_ffn, m.n_experts);
+      if (m.n_shared > 0) {
+        ok &= make_mat(L.sh_gu, W(i++), 2 * m.shared_ffn, d, m.n_shared);
+        ok &= make_mat(L.sh_down, W(i++), d, m.shared_ffn, m.n_shared);
+      } else {
+        i += 2;
+        L.sh_gu = L.exp_gu;
+        L.sh_down = L.exp_down;
+      }
     }
   }
   c->final_norm = W(i++);
-  c->lm_head = W(i++);
-  DraftW& d = c->dw;
-  d.norm_h = W(i++);
-  d.norm_e = W(i++);
-  d.fc = W(i++);
-  d.attn_norm = W(i++);
-  d.wqkv = W(i++);
-  d.wo = W(i++);
-  d.ffn_norm = W(i++);
-  d.w_gu = W(i++);
-  d.w_down = W(i++);
-  d.final_norm = W(i++);
+  ok &= make_mat(c->lm_head, W(i++), m.vocab, d, 1);
+  DraftW& dw = c->dw;
+  dw.norm_h = W(i++);
+  dw.norm_e = W(i++);
+  ok &= make_mat(dw.fc, W(i++), d, 2 * d, 1);
+  dw.attn_norm = W(i++);
+  ok &= make_mat(dw.wqkv, W(i++), 3 * d, d, 1);
+  ok &= make_mat(dw.wo, W(i++), d, d, 1);
+  dw.ffn_norm = W(i++);
+  ok &= make_mat(dw.w_gu, W(i++), 2 * m.draft_ffn, d, 1);
+  ok &= make_mat(dw.w_down, W(i++), d, m.draft_ffn, 1);
+  dw.final_norm = W(i++);
+  if (!ok) return OCRDEC_ECUDA;
   c->have_weights = true;
   c->drop_graphs();
   return OCRDEC_OK;
@@ -932,8 +901,7 @@ size_t ocrdec_op_scratch_bytes(void) {
 
 int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps, int R, int N, int K, float* y,
                         void* scratch, ocrdec_stream stream) {
-  if (!W || !x || !g || !y || !scratch || R < 1 || R > kRmax || N < kTR || N % kTR || K < 8 || K % 8 ||
-      K * 2 > 4096 * 2)
+  if (!W || !x || !g || !y || !scratch || R < 1 || R > kRmax || N < 1 || K < 8 || K % 8 || K > kGemvMaxK)
     return OCRDEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -941,7 +909,8 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
   CK(prepare_kernels());
   CK(cudaMemsetAsync(st, 0, 16, s));
   GemvLaunch gl;
-  gl.s.W = static_cast<const bf16*>(W);
+  CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
+  gl.tm_sh = gl.tm_w;
   gl.s.N = N;
   gl.s.K = K;
   gl.s.rows_static = R;
@@ -959,8 +928,7 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
 
 int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps, int R, int N, int K, int32_t* tok,
                         float* logits, void* scratch, ocrdec_stream stream) {
-  if (!W || !x || !g || !tok || !scratch || R < 1 || R > kRmax || N < kTR || N % kTR || K < 8 || K % 8 ||
-      K > 4096)
+  if (!W || !x || !g || !tok || !scratch || R < 1 || R > kRmax || N < 1 || K < 8 || K % 8 || K > kGemvMaxK)
     return OCRDEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -969,7 +937,8 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   CK(cudaMemsetAsync(st, 0, 16, s));
   int sms = device_sms();
   GemvLaunch gl;
-  gl.s.W = static_cast<const bf16*>(W);
+  CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
+  gl.tm_sh = gl.tm_w;
   gl.s.N = N;
   gl.s.K = K;
   gl.s.rows_static = R;

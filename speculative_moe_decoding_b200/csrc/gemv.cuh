@@ -1,45 +1,50 @@
 // Weight-streaming GEMV for a handful of rows (batch-1 speculative decoding).
 //
 // y[r][n] = sum_k W[n][k] * x[r][k] for the R <= kRmax rows of a pass.  The
-// work is HBM-bound: every weight byte is read once per pass, so the kernel is
-// built around the bulk-copy (TMA) unit:
-//   * one producer thread streams weight tiles (TR rows x one K-slice) into a
-//     kStages-deep ring of shared-memory stages with cp.async.bulk, each stage
-//     completing an mbarrier by transaction bytes;
-//   * kNW consumer warps own 16-byte K-chunks of the stage (thread t owns chunks
-//     t, t+256, ...), load the matching activation chunk of up to RG rows once
-//     and apply it to all TR weight rows of the tile;
-//   * each output is then reduced across the warp by a transpose-reduce whose
-//     shape depends on TR only, and across warps in warp order.
-// Every output's reduction order is therefore fixed by (K, TR) alone - never by
-// R, RG or which other rows share the pass - which is what makes the
-// speculative path bit-identical to k = 0.
+// work is HBM-bound: every weight byte is read once per pass.  The kernel is
+// built around the tensor-memory-access (TMA) unit:
+//   * one producer thread streams weight boxes of 32 rows x 256 columns
+//     (16 KB) into a kStages-deep shared-memory ring with
+//     cp.async.bulk.tensor (3-D tensor map: column, row, expert; no multicast),
+//     each stage completing an mbarrier by transaction bytes.  Columns past K
+//     and rows past N arrive zero-filled, so ragged shapes need no special case;
+//   * each of the kNW consumer warps owns 4 rows of every box: lane l handles
+//     the 16-byte chunk l of the 256-column slice for all 4 rows, with the
+//     matching activation chunk of every pass row loaded once per slice;
+//   * after the last slice a warp reduces its rows across lanes with a fixed
+//     transpose-reduce (xor 16, 8) and butterfly (xor 4, 2, 1), and runs the
+//     epilogue itself - no block-wide barrier per tile.
+// Every output's reduction order is fixed by K alone (slice order, lane, the
+// shuffle tree) - never by R, the row-group width or which rows share the
+// pass - which is what makes the speculative path bit-identical to k = 0.
 //
-// Work items are (matrix, tile) pairs handed to CTAs in contiguous ranges.
-// Dense mode has one matrix; expert mode walks a device-side list of touched
-// experts (shared experts first) so only the experts routed in this pass are
-// streamed.
+// Work items are (matrix, 32-row tile) pairs handed to CTAs in contiguous
+// ranges.  Dense mode has one matrix; expert mode walks a device-side list of
+// touched experts (shared experts first) so only the experts routed in this
+// pass are streamed.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
 namespace ocrdec {
 
-constexpr int kNW = 8;                      // consumer warps
-constexpr int kConsumers = kNW * 32;        // consumer threads
-constexpr int kGemvThreads = kConsumers + 32;  // + producer warp
-constexpr int kStages = 3;
-constexpr int kStageBytes = 24 * 1024;
-constexpr int kRmax = 8;                    // rows per pass on the GEMV path
+constexpr int kNW = 8;                          // consumer warps
+constexpr int kConsumers = kNW * 32;            // consumer threads
+constexpr int kGemvThreads = kConsumers + 32;   // + producer warp
+constexpr int kWarpRows = 4;                    // weight rows per warp per tile
+constexpr int kTile = kNW * kWarpRows;          // 32 rows per tile
+constexpr int kSlice = 256;                     // columns per stage
+constexpr int kBoxRows = 16;                    // rows per TMA box (two boxes per stage)
+constexpr int kStageBytes = kTile * kSlice * 2; // 16 KB
+constexpr int kStages = 6;
+constexpr int kRmax = 8;                        // rows per pass on the GEMV path
 
 struct GemvShape {
-  const bf16* W;        // dense matrix, or expert 0 of the routed experts
-  const bf16* W_sh;     // expert mode: shared expert 0
-  long long mat_stride; // elements between consecutive expert matrices
   int N, K;
-  int cps;              // 16-byte chunks per K-slice
-  int ns;               // K-slices (> 1 only in dense mode)
-  int pair_half;        // 0: tile = TR consecutive rows; else TR/2 rows + the TR/2 rows pair_half below
+  int ns;               // 256-column slices
+  int pair_half;        // 0: tile = 32 consecutive rows; else 16 rows + the 16 rows pair_half below
   int tiles_per_mat;
   // expert mode (mats != nullptr)
   const int* mats;      // mats[m] = routed expert id (< n_experts) or n_experts + shared index
@@ -66,36 +71,51 @@ __device__ __forceinline__ int pass_rows(const GemvShape& s) {
   return R < 0 ? 0 : (R > kRmax ? kRmax : R);
 }
 
-// Matrix row of tile-row i.
-template <int TR>
-__device__ __forceinline__ int tile_row(const GemvShape& s, int tile, int i) {
-  if (s.pair_half == 0) return tile * TR + i;
-  constexpr int H2 = TR / 2;
-  int per_blk = s.pair_half / H2;
-  int blk = tile / per_blk, j = tile - blk * per_blk;
-  int base = blk * 2 * s.pair_half + j * H2;
-  return i < H2 ? base + i : base + s.pair_half + (i - H2);
+// First matrix row of each of the two 16-row boxes of a tile.
+__device__ __forceinline__ void tile_boxes(const GemvShape& s, int tile, int* r0, int* r1) {
+  if (s.pair_half == 0) {
+    *r0 = tile * kTile;
+    *r1 = tile * kTile + kBoxRows;
+    return;
+  }
+  const int per_blk = s.pair_half / kBoxRows;
+  const int blk = tile / per_blk, j = tile - blk * per_blk;
+  *r0 = blk * 2 * s.pair_half + j * kBoxRows;
+  *r1 = *r0 + s.pair_half;
 }
 
-__device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, const bf16** Wm, int* expert,
+// Stage row of local row i (0..3) of warp w.  Plain tiles: 4 consecutive rows.
+// Paired tiles: rows 0,1 from the first box and their partners 2,3 from the
+// second box (local i and i + 2 form a pair).
+__device__ __forceinline__ int stage_row(bool paired, int w, int i) {
+  return paired ? (i < 2 ? 2 * w + i : kBoxRows + 2 * w + (i - 2)) : kWarpRows * w + i;
+}
+
+__device__ __forceinline__ int matrix_row(int r0, int r1, int srow) {
+  return srow < kBoxRows ? r0 + srow : r1 + (srow - kBoxRows);
+}
+
+__device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* coord_e, bool* shared,
                                          RowSet* rs) {
   if (!s.mats) {
-    *Wm = s.W;
-    *expert = 0;
+    *coord_e = 0;
+    *shared = false;
     if (rs) {
       rs->n = R;
+#pragma unroll
       for (int i = 0; i < kRmax; ++i) { rs->r[i] = i; rs->slot[i] = 0; }
     }
     return;
   }
   int e = s.mats[m];
-  *expert = e;
   if (e < s.n_experts) {
-    *Wm = s.W + (long long)e * s.mat_stride;
+    *coord_e = e;
+    *shared = false;
     if (rs) {
       int n = s.counts[e], off = s.offsets[e];
       n = n > kRmax ? kRmax : n;
       rs->n = n;
+#pragma unroll
       for (int i = 0; i < kRmax; ++i) {
         int v = i < n ? s.rowlist[off + i] : 0;
         rs->r[i] = v & 0xff;
@@ -104,16 +124,28 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, const
     }
   } else {
     int sh = e - s.n_experts;
-    *Wm = s.W_sh + (long long)sh * s.mat_stride;
+    *coord_e = sh;
+    *shared = true;
     if (rs) {
       rs->n = R;
+#pragma unroll
       for (int i = 0; i < kRmax; ++i) { rs->r[i] = i; rs->slot[i] = s.top_k + sh; }
     }
   }
 }
 
+// 3-D tensor-map load: box (256 columns, 16 rows, 1 matrix) at (c0, row, mat).
+__device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, int c0, int row, int mat,
+                                             uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(row), "r"(mat), "r"(smem_u32(bar))
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
-// activation sources
+// activation sources: 16-byte chunk c16 of pass row r (slot for expert outputs)
 // ---------------------------------------------------------------------------
 
 // Rows of a float32 matrix, RMS-normalised, scaled by a gain vector and rounded
@@ -181,16 +213,15 @@ struct SrcBf16 {
 };
 
 // ---------------------------------------------------------------------------
-// epilogues: called by all consumer threads with red[w][i][rg] complete
+// epilogues: run by one warp on its 4 reduced rows.  Lane L = 8 i + q holds
+// (in v) the result of local row i for pass-row slot q of the item's row set.
 // ---------------------------------------------------------------------------
 
-template <int TR, int RG>
-__device__ __forceinline__ float red_sum(const float* red, int i, int rg) {
-  float a = 0.f;
-#pragma unroll
-  for (int w = 0; w < kNW; ++w) a = __fadd_rn(a, red[(w * TR + i) * RG + rg]);
-  return a;
-}
+struct WarpOut {
+  float v;           // value for (local row i, row-set entry q) of this lane
+  int i, q;          // i = lane >> 3, q = lane & 7
+  int n[kWarpRows];  // matrix row of each local row (may be >= N in a ragged tile)
+};
 
 // out[(row(r) * nslot + slot) * ld + n] = v   (or += v when kAdd)
 template <bool kAdd>
@@ -201,23 +232,21 @@ struct EpiStore {
     int nslot;
     const int* row_dst;  // pass row r -> output row (nullptr: r)
   };
-  template <int TR, int RG>
-  __device__ static void apply(const Params& p, const GemvShape& s, int expert, int tile, const float* red,
-                               const RowSet& rs, int g, int tid) {
-    if (tid >= TR * RG) return;
-    int i = tid / RG, rg = tid % RG, j = g * RG + rg;
-    if (j >= rs.n) return;
-    float v = red_sum<TR, RG>(red, i, rg);
-    int r = rs.r[j];
-    long long row = (long long)(p.row_dst ? p.row_dst[r] : r) * p.nslot + rs.slot[j];
-    float* dst = p.y + row * p.ld + tile_row<TR>(s, tile, i);
-    if (kAdd) *dst = __fadd_rn(*dst, v);
-    else *dst = v;
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
+                               int lane) {
+    if (o.q >= rs.n) return;
+    int nrow = o.n[o.i];
+    if (nrow >= s.N) return;
+    int r = rs.r[o.q];
+    long long row = (long long)(p.row_dst ? p.row_dst[r] : r) * p.nslot + rs.slot[o.q];
+    float* dst = p.y + row * p.ld + nrow;
+    if (kAdd) *dst = __fadd_rn(*dst, o.v);
+    else *dst = o.v;
   }
   __device__ static void finish(const Params&, const GemvShape&, int, int) {}
 };
 
-// SwiGLU on paired tiles (gate rows i, up rows i + pair_half):
+// SwiGLU on paired tiles (gate row n, up row n + pair_half):
 // h[(r * nslot + slot) * ld + n] = bf16(silu(gate) * up)
 struct EpiSwiGLU {
   struct Params {
@@ -225,25 +254,20 @@ struct EpiSwiGLU {
     long long ld;
     int nslot;
   };
-  template <int TR, int RG>
-  __device__ static void apply(const Params& p, const GemvShape& s, int expert, int tile, const float* red,
-                               const RowSet& rs, int g, int tid) {
-    constexpr int H2 = TR / 2;
-    if (tid >= H2 * RG) return;
-    int i = tid / RG, rg = tid % RG, j = g * RG + rg;
-    if (j >= rs.n) return;
-    float gt = red_sum<TR, RG>(red, i, rg);
-    float up = red_sum<TR, RG>(red, i + H2, rg);
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
+                               int lane) {
+    float up = __shfl_down_sync(0xffffffffu, o.v, 16);
+    if (o.i >= 2 || o.q >= rs.n) return;
+    float gt = o.v;
     float act = __fdiv_rn(gt, __fadd_rn(1.f, expf(-gt)));
-    int n = tile_row<TR>(s, tile, i);  // gate row index = position in the hidden vector
-    long long row = (long long)rs.r[j] * p.nslot + rs.slot[j];
-    p.h[row * p.ld + n] = f2bf(__fmul_rn(act, up));
+    long long row = (long long)rs.r[o.q] * p.nslot + rs.slot[o.q];
+    p.h[row * p.ld + o.n[o.i]] = f2bf(__fmul_rn(act, up));
   }
   __device__ static void finish(const Params&, const GemvShape&, int, int) {}
 };
 
-// Q/K/V projection on paired tiles of one head (dims i and i + head_dim/2):
-// RoPE (rotate-half) on q and k with the table cos/sin[pos][i]; q -> float32
+// Q/K/V projection on paired tiles of one head (dims j and j + head_dim/2):
+// RoPE (rotate-half) on q and k with the table cos/sin[pos][j]; q -> float32
 // qbuf[r][H][Dh]; k, v -> bfloat16 KV cache at (slot, head, pos).
 struct EpiQKV {
   struct Params {
@@ -256,20 +280,16 @@ struct EpiQKV {
     const int* row_slot;  // pass row -> slot
     const int* row_pos;   // pass row -> position
   };
-  template <int TR, int RG>
-  __device__ static void apply(const Params& p, const GemvShape& s, int expert, int tile, const float* red,
-                               const RowSet& rs, int g, int tid) {
-    constexpr int H2 = TR / 2;
-    if (tid >= H2 * RG) return;
-    int i = tid / RG, rg = tid % RG, j = g * RG + rg;
-    if (j >= rs.n) return;
-    float a = red_sum<TR, RG>(red, i, rg);
-    float b = red_sum<TR, RG>(red, i + H2, rg);
-    int n = tile_row<TR>(s, tile, i);  // row of the first half
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
+                               int lane) {
+    float b = __shfl_down_sync(0xffffffffu, o.v, 16);
+    if (o.i >= 2 || o.q >= rs.n) return;
+    float a = o.v;
+    int n = o.n[o.i];                  // row of the first half
     int blk = n / p.Dh;                // 0..3H-1 : q heads, k heads, v heads
     int dim = n - blk * p.Dh;          // < Dh/2
     int half = p.Dh / 2;
-    int r = rs.r[j];
+    int r = rs.r[o.q];
     int pos = p.row_pos[r];
     if (blk < 2 * p.H) {
       float2 cs = p.rope[(long long)pos * half + dim];
@@ -293,9 +313,10 @@ struct EpiQKV {
   __device__ static void finish(const Params&, const GemvShape&, int, int) {}
 };
 
-// Greedy argmax over all rows of the matrix (LM head): per-CTA running maximum
-// (first index wins ties), then the last CTA to finish merges the per-CTA
-// partials (larger value, then lower index) and writes tok[r].
+// Greedy argmax over all rows of the matrix (LM head).  Each warp keeps a
+// running (value, index) per pass row; at the end the warps merge in order,
+// the CTA writes its partial, and the last CTA to finish merges the partials
+// (larger value, then lower index) and writes the tokens.
 struct EpiArgmax {
   struct Params {
     int* tok;           // token of pass row r at tok[row_dst(r) * tok_stride]
@@ -304,43 +325,53 @@ struct EpiArgmax {
     float2* partial;    // [gridDim][kRmax] (value, index as float bits)
     const int* row_dst; // pass row -> tok/logits row (nullptr: r)
   };
-  __device__ static float* best_v() { __shared__ float v[kRmax]; return v; }
-  __device__ static int* best_i() { __shared__ int v[kRmax]; return v; }
+  __device__ static float* best_v() { __shared__ float v[kNW * kRmax]; return v; }
+  __device__ static int* best_i() { __shared__ int v[kNW * kRmax]; return v; }
 
-  template <int TR, int RG>
-  __device__ static void apply(const Params& p, const GemvShape& s, int expert, int tile, const float* red,
-                               const RowSet& rs, int g, int tid) {
-    if (p.logits && tid < TR * RG) {
-      int i = tid / RG, rg = tid % RG, j = g * RG + rg;
-      if (j < rs.n) {
-        int r = rs.r[j];
-        int orow = p.row_dst ? p.row_dst[r] : r;
-        p.logits[(long long)orow * s.N + tile_row<TR>(s, tile, i)] = red_sum<TR, RG>(red, i, rg);
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
+                               int lane) {
+    int nrow = o.n[o.i];
+    bool valid = o.q < rs.n && nrow < s.N;
+    if (p.logits && valid) {
+      int r = rs.r[o.q];
+      p.logits[(long long)(p.row_dst ? p.row_dst[r] : r) * s.N + nrow] = o.v;
+    }
+    float bv = valid ? o.v : -INFINITY;
+    int bi = valid ? nrow : 0x7fffffff;
+#pragma unroll
+    for (int m = 8; m <= 16; m <<= 1) {
+      float ov = __shfl_xor_sync(0xffffffffu, bv, m);
+      int oi = __shfl_xor_sync(0xffffffffu, bi, m);
+      if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
+    }
+    if (lane < kRmax && lane < rs.n) {
+      const int w = threadIdx.x >> 5;
+      const int r = rs.r[lane];
+      float cv = best_v()[w * kRmax + r];
+      int ci = best_i()[w * kRmax + r];
+      if (bv > cv || (bv == cv && bi < ci)) {
+        best_v()[w * kRmax + r] = bv;
+        best_i()[w * kRmax + r] = bi;
       }
     }
-    if (tid >= RG) return;
-    int j = g * RG + tid;
-    if (j >= rs.n) return;
-    int r = rs.r[j];
-    float bv = best_v()[r];
-    int bi = best_i()[r];
-    for (int i = 0; i < TR; ++i) {
-      float v = red_sum<TR, RG>(red, i, tid);
-      int n = tile_row<TR>(s, tile, i);
-      if (v > bv || (v == bv && n < bi)) { bv = v; bi = n; }
-    }
-    best_v()[r] = bv;
-    best_i()[r] = bi;
   }
 
   __device__ static void init(int tid) {
-    if (tid < kRmax) { best_v()[tid] = -INFINITY; best_i()[tid] = 0x7fffffff; }
+    if (tid < kNW * kRmax) { best_v()[tid] = -INFINITY; best_i()[tid] = 0x7fffffff; }
   }
 
   __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
     __shared__ int last;
-    if (tid < kRmax)
-      p.partial[blockIdx.x * kRmax + tid] = make_float2(best_v()[tid], __int_as_float(best_i()[tid]));
+    if (tid < kRmax) {
+      float bv = -INFINITY;
+      int bi = 0x7fffffff;
+      for (int w = 0; w < kNW; ++w) {
+        float v = best_v()[w * kRmax + tid];
+        int i = best_i()[w * kRmax + tid];
+        if (v > bv || (v == bv && i < bi)) { bv = v; bi = i; }
+      }
+      p.partial[blockIdx.x * kRmax + tid] = make_float2(bv, __int_as_float(bi));
+    }
     __threadfence();
     named_sync(1, kConsumers);
     if (tid == 0) last = (atomicAdd(s.counter, 1) == (int)gridDim.x - 1);
@@ -352,9 +383,9 @@ struct EpiArgmax {
       int bi = 0x7fffffff;
       const volatile float2* part = p.partial;
       for (int b = 0; b < (int)gridDim.x; ++b) {
-        float2 e = const_cast<const float2&>(part[b * kRmax + tid]);
-        int ei = __float_as_int(e.y);
-        if (e.x > bv || (e.x == bv && ei < bi)) { bv = e.x; bi = ei; }
+        float ev = part[b * kRmax + tid].x;
+        int ei = __float_as_int(part[b * kRmax + tid].y);
+        if (ev > bv || (ev == bv && ei < bi)) { bv = ev; bi = ei; }
       }
       p.tok[(p.row_dst ? p.row_dst[tid] : tid) * p.tok_stride] = bi;
     }
@@ -371,59 +402,19 @@ __device__ __forceinline__ void epi_init<EpiArgmax>(int tid) { EpiArgmax::init(t
 // the kernel
 // ---------------------------------------------------------------------------
 
-// After log2(TR) halving stages (xor 16, 8, ...) every lane holds one
-// partially reduced value whose tile row is decoded from its lane bits; a
-// butterfly over the remaining lane bits finishes the sum.
-template <int N, int M>
-__device__ __forceinline__ void transpose_stage(float* v, int lane) {
-  if constexpr (N > 1) {
-    constexpr int H = N / 2;
-    const bool upper = (lane & M) != 0;
-#pragma unroll
-    for (int j = 0; j < H; ++j) {
-      float send = upper ? v[j] : v[j + H];
-      float keep = upper ? v[j + H] : v[j];
-      v[j] = __fadd_rn(keep, __shfl_xor_sync(0xffffffffu, send, M));
-    }
-    transpose_stage<H, M / 2>(v, lane);
-  }
-}
-
-template <int TR>
-__device__ __forceinline__ void warp_transpose_reduce(float* v, int lane) {
-  transpose_stage<TR, 16>(v, lane);
-}
-
-template <int TR>
-__device__ __forceinline__ int transpose_row(int lane) {
-  int i = 0, n = TR;
-#pragma unroll
-  for (int m = 16; m > 0; m >>= 1) {
-    if (n <= 1) break;
-    n >>= 1;
-    if (lane & m) i += n;
-  }
-  return i;
-}
-
-template <int TR>
-constexpr int transpose_stages() { return TR >= 16 ? 4 : TR >= 8 ? 3 : TR >= 4 ? 2 : TR >= 2 ? 1 : 0; }
-
-template <int TR, int RG, class Src, class Epi>
+template <int RG, class Src, class Epi>
 __global__ void __launch_bounds__(kGemvThreads, 1)
-gemv_kernel(const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
-  extern __shared__ __align__(128) unsigned char smem[];
+gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
+            const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
+  extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ float red[2][kNW * TR * RG];
   __shared__ float red_pro[kNW * kRmax];
-
   __shared__ int s_abort;
+
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-
   unsigned char* stages = smem;
   bf16* xs = reinterpret_cast<bf16*>(smem + kStages * kStageBytes);
-  const int stage_stride_row = s.cps * 16;  // bytes per tile row in a stage
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -437,49 +428,36 @@ gemv_kernel(const GemvShape s, const typename Src::Params sp, const typename Epi
   __syncthreads();
   if (s_abort) return;
   pdl_trigger();
+
   const int R = pass_rows(s);
   const int n_mats = s.mats ? *s.n_mats : 1;
   const int total = n_mats * s.tiles_per_mat;
   const int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
   const int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
-  const int ngroups_dense = (R + RG - 1) / RG;
   const int nch = s.K / 8;  // 16-byte chunks per row
+  const bool paired = s.pair_half != 0;
 
   if (warp == kNW) {
     // ---------------- producer ----------------
     if (lane == 0) {
       uint32_t it = 0;
-      bool ok = true;
-      for (int item = start; item < end && ok; ++item) {
+      for (int item = start; item < end; ++item) {
         int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
-        const bf16* Wm;
-        int e;
-        mat_info(s, m, R, &Wm, &e, nullptr);
-        int passes = s.ns == 1 ? 1 : ngroups_dense;
-        for (int ps = 0; ps < passes && ok; ++ps) {
-          for (int sl = 0; sl < s.ns && ok; ++sl, ++it) {
-            int st = it % kStages;
-            // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
-            // stays uniform so the block always terminates
-            if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
-            int c0 = sl * s.cps;
-            int cn = min(s.cps, nch - c0);
-            uint32_t seg = cn * 16;
-            mbar_arrive_expect_tx(&full_bar[st], seg * TR);
-            unsigned char* dst = stages + st * kStageBytes;
-            if (s.ns == 1 && s.pair_half == 0) {
-              bulk_g2s(dst, Wm + (long long)t * TR * s.K, seg * TR, &full_bar[st]);
-            } else if (s.ns == 1) {
-              constexpr int H2 = TR / 2;
-              bulk_g2s(dst, Wm + (long long)tile_row<TR>(s, t, 0) * s.K, seg * H2, &full_bar[st]);
-              bulk_g2s(dst + H2 * stage_stride_row, Wm + (long long)tile_row<TR>(s, t, H2) * s.K, seg * H2,
-                       &full_bar[st]);
-            } else {
-              for (int i = 0; i < TR; ++i)
-                bulk_g2s(dst + i * stage_stride_row, Wm + (long long)tile_row<TR>(s, t, i) * s.K + c0 * 8, seg,
-                         &full_bar[st]);
-            }
-          }
+        int ce;
+        bool sh;
+        mat_info(s, m, R, &ce, &sh, nullptr);
+        const CUtensorMap* map = sh ? &tm_sh : &tm_w;
+        int r0, r1;
+        tile_boxes(s, t, &r0, &r1);
+        for (int sl = 0; sl < s.ns; ++sl, ++it) {
+          int st = it % kStages;
+          // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control
+          // flow stays uniform so the block always terminates
+          if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
+          mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+          unsigned char* dst = stages + st * kStageBytes;
+          tma_load_box(dst, map, sl * kSlice, r0, ce, &full_bar[st]);
+          tma_load_box(dst + kStageBytes / 2, map, sl * kSlice, r1, ce, &full_bar[st]);
         }
       }
       // drain: every issued copy has landed before the block can exit
@@ -495,85 +473,87 @@ gemv_kernel(const GemvShape s, const typename Src::Params sp, const typename Epi
   else named_sync(1, kConsumers);
 
   uint32_t it = 0;
-  int red_buf = 0;
   int cur_m = -1;
   RowSet rs;
-  const bf16* Wm = nullptr;
-  int expert = 0;
-  bool ok = true;
-  for (int item = start; item < end && ok; ++item) {
+  int ce = 0;
+  bool sh = false;
+  int srow[kWarpRows];
+#pragma unroll
+  for (int i = 0; i < kWarpRows; ++i) srow[i] = stage_row(paired, warp, i);
+
+  for (int item = start; item < end; ++item) {
     int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
     if (m != cur_m) {
-      mat_info(s, m, R, &Wm, &expert, &rs);
+      mat_info(s, m, R, &ce, &sh, &rs);
       cur_m = m;
     }
-    const int ngroups = (rs.n + RG - 1) / RG;
-    const int passes = s.ns == 1 ? 1 : ngroups;
-    for (int ps = 0; ps < passes && ok; ++ps) {
-      const int g_lo = s.ns == 1 ? 0 : ps;
-      const int g_hi = s.ns == 1 ? ngroups : ps + 1;
-      float acc[TR][RG];
-      for (int sl = 0; sl < s.ns; ++sl, ++it) {
-        int st = it % kStages;
-        mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
-        const unsigned char* w_st = stages + st * kStageBytes;
-        int c0 = sl * s.cps;
-        int cn = min(s.cps, nch - c0);
-        for (int g = g_lo; g < g_hi; ++g) {
-          if (s.ns == 1 || sl == 0) {
+    float acc[kWarpRows][RG];
 #pragma unroll
-            for (int i = 0; i < TR; ++i)
+    for (int i = 0; i < kWarpRows; ++i)
 #pragma unroll
-              for (int q = 0; q < RG; ++q) acc[i][q] = 0.f;
-          }
-          for (int c = tid; c < cn; c += kConsumers) {
-            float xv[RG][8];
+      for (int q = 0; q < RG; ++q) acc[i][q] = 0.f;
+
+    for (int sl = 0; sl < s.ns; ++sl, ++it) {
+      const int st = it % kStages;
+      mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
+      const unsigned char* w_st = stages + st * kStageBytes;
+      const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
+      if (c < nch) {
+        float xv[RG][8];
 #pragma unroll
-            for (int q = 0; q < RG; ++q) {
-              int j = g * RG + q;
-              if (j < rs.n) {
-                uint4 u = Src::chunk(sp, xs, s.K, rs.r[j], rs.slot[j], c0 + c);
-                unpack8(u, xv[q]);
-              } else {
+        for (int q = 0; q < RG; ++q) {
+          if (q < rs.n) {
+            uint4 u = Src::chunk(sp, xs, s.K, rs.r[q], rs.slot[q], c);
+            unpack8(u, xv[q]);
+          } else {
 #pragma unroll
-                for (int e = 0; e < 8; ++e) xv[q][e] = 0.f;
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < TR; ++i) {
-              uint4 u = *reinterpret_cast<const uint4*>(w_st + i * stage_stride_row + c * 16);
-              float wv[8];
-              unpack8(u, wv);
-#pragma unroll
-              for (int e = 0; e < 8; ++e)
-#pragma unroll
-                for (int q = 0; q < RG; ++q) acc[i][q] = __fmaf_rn(wv[e], xv[q][e], acc[i][q]);
-            }
-          }
-          if (sl == s.ns - 1) {
-            // reduce: warp transpose-reduce per row of the group, then warps in order
-            float* rb = red[red_buf];
-#pragma unroll
-            for (int q = 0; q < RG; ++q) {
-              float v[TR];
-#pragma unroll
-              for (int i = 0; i < TR; ++i) v[i] = acc[i][q];
-              warp_transpose_reduce<TR>(v, lane);
-#pragma unroll
-              for (int m2 = (32 >> transpose_stages<TR>()) / 2; m2 > 0; m2 >>= 1)
-                v[0] = __fadd_rn(v[0], __shfl_xor_sync(0xffffffffu, v[0], m2));
-              if ((lane & ((32 >> transpose_stages<TR>()) - 1)) == 0)
-                rb[(warp * TR + transpose_row<TR>(lane)) * RG + q] = v[0];
-            }
-            named_sync(1, kConsumers);
-            Epi::template apply<TR, RG>(ep, s, expert, t, rb, rs, g, tid);
-            red_buf ^= 1;
+            for (int e = 0; e < 8; ++e) xv[q][e] = 0.f;
           }
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[st]);
+#pragma unroll
+        for (int i = 0; i < kWarpRows; ++i) {
+          uint4 u = *reinterpret_cast<const uint4*>(w_st + srow[i] * (kSlice * 2) + lane * 16);
+          float wv[8];
+          unpack8(u, wv);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+#pragma unroll
+            for (int q = 0; q < RG; ++q) acc[i][q] = __fmaf_rn(wv[e], xv[q][e], acc[i][q]);
+        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
+
+    // reduce the warp's 4 rows: transpose over lane bits 4, 3, then butterfly over bits 2..0;
+    // afterwards lane L holds the full sum of local row (L >> 3)
+    float v[RG];
+#pragma unroll
+    for (int q = 0; q < RG; ++q) {
+      const bool up16 = lane & 16;
+      float a0 = __fadd_rn(up16 ? acc[2][q] : acc[0][q],
+                           __shfl_xor_sync(0xffffffffu, up16 ? acc[0][q] : acc[2][q], 16));
+      float a1 = __fadd_rn(up16 ? acc[3][q] : acc[1][q],
+                           __shfl_xor_sync(0xffffffffu, up16 ? acc[1][q] : acc[3][q], 16));
+      const bool up8 = lane & 8;
+      float b = __fadd_rn(up8 ? a1 : a0, __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8));
+      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 4));
+      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 2));
+      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 1));
+      v[q] = b;
+    }
+    WarpOut o;
+    o.i = lane >> 3;
+    o.q = lane & 7;
+    o.v = 0.f;
+#pragma unroll
+    for (int q = 0; q < RG; ++q)
+      if (o.q == q) o.v = v[q];
+    int r0, r1;
+    tile_boxes(s, t, &r0, &r1);
+#pragma unroll
+    for (int i = 0; i < kWarpRows; ++i) o.n[i] = matrix_row(r0, r1, srow[i]);
+    Epi::apply(ep, s, o, rs, lane);
   }
   named_sync(1, kConsumers);
   Epi::finish(ep, s, R, tid);

@@ -6,11 +6,32 @@
 namespace ocrdec {
 
 void gemv_plan(GemvShape& s) {
-  const int nch = s.K / 8;
-  const int max_cps = kStageBytes / (kTR * 16);
-  s.ns = (nch + max_cps - 1) / max_cps;
-  s.cps = (nch + s.ns - 1) / s.ns;
-  s.tiles_per_mat = s.N / kTR;
+  s.ns = (s.K + kSlice - 1) / kSlice;
+  s.tiles_per_mat = s.pair_half ? (s.N / (2 * s.pair_half)) * (s.pair_half / kBoxRows) : (s.N + kTile - 1) / kTile;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || K % 8 || K <= 0 || N <= 0 || E <= 0) return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)E};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)K * 2 * N};
+  cuuint32_t box[3] = {kSlice, kBoxRows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <class Src>
@@ -20,7 +41,7 @@ static size_t smem_max() {
 
 template <int RG, class Src, class Epi>
 static cudaError_t configure_one() {
-  return cudaFuncSetAttribute(gemv_kernel<kTR, RG, Src, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(gemv_kernel<RG, Src, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)smem_max<Src>());
 }
 
@@ -29,6 +50,7 @@ static cudaError_t configure_rg() {
   cudaError_t e = configure_one<1, Src, Epi>();
   if (e == cudaSuccess) e = configure_one<2, Src, Epi>();
   if (e == cudaSuccess) e = configure_one<4, Src, Epi>();
+  if (e == cudaSuccess) e = configure_one<8, Src, Epi>();
   return e;
 }
 
@@ -45,12 +67,12 @@ cudaError_t gemv_prepare() {
 template <int RG, class Src, class Epi>
 static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& sp, const typename Epi::Params& ep,
                               const LaunchCfg& lc) {
-  auto kern = gemv_kernel<kTR, RG, Src, Epi>;
+  auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
   size_t smem = (size_t)kStages * kStageBytes + (Src::kSmem ? (size_t)kRmax * g.s.K * 2 : 0);
   int grid = g.grid;
   if (grid <= 0) grid = g.s.mats ? lc.num_sms : std::min(g.s.tiles_per_mat, lc.num_sms);
-  return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.s, sp, ep);
+  return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
 }
 
 template <class Src, class Epi>
@@ -58,12 +80,14 @@ static cudaError_t launch_rg(const GemvLaunch& g, const typename Src::Params& sp
                              const LaunchCfg& lc) {
   if (g.rows_bound <= 1) return launch_one<1, Src, Epi>(g, sp, ep, lc);
   if (g.rows_bound <= 2) return launch_one<2, Src, Epi>(g, sp, ep, lc);
-  return launch_one<4, Src, Epi>(g, sp, ep, lc);
+  if (g.rows_bound <= 4) return launch_one<4, Src, Epi>(g, sp, ep, lc);
+  return launch_one<8, Src, Epi>(g, sp, ep, lc);
 }
 
 cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
-  if (g.s.N % kTR || g.s.K % 8 || (g.s.pair_half && g.s.pair_half % (kTR / 2))) return cudaErrorInvalidValue;
-  if (g.s.ns > 1 && g.s.mats) return cudaErrorInvalidValue;
+  if (g.s.K % 8 || (g.s.pair_half && (g.s.pair_half % kBoxRows || g.s.N % (2 * g.s.pair_half))))
+    return cudaErrorInvalidValue;
+  if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
   if (g.src == SrcKind::Norm) {
     switch (g.epi) {
       case EpiKind::QKV: return launch_rg<SrcNorm, EpiQKV>(g, g.norm, g.qkv, lc);

@@ -35,6 +35,8 @@ enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.
 struct GemvLaunch {
+  CUtensorMap tm_w;   // routed experts / dense matrix
+  CUtensorMap tm_sh;  // shared experts (expert mode); unused otherwise
   GemvShape s{};
   SrcKind src = SrcKind::Norm;
   EpiKind epi = EpiKind::Store;
@@ -48,14 +50,16 @@ struct GemvLaunch {
   int grid = 0;            // 0: derived from the work and the SM count
 };
 
-// Fills cps/ns/tiles_per_mat for tile height kTR and stage size.
+// Fills ns / tiles_per_mat from N, K and pair_half.
 void gemv_plan(GemvShape& s);
+// 3-D tensor map (columns K, rows N, matrices E) of a bfloat16 weight array with
+// the GEMV's 256 x 16 box; base 16-byte aligned.
+cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap* out);
 cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
 // Raises the dynamic shared-memory limit of every GEMV instantiation to the
 // largest size any launch uses (call outside stream capture, once per device).
 cudaError_t gemv_prepare();
 constexpr int kGemvMaxK = 4096;  // largest K of a normalised (shared-memory) source
 
-constexpr int kTR = 8;  // weight rows per tile on every GEMV
 
 }  // namespace ocrdec
