@@ -266,10 +266,12 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed_steps")
     e0.record(stream)
     for _ in range(args.steps):
         dec.step(1, k)
     e1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     barrier()
     clk = clocks.stop()
