@@ -200,6 +200,11 @@ OCRDEC_API int ocrdec_step_kernel_count(ocrdec_ctx* ctx, int batch, int k, int32
  * max_batch*(max_k+1) or the prefill chunk of 8).  NULL switches a tap off. */
 OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* dev_logits);
 
+/* Parity tap for the draft: when set, recursion j (1-based) of every draft
+ * also writes its LM-head logits to dev_logits[j-1][slot][V] (float32,
+ * max_k * max_batch * V entries).  NULL switches it off. */
+OCRDEC_API int ocrdec_set_draft_taps(ocrdec_ctx* ctx, float* dev_logits);
+
 OCRDEC_API const char* ocrdec_strerror(int status);
 
 /* ---- single-kernel entry points (kernel-level parity tests) ----------------- */

@@ -281,7 +281,7 @@ class Oracle:
     def draft_token(self, hprime_row: np.ndarray, margins: Optional[list] = None) -> int:
         logits = self.lm_logits(hprime_row[None, :], "draft.final_norm")[0]
         if margins is not None:
-            margins.append(top2_margin(logits))
+            margins.append(logits)
         return greedy_argmax(logits)
 
 
@@ -336,6 +336,7 @@ def prefill(orc: Oracle, visual: np.ndarray, prompt: Sequence[int], with_draft: 
 
 
 def draft_propose(orc: Oracle, st: SeqState, k: int, margins: Optional[list] = None) -> List[int]:
+    """(``margins``, if given, receives each recursion's draft logits.)"""
     """k recursions of the shared draft block.  Recursion 1 consumes the pending
     pairs (verifier hidden at p, committed token at p+1); recursion j >= 2 feeds
     the block's own output hidden with the previous draft token."""

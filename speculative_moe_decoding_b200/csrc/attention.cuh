@@ -15,7 +15,7 @@
 
 namespace ocrdec {
 
-constexpr int kAttnChunk = 128;
+constexpr int kAttnChunk = 64;
 constexpr int kAttnThreads = 128;
 constexpr int kAttnRows = 8;  // rows of one slot in a pass
 
@@ -43,6 +43,7 @@ attention_kernel(const AttnParams p) {
   __shared__ int s_abort;
   __shared__ float qs[kAttnRows][128];
   __shared__ float sc[kAttnRows][kAttnChunk];
+  __shared__ float ored[4][kAttnRows][128];
   __shared__ float s_m[kAttnRows], s_l[kAttnRows];
   __shared__ int s_last;
 
@@ -96,7 +97,7 @@ attention_kernel(const AttnParams p) {
         int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
         qr[i][e] = (rb + i < nr && (e < 8 || l8 + 8 < ndc)) ? qs[rb + i][d] : 0.f;
       }
-    for (int j0 = warp * 32; j0 < warp * 32 + 32; j0 += 4) {
+    for (int j0 = warp * 16; j0 < warp * 16 + 16; j0 += 4) {
       int j = j0 + g;
       float kv[16];
       if (j < npos) {
@@ -148,7 +149,7 @@ attention_kernel(const AttnParams p) {
     for (int j = lane; j < kAttnChunk; j += 32) {
       float e = 0.f;
       if (j < lim) e = expf(__fsub_rn(sc[r][j], m));
-      if (j < npos) sc[r][j] = e;
+      sc[r][j] = e;
       l = __fadd_rn(l, e);
     }
 #pragma unroll
@@ -157,17 +158,52 @@ attention_kernel(const AttnParams p) {
   }
   __syncthreads();
 
-  // ---- o = sum_j p_j v_j, thread per dim, positions in order ----
+  // ---- o = sum_j p_j v_j: warp w takes positions 16w..16w+15 in order, lane l
+  // dims [l*dpl, (l+1)*dpl); the 4 warp partials are then added in warp order ----
   const int ld = Dh + 2;
+  const int dpl = Dh / 32;  // dims per lane: 4 (Dh 128) or 2 (Dh 64)
+  {
+    float o[kAttnRows][4];
+#pragma unroll
+    for (int r = 0; r < kAttnRows; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) o[r][e] = 0.f;
+    int lim[kAttnRows];
+#pragma unroll
+    for (int r = 0; r < kAttnRows; ++r) lim[r] = r < nr ? min(p.row_pos[r0 + r] - p0 + 1, npos) : 0;
+    const int jb = warp * 16;
+    for (int jj = 0; jj < 16; ++jj) {
+      const int j = jb + jj;
+      if (j >= npos) break;
+      float vv[4];
+      if (dpl == 4) {
+        uint2 u = *reinterpret_cast<const uint2*>(Vs + j * Dh + lane * 4);
+        vv[0] = bf_lo(u.x); vv[1] = bf_hi(u.x); vv[2] = bf_lo(u.y); vv[3] = bf_hi(u.y);
+      } else {
+        uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + j * Dh + lane * 2);
+        vv[0] = bf_lo(u); vv[1] = bf_hi(u); vv[2] = 0.f; vv[3] = 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < kAttnRows; ++r) {
+        if (j < lim[r]) {
+          const float pj = sc[r][j];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[r][e] = __fmaf_rn(pj, vv[e], o[r][e]);
+        }
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < kAttnRows; ++r)
+      if (r < nr)
+        for (int e = 0; e < dpl; ++e) ored[warp][r][lane * dpl + e] = o[r][e];
+  }
+  __syncthreads();
   for (int r = 0; r < nr; ++r) {
     int lim = min(p.row_pos[r0 + r] - p0 + 1, npos);
     if (lim <= 0) continue;
     float* dst = p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + c) * ld;
-    for (int d = tid; d < Dh; d += kAttnThreads) {
-      float o = 0.f;
-      for (int j = 0; j < lim; ++j) o = __fmaf_rn(sc[r][j], bf2f(Vs[j * Dh + d]), o);
-      dst[d] = o;
-    }
+    for (int d = tid; d < Dh; d += kAttnThreads)
+      dst[d] = __fadd_rn(__fadd_rn(__fadd_rn(ored[0][r][d], ored[1][r][d]), ored[2][r][d]), ored[3][r][d]);
     if (tid == 0) { dst[Dh] = s_m[r]; dst[Dh + 1] = s_l[r]; }
   }
 

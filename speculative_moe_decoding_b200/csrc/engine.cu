@@ -15,7 +15,7 @@
 
 #include "attention.cuh"
 #include "launch.cuh"
-#include "step_kernels.cuh"
+#include "step_globals.cuh"
 
 using namespace ocrdec;
 
@@ -184,7 +184,7 @@ struct ocrdec_ctx {
   char* ws = nullptr;
   bool have_weights = false;
   int num_sms = 0;
-  bool pdl = false;
+  bool pdl = true;
   const bf16 *embed = nullptr, *final_norm = nullptr;
   Mat lm_head;
   std::vector<LayerW> layers;
@@ -199,6 +199,7 @@ struct ocrdec_ctx {
   float f_p[3] = {0, 0, 0};
   float* dbg_hidden = nullptr;
   float* dbg_logits = nullptr;
+  float* dbg_draft_logits = nullptr;
 
   template <class T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
@@ -324,13 +325,6 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   float* x = c->at<float>(c->L.x);
   const int nslot = m.top_k + m.n_shared;
 
-  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax);
-  r.src = SrcKind::Norm;
-  r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
-  r.epi = EpiKind::Store;
-  r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
-  CK(launch_gemv(r, lc));
-
   RouteParams rp{};
   rp.logits = c->at<float>(c->L.rlogits);
   rp.nrows = &rows->n;
@@ -346,7 +340,16 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   rp.n_mats = c->at<int>(c->L.n_mats);
   rp.touched = count ? c->misc() : nullptr;
   rp.status = c->status();
-  CK(launch_ex(route_kernel, dim3(1), dim3(256), 0, lc, rp));
+
+  // router logits + (last CTA) softmax / top-k / bucketing
+  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax);
+  r.s.counter = c->am_counter(2);
+  r.src = SrcKind::Norm;
+  r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
+  r.epi = EpiKind::Route;
+  r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
+  r.route = rp;
+  CK(launch_gemv(r, lc));
 
   auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half) {
     GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax);
@@ -417,7 +420,7 @@ int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const 
 
 // The draft block over the rows prepared by draft_setup (fcin, rows).
 // kv_only: stop after the draft KV append (prefill pairs whose outputs are unused).
-int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int* tok, int tok_stride) {
+int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int* tok, int tok_stride, int j) {
   const ocrdec_config& m = c->cfg;
   const DraftW& w = c->dw;
   PassRows* rows = c->rows();
@@ -445,7 +448,8 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   if (st) return st;
   st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down);
   if (st) return st;
-  return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, nullptr, 1);
+  float* dl = c->dbg_draft_logits ? c->dbg_draft_logits + (size_t)(j - 1) * m.max_batch * m.vocab : nullptr;
+  return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, dl, 1);
 }
 
 int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) {
@@ -474,7 +478,7 @@ int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) 
     dp.status = c->status();
     CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
     int rmax = j == 1 ? std::min(kRmax, B * (m.max_k + 1)) : B;
-    int st = draft_block(c, lc, rmax, false, props + (j - 1), k);
+    int st = draft_block(c, lc, rmax, false, props + (j - 1), k, j);
     if (st) return st;
   }
   return OCRDEC_OK;
@@ -497,12 +501,17 @@ int enqueue_verify(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, const int* 
   CK(launch_ex(verify_setup_kernel, dim3(1), dim3(256), 0, lc, vp));
   int st = verifier_layers(c, lc, R, true);
   if (st) return st;
-  st = lm_head(c, lc, R, c->at<float>(c->L.x), c->final_norm, nullptr, &c->rows()->n, 0, c->at<int>(c->L.gtok), 1,
-               c->dbg_logits, 0);
-  if (st) return st;
   AcceptParams ap{c->slots(), c->at<int>(c->L.gtok), props, B, k, m.d_model, m.max_k, c->hist(), c->L.hist_ld,
                   c->at<float>(c->L.x), c->at<float>(c->L.hpend), committed, ncommitted, c->status()};
-  CK(launch_ex(accept_kernel, dim3(1), dim3(256), 0, lc, ap));
+  GemvLaunch g = dense_launch(c, c->lm_head, 0, &c->rows()->n, 0, R);
+  g.s.counter = c->am_counter(0);
+  g.src = SrcKind::Norm;
+  g.norm = SrcNorm::Params{c->at<float>(c->L.x), m.d_model, nullptr, c->final_norm, m.rms_eps};
+  g.epi = EpiKind::ArgmaxAccept;
+  g.argmax = EpiArgmax::Params{c->at<int>(c->L.gtok), 1, c->dbg_logits, c->at<float2>(c->L.am_part), nullptr};
+  g.accept = ap;
+  g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
+  CK(launch_gemv(g, lc));
   return OCRDEC_OK;
 }
 
@@ -712,7 +721,7 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
         CK(launch_ex(prefill_finish_kernel, dim3(1), dim3(256), 0, lc, pf));
       }
       CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
-      st = draft_block(c, lc, q1 - p0, true, nullptr, 0);
+      st = draft_block(c, lc, q1 - p0, true, nullptr, 0, 0);
       if (st) return st;
     } else if (p0 + n == C) {
       PrefillFinishParams pf{c->slots(), slot, C, C - 1 - p0, m.d_model, m.max_k, c->at<int>(c->L.gtok),
@@ -868,6 +877,13 @@ int ocrdec_step_kernel_count(ocrdec_ctx* c, int batch, int k, int32_t* dev_commi
   auto it = c->graph_kernels.find(std::make_tuple(batch, k, (void*)dev_committed, (void*)dev_n_committed));
   if (it == c->graph_kernels.end()) return OCRDEC_ESTATE;
   *count = it->second;
+  return OCRDEC_OK;
+}
+
+int ocrdec_set_draft_taps(ocrdec_ctx* c, float* logits) {
+  if (!c) return OCRDEC_EINVAL;
+  c->dbg_draft_logits = logits;
+  c->drop_graphs();
   return OCRDEC_OK;
 }
 

@@ -1,0 +1,58 @@
+// GEMV epilogues that finish a pass step in the GEMV's last CTA: routing after
+// the router logits, greedy acceptance after the verifier's LM-head argmax.
+// Each saves one launch per use.
+#pragma once
+
+#include "gemv.cuh"
+#include "step_kernels.cuh"
+
+namespace ocrdec {
+
+struct ConsumerSync {
+  __device__ void operator()() const { named_sync(1, kConsumers); }
+};
+
+// Router logits (stored like EpiStore), then - in the last CTA to finish -
+// softmax, top-k and bucketing of every row.
+struct EpiRoute {
+  struct Params {
+    EpiStore<false>::Params store;
+    RouteParams route;
+  };
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs, int lane) {
+    EpiStore<false>::apply(p.store, s, o, rs, lane);
+  }
+  __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
+    __shared__ int last;
+    __threadfence();
+    named_sync(1, kConsumers);
+    if (tid == 0) last = (atomicAdd(s.counter, 1) == (int)gridDim.x - 1);
+    named_sync(1, kConsumers);
+    if (!last) return;
+    __threadfence();
+    route_rows(p.route, R, tid, kConsumers, ConsumerSync{});
+    if (tid == 0) *s.counter = 0;
+  }
+};
+
+// LM-head argmax, then - in the last CTA - acceptance, commit and rollback.
+struct EpiArgmaxAccept {
+  struct Params {
+    EpiArgmax::Params am;
+    AcceptParams accept;
+  };
+  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs, int lane) {
+    EpiArgmax::apply(p.am, s, o, rs, lane);
+  }
+  __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
+    __shared__ int s_tok[kRmax];
+    if (!EpiArgmax::merge(p.am, s, R, tid, s_tok)) return;
+    named_sync(1, kConsumers);
+    accept_rows(p.accept, s_tok, tid, kConsumers, ConsumerSync{});
+  }
+};
+
+template <>
+__device__ __forceinline__ void epi_init<EpiArgmaxAccept>(int tid) { EpiArgmax::init(tid); }
+
+}  // namespace ocrdec

@@ -38,7 +38,7 @@ constexpr int kTile = kNW * kWarpRows;          // 32 rows per tile
 constexpr int kSlice = 256;                     // columns per stage
 constexpr int kBoxRows = 16;                    // rows per TMA box (two boxes per stage)
 constexpr int kStageBytes = kTile * kSlice * 2; // 16 KB
-constexpr int kStages = 6;
+constexpr int kStages = 4;
 constexpr int kRmax = 8;                        // rows per pass on the GEMV path
 
 struct GemvShape {
@@ -144,12 +144,51 @@ __device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, 
       : "memory");
 }
 
+// ---- packed float pairs (Blackwell f32x2 FMA) -------------------------------
+typedef unsigned long long f2_t;
+__device__ __forceinline__ f2_t pk2(float lo, float hi) {
+  f2_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ float2 upk2(f2_t v) {
+  float2 f;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
+  return f;
+}
+// acc.{x,y} = fma(a.{x,y}, b.{x,y}, acc.{x,y}), each rounded like a scalar fma
+__device__ __forceinline__ void ffma2(f2_t& acc, f2_t a, f2_t b) {
+  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
+}
+// a bfloat16 pair (low half = element 0) as a float pair
+__device__ __forceinline__ f2_t bf2_to_f2(uint32_t u) {
+  return pk2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+}
+
+// The 8 elements of one 16-byte weight chunk, or of the matching activation
+// chunk, as 4 float pairs (0,1), (2,3), (4,5), (6,7).
+struct Pairs8 {
+  f2_t p[4];
+};
+
+__device__ __forceinline__ Pairs8 pairs_from_bf16(const uint4& u) {
+  Pairs8 r;
+  r.p[0] = bf2_to_f2(u.x);
+  r.p[1] = bf2_to_f2(u.y);
+  r.p[2] = bf2_to_f2(u.z);
+  r.p[3] = bf2_to_f2(u.w);
+  return r;
+}
+
 // ---------------------------------------------------------------------------
 // activation sources: 16-byte chunk c16 of pass row r (slot for expert outputs)
 // ---------------------------------------------------------------------------
 
 // Rows of a float32 matrix, RMS-normalised, scaled by a gain vector and rounded
-// to bfloat16 into shared memory once per kernel (K = model width).
+// to bfloat16 (the GEMV input precision), kept as float32 in shared memory once
+// per kernel (K = model width).  Each row is stored as two planes: plane 0
+// holds elements 8c..8c+3 of every 16-byte chunk c, plane 1 elements 8c+4..8c+7,
+// so a lane's two 16-byte loads are consecutive across the warp.
 struct SrcNorm {
   struct Params {
     const float* x;
@@ -159,8 +198,9 @@ struct SrcNorm {
     float eps;
   };
   static constexpr bool kSmem = true;
+  static constexpr int kBytesPerElem = 4;
 
-  __device__ static void prologue(const Params& p, int K, int R, bf16* xs, float* red, int tid) {
+  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, int tid) {
     // per-row sum of squares: thread-strided partials, warp butterfly, warps in order
     __shared__ float scale[kRmax];
     int lane = tid & 31, warp = tid >> 5;
@@ -182,17 +222,29 @@ struct SrcNorm {
       scale[tid] = rsqrtf(__fadd_rn(__fdiv_rn(a, (float)K), p.eps));
     }
     named_sync(1, kConsumers);
+    const int half = K / 2;
     for (int r = 0; r < R; ++r) {
       const float* xr = p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx;
       float sc = scale[r];
-      for (int k = tid; k < K; k += kConsumers)
-        xs[r * K + k] = f2bf(__fmul_rn(__fmul_rn(xr[k], sc), bf2f(p.gain[k])));
+      for (int k = tid; k < K; k += kConsumers) {
+        float v = round_bf(__fmul_rn(__fmul_rn(xr[k], sc), bf2f(p.gain[k])));
+        int c = k >> 3, e = k & 7;
+        xs[r * K + (e >> 2) * half + c * 4 + (e & 3)] = v;
+      }
     }
     named_sync(1, kConsumers);
   }
 
-  __device__ static uint4 chunk(const Params& p, const bf16* xs, int K, int r, int slot, int c16) {
-    return *reinterpret_cast<const uint4*>(xs + r * K + c16 * 8);
+  __device__ static Pairs8 chunk(const Params& p, const float* xs, int K, int r, int slot, int c16) {
+    const float* base = xs + r * K + c16 * 4;
+    float4 lo = *reinterpret_cast<const float4*>(base);
+    float4 hi = *reinterpret_cast<const float4*>(base + K / 2);
+    Pairs8 q;
+    q.p[0] = pk2(lo.x, lo.y);
+    q.p[1] = pk2(lo.z, lo.w);
+    q.p[2] = pk2(hi.x, hi.y);
+    q.p[3] = pk2(hi.z, hi.w);
+    return q;
   }
 };
 
@@ -205,10 +257,11 @@ struct SrcBf16 {
     const int* row_src;
   };
   static constexpr bool kSmem = false;
-  __device__ static void prologue(const Params&, int, int, bf16*, float*, int) {}
-  __device__ static uint4 chunk(const Params& p, const bf16*, int K, int r, int slot, int c16) {
+  static constexpr int kBytesPerElem = 0;
+  __device__ static void prologue(const Params&, int, int, float*, float*, int) {}
+  __device__ static Pairs8 chunk(const Params& p, const float*, int K, int r, int slot, int c16) {
     int row = (p.row_src ? p.row_src[r] : r) * p.nslot + slot;
-    return ld_v4(p.x + (long long)row * p.ld + c16 * 8);
+    return pairs_from_bf16(ld_v4(p.x + (long long)row * p.ld + c16 * 8));
   }
 };
 
@@ -360,7 +413,9 @@ struct EpiArgmax {
     if (tid < kNW * kRmax) { best_v()[tid] = -INFINITY; best_i()[tid] = 0x7fffffff; }
   }
 
-  __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
+  // Per-CTA partial, then the last CTA merges all partials; returns true in the
+  // last CTA, where s_tok[r] holds the token of pass row r (r < R).
+  __device__ static bool merge(const Params& p, const GemvShape& s, int R, int tid, int* s_tok) {
     __shared__ int last;
     if (tid < kRmax) {
       float bv = -INFINITY;
@@ -376,7 +431,7 @@ struct EpiArgmax {
     named_sync(1, kConsumers);
     if (tid == 0) last = (atomicAdd(s.counter, 1) == (int)gridDim.x - 1);
     named_sync(1, kConsumers);
-    if (!last) return;
+    if (!last) return false;
     __threadfence();
     if (tid < R) {
       float bv = -INFINITY;
@@ -388,8 +443,15 @@ struct EpiArgmax {
         if (ev > bv || (ev == bv && ei < bi)) { bv = ev; bi = ei; }
       }
       p.tok[(p.row_dst ? p.row_dst[tid] : tid) * p.tok_stride] = bi;
+      s_tok[tid] = bi;
     }
     if (tid == 0) *s.counter = 0;
+    return true;
+  }
+
+  __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
+    __shared__ int s_tok[kRmax];
+    merge(p, s, R, tid, s_tok);
   }
 };
 
@@ -401,6 +463,85 @@ __device__ __forceinline__ void epi_init<EpiArgmax>(int tid) { EpiArgmax::init(t
 // ---------------------------------------------------------------------------
 // the kernel
 // ---------------------------------------------------------------------------
+
+// Streams the tiles of one work item through the ring and returns the warp's
+// reduced values: lane L = 8 i + q gets local row i (0..3) for row-set entry q.
+// NR = live rows of the item (row-set entries 0..NR-1); the arithmetic of a
+// row does not depend on NR.
+template <int NR, class Src>
+__device__ __forceinline__ float consume_item(const GemvShape& s, const typename Src::Params& sp, const float* xs,
+                                              const unsigned char* stages, uint64_t* full_bar, uint64_t* empty_bar,
+                                              uint32_t& it, const RowSet& rs, const int (&srow)[kWarpRows],
+                                              int nch, int lane) {
+  f2_t acc[kWarpRows][NR > 0 ? NR : 1];
+#pragma unroll
+  for (int i = 0; i < kWarpRows; ++i)
+#pragma unroll
+    for (int q = 0; q < (NR > 0 ? NR : 1); ++q) acc[i][q] = 0ull;
+
+  for (int sl = 0; sl < s.ns; ++sl, ++it) {
+    const int st = it % kStages;
+    mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
+    const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
+    if (NR > 0 && c < nch) {
+      Pairs8 xv[NR > 0 ? NR : 1];
+#pragma unroll
+      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, s.K, rs.r[q], rs.slot[q], c);
+      const unsigned char* w_st = stages + st * kStageBytes + lane * 16;
+#pragma unroll
+      for (int i = 0; i < kWarpRows; ++i) {
+        Pairs8 wv = pairs_from_bf16(*reinterpret_cast<const uint4*>(w_st + srow[i] * (kSlice * 2)));
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+#pragma unroll
+          for (int q = 0; q < NR; ++q) ffma2(acc[i][q], wv.p[e], xv[q].p[e]);
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty_bar[st]);
+  }
+
+  // per lane: even + odd partial; then transpose over lane bits 4, 3 and a
+  // butterfly over bits 2..0, after which lane L holds local row L >> 3
+  float out = 0.f;
+#pragma unroll
+  for (int q = 0; q < NR; ++q) {
+    float r4[kWarpRows];
+#pragma unroll
+    for (int i = 0; i < kWarpRows; ++i) {
+      float2 t = upk2(acc[i][q]);
+      r4[i] = __fadd_rn(t.x, t.y);
+    }
+    const bool up16 = lane & 16;
+    float a0 = __fadd_rn(up16 ? r4[2] : r4[0], __shfl_xor_sync(0xffffffffu, up16 ? r4[0] : r4[2], 16));
+    float a1 = __fadd_rn(up16 ? r4[3] : r4[1], __shfl_xor_sync(0xffffffffu, up16 ? r4[1] : r4[3], 16));
+    const bool up8 = lane & 8;
+    float b = __fadd_rn(up8 ? a1 : a0, __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8));
+    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 4));
+    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 2));
+    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 1));
+    if ((lane & 7) == q) out = b;
+  }
+  return out;
+}
+
+template <int RG, class Src>
+__device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, const typename Src::Params& sp,
+                                                  const float* xs, const unsigned char* stages, uint64_t* full_bar,
+                                                  uint64_t* empty_bar, uint32_t& it, const RowSet& rs,
+                                                  const int (&srow)[kWarpRows], int nch, int lane) {
+#define OCRDEC_CONSUME(NRV) consume_item<NRV, Src>(s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane)
+  if (n <= 0) return OCRDEC_CONSUME(0);
+  if (n == 1 || RG == 1) return OCRDEC_CONSUME(1);
+  if (n == 2 || RG == 2) return OCRDEC_CONSUME((RG >= 2 ? 2 : 1));
+  if (n == 3) return OCRDEC_CONSUME((RG >= 3 ? 3 : 1));
+  if (n == 4 || RG == 4) return OCRDEC_CONSUME((RG >= 4 ? 4 : 1));
+  if (n == 5) return OCRDEC_CONSUME((RG >= 5 ? 5 : 1));
+  if (n == 6) return OCRDEC_CONSUME((RG >= 6 ? 6 : 1));
+  if (n == 7) return OCRDEC_CONSUME((RG >= 7 ? 7 : 1));
+  return OCRDEC_CONSUME((RG >= 8 ? 8 : 1));
+#undef OCRDEC_CONSUME
+}
 
 template <int RG, class Src, class Epi>
 __global__ void __launch_bounds__(kGemvThreads, 1)
@@ -414,7 +555,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   unsigned char* stages = smem;
-  bf16* xs = reinterpret_cast<bf16*>(smem + kStages * kStageBytes);
+  float* xs = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  const bool paired = s.pair_half != 0;
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -423,9 +565,67 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     }
     fence_mbar_init();
   }
+  __syncthreads();
+
+  if (warp == kNW) {
+    // ---------------- producer ----------------
+    if (lane != 0) return;
+    uint32_t it = 0;
+    // Dense weights do not depend on earlier kernels: start streaming the first
+    // stages before waiting for the previous kernel (programmatic dependent
+    // launch lets this overlap its tail).
+    int total = s.mats ? 0 : s.tiles_per_mat;
+    int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
+    int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
+    int item = start, sl = 0;
+    auto issue = [&](int m, int t, int slc) {
+      int ce;
+      bool sh;
+      mat_info(s, m, 0, &ce, &sh, nullptr);
+      const CUtensorMap* map = sh ? &tm_sh : &tm_w;
+      int r0, r1;
+      tile_boxes(s, t, &r0, &r1);
+      const int st = it % kStages;
+      // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
+      // stays uniform so the block always terminates
+      if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
+      mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
+      unsigned char* dst = stages + st * kStageBytes;
+      tma_load_box(dst, map, slc * kSlice, r0, ce, &full_bar[st]);
+      tma_load_box(dst + kStageBytes / 2, map, slc * kSlice, r1, ce, &full_bar[st]);
+      ++it;
+    };
+    if (!s.mats) {
+      for (; item < end && it < (uint32_t)kStages;) {
+        issue(0, item, sl);
+        if (++sl == s.ns) { sl = 0; ++item; }
+      }
+    }
+    pdl_wait();
+    if (!status_bad(s.status)) {
+      if (s.mats) {
+        total = *s.n_mats * s.tiles_per_mat;
+        start = (int)(((long long)blockIdx.x * total) / gridDim.x);
+        end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
+        item = start;
+        sl = 0;
+      }
+      for (; item < end;) {
+        int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
+        issue(m, t, sl);
+        if (++sl == s.ns) { sl = 0; ++item; }
+      }
+    }
+    // drain: every issued copy has landed before the block can exit
+    for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
+      mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, s.status);
+    return;
+  }
+
+  // ---------------- consumers ----------------
   pdl_wait();
   if (tid == 0) s_abort = status_bad(s.status);
-  __syncthreads();
+  named_sync(1, kConsumers);
   if (s_abort) return;
   pdl_trigger();
 
@@ -435,39 +635,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
   const int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
   const int nch = s.K / 8;  // 16-byte chunks per row
-  const bool paired = s.pair_half != 0;
 
-  if (warp == kNW) {
-    // ---------------- producer ----------------
-    if (lane == 0) {
-      uint32_t it = 0;
-      for (int item = start; item < end; ++item) {
-        int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
-        int ce;
-        bool sh;
-        mat_info(s, m, R, &ce, &sh, nullptr);
-        const CUtensorMap* map = sh ? &tm_sh : &tm_w;
-        int r0, r1;
-        tile_boxes(s, t, &r0, &r1);
-        for (int sl = 0; sl < s.ns; ++sl, ++it) {
-          int st = it % kStages;
-          // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control
-          // flow stays uniform so the block always terminates
-          if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
-          mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
-          unsigned char* dst = stages + st * kStageBytes;
-          tma_load_box(dst, map, sl * kSlice, r0, ce, &full_bar[st]);
-          tma_load_box(dst + kStageBytes / 2, map, sl * kSlice, r1, ce, &full_bar[st]);
-        }
-      }
-      // drain: every issued copy has landed before the block can exit
-      for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
-        mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, s.status);
-    }
-    return;
-  }
-
-  // ---------------- consumers ----------------
   epi_init<Epi>(tid);
   if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, tid);
   else named_sync(1, kConsumers);
@@ -487,68 +655,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       mat_info(s, m, R, &ce, &sh, &rs);
       cur_m = m;
     }
-    float acc[kWarpRows][RG];
-#pragma unroll
-    for (int i = 0; i < kWarpRows; ++i)
-#pragma unroll
-      for (int q = 0; q < RG; ++q) acc[i][q] = 0.f;
-
-    for (int sl = 0; sl < s.ns; ++sl, ++it) {
-      const int st = it % kStages;
-      mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
-      const unsigned char* w_st = stages + st * kStageBytes;
-      const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
-      if (c < nch) {
-        float xv[RG][8];
-#pragma unroll
-        for (int q = 0; q < RG; ++q) {
-          if (q < rs.n) {
-            uint4 u = Src::chunk(sp, xs, s.K, rs.r[q], rs.slot[q], c);
-            unpack8(u, xv[q]);
-          } else {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xv[q][e] = 0.f;
-          }
-        }
-#pragma unroll
-        for (int i = 0; i < kWarpRows; ++i) {
-          uint4 u = *reinterpret_cast<const uint4*>(w_st + srow[i] * (kSlice * 2) + lane * 16);
-          float wv[8];
-          unpack8(u, wv);
-#pragma unroll
-          for (int e = 0; e < 8; ++e)
-#pragma unroll
-            for (int q = 0; q < RG; ++q) acc[i][q] = __fmaf_rn(wv[e], xv[q][e], acc[i][q]);
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty_bar[st]);
-    }
-
-    // reduce the warp's 4 rows: transpose over lane bits 4, 3, then butterfly over bits 2..0;
-    // afterwards lane L holds the full sum of local row (L >> 3)
-    float v[RG];
-#pragma unroll
-    for (int q = 0; q < RG; ++q) {
-      const bool up16 = lane & 16;
-      float a0 = __fadd_rn(up16 ? acc[2][q] : acc[0][q],
-                           __shfl_xor_sync(0xffffffffu, up16 ? acc[0][q] : acc[2][q], 16));
-      float a1 = __fadd_rn(up16 ? acc[3][q] : acc[1][q],
-                           __shfl_xor_sync(0xffffffffu, up16 ? acc[1][q] : acc[3][q], 16));
-      const bool up8 = lane & 8;
-      float b = __fadd_rn(up8 ? a1 : a0, __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8));
-      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 4));
-      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 2));
-      b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 1));
-      v[q] = b;
-    }
     WarpOut o;
+    o.v = consume_dispatch<RG, Src>(rs.n, s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane);
     o.i = lane >> 3;
     o.q = lane & 7;
-    o.v = 0.f;
-#pragma unroll
-    for (int q = 0; q < RG; ++q)
-      if (o.q == q) o.v = v[q];
     int r0, r1;
     tile_boxes(s, t, &r0, &r1);
 #pragma unroll

@@ -36,7 +36,7 @@ cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap
 
 template <class Src>
 static size_t smem_max() {
-  return (size_t)kStages * kStageBytes + (Src::kSmem ? (size_t)kRmax * kGemvMaxK * 2 : 0);
+  return (size_t)kStages * kStageBytes + (size_t)kRmax * kGemvMaxK * Src::kBytesPerElem;
 }
 
 template <int RG, class Src, class Epi>
@@ -59,6 +59,8 @@ cudaError_t gemv_prepare() {
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiSwiGLU>();
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmax>();
+  if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiRoute>();
+  if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmaxAccept>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<true>>();
   return e;
@@ -69,7 +71,7 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
                               const LaunchCfg& lc) {
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
-  size_t smem = (size_t)kStages * kStageBytes + (Src::kSmem ? (size_t)kRmax * g.s.K * 2 : 0);
+  size_t smem = (size_t)kStages * kStageBytes + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
   int grid = g.grid;
   if (grid <= 0) grid = g.s.mats ? lc.num_sms : std::min(g.s.tiles_per_mat, lc.num_sms);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
@@ -94,6 +96,14 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
       case EpiKind::Store: return launch_rg<SrcNorm, EpiStore<false>>(g, g.norm, g.store, lc);
       case EpiKind::SwiGLU: return launch_rg<SrcNorm, EpiSwiGLU>(g, g.norm, g.swiglu, lc);
       case EpiKind::Argmax: return launch_rg<SrcNorm, EpiArgmax>(g, g.norm, g.argmax, lc);
+      case EpiKind::Route: {
+        EpiRoute::Params ep{g.store, g.route};
+        return launch_rg<SrcNorm, EpiRoute>(g, g.norm, ep, lc);
+      }
+      case EpiKind::ArgmaxAccept: {
+        EpiArgmaxAccept::Params ep{g.argmax, g.accept};
+        return launch_rg<SrcNorm, EpiArgmaxAccept>(g, g.norm, ep, lc);
+      }
       default: return cudaErrorInvalidValue;
     }
   }

@@ -3,7 +3,7 @@
 
 #include <cuda_runtime.h>
 
-#include "gemv.cuh"
+#include "fused_epi.cuh"
 
 namespace ocrdec {
 
@@ -31,7 +31,7 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
 }
 
 enum class SrcKind { Norm, Bf16 };
-enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax };
+enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, Route, ArgmaxAccept };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.
 struct GemvLaunch {
@@ -46,6 +46,8 @@ struct GemvLaunch {
   EpiSwiGLU::Params swiglu{};
   EpiQKV::Params qkv{};
   EpiArgmax::Params argmax{};
+  RouteParams route{};    // EpiKind::Route (with store)
+  AcceptParams accept{};  // EpiKind::ArgmaxAccept (with argmax)
   int rows_bound = kRmax;  // static bound on rows of one work item (selects the row-group width)
   int grid = 0;            // 0: derived from the work and the SM count
 };

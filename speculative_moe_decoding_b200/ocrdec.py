@@ -66,6 +66,7 @@ ocrdec_get_counters = _sig("ocrdec_get_counters", _i32, _vp, ctypes.POINTER(_i32
 ocrdec_reset_counters = _sig("ocrdec_reset_counters", _i32, _vp, _vp)
 ocrdec_step_kernel_count = _sig("ocrdec_step_kernel_count", _i32, _vp, _i32, _i32, _vp, _vp, ctypes.POINTER(_i32))
 ocrdec_set_debug_taps = _sig("ocrdec_set_debug_taps", _i32, _vp, _vp, _vp)
+ocrdec_set_draft_taps = _sig("ocrdec_set_draft_taps", _i32, _vp, _vp)
 ocrdec_strerror = _sig("ocrdec_strerror", ctypes.c_char_p, _i32)
 ocrdec_op_scratch_bytes = _sig("ocrdec_op_scratch_bytes", _sz)
 ocrdec_op_norm_gemv = _sig("ocrdec_op_norm_gemv", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp)
@@ -240,6 +241,10 @@ class Decoder:
         check(ocrdec_step_kernel_count(self.ctx, batch, k, self.committed.data_ptr(), self.n_committed.data_ptr(),
                                        ctypes.byref(n)), "ocrdec_step_kernel_count")
         return n.value
+
+    def set_draft_taps(self, logits=None):
+        self._dtaps = logits
+        check(ocrdec_set_draft_taps(self.ctx, _ptr(logits)), "ocrdec_set_draft_taps")
 
     def set_debug_taps(self, hidden=None, logits=None):
         self._taps = (hidden, logits)
