@@ -71,7 +71,7 @@ typedef struct {
   int32_t expert_ffn, shared_ffn, dense_ffn, draft_ffn, vocab;
   int32_t max_k;       /* largest number of draft tokens per step, 0..3 */
   int32_t max_batch;   /* number of sequence slots */
-  int32_t kv_capacity; /* positions per slot (context + generated + max_k) */
+  int32_t kv_capacity; /* positions per slot (context + generated + max_k), <= 8192 */
   float rope_theta, rms_eps;
 } ocrdec_config;
 

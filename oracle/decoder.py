@@ -358,10 +358,11 @@ def draft_propose(orc: Oracle, st: SeqState, k: int, margins: Optional[list] = N
 
 
 def verify_commit(orc: Oracle, st: SeqState, proposals: Sequence[int],
-                  record: Optional[list] = None) -> List[int]:
+                  record: Optional[list] = None, forced_g: Optional[Sequence[int]] = None) -> List[int]:
     """One verifier pass over [bonus, d_1..d_k] at positions n..n+k, processed one
     row at a time; commits the longest agreeing prefix plus the bonus token and
-    rolls the KV length back to n + a + 1."""
+    rolls the KV length back to n + a + 1.  ``forced_g`` (tests only) replaces the
+    rows' greedy tokens - teacher forcing onto another implementation's choices."""
     n = st.kv_len
     rows = [st.bonus] + list(proposals)
     g, hs = [], []
@@ -371,6 +372,8 @@ def verify_commit(orc: Oracle, st: SeqState, proposals: Sequence[int],
         hs.append(out.hidden[0])
         if record is not None:
             record.append((n + i, tok, out))
+    if forced_g is not None:
+        g = [int(t) for t in forced_g]
     a = 0
     while a < len(proposals) and proposals[a] == g[a]:
         a += 1

@@ -18,6 +18,7 @@ namespace ocrdec {
 constexpr int kAttnChunk = 64;
 constexpr int kAttnThreads = 128;
 constexpr int kAttnRows = 8;  // rows of one slot in a pass
+constexpr int kAttnMaxChunks = 128;  // chunks per sequence: kv_capacity <= 8192
 
 struct AttnParams {
   const float* q;          // [R][H*Dh]
@@ -78,9 +79,10 @@ attention_kernel(const AttnParams p) {
     bulk_g2s(Ks, p.kc + base, bytes, &bar);
     bulk_g2s(Vs, p.vc + base, bytes, &bar);
   }
-  // queries of this slot's rows
-  for (int i = 0; i < nr; ++i)
-    for (int d = tid; d < Dh; d += kAttnThreads) qs[i][d] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + d];
+  // queries of this slot's rows (all loads in flight together)
+#pragma unroll
+  for (int i = 0; i < kAttnRows; ++i)
+    if (i < nr && tid < Dh) qs[i][tid] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + tid];
   __syncthreads();
   mbar_wait(&bar, 0, p.status);  // gives up with OCRDEC_ETIMEOUT recorded; control flow stays uniform
 
@@ -214,20 +216,41 @@ attention_kernel(const AttnParams p) {
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int r = 0; r < nr; ++r) {
-    int pos = p.row_pos[r0 + r];
-    int nc = pos / kAttnChunk + 1;
-    const volatile float* pr = p.part + ((long long)(r0 + r) * p.H + h) * p.max_chunks * ld;
+  // stage every (row, chunk) max and sum, then the per-chunk rescale factors
+  __shared__ float s_m2[kAttnRows][kAttnMaxChunks];
+  __shared__ float s_f[kAttnRows][kAttnMaxChunks];
+  __shared__ float s_L[kAttnRows];
+  const int maxc = min(nchunks, kAttnMaxChunks);
+  for (int idx = tid; idx < nr * maxc; idx += kAttnThreads) {
+    int r = idx / maxc, cc = idx - r * maxc;
+    const float* pr = p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + cc) * ld;
+    int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
+    s_m2[r][cc] = cc < nc ? __ldcg(pr + Dh) : -INFINITY;     // m
+    s_f[r][cc] = cc < nc ? __ldcg(pr + Dh + 1) : 0.f;       // l
+  }
+  __syncthreads();
+  if (tid < nr) {
+    const int r = tid;
+    int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
     float M = -INFINITY;
-    for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, pr[cc * ld + Dh]);
+    for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, s_m2[r][cc]);
+    float L = 0.f;
+    for (int cc = 0; cc < nc; ++cc) {
+      float f = expf(__fsub_rn(s_m2[r][cc], M));
+      L = __fmaf_rn(s_f[r][cc], f, L);
+      s_m2[r][cc] = f;
+    }
+    s_L[r] = L;
+  }
+  __syncthreads();
+  for (int r = 0; r < nr; ++r) {
+    const int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
+    const float* pr = p.part + ((long long)(r0 + r) * p.H + h) * p.max_chunks * ld;
     for (int d = tid; d < Dh; d += kAttnThreads) {
-      float L = 0.f, O = 0.f;
-      for (int cc = 0; cc < nc; ++cc) {
-        float f = expf(__fsub_rn(pr[cc * ld + Dh], M));
-        L = __fmaf_rn(pr[cc * ld + Dh + 1], f, L);
-        O = __fmaf_rn(pr[cc * ld + d], f, O);
-      }
-      p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, L));
+      float O = 0.f;
+#pragma unroll 4
+      for (int cc = 0; cc < nc; ++cc) O = __fmaf_rn(__ldcg(pr + cc * ld + d), s_m2[r][cc], O);
+      p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, s_L[r]));
     }
   }
   if (tid == 0) p.counters[b * p.H + h] = 0;

@@ -100,7 +100,8 @@ bool config_ok(const ocrdec_config* c) {
   if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > 256 || c->top_k + c->n_shared > 127) return false;
   if (c->max_k < 0 || c->max_k > 3) return false;
   if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
-  if (c->d_model * 2 > 4096) return false;  // shared-memory copy of the normalised rows
+  if (c->d_model > kGemvMaxK) return false;  // shared-memory copy of the normalised rows
+  if ((c->kv_capacity + kAttnChunk - 1) / kAttnChunk > kAttnMaxChunks) return false;
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
   return true;
 }

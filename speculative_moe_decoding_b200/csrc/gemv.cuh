@@ -37,9 +37,10 @@ constexpr int kWarpRows = 4;                    // weight rows per warp per tile
 constexpr int kTile = kNW * kWarpRows;          // 32 rows per tile
 constexpr int kSlice = 256;                     // columns per stage
 constexpr int kBoxRows = 16;                    // rows per TMA box (two boxes per stage)
-constexpr int kStageBytes = kTile * kSlice * 2; // 16 KB
+constexpr int kStageBytes = kTile * kSlice * 2; // 16 KB of weights per stage
 constexpr int kStages = 4;
 constexpr int kRmax = 8;                        // rows per pass on the GEMV path
+constexpr int kXSliceBytes = kSlice * 2;        // one activation row of a staged bf16 slice (512 B)
 
 struct GemvShape {
   int N, K;
@@ -185,10 +186,11 @@ __device__ __forceinline__ Pairs8 pairs_from_bf16(const uint4& u) {
 // ---------------------------------------------------------------------------
 
 // Rows of a float32 matrix, RMS-normalised, scaled by a gain vector and rounded
-// to bfloat16 (the GEMV input precision), kept as float32 in shared memory once
-// per kernel (K = model width).  Each row is stored as two planes: plane 0
-// holds elements 8c..8c+3 of every 16-byte chunk c, plane 1 elements 8c+4..8c+7,
-// so a lane's two 16-byte loads are consecutive across the warp.
+// to bfloat16 (the GEMV input precision), kept as float32 in shared memory for
+// the whole kernel (K = model width).  The raw rows arrive by bulk copy; each
+// is then normalised in place into two planes: plane 0 holds elements
+// 8c..8c+3 of every 16-byte chunk c, plane 1 elements 8c+4..8c+7, so a lane's
+// two 16-byte loads are consecutive across the warp.
 struct SrcNorm {
   struct Params {
     const float* x;
@@ -197,58 +199,79 @@ struct SrcNorm {
     const bf16* gain;
     float eps;
   };
-  static constexpr bool kSmem = true;
+  static constexpr bool kSmem = true;    // activations live in shared memory (prologue)
+  static constexpr bool kStaged = false; // activations are not part of the weight stages
   static constexpr int kBytesPerElem = 4;
+  static constexpr int kMaxPer = 16;     // elements per thread per row: K <= 16 * 256
 
-  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, int tid) {
-    // per-row sum of squares: thread-strided partials, warp butterfly, warps in order
-    __shared__ float scale[kRmax];
-    int lane = tid & 31, warp = tid >> 5;
+  // Called by all consumer threads after the dependency wait.
+  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, uint64_t* xbar,
+                                  int* status, int tid) {
+    if (tid == 0) {
+      mbar_init(xbar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(xbar, (uint32_t)(R * K * 4));
+      for (int r = 0; r < R; ++r)
+        bulk_g2s(xs + r * K, p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx, K * 4, xbar);
+    }
+    float g[kMaxPer];
 #pragma unroll
-    for (int r = 0; r < kRmax; ++r) {
+    for (int j = 0; j < kMaxPer; ++j) {
+      int k = tid + j * kConsumers;
+      g[j] = k < K ? bf2f(p.gain[k]) : 0.f;
+    }
+    named_sync(1, kConsumers);
+    if (R > 0) mbar_wait(xbar, 0, status);
+    const int lane = tid & 31, warp = tid >> 5;
+    const int half = K / 2;
+    for (int r = 0; r < R; ++r) {
+      float* row = xs + r * K;
+      float v[kMaxPer];
       float a = 0.f;
-      if (r < R) {
-        const float* xr = p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx;
-        for (int k = tid; k < K; k += kConsumers) a = __fmaf_rn(xr[k], xr[k], a);
+#pragma unroll
+      for (int j = 0; j < kMaxPer; ++j) {
+        int k = tid + j * kConsumers;
+        v[j] = k < K ? row[k] : 0.f;
+        a = __fmaf_rn(v[j], v[j], a);
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (lane == 0) red[warp * kRmax + r] = a;
-    }
-    named_sync(1, kConsumers);
-    if (tid < kRmax) {
-      float a = 0.f;
-      for (int w = 0; w < kNW; ++w) a = __fadd_rn(a, red[w * kRmax + tid]);
-      scale[tid] = rsqrtf(__fadd_rn(__fdiv_rn(a, (float)K), p.eps));
-    }
-    named_sync(1, kConsumers);
-    const int half = K / 2;
-    for (int r = 0; r < R; ++r) {
-      const float* xr = p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx;
-      float sc = scale[r];
-      for (int k = tid; k < K; k += kConsumers) {
-        float v = round_bf(__fmul_rn(__fmul_rn(xr[k], sc), bf2f(p.gain[k])));
-        int c = k >> 3, e = k & 7;
-        xs[r * K + (e >> 2) * half + c * 4 + (e & 3)] = v;
+      if (lane == 0) red[r * kNW + warp] = a;
+      named_sync(1, kConsumers);  // every thread has read row r and posted its sum
+      float ss = 0.f;
+#pragma unroll
+      for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
+      const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
+#pragma unroll
+      for (int j = 0; j < kMaxPer; ++j) {
+        int k = tid + j * kConsumers;
+        if (k < K) {
+          int c = k >> 3, e = k & 7;
+          row[(e >> 2) * half + c * 4 + (e & 3)] = round_bf(__fmul_rn(__fmul_rn(v[j], sc), g[j]));
+        }
       }
     }
     named_sync(1, kConsumers);
   }
 
-  __device__ static Pairs8 chunk(const Params& p, const float* xs, int K, int r, int slot, int c16) {
+  __device__ static Pairs8 chunk(const Params& p, const float* xs, const unsigned char* xstage, int K, int q, int r,
+                                 int slot, int c16, int lane) {
     const float* base = xs + r * K + c16 * 4;
     float4 lo = *reinterpret_cast<const float4*>(base);
     float4 hi = *reinterpret_cast<const float4*>(base + K / 2);
-    Pairs8 q;
-    q.p[0] = pk2(lo.x, lo.y);
-    q.p[1] = pk2(lo.z, lo.w);
-    q.p[2] = pk2(hi.x, hi.y);
-    q.p[3] = pk2(hi.z, hi.w);
-    return q;
+    Pairs8 o;
+    o.p[0] = pk2(lo.x, lo.y);
+    o.p[1] = pk2(lo.z, lo.w);
+    o.p[2] = pk2(hi.x, hi.y);
+    o.p[3] = pk2(hi.z, hi.w);
+    return o;
   }
 };
 
 // Rows of a bfloat16 matrix in global memory: row (row_src[r] * nslot + slot).
+// The producer copies each slice of the item's rows into the stage next to the
+// weight box (row-set entry q at offset q * 512 B), so consumers read them from
+// shared memory.
 struct SrcBf16 {
   struct Params {
     const bf16* x;
@@ -257,11 +280,15 @@ struct SrcBf16 {
     const int* row_src;
   };
   static constexpr bool kSmem = false;
+  static constexpr bool kStaged = true;
   static constexpr int kBytesPerElem = 0;
-  __device__ static void prologue(const Params&, int, int, float*, float*, int) {}
-  __device__ static Pairs8 chunk(const Params& p, const float*, int K, int r, int slot, int c16) {
-    int row = (p.row_src ? p.row_src[r] : r) * p.nslot + slot;
-    return pairs_from_bf16(ld_v4(p.x + (long long)row * p.ld + c16 * 8));
+  __device__ static void prologue(const Params&, int, int, float*, float*, uint64_t*, int*, int) {}
+  __device__ static const bf16* row_ptr(const Params& p, int r, int slot) {
+    return p.x + (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
+  }
+  __device__ static Pairs8 chunk(const Params& p, const float*, const unsigned char* xstage, int K, int q, int r,
+                                 int slot, int c16, int lane) {
+    return pairs_from_bf16(*reinterpret_cast<const uint4*>(xstage + q * kXSliceBytes + lane * 16));
   }
 };
 
@@ -468,6 +495,11 @@ __device__ __forceinline__ void epi_init<EpiArgmax>(int tid) { EpiArgmax::init(t
 // reduced values: lane L = 8 i + q gets local row i (0..3) for row-set entry q.
 // NR = live rows of the item (row-set entries 0..NR-1); the arithmetic of a
 // row does not depend on NR.
+template <class Src>
+constexpr int stage_stride() {
+  return kStageBytes + (Src::kStaged ? kRmax * kXSliceBytes : 0);
+}
+
 template <int NR, class Src>
 __device__ __forceinline__ float consume_item(const GemvShape& s, const typename Src::Params& sp, const float* xs,
                                               const unsigned char* stages, uint64_t* full_bar, uint64_t* empty_bar,
@@ -484,10 +516,11 @@ __device__ __forceinline__ float consume_item(const GemvShape& s, const typename
     mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
     const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
     if (NR > 0 && c < nch) {
+      const unsigned char* stg = stages + st * stage_stride<Src>();
       Pairs8 xv[NR > 0 ? NR : 1];
 #pragma unroll
-      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, s.K, rs.r[q], rs.slot[q], c);
-      const unsigned char* w_st = stages + st * kStageBytes + lane * 16;
+      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, stg + kStageBytes, s.K, q, rs.r[q], rs.slot[q], c, lane);
+      const unsigned char* w_st = stg + lane * 16;
 #pragma unroll
       for (int i = 0; i < kWarpRows; ++i) {
         Pairs8 wv = pairs_from_bf16(*reinterpret_cast<const uint4*>(w_st + srow[i] * (kSlice * 2)));
@@ -548,19 +581,20 @@ __global__ void __launch_bounds__(kGemvThreads, 1)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
-  __shared__ float red_pro[kNW * kRmax];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], xbar;
+  __shared__ float red_pro[kRmax * kNW];
   __shared__ int s_abort;
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  constexpr int kStride = stage_stride<Src>();
   unsigned char* stages = smem;
-  float* xs = reinterpret_cast<float*>(smem + kStages * kStageBytes);
+  float* xs = reinterpret_cast<float*>(smem + kStages * kStride);
   const bool paired = s.pair_half != 0;
 
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full_bar[i], 1);
+      mbar_init(&full_bar[i], Src::kStaged ? 2 : 1);
       mbar_init(&empty_bar[i], kNW);
     }
     fence_mbar_init();
@@ -578,7 +612,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
     int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
     int item = start, sl = 0;
-    auto issue = [&](int m, int t, int slc) {
+    int R = 0;
+    RowSet prs;  // rows of the current item (bf16 sources staged with the weights)
+    int prs_m = -1;
+    // Stage = weight box (one arrival with its transaction bytes) and, for a
+    // staged bf16 source, the item's activation slice rows (a second arrival,
+    // declared only after the dependency wait).
+    auto issue_w = [&](int m, int t, int slc) {
       int ce;
       bool sh;
       mat_info(s, m, 0, &ce, &sh, nullptr);
@@ -590,19 +630,46 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       // stays uniform so the block always terminates
       if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
       mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
-      unsigned char* dst = stages + st * kStageBytes;
+      unsigned char* dst = stages + st * kStride;
       tma_load_box(dst, map, slc * kSlice, r0, ce, &full_bar[st]);
       tma_load_box(dst + kStageBytes / 2, map, slc * kSlice, r1, ce, &full_bar[st]);
       ++it;
     };
+    auto issue_x = [&](uint32_t j, int m, int slc) {
+      if (!Src::kStaged) return;
+      if (m != prs_m) {
+        int ce;
+        bool sh;
+        mat_info(s, m, R, &ce, &sh, &prs);
+        prs_m = m;
+      }
+      const int st = j % kStages;
+      unsigned char* dst = stages + st * kStride + kStageBytes;
+      const int cols = min(kSlice, s.K - slc * kSlice);
+      mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(prs.n * cols * 2));
+      for (int q = 0; q < prs.n; ++q)
+        bulk_g2s(dst + q * kXSliceBytes,
+                 SrcBf16::row_ptr(reinterpret_cast<const SrcBf16::Params&>(sp), prs.r[q], prs.slot[q]) + slc * kSlice,
+                 cols * 2, &full_bar[st]);
+    };
+    // dense weights do not depend on earlier kernels: the first stages are
+    // requested before the dependency wait
+    int pre_item[kStages], pre_sl[kStages];
+    int npre = 0;
     if (!s.mats) {
       for (; item < end && it < (uint32_t)kStages;) {
-        issue(0, item, sl);
+        pre_item[npre] = item;
+        pre_sl[npre] = sl;
+        ++npre;
+        issue_w(0, item, sl);
         if (++sl == s.ns) { sl = 0; ++item; }
       }
     }
     pdl_wait();
-    if (!status_bad(s.status)) {
+    const bool ok = !status_bad(s.status);
+    if (ok) {
+      R = pass_rows(s);
+      for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j]);
       if (s.mats) {
         total = *s.n_mats * s.tiles_per_mat;
         start = (int)(((long long)blockIdx.x * total) / gridDim.x);
@@ -612,10 +679,16 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       }
       for (; item < end;) {
         int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
-        issue(m, t, sl);
+        const uint32_t j = it;
+        issue_w(m, t, sl);
+        issue_x(j, m, sl);
         if (++sl == s.ns) { sl = 0; ++item; }
       }
+    } else if (Src::kStaged) {
+      // aborting: complete the second arrival of every prefetched stage so the drain below can finish
+      for (int j = 0; j < npre; ++j) mbar_arrive(&full_bar[j]);
     }
+    (void)pre_item;
     // drain: every issued copy has landed before the block can exit
     for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
       mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, s.status);
@@ -637,7 +710,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int nch = s.K / 8;  // 16-byte chunks per row
 
   epi_init<Epi>(tid);
-  if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, tid);
+  if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid);
   else named_sync(1, kConsumers);
 
   uint32_t it = 0;

@@ -36,7 +36,7 @@ cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap
 
 template <class Src>
 static size_t smem_max() {
-  return (size_t)kStages * kStageBytes + (size_t)kRmax * kGemvMaxK * Src::kBytesPerElem;
+  return (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * kGemvMaxK * Src::kBytesPerElem;
 }
 
 template <int RG, class Src, class Epi>
@@ -71,7 +71,7 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
                               const LaunchCfg& lc) {
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
-  size_t smem = (size_t)kStages * kStageBytes + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
+  size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
   int grid = g.grid;
   if (grid <= 0) grid = g.s.mats ? lc.num_sms : std::min(g.s.tiles_per_mat, lc.num_sms);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);

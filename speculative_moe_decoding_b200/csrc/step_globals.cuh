@@ -83,9 +83,14 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   __syncthreads();
   if (s_bad) return;
   pdl_trigger();
-  for (int idx = tid; idx < R * p.d; idx += blockDim.x) {
-    int r = idx / p.d, n = idx - r * p.d;
-    p.x[idx] = bf2f(p.embed[(long long)s_tok[r] * p.d + n]);
+  // embedding gather: every row's loads are issued before any is consumed
+#pragma unroll
+  for (int r = 0; r < kRmax; ++r) {
+    if (r >= R) break;
+    const bf16* e = p.embed + (long long)s_tok[r] * p.d;
+    float* xr = p.x + (long long)r * p.d;
+#pragma unroll 8
+    for (int n = tid; n < p.d; n += 256) xr[n] = bf2f(e[n]);
   }
 }
 
@@ -197,32 +202,63 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
     pr.last_row[b] = p.mode == 2 ? p.n - 1 : (nrows > 0 ? row0 + nrows - 1 : 0);
   }
   __syncthreads();
-  // warp r: fcin[r] = [bf16(RMSNorm(h_r) * g_h) ; bf16(RMSNorm(e_r) * g_e)]
+  // fcin[r] = [bf16(RMSNorm(h_r) * g_h) ; bf16(RMSNorm(e_r) * g_e)]: all 256
+  // threads per row, the sums of every row reduced in one round
   const int d = p.d;
-  for (int r = warp; r < pr.n; r += 8) {
-    const int b = pr.slot[r];
+  const int nrow = pr.n;
+  __shared__ float red[8][kRmax][2];
+  __shared__ const float* s_h[kRmax];
+  __shared__ const float* s_ev[kRmax];
+  __shared__ const bf16* s_eb[kRmax];
+  if (tid < nrow) {
+    const int r = tid, b = pr.slot[r];
     const float* h;
     if (p.mode == 0) h = p.hpend + ((long long)b * (p.max_k + 1) + (r - pr.slot_row0[b])) * d;
     else if (p.mode == 1) h = p.xd + (long long)s_prev_last[b] * d;
     else h = p.xv + (long long)r * d;
     const int tok = pr.tok[r];
-    const float* ev = (p.mode == 2 && tok < 0) ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
-    const bf16* eb = p.embed + (long long)(tok < 0 ? 0 : tok) * d;
-    float sh = 0.f, se = 0.f;
-    for (int n = lane; n < d; n += 32) {
-      float hv = h[n];
-      float e = ev ? ev[n] : bf2f(eb[n]);
-      sh = __fmaf_rn(hv, hv, sh);
-      se = __fmaf_rn(e, e, se);
+    s_h[r] = h;
+    s_ev[r] = (p.mode == 2 && tok < 0) ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
+    s_eb[r] = p.embed + (long long)(tok < 0 ? 0 : tok) * d;
+  }
+  __syncthreads();
+  float sh[kRmax], se[kRmax];
+#pragma unroll
+  for (int r = 0; r < kRmax; ++r) {
+    sh[r] = 0.f;
+    se[r] = 0.f;
+    if (r < nrow) {
+      const float* h = s_h[r];
+      const float* ev = s_ev[r];
+      const bf16* eb = s_eb[r];
+#pragma unroll 4
+      for (int n = tid; n < d; n += 256) {
+        float hv = h[n];
+        float e = ev ? ev[n] : bf2f(eb[n]);
+        sh[r] = __fmaf_rn(hv, hv, sh[r]);
+        se[r] = __fmaf_rn(e, e, se[r]);
+      }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      sh = __fadd_rn(sh, __shfl_xor_sync(0xffffffffu, sh, o));
-      se = __fadd_rn(se, __shfl_xor_sync(0xffffffffu, se, o));
+      sh[r] = __fadd_rn(sh[r], __shfl_xor_sync(0xffffffffu, sh[r], o));
+      se[r] = __fadd_rn(se[r], __shfl_xor_sync(0xffffffffu, se[r], o));
     }
-    const float ch = rsqrtf(__fadd_rn(__fdiv_rn(sh, (float)d), p.eps));
-    const float ce = rsqrtf(__fadd_rn(__fdiv_rn(se, (float)d), p.eps));
-    for (int n = lane; n < d; n += 32) {
+    if (lane == 0) { red[warp][r][0] = sh[r]; red[warp][r][1] = se[r]; }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int r = 0; r < kRmax; ++r) {
+    if (r >= nrow) break;
+    float a = 0.f, c = 0.f;
+    for (int w = 0; w < 8; ++w) { a = __fadd_rn(a, red[w][r][0]); c = __fadd_rn(c, red[w][r][1]); }
+    const float ch = rsqrtf(__fadd_rn(__fdiv_rn(a, (float)d), p.eps));
+    const float ce = rsqrtf(__fadd_rn(__fdiv_rn(c, (float)d), p.eps));
+    const float* h = s_h[r];
+    const float* ev = s_ev[r];
+    const bf16* eb = s_eb[r];
+#pragma unroll 4
+    for (int n = tid; n < d; n += 256) {
       float e = ev ? ev[n] : bf2f(eb[n]);
       p.fcin[(long long)r * 2 * d + n] = f2bf(__fmul_rn(__fmul_rn(h[n], ch), bf2f(p.g_h[n])));
       p.fcin[(long long)r * 2 * d + d + n] = f2bf(__fmul_rn(__fmul_rn(e, ce), bf2f(p.g_e[n])));
