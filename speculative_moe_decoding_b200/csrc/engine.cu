@@ -170,9 +170,24 @@ int device_sms() {
   return n;
 }
 
+template <class K>
+cudaError_t max_carveout(K kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
+}
+
 cudaError_t prepare_kernels() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * kAttnChunk * 128 * 2);
+  // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
+  if (e == cudaSuccess) e = max_carveout(attention_kernel);
+  if (e == cudaSuccess) e = max_carveout(route_kernel);
+  if (e == cudaSuccess) e = max_carveout(combine_kernel);
+  if (e == cudaSuccess) e = max_carveout(verify_setup_kernel);
+  if (e == cudaSuccess) e = max_carveout(prefill_setup_kernel);
+  if (e == cudaSuccess) e = max_carveout(draft_setup_kernel);
+  if (e == cudaSuccess) e = max_carveout(accept_kernel);
+  if (e == cudaSuccess) e = max_carveout(force_kernel);
+  if (e == cudaSuccess) e = max_carveout(prefill_finish_kernel);
   if (e != cudaSuccess) return e;
   return gemv_prepare();
 }

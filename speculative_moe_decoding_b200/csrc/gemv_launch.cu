@@ -41,8 +41,14 @@ static size_t smem_max() {
 
 template <int RG, class Src, class Epi>
 static cudaError_t configure_one() {
-  return cudaFuncSetAttribute(gemv_kernel<RG, Src, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                              (int)smem_max<Src>());
+  cudaError_t e = cudaFuncSetAttribute(gemv_kernel<RG, Src, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem_max<Src>());
+  // every kernel of the library asks for the same (maximal) shared-memory
+  // carveout, so consecutive kernels never wait for an SM reconfiguration
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(gemv_kernel<RG, Src, Epi>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+  return e;
 }
 
 template <class Src, class Epi>

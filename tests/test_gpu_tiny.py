@@ -225,8 +225,8 @@ def test_capacity_overflow_sets_status_and_stops(tiny_bits, inputs):
     d = make_decoder(synth.TINY, tiny_bits, max_k=3, max_batch=1, kv_capacity=96)
     try:
         vis, prm = to_dev(inputs)
-        d.prefill(0, vis, prm)  # C = 80
-        for _ in range(8):
+        d.prefill(0, vis, prm)  # C = 80; every step commits >= 1 token
+        for _ in range(20):
             d.step(1, 3)
         torch.cuda.synchronize()
         from speculative_moe_decoding_b200 import ocrdec
