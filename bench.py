@@ -307,16 +307,22 @@ def main():
     tok = torch.empty(R, dtype=torch.int32, device="cuda")
     scratch = ocrdec.op_scratch()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)  # one-time kernel set-up
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
     times = []
     for i in range(23):
         flush.fill_(i & 0xff)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
+        graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
         if i >= 3:
             times.append(a.elapsed_time(b))
+    del graph
     lm_ms = float(np.mean(times))
     lm_bytes = dims.vocab * dims.d_model * 2 + R * dims.d_model * 4 + dims.d_model * 2
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
@@ -378,8 +384,9 @@ def main():
                          "bound": "hbm", "achieved": lm_gbs, "peak": peak_gbs, "unit": "GB/s",
                          "frac": lm_gbs / peak_gbs, "traffic": None, "peak_source": peak_src,
                          "launch_ms": lm_ms, "bytes_per_launch": lm_bytes,
-                         "timing": "same kernel instantiation as in the step, launched alone through ocrdec_op_lm_argmax, "
-                                   "L2 flushed before each launch, CUDA events on the launching stream"},
+                         "timing": "same kernel instantiation as in the step, launched alone through ocrdec_op_lm_argmax "
+                                   "replayed from a CUDA graph, L2 flushed before each launch, CUDA events on the "
+                                   "launching stream"},
             "gpu_launches": kernels * args.steps,
             "kernels_per_step": kernels,
             "clocks": clk,

@@ -9,6 +9,8 @@
 #include <cmath>
 #include <cstring>
 #include <map>
+#include <mutex>
+#include <set>
 #include <new>
 #include <tuple>
 #include <vector>
@@ -175,7 +177,7 @@ cudaError_t max_carveout(K kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
 }
 
-cudaError_t prepare_kernels() {
+cudaError_t prepare_kernels_now() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        2 * kAttnChunk * 128 * 2);
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
@@ -190,6 +192,20 @@ cudaError_t prepare_kernels() {
   if (e == cudaSuccess) e = max_carveout(prefill_finish_kernel);
   if (e != cudaSuccess) return e;
   return gemv_prepare();
+}
+
+// Kernel attributes are per device: set them once for each device a call runs on.
+cudaError_t prepare_kernels() {
+  static std::mutex mu;
+  static std::set<int> done;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (done.count(dev)) return cudaSuccess;
+  e = prepare_kernels_now();
+  if (e == cudaSuccess) done.insert(dev);
+  return e;
 }
 
 }  // namespace
@@ -571,7 +587,7 @@ int ocrdec_create(const ocrdec_config* cfg, ocrdec_ctx** out) {
   c->cfg = *cfg;
   c->num_sms = device_sms();
   if (c->num_sms <= 0) c->num_sms = 148;
-  c->L = make_layout(*cfg, c->num_sms);
+  c->L = make_layout(*cfg, 2 * c->num_sms);
   *out = c;
   return OCRDEC_OK;
 }
@@ -603,7 +619,7 @@ int ocrdec_weight_info(const ocrdec_config* cfg, int index, int64_t dims[3], int
 size_t ocrdec_workspace_bytes(const ocrdec_config* cfg) {
   if (!config_ok(cfg)) return 0;
   int sms = device_sms();
-  return make_layout(*cfg, sms > 0 ? sms : 148).total;
+  return make_layout(*cfg, 2 * (sms > 0 ? sms : 148)).total;
 }
 
 int ocrdec_bind_workspace(ocrdec_ctx* c, void* ws, size_t bytes, ocrdec_stream stream) {
@@ -928,7 +944,7 @@ const char* ocrdec_strerror(int s) {
 
 size_t ocrdec_op_scratch_bytes(void) {
   int sms = device_sms();
-  return 256 + sizeof(float2) * (size_t)(sms > 0 ? sms : 148) * kRmax;
+  return 256 + sizeof(float2) * (size_t)(2 * (sms > 0 ? sms : 148)) * kRmax;
 }
 
 int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps, int R, int N, int K, float* y,
@@ -982,7 +998,7 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   gl.epi = EpiKind::Argmax;
   gl.argmax = EpiArgmax::Params{tok, 1, logits, reinterpret_cast<float2*>(static_cast<char*>(scratch) + 256), nullptr};
   gl.rows_bound = R;
-  gl.grid = std::min(gl.s.tiles_per_mat, sms);
+  gl.grid = std::min(gl.s.tiles_per_mat, 2 * sms);
   LaunchCfg lc{s, false, sms};
   CK(launch_gemv(gl, lc));
   return OCRDEC_OK;

@@ -577,7 +577,7 @@ __device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, con
 }
 
 template <int RG, class Src, class Epi>
-__global__ void __launch_bounds__(kGemvThreads, 1)
+__global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem[];

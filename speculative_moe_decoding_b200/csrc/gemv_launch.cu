@@ -79,7 +79,8 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
   size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
   int grid = g.grid;
-  if (grid <= 0) grid = g.s.mats ? lc.num_sms : std::min(g.s.tiles_per_mat, lc.num_sms);
+  // two CTAs per SM (register-capped): the second hides the first's latencies
+  if (grid <= 0) grid = g.s.mats ? 2 * lc.num_sms : std::min(g.s.tiles_per_mat, 2 * lc.num_sms);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
 }
 
