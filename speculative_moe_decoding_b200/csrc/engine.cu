@@ -111,7 +111,7 @@ bool config_ok(const ocrdec_config* c) {
 size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t status, counters, slots, rows, hist, rope, kvk, kvv, dkvk, dkvv, x, xd, q, part, attn_out, rlogits,
+  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, part, attn_out, rlogits,
       topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, ybuf, hdense, fcin, am_part, gtok, props,
       committed, ncommitted, hpend, total;
   int hist_ld, max_chunks, am_blocks;
@@ -130,10 +130,12 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.status = take(64);
   L.counters = take(sizeof(int) * (2 * B * H + 16));
+  L.tile_ctr = take(sizeof(int) * kSplitMaxTiles);
   L.slots = take(sizeof(SlotState) * B);
   L.rows = take(sizeof(PassRows));
   L.hist = take(sizeof(int) * B * L.hist_ld);
   L.rope = take(sizeof(float2) * cap * (Dh / 2));
+  L.split_part = take(sizeof(float) * kSplitPartFloats);
   L.kvk = take(2 * B * c.n_layers * H * cap * Dh);
   L.kvv = take(2 * B * c.n_layers * H * cap * Dh);
   L.dkvk = take(2 * B * H * cap * Dh);
@@ -285,6 +287,9 @@ GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* n
   g.s.status = c->status();
   g.rows_bound = rmax;
   gemv_plan(g.s);
+  g.s.kparts = gemv_kparts(g.s, 2 * c->num_sms);
+  g.s.part = c->at<float>(c->L.split_part);
+  g.s.tile_counter = c->at<int>(c->L.tile_ctr);
   return g;
 }
 
@@ -385,6 +390,7 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
 
   auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half) {
     GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax);
+    g.s.kparts = 1;
     g.tm_sh = shared.map;
     g.s.n_experts = m.n_experts;
     g.s.top_k = m.top_k;
@@ -557,6 +563,18 @@ int enqueue_step(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* committe
     if (st) return st;
   }
   return enqueue_verify(c, lc, B, k, props, committed, ncommitted);
+}
+
+// Scratch of the single-kernel entry points: status/counter words, argmax
+// partials, split-K tile counters and partial sums.  Returns the byte size.
+size_t op_scratch_layout(int sms, size_t* am, size_t* ctr, size_t* part) {
+  size_t o = 256;
+  if (am) *am = o;
+  o = align_up(o + sizeof(float2) * 2 * sms * kRmax);
+  if (ctr) *ctr = o;
+  o = align_up(o + sizeof(int) * kSplitMaxTiles);
+  if (part) *part = o;
+  return align_up(o + sizeof(float) * kSplitPartFloats);
 }
 
 int check_ready(const ocrdec_ctx* c) {
@@ -944,7 +962,7 @@ const char* ocrdec_strerror(int s) {
 
 size_t ocrdec_op_scratch_bytes(void) {
   int sms = device_sms();
-  return 256 + sizeof(float2) * (size_t)(2 * (sms > 0 ? sms : 148)) * kRmax;
+  return op_scratch_layout(sms > 0 ? sms : 148, nullptr, nullptr, nullptr);
 }
 
 int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps, int R, int N, int K, float* y,
@@ -955,7 +973,10 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int* st = static_cast<int*>(scratch);
   CK(prepare_kernels());
-  CK(cudaMemsetAsync(st, 0, 16, s));
+  const int sms = device_sms();
+  size_t am_off, ctr_off, part_off;
+  op_scratch_layout(sms, &am_off, &ctr_off, &part_off);
+  CK(cudaMemsetAsync(st, 0, part_off, s));  // status, counters, tile counters
   GemvLaunch gl;
   CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
   gl.tm_sh = gl.tm_w;
@@ -964,12 +985,15 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
   gl.s.rows_static = R;
   gl.s.status = st;
   gemv_plan(gl.s);
+  gl.s.kparts = gemv_kparts(gl.s, 2 * sms);
+  gl.s.part = reinterpret_cast<float*>(static_cast<char*>(scratch) + part_off);
+  gl.s.tile_counter = reinterpret_cast<int*>(static_cast<char*>(scratch) + ctr_off);
   gl.src = SrcKind::Norm;
   gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};
   gl.epi = EpiKind::Store;
   gl.store = EpiStore<false>::Params{y, N, 1, nullptr};
   gl.rows_bound = R;
-  LaunchCfg lc{s, false, device_sms()};
+  LaunchCfg lc{s, false, sms};
   CK(launch_gemv(gl, lc));
   return OCRDEC_OK;
 }
@@ -982,8 +1006,10 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   int* st = static_cast<int*>(scratch);
   CK(prepare_kernels());
+  const int sms = device_sms();
+  size_t am_off;
+  op_scratch_layout(sms, &am_off, nullptr, nullptr);
   CK(cudaMemsetAsync(st, 0, 16, s));
-  int sms = device_sms();
   GemvLaunch gl;
   CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
   gl.tm_sh = gl.tm_w;
@@ -996,7 +1022,7 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   gl.src = SrcKind::Norm;
   gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};
   gl.epi = EpiKind::Argmax;
-  gl.argmax = EpiArgmax::Params{tok, 1, logits, reinterpret_cast<float2*>(static_cast<char*>(scratch) + 256), nullptr};
+  gl.argmax = EpiArgmax::Params{tok, 1, logits, reinterpret_cast<float2*>(static_cast<char*>(scratch) + am_off), nullptr};
   gl.rows_bound = R;
   gl.grid = std::min(gl.s.tiles_per_mat, 2 * sms);
   LaunchCfg lc{s, false, sms};

@@ -58,7 +58,13 @@ struct GemvShape {
   const int* nrows;     // device row count, or nullptr to use rows_static
   int rows_static;
   int* status;
-  int* counter;         // last-block counter (argmax epilogue)
+  int* counter;         // last-block counter (argmax / routing epilogues)
+  // split-K (dense mode): each tile's K-slices are cut into kparts contiguous
+  // parts handled by separate work items; the last part of a tile to finish
+  // adds the parts' partial sums in part order and runs the epilogue
+  int kparts;           // 1 = no split
+  float* part;          // [tiles][kparts][kNW * 32] partial sums
+  int* tile_counter;    // [tiles], zero between launches
 };
 
 struct RowSet {
@@ -204,7 +210,10 @@ struct SrcNorm {
   static constexpr int kBytesPerElem = 4;
   static constexpr int kMaxPer = 16;     // elements per thread per row: K <= 16 * 256
 
-  // Called by all consumer threads after the dependency wait.
+  // Called by all consumer threads after the dependency wait.  Thread t owns
+  // the float4 groups t, t + 256, ... of each row; a group of raw elements
+  // [4m, 4m + 4) is plane (m & 1) at offset (m >> 1) * 4 - contiguous in both
+  // layouts - so each group is read, scaled and written back as one float4.
   __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, uint64_t* xbar,
                                   int* status, int tid) {
     if (tid == 0) {
@@ -214,11 +223,16 @@ struct SrcNorm {
       for (int r = 0; r < R; ++r)
         bulk_g2s(xs + r * K, p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx, K * 4, xbar);
     }
-    float g[kMaxPer];
+    constexpr int kG = kMaxPer / 4;  // float4 groups per thread per row (K <= 4096)
+    const int ng = K / 4;
+    float4 g[kG];
 #pragma unroll
-    for (int j = 0; j < kMaxPer; ++j) {
-      int k = tid + j * kConsumers;
-      g[j] = k < K ? bf2f(p.gain[k]) : 0.f;
+    for (int j = 0; j < kG; ++j) {
+      int m = tid + j * kConsumers;
+      if (m < ng) {
+        uint2 u = *reinterpret_cast<const uint2*>(p.gain + 4 * m);
+        g[j] = make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+      }
     }
     named_sync(1, kConsumers);
     if (R > 0) mbar_wait(xbar, 0, status);
@@ -226,13 +240,18 @@ struct SrcNorm {
     const int half = K / 2;
     for (int r = 0; r < R; ++r) {
       float* row = xs + r * K;
-      float v[kMaxPer];
+      float4 v[kG];
       float a = 0.f;
 #pragma unroll
-      for (int j = 0; j < kMaxPer; ++j) {
-        int k = tid + j * kConsumers;
-        v[j] = k < K ? row[k] : 0.f;
-        a = __fmaf_rn(v[j], v[j], a);
+      for (int j = 0; j < kG; ++j) {
+        int m = tid + j * kConsumers;
+        if (m < ng) {
+          v[j] = reinterpret_cast<const float4*>(row)[m];
+          a = __fmaf_rn(v[j].x, v[j].x, a);
+          a = __fmaf_rn(v[j].y, v[j].y, a);
+          a = __fmaf_rn(v[j].z, v[j].z, a);
+          a = __fmaf_rn(v[j].w, v[j].w, a);
+        }
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
@@ -243,11 +262,15 @@ struct SrcNorm {
       for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
       const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
 #pragma unroll
-      for (int j = 0; j < kMaxPer; ++j) {
-        int k = tid + j * kConsumers;
-        if (k < K) {
-          int c = k >> 3, e = k & 7;
-          row[(e >> 2) * half + c * 4 + (e & 3)] = round_bf(__fmul_rn(__fmul_rn(v[j], sc), g[j]));
+      for (int j = 0; j < kG; ++j) {
+        int m = tid + j * kConsumers;
+        if (m < ng) {
+          float4 o;
+          o.x = round_bf(__fmul_rn(__fmul_rn(v[j].x, sc), g[j].x));
+          o.y = round_bf(__fmul_rn(__fmul_rn(v[j].y, sc), g[j].y));
+          o.z = round_bf(__fmul_rn(__fmul_rn(v[j].z, sc), g[j].z));
+          o.w = round_bf(__fmul_rn(__fmul_rn(v[j].w, sc), g[j].w));
+          *reinterpret_cast<float4*>(row + (m & 1) * half + (m >> 1) * 4) = o;
         }
       }
     }
@@ -495,6 +518,31 @@ __device__ __forceinline__ void epi_init<EpiArgmax>(int tid) { EpiArgmax::init(t
 // reduced values: lane L = 8 i + q gets local row i (0..3) for row-set entry q.
 // NR = live rows of the item (row-set entries 0..NR-1); the arithmetic of a
 // row does not depend on NR.
+// Work item -> (matrix, tile, slice range).  Dense mode may split a tile's
+// slices into s.kparts parts (items tile * kparts + part).
+struct ItemPos {
+  int m, t, kp, sl0, sl1;
+};
+
+__device__ __forceinline__ ItemPos item_pos(const GemvShape& s, int item) {
+  ItemPos ip;
+  if (s.kparts > 1) {
+    ip.m = 0;
+    ip.t = item / s.kparts;
+    ip.kp = item - ip.t * s.kparts;
+    const int spp = (s.ns + s.kparts - 1) / s.kparts;
+    ip.sl0 = ip.kp * spp;
+    ip.sl1 = min(s.ns, ip.sl0 + spp);
+  } else {
+    ip.m = item / s.tiles_per_mat;
+    ip.t = item - ip.m * s.tiles_per_mat;
+    ip.kp = 0;
+    ip.sl0 = 0;
+    ip.sl1 = s.ns;
+  }
+  return ip;
+}
+
 template <class Src>
 constexpr int stage_stride() {
   return kStageBytes + (Src::kStaged ? kRmax * kXSliceBytes : 0);
@@ -504,14 +552,14 @@ template <int NR, class Src>
 __device__ __forceinline__ float consume_item(const GemvShape& s, const typename Src::Params& sp, const float* xs,
                                               const unsigned char* stages, uint64_t* full_bar, uint64_t* empty_bar,
                                               uint32_t& it, const RowSet& rs, const int (&srow)[kWarpRows],
-                                              int nch, int lane) {
+                                              int nch, int lane, int sl0, int sl1) {
   f2_t acc[kWarpRows][NR > 0 ? NR : 1];
 #pragma unroll
   for (int i = 0; i < kWarpRows; ++i)
 #pragma unroll
     for (int q = 0; q < (NR > 0 ? NR : 1); ++q) acc[i][q] = 0ull;
 
-  for (int sl = 0; sl < s.ns; ++sl, ++it) {
+  for (int sl = sl0; sl < sl1; ++sl, ++it) {
     const int st = it % kStages;
     mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
     const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
@@ -562,8 +610,10 @@ template <int RG, class Src>
 __device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, const typename Src::Params& sp,
                                                   const float* xs, const unsigned char* stages, uint64_t* full_bar,
                                                   uint64_t* empty_bar, uint32_t& it, const RowSet& rs,
-                                                  const int (&srow)[kWarpRows], int nch, int lane) {
-#define OCRDEC_CONSUME(NRV) consume_item<NRV, Src>(s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane)
+                                                  const int (&srow)[kWarpRows], int nch, int lane, int sl0,
+                                                  int sl1) {
+#define OCRDEC_CONSUME(NRV) \
+  consume_item<NRV, Src>(s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane, sl0, sl1)
   if (n <= 0) return OCRDEC_CONSUME(0);
   if (n == 1 || RG == 1) return OCRDEC_CONSUME(1);
   if (n == 2 || RG == 2) return OCRDEC_CONSUME((RG >= 2 ? 2 : 1));
@@ -608,10 +658,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // Dense weights do not depend on earlier kernels: start streaming the first
     // stages before waiting for the previous kernel (programmatic dependent
     // launch lets this overlap its tail).
-    int total = s.mats ? 0 : s.tiles_per_mat;
+    int total = s.mats ? 0 : s.tiles_per_mat * s.kparts;
     int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
     int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
-    int item = start, sl = 0;
+    int item = start;
+    int sl = item < end ? item_pos(s, item).sl0 : 0;
     int R = 0;
     RowSet prs;  // rows of the current item (bf16 sources staged with the weights)
     int prs_m = -1;
@@ -658,11 +709,15 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     int npre = 0;
     if (!s.mats) {
       for (; item < end && it < (uint32_t)kStages;) {
+        const ItemPos ip = item_pos(s, item);
         pre_item[npre] = item;
         pre_sl[npre] = sl;
         ++npre;
-        issue_w(0, item, sl);
-        if (++sl == s.ns) { sl = 0; ++item; }
+        issue_w(0, ip.t, sl);
+        if (++sl == ip.sl1) {
+          ++item;
+          if (item < end) sl = item_pos(s, item).sl0;
+        }
       }
     }
     pdl_wait();
@@ -678,11 +733,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
         sl = 0;
       }
       for (; item < end;) {
-        int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
+        const ItemPos ip = item_pos(s, item);
         const uint32_t j = it;
-        issue_w(m, t, sl);
-        issue_x(j, m, sl);
-        if (++sl == s.ns) { sl = 0; ++item; }
+        issue_w(ip.m, ip.t, sl);
+        issue_x(j, ip.m, sl);
+        if (++sl == ip.sl1) {
+          ++item;
+          if (item < end) sl = item_pos(s, item).sl0;
+        }
       }
     } else if (Src::kStaged) {
       // aborting: complete the second arrival of every prefetched stage so the drain below can finish
@@ -704,10 +762,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int R = pass_rows(s);
   const int n_mats = s.mats ? *s.n_mats : 1;
-  const int total = n_mats * s.tiles_per_mat;
+  const int total = n_mats * s.tiles_per_mat * (s.mats ? 1 : s.kparts);
   const int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
   const int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
   const int nch = s.K / 8;  // 16-byte chunks per row
+  __shared__ int s_last_part;
 
   epi_init<Epi>(tid);
   if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid);
@@ -723,17 +782,33 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   for (int i = 0; i < kWarpRows; ++i) srow[i] = stage_row(paired, warp, i);
 
   for (int item = start; item < end; ++item) {
-    int m = item / s.tiles_per_mat, t = item - m * s.tiles_per_mat;
-    if (m != cur_m) {
-      mat_info(s, m, R, &ce, &sh, &rs);
-      cur_m = m;
+    const ItemPos ip = item_pos(s, item);
+    if (ip.m != cur_m) {
+      mat_info(s, ip.m, R, &ce, &sh, &rs);
+      cur_m = ip.m;
     }
     WarpOut o;
-    o.v = consume_dispatch<RG, Src>(rs.n, s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane);
+    o.v = consume_dispatch<RG, Src>(rs.n, s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane, ip.sl0,
+                                    ip.sl1);
+    if (s.kparts > 1) {
+      // post this part; the tile's last part adds all parts in part order
+      float* pt = s.part + ((long long)ip.t * s.kparts) * (kNW * 32);
+      pt[ip.kp * (kNW * 32) + warp * 32 + lane] = o.v;
+      __threadfence();
+      named_sync(1, kConsumers);
+      if (tid == 0) s_last_part = (atomicAdd(&s.tile_counter[ip.t], 1) == s.kparts - 1);
+      named_sync(1, kConsumers);
+      if (!s_last_part) continue;
+      __threadfence();
+      float v = 0.f;
+      for (int kp = 0; kp < s.kparts; ++kp) v = __fadd_rn(v, __ldcg(pt + kp * (kNW * 32) + warp * 32 + lane));
+      o.v = v;
+      if (tid == 0) s.tile_counter[ip.t] = 0;
+    }
     o.i = lane >> 3;
     o.q = lane & 7;
     int r0, r1;
-    tile_boxes(s, t, &r0, &r1);
+    tile_boxes(s, ip.t, &r0, &r1);
 #pragma unroll
     for (int i = 0; i < kWarpRows; ++i) o.n[i] = matrix_row(r0, r1, srow[i]);
     Epi::apply(ep, s, o, rs, lane);

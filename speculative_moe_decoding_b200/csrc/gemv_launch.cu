@@ -8,6 +8,17 @@ namespace ocrdec {
 void gemv_plan(GemvShape& s) {
   s.ns = (s.K + kSlice - 1) / kSlice;
   s.tiles_per_mat = s.pair_half ? (s.N / (2 * s.pair_half)) * (s.pair_half / kBoxRows) : (s.N + kTile - 1) / kTile;
+  s.kparts = 1;
+}
+
+int gemv_kparts(const GemvShape& s, int target_items) {
+  if (s.mats || s.tiles_per_mat >= target_items / 2 || s.ns < 2) return 1;
+  int want = (target_items + s.tiles_per_mat - 1) / s.tiles_per_mat;
+  want = std::min(want, s.ns);
+  const int spp = (s.ns + want - 1) / want;  // slices per part
+  int kp = (s.ns + spp - 1) / spp;           // parts, all non-empty
+  if ((long long)s.tiles_per_mat * kp * kNW * 32 > kSplitPartFloats || s.tiles_per_mat > kSplitMaxTiles) return 1;
+  return kp;
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -80,7 +91,7 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
   size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
   int grid = g.grid;
   // two CTAs per SM (register-capped): the second hides the first's latencies
-  if (grid <= 0) grid = g.s.mats ? 2 * lc.num_sms : std::min(g.s.tiles_per_mat, 2 * lc.num_sms);
+  if (grid <= 0) grid = g.s.mats ? 2 * lc.num_sms : std::min(g.s.tiles_per_mat * g.s.kparts, 2 * lc.num_sms);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
 }
 
@@ -97,6 +108,7 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
   if (g.s.K % 8 || (g.s.pair_half && (g.s.pair_half % kBoxRows || g.s.N % (2 * g.s.pair_half))))
     return cudaErrorInvalidValue;
   if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
+  if (g.s.kparts > 1 && (g.s.mats || !g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;
   if (g.src == SrcKind::Norm) {
     switch (g.epi) {
       case EpiKind::QKV: return launch_rg<SrcNorm, EpiQKV>(g, g.norm, g.qkv, lc);

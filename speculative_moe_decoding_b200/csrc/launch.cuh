@@ -52,8 +52,14 @@ struct GemvLaunch {
   int grid = 0;            // 0: derived from the work and the SM count
 };
 
-// Fills ns / tiles_per_mat from N, K and pair_half.
+// Fills ns / tiles_per_mat from N, K and pair_half (and kparts = 1).
 void gemv_plan(GemvShape& s);
+// Split-K for a dense launch with few tiles: the number of K-parts (every part
+// non-empty) that brings the item count near `target_items`.  Depends on the
+// shape alone, so every launch of a matrix reduces in the same order.
+int gemv_kparts(const GemvShape& s, int target_items);
+constexpr int kSplitPartFloats = 1 << 19;  // partial-sum buffer (floats) shared by split launches
+constexpr int kSplitMaxTiles = 4096;       // per-tile counters
 // 3-D tensor map (columns K, rows N, matrices E) of a bfloat16 weight array with
 // the GEMV's 256 x 16 box; base 16-byte aligned.
 cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap* out);
