@@ -178,6 +178,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", action="store_true", help="skip e2e and the CPU baseline (for ncu)")
+    ap.add_argument("--trace", type=int, default=8, help="steps replayed with the device timeline tracer after the "
+                    "timed region (0 = off)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     dims = synth.FULL
@@ -294,6 +296,20 @@ def main():
     kv_mid = C + (st0.n_generated + st1.n_generated) / 2
     union_b, dep_b = step_bytes(dims, k, U, kv_mid)
 
+    # ---- device timeline of a few more steps (outside the timed region) ----
+    timeline = None
+    if args.trace > 0:
+        from speculative_moe_decoding_b200 import timeline as tl
+        dec.set_trace(True)
+        for _ in range(args.trace):
+            dec.step(1, k)
+        torch.cuda.synchronize()
+        rec = dec.read_trace()
+        dec.set_trace(False)
+        timeline = tl.summary(rec, args.trace)
+        if rank == 0:
+            print(tl.format_summary(timeline), file=sys.stderr)
+
     # ---- dominant kernel: LM head + argmax over k+1 rows, timed alone ----
     import math
     peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
@@ -387,6 +403,7 @@ def main():
                          "timing": "same kernel instantiation as in the step, launched alone through ocrdec_op_lm_argmax "
                                    "replayed from a CUDA graph, L2 flushed before each launch, CUDA events on the "
                                    "launching stream"},
+            "timeline": timeline,
             "gpu_launches": kernels * args.steps,
             "kernels_per_step": kernels,
             "clocks": clk,

@@ -16,6 +16,7 @@
 namespace ocrdec {
 
 constexpr int kAttnChunk = 64;
+constexpr int kTagAttention = 40;
 constexpr int kAttnThreads = 128;
 constexpr int kAttnRows = 8;  // rows of one slot in a pass
 constexpr int kAttnMaxChunks = 128;  // chunks per sequence: kv_capacity <= 8192
@@ -50,6 +51,7 @@ attention_kernel(const AttnParams p) {
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   const int Dh = p.Dh;
 
   pdl_wait();
@@ -214,7 +216,10 @@ attention_kernel(const AttnParams p) {
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&p.counters[b * p.H + h], 1) == nchunks - 1);
   __syncthreads();
-  if (!s_last) return;
+  if (!s_last) {
+    if (tid == 0) trace_end(p.status, kTagAttention, t_start);
+    return;
+  }
   __threadfence();
   // stage every (row, chunk) max and sum, then the per-chunk rescale factors
   __shared__ float s_m2[kAttnRows][kAttnMaxChunks];
@@ -253,7 +258,10 @@ attention_kernel(const AttnParams p) {
       p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, s_L[r]));
     }
   }
-  if (tid == 0) p.counters[b * p.H + h] = 0;
+  if (tid == 0) {
+    p.counters[b * p.H + h] = 0;
+    trace_end(p.status, kTagAttention, t_start);
+  }
 }
 
 }  // namespace ocrdec

@@ -31,6 +31,41 @@ __device__ __forceinline__ bool status_bad(const int* status) {
   return status && *(volatile const int*)status != 0;
 }
 
+// ---- timeline tracer ---------------------------------------------------------
+// The status word heads a small region: status[1] != 0 enables tracing,
+// status[2] counts records, and TraceRec entries start 256 bytes in.  Each
+// traced CTA appends (start time, duration, kernel tag, SM) when it finishes.
+constexpr int kTraceCap = 1 << 16;
+struct TraceRec {
+  unsigned long long t0;
+  unsigned int dt;
+  unsigned short tag;
+  unsigned short sm;
+};
+
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned int sm_id() {
+  unsigned int r;
+  asm volatile("mov.u32 %0, %%smid;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void trace_end(int* status, int tag, unsigned long long t0) {
+  if (!status || !*(volatile int*)(status + 1)) return;
+  unsigned int i = atomicAdd(reinterpret_cast<unsigned int*>(status + 2), 1u);
+  if (i >= (unsigned)kTraceCap) return;
+  TraceRec* r = reinterpret_cast<TraceRec*>(reinterpret_cast<char*>(status) + 256) + i;
+  r->t0 = t0;
+  r->dt = (unsigned int)(gtimer() - t0);
+  r->tag = (unsigned short)tag;
+  r->sm = (unsigned short)sm_id();
+}
+
 // ---- mbarrier -------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");

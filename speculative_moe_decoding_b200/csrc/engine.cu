@@ -128,7 +128,7 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.am_blocks = am_blocks;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
-  L.status = take(64);
+  L.status = take(256 + sizeof(TraceRec) * kTraceCap);  // status word + timeline trace
   L.counters = take(sizeof(int) * (2 * B * H + 16));
   L.tile_ctr = take(sizeof(int) * kSplitMaxTiles);
   L.slots = take(sizeof(SlotState) * B);
@@ -266,6 +266,12 @@ namespace {
 // building blocks
 // ---------------------------------------------------------------------------
 
+// Timeline-trace tags of the launches (ocrdec_read_trace).
+enum Tag {
+  kTagQKV = 1, kTagOProj = 2, kTagRouter = 3, kTagExpGU = 4, kTagExpDown = 5, kTagDenseGU = 6, kTagDenseDown = 7,
+  kTagLMVerify = 8, kTagLMDraft = 9, kTagFC = 10
+};
+
 struct BlockIO {
   float* x;            // residual rows of the pass
   bf16* kc;            // K cache of this block, slot 0 (layer offset applied)
@@ -275,8 +281,10 @@ struct BlockIO {
 };
 
 // A GEMV launch over one dense matrix.
-GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* nrows, int rows_static, int rmax) {
+GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* nrows, int rows_static, int rmax,
+                        int tag) {
   GemvLaunch g;
+  g.s.tag = tag;
   g.tm_w = m.map;
   g.tm_sh = m.map;
   g.s.N = m.N;
@@ -297,7 +305,7 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
                    const Mat& wo, const BlockIO& io) {
   const ocrdec_config& m = c->cfg;
   PassRows* rows = c->rows();
-  GemvLaunch g = dense_launch(c, wqkv, m.head_dim / 2, &rows->n, 0, rmax);
+  GemvLaunch g = dense_launch(c, wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{io.x, m.d_model, nullptr, attn_norm, m.rms_eps};
   g.epi = EpiKind::QKV;
@@ -325,7 +333,7 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   CK(launch_ex(attention_kernel, dim3(c->L.max_chunks, m.n_heads, m.max_batch), dim3(kAttnThreads),
                (size_t)2 * kAttnChunk * m.head_dim * 2, lc, a));
 
-  GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax);
+  GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax, kTagOProj);
   o.src = SrcKind::Bf16;
   o.bf = SrcBf16::Params{c->at<bf16>(c->L.attn_out), m.d_model, 1, nullptr};
   o.epi = EpiKind::StoreAdd;
@@ -340,14 +348,14 @@ int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16
   PassRows* rows = c->rows();
   const int F = w_down.K;
   bf16* h = c->at<bf16>(c->L.hdense);
-  GemvLaunch g = dense_launch(c, w_gu, F, &rows->n, 0, rmax);
+  GemvLaunch g = dense_launch(c, w_gu, F, &rows->n, 0, rmax, kTagDenseGU);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{x, m.d_model, nullptr, norm, m.rms_eps};
   g.epi = EpiKind::SwiGLU;
   g.swiglu = EpiSwiGLU::Params{h, F, 1};
   CK(launch_gemv(g, lc));
 
-  GemvLaunch dn = dense_launch(c, w_down, 0, &rows->n, 0, rmax);
+  GemvLaunch dn = dense_launch(c, w_down, 0, &rows->n, 0, rmax, kTagDenseDown);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{h, F, 1, nullptr};
   dn.epi = EpiKind::StoreAdd;
@@ -379,7 +387,7 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   rp.status = c->status();
 
   // router logits + (last CTA) softmax / top-k / bucketing
-  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax);
+  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax, kTagRouter);
   r.s.counter = c->am_counter(2);
   r.src = SrcKind::Norm;
   r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
@@ -388,8 +396,8 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   r.route = rp;
   CK(launch_gemv(r, lc));
 
-  auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half) {
-    GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax);
+  auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half, int tag) {
+    GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax, tag);
     g.s.kparts = 1;
     g.tm_sh = shared.map;
     g.s.n_experts = m.n_experts;
@@ -402,14 +410,14 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
     return g;
   };
 
-  GemvLaunch gu = expert_launch(w.exp_gu, w.sh_gu, m.expert_ffn);
+  GemvLaunch gu = expert_launch(w.exp_gu, w.sh_gu, m.expert_ffn, kTagExpGU);
   gu.src = SrcKind::Norm;
   gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   gu.epi = EpiKind::SwiGLU;
   gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot};
   CK(launch_gemv(gu, lc));
 
-  GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0);
+  GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0, kTagExpDown);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot, nullptr};
   dn.epi = EpiKind::Store;
@@ -445,7 +453,7 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
 int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const bf16* norm, const int* row_src,
             const int* nrows, int rows_static, int* tok, int tok_stride, float* logits, int which_counter) {
   const ocrdec_config& m = c->cfg;
-  GemvLaunch g = dense_launch(c, c->lm_head, 0, nrows, rows_static, rmax);
+  GemvLaunch g = dense_launch(c, c->lm_head, 0, nrows, rows_static, rmax, kTagLMDraft);
   g.s.counter = c->am_counter(which_counter);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{x, m.d_model, row_src, norm, m.rms_eps};
@@ -463,7 +471,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   const DraftW& w = c->dw;
   PassRows* rows = c->rows();
   float* xd = c->at<float>(c->L.xd);
-  GemvLaunch fc = dense_launch(c, w.fc, 0, &rows->n, 0, rmax);
+  GemvLaunch fc = dense_launch(c, w.fc, 0, &rows->n, 0, rmax, kTagFC);
   fc.src = SrcKind::Bf16;
   fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), 2 * m.d_model, 1, nullptr};
   fc.epi = EpiKind::Store;
@@ -473,7 +481,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   const long long slot_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
   BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems, c->attn_counters(1)};
   if (kv_only) {
-    GemvLaunch g = dense_launch(c, w.wqkv, m.head_dim / 2, &rows->n, 0, rmax);
+    GemvLaunch g = dense_launch(c, w.wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
     g.src = SrcKind::Norm;
     g.norm = SrcNorm::Params{xd, m.d_model, nullptr, w.attn_norm, m.rms_eps};
     g.epi = EpiKind::QKV;
@@ -541,7 +549,7 @@ int enqueue_verify(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, const int* 
   if (st) return st;
   AcceptParams ap{c->slots(), c->at<int>(c->L.gtok), props, B, k, m.d_model, m.max_k, c->hist(), c->L.hist_ld,
                   c->at<float>(c->L.x), c->at<float>(c->L.hpend), committed, ncommitted, c->status()};
-  GemvLaunch g = dense_launch(c, c->lm_head, 0, &c->rows()->n, 0, R);
+  GemvLaunch g = dense_launch(c, c->lm_head, 0, &c->rows()->n, 0, R, kTagLMVerify);
   g.s.counter = c->am_counter(0);
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{c->at<float>(c->L.x), m.d_model, nullptr, c->final_norm, m.rms_eps};
@@ -927,6 +935,32 @@ int ocrdec_step_kernel_count(ocrdec_ctx* c, int batch, int k, int32_t* dev_commi
   auto it = c->graph_kernels.find(std::make_tuple(batch, k, (void*)dev_committed, (void*)dev_n_committed));
   if (it == c->graph_kernels.end()) return OCRDEC_ESTATE;
   *count = it->second;
+  return OCRDEC_OK;
+}
+
+int ocrdec_set_trace(ocrdec_ctx* c, int enable, ocrdec_stream stream) {
+  if (!c) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  int v[2] = {enable ? 1 : 0, 0};
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemcpyAsync(c->status() + 1, v, sizeof(v), cudaMemcpyHostToDevice, s));
+  CK(cudaStreamSynchronize(s));
+  return OCRDEC_OK;
+}
+
+int ocrdec_read_trace(ocrdec_ctx* c, void* host_records, int max_records, int32_t* n, ocrdec_stream stream) {
+  if (!c || !n || max_records < 0 || (max_records > 0 && !host_records)) return OCRDEC_EINVAL;
+  if (!c->ws) return OCRDEC_ESTATE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  unsigned int cnt = 0;
+  CK(cudaMemcpyAsync(&cnt, c->status() + 2, sizeof(cnt), cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  int take = (int)std::min<unsigned>(std::min<unsigned>(cnt, (unsigned)kTraceCap), (unsigned)max_records);
+  if (take > 0)
+    CK(cudaMemcpyAsync(host_records, reinterpret_cast<char*>(c->status()) + 256, sizeof(TraceRec) * take,
+                       cudaMemcpyDeviceToHost, s));
+  CK(cudaStreamSynchronize(s));
+  *n = (int32_t)std::min<unsigned>(cnt, (unsigned)kTraceCap);
   return OCRDEC_OK;
 }
 

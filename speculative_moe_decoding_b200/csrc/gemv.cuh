@@ -65,6 +65,7 @@ struct GemvShape {
   int kparts;           // 1 = no split
   float* part;          // [tiles][kparts][kNW * 32] partial sums
   int* tile_counter;    // [tiles], zero between launches
+  int tag;              // timeline-trace tag of this launch
 };
 
 struct RowSet {
@@ -637,6 +638,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
+  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   constexpr int kStride = stage_stride<Src>();
   unsigned char* stages = smem;
   float* xs = reinterpret_cast<float*>(smem + kStages * kStride);
@@ -815,6 +817,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   }
   named_sync(1, kConsumers);
   Epi::finish(ep, s, R, tid);
+  if (tid == 0) trace_end(s.status, s.tag, t_start);
 }
 
 }  // namespace ocrdec

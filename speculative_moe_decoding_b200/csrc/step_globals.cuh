@@ -21,16 +21,19 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   pdl_wait();
   if (status_bad(p.status)) return;
   pdl_trigger();
+  const unsigned long long t_start = threadIdx.x == 0 ? gtimer() : 0ull;
   const int R = min(*p.nrows, kRmax);
   const int nslot = p.top_k + p.S;
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= R * p.d) return;
-  int r = idx / p.d, n = idx - r * p.d;
-  const float* yr = p.y + (long long)r * nslot * p.d + n;
-  float t = 0.f;
-  for (int s = 0; s < p.top_k; ++s) t = __fmaf_rn(p.gates[r * p.top_k + s], yr[(long long)s * p.d], t);
-  for (int s = 0; s < p.S; ++s) t = __fadd_rn(t, yr[(long long)(p.top_k + s) * p.d]);
-  p.x[idx] = __fadd_rn(p.x[idx], t);
+  if (idx < R * p.d) {
+    int r = idx / p.d, n = idx - r * p.d;
+    const float* yr = p.y + (long long)r * nslot * p.d + n;
+    float t = 0.f;
+    for (int s = 0; s < p.top_k; ++s) t = __fmaf_rn(p.gates[r * p.top_k + s], yr[(long long)s * p.d], t);
+    for (int s = 0; s < p.S; ++s) t = __fadd_rn(t, yr[(long long)(p.top_k + s) * p.d]);
+    p.x[idx] = __fadd_rn(p.x[idx], t);
+  }
+  if (threadIdx.x == 0) trace_end(p.status, 41, t_start);
 }
 
 __global__ void rope_table_kernel(float2* tab, int cap, int Dh, double theta) {
@@ -83,6 +86,7 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   __syncthreads();
   if (s_bad) return;
   pdl_trigger();
+  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   // embedding gather: every row's loads are issued before any is consumed
 #pragma unroll
   for (int r = 0; r < kRmax; ++r) {
@@ -92,6 +96,7 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
 #pragma unroll 8
     for (int n = tid; n < p.d; n += 256) xr[n] = bf2f(e[n]);
   }
+  if (tid == 0) trace_end(p.status, 42, t_start);
 }
 
 __global__ void __launch_bounds__(256) prefill_setup_kernel(const PrefillSetupParams p) {
@@ -143,6 +148,7 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
   __shared__ PassRows pr;
   __shared__ int s_pend[kRmax], s_ppos[kRmax], s_kv[kRmax], s_prev_last[kRmax];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   pdl_wait();
   if (tid == 0) s_bad = status_bad(p.status);
   if (tid < kRmax) {
@@ -268,6 +274,7 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
   int* dst = reinterpret_cast<int*>(p.rows);
   const int* src = reinterpret_cast<const int*>(&pr);
   for (int i = tid; i < (int)(sizeof(PassRows) / sizeof(int)); i += 256) dst[i] = src[i];
+  if (tid == 0) trace_end(p.status, 43, t_start);
 }
 
 __global__ void __launch_bounds__(256) accept_kernel(const AcceptParams p) {

@@ -67,6 +67,10 @@ ocrdec_reset_counters = _sig("ocrdec_reset_counters", _i32, _vp, _vp)
 ocrdec_step_kernel_count = _sig("ocrdec_step_kernel_count", _i32, _vp, _i32, _i32, _vp, _vp, ctypes.POINTER(_i32))
 ocrdec_set_debug_taps = _sig("ocrdec_set_debug_taps", _i32, _vp, _vp, _vp)
 ocrdec_set_draft_taps = _sig("ocrdec_set_draft_taps", _i32, _vp, _vp)
+ocrdec_set_trace = _sig("ocrdec_set_trace", _i32, _vp, _i32, _vp)
+ocrdec_read_trace = _sig("ocrdec_read_trace", _i32, _vp, _vp, _i32, ctypes.POINTER(_i32), _vp)
+
+TRACE_DTYPE = np.dtype([("t0", "<u8"), ("dt", "<u4"), ("tag", "<u2"), ("sm", "<u2")])
 ocrdec_strerror = _sig("ocrdec_strerror", ctypes.c_char_p, _i32)
 ocrdec_op_scratch_bytes = _sig("ocrdec_op_scratch_bytes", _sz)
 ocrdec_op_norm_gemv = _sig("ocrdec_op_norm_gemv", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp)
@@ -241,6 +245,16 @@ class Decoder:
         check(ocrdec_step_kernel_count(self.ctx, batch, k, self.committed.data_ptr(), self.n_committed.data_ptr(),
                                        ctypes.byref(n)), "ocrdec_step_kernel_count")
         return n.value
+
+    def set_trace(self, enable: bool, stream=None):
+        check(ocrdec_set_trace(self.ctx, 1 if enable else 0, _stream(stream)), "ocrdec_set_trace")
+
+    def read_trace(self, max_records: int = 1 << 16, stream=None) -> np.ndarray:
+        buf = np.zeros(max_records, dtype=TRACE_DTYPE)
+        n = _i32()
+        check(ocrdec_read_trace(self.ctx, buf.ctypes.data, max_records, ctypes.byref(n), _stream(stream)),
+              "ocrdec_read_trace")
+        return buf[:min(n.value, max_records)]
 
     def set_draft_taps(self, logits=None):
         self._dtaps = logits
