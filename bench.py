@@ -178,7 +178,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", action="store_true", help="skip e2e and the CPU baseline (for ncu)")
-    ap.add_argument("--trace", type=int, default=8, help="steps replayed with the device timeline tracer after the "
+    ap.add_argument("--trace", type=int, default=4, help="steps replayed with the device timeline tracer after the "
                     "timed region (0 = off)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

@@ -203,7 +203,7 @@ OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* 
 /* Timeline tracer (diagnostics).  While enabled, every CTA of the library's
  * kernels appends one 16-byte record {uint64 start_ns (%globaltimer),
  * uint32 duration_ns, uint16 kernel tag, uint16 SM id} to a device buffer of
- * 65536 records; enabling clears it.  ocrdec_read_trace copies up to
+ * 1,048,576 records; enabling clears it.  ocrdec_read_trace copies up to
  * max_records records to host memory and sets *n to the number recorded
  * (synchronises `stream`).  Tags: 1 QKV, 2 O-proj, 3 router+routing, 4 expert
  * gate/up, 5 expert down, 6 dense gate/up, 7 dense down, 8 verify LM head +

@@ -35,7 +35,7 @@ __device__ __forceinline__ bool status_bad(const int* status) {
 // The status word heads a small region: status[1] != 0 enables tracing,
 // status[2] counts records, and TraceRec entries start 256 bytes in.  Each
 // traced CTA appends (start time, duration, kernel tag, SM) when it finishes.
-constexpr int kTraceCap = 1 << 16;
+constexpr int kTraceCap = 1 << 20;
 struct TraceRec {
   unsigned long long t0;
   unsigned int dt;

@@ -573,8 +573,9 @@ int enqueue_step(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* committe
   return enqueue_verify(c, lc, B, k, props, committed, ncommitted);
 }
 
-// Scratch of the single-kernel entry points: status/counter words, argmax
-// partials, split-K tile counters and partial sums.  Returns the byte size.
+// Scratch of the single-kernel entry points: status word, trace header (kept
+// zero: tracing off), last-block counter at word 8, argmax partials, split-K
+// tile counters and partial sums.  Returns the byte size.
 size_t op_scratch_layout(int sms, size_t* am, size_t* ctr, size_t* part) {
   size_t o = 256;
   if (am) *am = o;
@@ -1043,7 +1044,7 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   const int sms = device_sms();
   size_t am_off;
   op_scratch_layout(sms, &am_off, nullptr, nullptr);
-  CK(cudaMemsetAsync(st, 0, 16, s));
+  CK(cudaMemsetAsync(st, 0, 64, s));  // status, trace header (off), counter
   GemvLaunch gl;
   CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
   gl.tm_sh = gl.tm_w;
@@ -1051,7 +1052,7 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   gl.s.K = K;
   gl.s.rows_static = R;
   gl.s.status = st;
-  gl.s.counter = st + 1;
+  gl.s.counter = st + 8;  // clear of the trace header (st[1], st[2])
   gemv_plan(gl.s);
   gl.src = SrcKind::Norm;
   gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};

@@ -638,7 +638,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
+  unsigned long long t_start = 0ull;  // trace: when the dependency wait returned
   constexpr int kStride = stage_stride<Src>();
   unsigned char* stages = smem;
   float* xs = reinterpret_cast<float*>(smem + kStages * kStride);
@@ -757,7 +757,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   // ---------------- consumers ----------------
   pdl_wait();
-  if (tid == 0) s_abort = status_bad(s.status);
+  if (tid == 0) {
+    t_start = gtimer();
+    s_abort = status_bad(s.status);
+  }
   named_sync(1, kConsumers);
   if (s_abort) return;
   pdl_trigger();

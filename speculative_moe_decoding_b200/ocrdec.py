@@ -249,7 +249,7 @@ class Decoder:
     def set_trace(self, enable: bool, stream=None):
         check(ocrdec_set_trace(self.ctx, 1 if enable else 0, _stream(stream)), "ocrdec_set_trace")
 
-    def read_trace(self, max_records: int = 1 << 16, stream=None) -> np.ndarray:
+    def read_trace(self, max_records: int = 1 << 20, stream=None) -> np.ndarray:
         buf = np.zeros(max_records, dtype=TRACE_DTYPE)
         n = _i32()
         check(ocrdec_read_trace(self.ctx, buf.ctypes.data, max_records, ctypes.byref(n), _stream(stream)),
