@@ -51,10 +51,10 @@ attention_kernel(const AttnParams p) {
 
   const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   const int Dh = p.Dh;
 
   pdl_wait();
+  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;  // trace: after the dependency wait
   if (tid == 0) s_abort = status_bad(p.status);
   __syncthreads();
   if (s_abort) return;
