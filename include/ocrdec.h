@@ -201,14 +201,16 @@ OCRDEC_API int ocrdec_step_kernel_count(ocrdec_ctx* ctx, int batch, int k, int32
 OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* dev_logits);
 
 /* Timeline tracer (diagnostics).  While enabled, every CTA of the library's
- * kernels appends one 16-byte record {uint64 start_ns (%globaltimer),
- * uint32 duration_ns, uint16 kernel tag, uint16 SM id} to a device buffer of
- * 1,048,576 records; enabling clears it.  ocrdec_read_trace copies up to
+ * kernels appends one 24-byte record {uint64 t0_ns (%globaltimer, when the CTA
+ * passed its dependency wait), uint32 ns to the end of phase 1, phase 2 and
+ * phase 3 (= CTA end), uint16 kernel tag, uint16 SM id} to a device buffer of
+ * 524,288 records; enabling clears it.  GEMV phases: activation prologue, main
+ * loop, epilogue/finish; attention: K/V landed, partials written, end.  ocrdec_read_trace copies up to
  * max_records records to host memory and sets *n to the number recorded
  * (synchronises `stream`).  Tags: 1 QKV, 2 O-proj, 3 router+routing, 4 expert
  * gate/up, 5 expert down, 6 dense gate/up, 7 dense down, 8 verify LM head +
- * acceptance, 9 draft LM head, 10 draft input fc, 40 attention, 41 MoE combine,
- * 42 verify setup, 43 draft setup. */
+ * acceptance, 9 draft LM head, 10 draft input fc, 40 attention, 41 attention
+ * CTA that merged the chunks, 42 verify setup, 43 draft setup, 44 MoE combine. */
 OCRDEC_API int ocrdec_set_trace(ocrdec_ctx* ctx, int enable, ocrdec_stream stream);
 OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_records, int32_t* n,
                                  ocrdec_stream stream);

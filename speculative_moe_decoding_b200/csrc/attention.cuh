@@ -54,7 +54,8 @@ attention_kernel(const AttnParams p) {
   const int Dh = p.Dh;
 
   pdl_wait();
-  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;  // trace: after the dependency wait
+  TraceMarks tm;  // trace: wait returned, K/V landed, partials written
+  if (tid == 0) tm.t0 = gtimer();
   if (tid == 0) s_abort = status_bad(p.status);
   __syncthreads();
   if (s_abort) return;
@@ -87,6 +88,7 @@ attention_kernel(const AttnParams p) {
     if (i < nr && tid < Dh) qs[i][tid] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + tid];
   __syncthreads();
   mbar_wait(&bar, 0, p.status);  // gives up with OCRDEC_ETIMEOUT recorded; control flow stays uniform
+  if (tid == 0) tm.t1 = gtimer();
 
   // ---- scores: 4 lanes-groups of 8 per warp, one position per group ----
   // lane l8 of a group owns the 16-byte dim-chunks l8 and l8 + 8 of a key row
@@ -212,12 +214,13 @@ attention_kernel(const AttnParams p) {
   }
 
   // ---- last CTA of (slot, head) merges the chunks of every row ----
+  if (tid == 0) tm.t2 = gtimer();
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&p.counters[b * p.H + h], 1) == nchunks - 1);
   __syncthreads();
   if (!s_last) {
-    if (tid == 0) trace_end(p.status, kTagAttention, t_start);
+    if (tid == 0) trace_end(p.status, kTagAttention, tm);
     return;
   }
   __threadfence();
@@ -260,7 +263,7 @@ attention_kernel(const AttnParams p) {
   }
   if (tid == 0) {
     p.counters[b * p.H + h] = 0;
-    trace_end(p.status, kTagAttention, t_start);
+    trace_end(p.status, kTagAttention + 1, tm);  // the merging CTA
   }
 }
 

@@ -35,10 +35,10 @@ __device__ __forceinline__ bool status_bad(const int* status) {
 // The status word heads a small region: status[1] != 0 enables tracing,
 // status[2] counts records, and TraceRec entries start 256 bytes in.  Each
 // traced CTA appends (start time, duration, kernel tag, SM) when it finishes.
-constexpr int kTraceCap = 1 << 20;
+constexpr int kTraceCap = 1 << 19;
 struct TraceRec {
-  unsigned long long t0;
-  unsigned int dt;
+  unsigned long long t0;   // the CTA passed its dependency wait
+  unsigned int d1, d2, d3; // ns from t0 to the end of phases 1, 2, 3 (3 = CTA end)
   unsigned short tag;
   unsigned short sm;
 };
@@ -55,13 +55,21 @@ __device__ __forceinline__ unsigned int sm_id() {
   return r;
 }
 
-__device__ __forceinline__ void trace_end(int* status, int tag, unsigned long long t0) {
+// Phase marks of one CTA (kept by the thread that records).
+struct TraceMarks {
+  unsigned long long t0 = 0, t1 = 0, t2 = 0;
+};
+
+__device__ __forceinline__ void trace_end(int* status, int tag, const TraceMarks& m) {
   if (!status || !*(volatile int*)(status + 1)) return;
   unsigned int i = atomicAdd(reinterpret_cast<unsigned int*>(status + 2), 1u);
   if (i >= (unsigned)kTraceCap) return;
   TraceRec* r = reinterpret_cast<TraceRec*>(reinterpret_cast<char*>(status) + 256) + i;
-  r->t0 = t0;
-  r->dt = (unsigned int)(gtimer() - t0);
+  const unsigned long long t3 = gtimer();
+  r->t0 = m.t0;
+  r->d1 = (unsigned int)((m.t1 ? m.t1 : t3) - m.t0);
+  r->d2 = (unsigned int)((m.t2 ? m.t2 : t3) - m.t0);
+  r->d3 = (unsigned int)(t3 - m.t0);
   r->tag = (unsigned short)tag;
   r->sm = (unsigned short)sm_id();
 }

@@ -638,7 +638,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
-  unsigned long long t_start = 0ull;  // trace: when the dependency wait returned
+  TraceMarks tm;  // trace (consumer thread 0): wait returned, prologue done, main loop done
   constexpr int kStride = stage_stride<Src>();
   unsigned char* stages = smem;
   float* xs = reinterpret_cast<float*>(smem + kStages * kStride);
@@ -758,7 +758,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   // ---------------- consumers ----------------
   pdl_wait();
   if (tid == 0) {
-    t_start = gtimer();
+    tm.t0 = gtimer();
     s_abort = status_bad(s.status);
   }
   named_sync(1, kConsumers);
@@ -776,6 +776,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   epi_init<Epi>(tid);
   if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid);
   else named_sync(1, kConsumers);
+  if (tid == 0) tm.t1 = gtimer();
 
   uint32_t it = 0;
   int cur_m = -1;
@@ -819,8 +820,9 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     Epi::apply(ep, s, o, rs, lane);
   }
   named_sync(1, kConsumers);
+  if (tid == 0) tm.t2 = gtimer();
   Epi::finish(ep, s, R, tid);
-  if (tid == 0) trace_end(s.status, s.tag, t_start);
+  if (tid == 0) trace_end(s.status, s.tag, tm);
 }
 
 }  // namespace ocrdec

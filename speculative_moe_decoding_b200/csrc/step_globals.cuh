@@ -21,7 +21,8 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   pdl_wait();
   if (status_bad(p.status)) return;
   pdl_trigger();
-  const unsigned long long t_start = threadIdx.x == 0 ? gtimer() : 0ull;
+  TraceMarks tm;
+  if (threadIdx.x == 0) tm.t0 = gtimer();  // trace: after the dependency wait
   const int R = min(*p.nrows, kRmax);
   const int nslot = p.top_k + p.S;
   int idx = blockIdx.x * blockDim.x + threadIdx.x;
@@ -33,7 +34,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
     for (int s = 0; s < p.S; ++s) t = __fadd_rn(t, yr[(long long)(p.top_k + s) * p.d]);
     p.x[idx] = __fadd_rn(p.x[idx], t);
   }
-  if (threadIdx.x == 0) trace_end(p.status, 41, t_start);
+  if (threadIdx.x == 0) trace_end(p.status, 44, tm);
 }
 
 __global__ void rope_table_kernel(float2* tab, int cap, int Dh, double theta) {
@@ -52,6 +53,8 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   const int tid = threadIdx.x;
   const int K1 = p.k + 1, R = p.B * K1;
   pdl_wait();
+  TraceMarks tm;
+  if (tid == 0) tm.t0 = gtimer();
   if (tid == 0) s_bad = status_bad(p.status);
   __syncthreads();
   if (s_bad) return;
@@ -86,7 +89,6 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   __syncthreads();
   if (s_bad) return;
   pdl_trigger();
-  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   // embedding gather: every row's loads are issued before any is consumed
 #pragma unroll
   for (int r = 0; r < kRmax; ++r) {
@@ -96,7 +98,7 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
 #pragma unroll 8
     for (int n = tid; n < p.d; n += 256) xr[n] = bf2f(e[n]);
   }
-  if (tid == 0) trace_end(p.status, 42, t_start);
+  if (tid == 0) trace_end(p.status, 42, tm);
 }
 
 __global__ void __launch_bounds__(256) prefill_setup_kernel(const PrefillSetupParams p) {
@@ -148,8 +150,9 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
   __shared__ PassRows pr;
   __shared__ int s_pend[kRmax], s_ppos[kRmax], s_kv[kRmax], s_prev_last[kRmax];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const unsigned long long t_start = tid == 0 ? gtimer() : 0ull;
   pdl_wait();
+  TraceMarks tm;
+  if (tid == 0) tm.t0 = gtimer();
   if (tid == 0) s_bad = status_bad(p.status);
   if (tid < kRmax) {
     const bool live = tid < p.B;
@@ -274,7 +277,7 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
   int* dst = reinterpret_cast<int*>(p.rows);
   const int* src = reinterpret_cast<const int*>(&pr);
   for (int i = tid; i < (int)(sizeof(PassRows) / sizeof(int)); i += 256) dst[i] = src[i];
-  if (tid == 0) trace_end(p.status, 43, t_start);
+  if (tid == 0) trace_end(p.status, 43, tm);
 }
 
 __global__ void __launch_bounds__(256) accept_kernel(const AcceptParams p) {

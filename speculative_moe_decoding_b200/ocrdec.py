@@ -70,7 +70,8 @@ ocrdec_set_draft_taps = _sig("ocrdec_set_draft_taps", _i32, _vp, _vp)
 ocrdec_set_trace = _sig("ocrdec_set_trace", _i32, _vp, _i32, _vp)
 ocrdec_read_trace = _sig("ocrdec_read_trace", _i32, _vp, _vp, _i32, ctypes.POINTER(_i32), _vp)
 
-TRACE_DTYPE = np.dtype([("t0", "<u8"), ("dt", "<u4"), ("tag", "<u2"), ("sm", "<u2")])
+TRACE_DTYPE = np.dtype([("t0", "<u8"), ("d1", "<u4"), ("d2", "<u4"), ("dt", "<u4"), ("tag", "<u2"),
+                        ("sm", "<u2")])
 ocrdec_strerror = _sig("ocrdec_strerror", ctypes.c_char_p, _i32)
 ocrdec_op_scratch_bytes = _sig("ocrdec_op_scratch_bytes", _sz)
 ocrdec_op_norm_gemv = _sig("ocrdec_op_norm_gemv", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp)
@@ -249,7 +250,7 @@ class Decoder:
     def set_trace(self, enable: bool, stream=None):
         check(ocrdec_set_trace(self.ctx, 1 if enable else 0, _stream(stream)), "ocrdec_set_trace")
 
-    def read_trace(self, max_records: int = 1 << 20, stream=None) -> np.ndarray:
+    def read_trace(self, max_records: int = 1 << 19, stream=None) -> np.ndarray:
         buf = np.zeros(max_records, dtype=TRACE_DTYPE)
         n = _i32()
         check(ocrdec_read_trace(self.ctx, buf.ctypes.data, max_records, ctypes.byref(n), _stream(stream)),

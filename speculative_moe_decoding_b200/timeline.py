@@ -15,7 +15,7 @@ import numpy as np
 
 TAGS = {1: "qkv", 2: "o_proj", 3: "router+routing", 4: "expert_gate_up", 5: "expert_down", 6: "dense_gate_up",
         7: "dense_down", 8: "lm_head_verify+accept", 9: "lm_head_draft", 10: "draft_fc", 40: "attention",
-        41: "moe_combine", 42: "verify_setup", 43: "draft_setup"}
+        41: "attention_merge", 42: "verify_setup", 43: "draft_setup", 44: "moe_combine"}
 
 
 def launches(rec: np.ndarray) -> List[dict]:
@@ -64,6 +64,12 @@ def summary(rec: np.ndarray, steps: int) -> Dict:
         e = per_tag.setdefault(name, {"launches": 0, "span_us": 0.0})
         e["launches"] += 1
         e["span_us"] += (d["t1"] - d["t0"]) / 1e3
+    for tag in np.unique(rec["tag"]):
+        r = rec[rec["tag"] == tag]
+        e = per_tag[TAGS.get(int(tag), str(int(tag)))]
+        # mean per-CTA phase ends (us after the CTA's dependency wait)
+        e["cta_phase_us"] = [round(float(np.mean(r[f])) / 1e3, 2) for f in ("d1", "d2", "dt")]
+        e["ctas_per_launch"] = round(len(r) / e["launches"], 1)
     for e in per_tag.values():
         e["mean_us"] = e["span_us"] / e["launches"]
         e["per_step_us"] = e["span_us"] / steps
@@ -77,5 +83,6 @@ def format_summary(s: Dict) -> str:
              f"idle {s['idle_us_per_step']:.1f} us/step, {s['launches_per_step']:.1f} launches/step"]
     for name, e in s["per_tag"].items():
         lines.append(f"  {name:24s} {e['launches']:5d} launches  mean {e['mean_us']:8.2f} us  "
-                     f"{e['per_step_us']:8.1f} us/step")
+                     f"{e['per_step_us']:8.1f} us/step  ctas {e.get('ctas_per_launch')}  "
+                     f"cta phases {e.get('cta_phase_us')}")
     return "\n".join(lines)
