@@ -61,11 +61,14 @@ attention_kernel(const AttnParams p) {
   if (s_abort) return;
   pdl_trigger();
 
+  __shared__ int s_pos[kAttnRows];
   const int r0 = p.slot_row0[b];
   const int nr = min(p.slot_nrows[b], kAttnRows);
   if (nr <= 0) return;
+  if (tid < nr) s_pos[tid] = p.row_pos[r0 + tid];
+  __syncthreads();
   int maxpos = 0;
-  for (int i = 0; i < nr; ++i) maxpos = max(maxpos, p.row_pos[r0 + i]);
+  for (int i = 0; i < nr; ++i) maxpos = max(maxpos, s_pos[i]);
   const int nchunks = maxpos / kAttnChunk + 1;
   if (c >= nchunks) return;
   const int p0 = c * kAttnChunk;
@@ -135,7 +138,7 @@ attention_kernel(const AttnParams p) {
         a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
         int r = rb + i;
         if (l8 == 0 && r < nr && j < kAttnChunk) {
-          bool valid = j < npos && p0 + j <= p.row_pos[r0 + r];
+          bool valid = j < npos && p0 + j <= s_pos[r];
           sc[r][j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
         }
       }
@@ -145,7 +148,7 @@ attention_kernel(const AttnParams p) {
 
   // ---- per-row chunk max and exp-sum (warp w takes rows w, w+4) ----
   for (int r = warp; r < nr; r += 4) {
-    int lim = p.row_pos[r0 + r] - p0 + 1;  // visible positions of this row in the chunk
+    int lim = s_pos[r] - p0 + 1;  // visible positions of this row in the chunk
     lim = min(lim, npos);
     float m = -INFINITY;
     for (int j = lane; j < lim; j += 32) m = fmaxf(m, sc[r][j]);
@@ -176,7 +179,7 @@ attention_kernel(const AttnParams p) {
       for (int e = 0; e < 4; ++e) o[r][e] = 0.f;
     int lim[kAttnRows];
 #pragma unroll
-    for (int r = 0; r < kAttnRows; ++r) lim[r] = r < nr ? min(p.row_pos[r0 + r] - p0 + 1, npos) : 0;
+    for (int r = 0; r < kAttnRows; ++r) lim[r] = r < nr ? min(s_pos[r] - p0 + 1, npos) : 0;
     const int jb = warp * 16;
     for (int jj = 0; jj < 16; ++jj) {
       const int j = jb + jj;
@@ -205,7 +208,7 @@ attention_kernel(const AttnParams p) {
   }
   __syncthreads();
   for (int r = 0; r < nr; ++r) {
-    int lim = min(p.row_pos[r0 + r] - p0 + 1, npos);
+    int lim = min(s_pos[r] - p0 + 1, npos);
     if (lim <= 0) continue;
     float* dst = p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + c) * ld;
     for (int d = tid; d < Dh; d += kAttnThreads)
@@ -232,14 +235,14 @@ attention_kernel(const AttnParams p) {
   for (int idx = tid; idx < nr * maxc; idx += kAttnThreads) {
     int r = idx / maxc, cc = idx - r * maxc;
     const float* pr = p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + cc) * ld;
-    int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
+    int nc = s_pos[r] / kAttnChunk + 1;
     s_m2[r][cc] = cc < nc ? __ldcg(pr + Dh) : -INFINITY;     // m
     s_f[r][cc] = cc < nc ? __ldcg(pr + Dh + 1) : 0.f;       // l
   }
   __syncthreads();
   if (tid < nr) {
     const int r = tid;
-    int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
+    int nc = s_pos[r] / kAttnChunk + 1;
     float M = -INFINITY;
     for (int cc = 0; cc < nc; ++cc) M = fmaxf(M, s_m2[r][cc]);
     float L = 0.f;
@@ -251,15 +254,25 @@ attention_kernel(const AttnParams p) {
     s_L[r] = L;
   }
   __syncthreads();
-  for (int r = 0; r < nr; ++r) {
-    const int nc = p.row_pos[r0 + r] / kAttnChunk + 1;
-    const float* pr = p.part + ((long long)(r0 + r) * p.H + h) * p.max_chunks * ld;
-    for (int d = tid; d < Dh; d += kAttnThreads) {
-      float O = 0.f;
-#pragma unroll 4
-      for (int cc = 0; cc < nc; ++cc) O = __fmaf_rn(__ldcg(pr + cc * ld + d), s_m2[r][cc], O);
-      p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, s_L[r]));
+  // O[r][d] = sum_c o_c[r][d] f[r][c]: the loads of all rows of a chunk are independent
+  for (int d = tid; d < Dh; d += kAttnThreads) {
+    float O[kAttnRows];
+#pragma unroll
+    for (int r = 0; r < kAttnRows; ++r) O[r] = 0.f;
+    for (int cc = 0; cc < maxc; ++cc) {
+      float v[kAttnRows];
+#pragma unroll
+      for (int r = 0; r < kAttnRows; ++r)
+        v[r] = (r < nr && cc <= s_pos[r] / kAttnChunk)
+                   ? __ldcg(p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + cc) * ld + d)
+                   : 0.f;
+#pragma unroll
+      for (int r = 0; r < kAttnRows; ++r)
+        if (r < nr && cc <= s_pos[r] / kAttnChunk) O[r] = __fmaf_rn(v[r], s_m2[r][cc], O[r]);
     }
+#pragma unroll
+    for (int r = 0; r < kAttnRows; ++r)
+      if (r < nr) p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O[r], s_L[r]));
   }
   if (tid == 0) {
     p.counters[b * p.H + h] = 0;

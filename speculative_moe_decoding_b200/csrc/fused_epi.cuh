@@ -29,9 +29,14 @@ struct EpiRoute {
     if (tid == 0) last = (atomicAdd(s.counter, 1) == (int)gridDim.x - 1);
     named_sync(1, kConsumers);
     if (!last) return;
+    TraceMarks tm;
+    if (tid == 0) tm.t0 = gtimer();
     __threadfence();
     route_rows(p.route, R, tid, kConsumers, ConsumerSync{});
-    if (tid == 0) *s.counter = 0;
+    if (tid == 0) {
+      *s.counter = 0;
+      trace_end(s.status, 45, tm);  // the routing step alone
+    }
   }
 };
 

@@ -15,7 +15,8 @@ import numpy as np
 
 TAGS = {1: "qkv", 2: "o_proj", 3: "router+routing", 4: "expert_gate_up", 5: "expert_down", 6: "dense_gate_up",
         7: "dense_down", 8: "lm_head_verify+accept", 9: "lm_head_draft", 10: "draft_fc", 40: "attention",
-        41: "attention_merge", 42: "verify_setup", 43: "draft_setup", 44: "moe_combine"}
+        41: "attention_merge", 42: "verify_setup", 43: "draft_setup", 44: "moe_combine",
+        45: "routing (last router CTA)"}
 
 
 def launches(rec: np.ndarray) -> List[dict]:
@@ -69,6 +70,7 @@ def summary(rec: np.ndarray, steps: int) -> Dict:
         e = per_tag[TAGS.get(int(tag), str(int(tag)))]
         # mean per-CTA phase ends (us after the CTA's dependency wait)
         e["cta_phase_us"] = [round(float(np.mean(r[f])) / 1e3, 2) for f in ("d1", "d2", "dt")]
+        e["cta_phase_max_us"] = [round(float(np.max(r[f])) / 1e3, 2) for f in ("d1", "d2", "dt")]
         e["ctas_per_launch"] = round(len(r) / e["launches"], 1)
     for e in per_tag.values():
         e["mean_us"] = e["span_us"] / e["launches"]
@@ -84,5 +86,5 @@ def format_summary(s: Dict) -> str:
     for name, e in s["per_tag"].items():
         lines.append(f"  {name:24s} {e['launches']:5d} launches  mean {e['mean_us']:8.2f} us  "
                      f"{e['per_step_us']:8.1f} us/step  ctas {e.get('ctas_per_launch')}  "
-                     f"cta phases {e.get('cta_phase_us')}")
+                     f"cta phases {e.get('cta_phase_us')} max {e.get('cta_phase_max_us')}")
     return "\n".join(lines)
