@@ -167,6 +167,7 @@ attention_kernel(const AttnParams p) {
   }
   __syncthreads();
 
+  if (tid == 0) tm.t2 = gtimer();  // trace: scores and softmax done
   // ---- o = sum_j p_j v_j: warp w takes positions 16w..16w+15 in order, lane l
   // dims [l*dpl, (l+1)*dpl); the 4 warp partials are then added in warp order ----
   const int ld = Dh + 2;
@@ -217,7 +218,6 @@ attention_kernel(const AttnParams p) {
   }
 
   // ---- last CTA of (slot, head) merges the chunks of every row ----
-  if (tid == 0) tm.t2 = gtimer();
   __threadfence();
   __syncthreads();
   if (tid == 0) s_last = (atomicAdd(&p.counters[b * p.H + h], 1) == nchunks - 1);
@@ -254,21 +254,30 @@ attention_kernel(const AttnParams p) {
     s_L[r] = L;
   }
   __syncthreads();
-  // O[r][d] = sum_c o_c[r][d] f[r][c]: the loads of all rows of a chunk are independent
+  // O[r][d] = sum_c o_c[r][d] f[r][c]: the partials of 4 chunks x all rows are
+  // requested before any is used, so the loads overlap
+  int ncr[kAttnRows];
+#pragma unroll
+  for (int r = 0; r < kAttnRows; ++r) ncr[r] = r < nr ? s_pos[r] / kAttnChunk + 1 : 0;
+  constexpr int kCB = 4;
   for (int d = tid; d < Dh; d += kAttnThreads) {
     float O[kAttnRows];
 #pragma unroll
     for (int r = 0; r < kAttnRows; ++r) O[r] = 0.f;
-    for (int cc = 0; cc < maxc; ++cc) {
-      float v[kAttnRows];
+    for (int c0 = 0; c0 < maxc; c0 += kCB) {
+      float v[kCB][kAttnRows];
 #pragma unroll
-      for (int r = 0; r < kAttnRows; ++r)
-        v[r] = (r < nr && cc <= s_pos[r] / kAttnChunk)
-                   ? __ldcg(p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + cc) * ld + d)
-                   : 0.f;
+      for (int j = 0; j < kCB; ++j)
 #pragma unroll
-      for (int r = 0; r < kAttnRows; ++r)
-        if (r < nr && cc <= s_pos[r] / kAttnChunk) O[r] = __fmaf_rn(v[r], s_m2[r][cc], O[r]);
+        for (int r = 0; r < kAttnRows; ++r)
+          v[j][r] = (c0 + j < ncr[r])
+                        ? __ldcg(p.part + (((long long)(r0 + r) * p.H + h) * p.max_chunks + c0 + j) * ld + d)
+                        : 0.f;
+#pragma unroll
+      for (int j = 0; j < kCB; ++j)
+#pragma unroll
+        for (int r = 0; r < kAttnRows; ++r)
+          if (c0 + j < ncr[r]) O[r] = __fmaf_rn(v[j][r], s_m2[r][c0 + j], O[r]);
     }
 #pragma unroll
     for (int r = 0; r < kAttnRows; ++r)

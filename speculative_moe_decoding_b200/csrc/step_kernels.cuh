@@ -82,11 +82,11 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
     for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
 #pragma unroll
     for (int i = 0; i < 8; ++i) pe[i] = __fdiv_rn(pe[i], sum);
-    int sel[8];
-    float selg[8];
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      if (s >= K) break;
+    // top-k rounds: round s's winner (value, id) stays in lane s - no
+    // dynamically indexed arrays (they would live in local memory)
+    int my_id = 0x7fffffff;
+    float my_g = 0.f;
+    for (int s = 0; s < K; ++s) {
       float bv = -1.f;
       int bi = 0x7fffffff;
 #pragma unroll
@@ -100,28 +100,21 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
         int oi = __shfl_xor_sync(0xffffffffu, bi, o);
         if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
       }
-      sel[s] = bi;
-      selg[s] = bv;
+      if (lane == s) { my_id = bi; my_g = bv; }
 #pragma unroll
       for (int i = 0; i < 8; ++i)
         if (lane + 32 * i == bi) pe[i] = -2.f;  // taken
     }
-    // slot order = ascending expert id; lane s < K writes slot s
-    int my_id = 0;
-    float my_g = 0.f;
-#pragma unroll
-    for (int s = 0; s < 8; ++s) {
-      if (s >= K) break;
-      int rank = 0;
-#pragma unroll
-      for (int t = 0; t < 8; ++t)
-        if (t < K && sel[t] < sel[s]) ++rank;
-      if (lane == rank) { my_id = sel[s]; my_g = selg[s]; }
+    // slot order = ascending expert id: lane s < K moves to slot rank(s)
+    int rank = 0;
+    for (int t = 0; t < K; ++t) {
+      int other = __shfl_sync(0xffffffffu, my_id, t);
+      if (other < my_id) ++rank;
     }
     if (lane < K) {
-      p.ids[warp * K + lane] = my_id;
-      p.gates[warp * K + lane] = my_g;
-      s_ids[warp][lane] = my_id;
+      p.ids[warp * K + rank] = my_id;
+      p.gates[warp * K + rank] = my_g;
+      s_ids[warp][rank] = my_id;
     }
   }
   sync();
