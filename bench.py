@@ -180,6 +180,7 @@ def main():
     ap.add_argument("--profile-only", action="store_true", help="skip e2e and the CPU baseline (for ncu)")
     ap.add_argument("--trace", type=int, default=4, help="steps replayed with the device timeline tracer after the "
                     "timed region (0 = off)")
+    ap.add_argument("--trace-dump", default=None, help="also save the raw trace records (numpy .npy) to this path")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     dims = synth.FULL
@@ -306,6 +307,8 @@ def main():
         torch.cuda.synchronize()
         rec = dec.read_trace()
         dec.set_trace(False)
+        if args.trace_dump and rank == 0:
+            np.save(args.trace_dump, rec)
         timeline = tl.summary(rec, args.trace)
         if rank == 0:
             print(tl.format_summary(timeline), file=sys.stderr)

@@ -94,16 +94,16 @@ bool config_ok(const ocrdec_config* c) {
   for (int v : pos)
     if (v <= 0) return false;
   if (c->n_heads * c->head_dim != c->d_model) return false;
-  if (c->head_dim % 16 || c->head_dim > 128) return false;
+  if (c->head_dim != 64 && c->head_dim != 128) return false;
   if (c->d_model % 8 || c->expert_ffn % 8 || c->draft_ffn % 8 || c->vocab % 8) return false;
   if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
   if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % 8)) return false;
   if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
-  if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > 256 || c->top_k + c->n_shared > 127) return false;
+  if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > kMaxExperts || c->top_k + c->n_shared > 127) return false;
   if (c->max_k < 0 || c->max_k > 3) return false;
   if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
   if (c->d_model > kGemvMaxK) return false;  // shared-memory copy of the normalised rows
-  if ((c->kv_capacity + kAttnChunk - 1) / kAttnChunk > kAttnMaxChunks) return false;
+  if (c->kv_capacity > 8192) return false;  // documented limit of the C ABI
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
   return true;
 }
@@ -114,7 +114,7 @@ struct Layout {
   size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, part, attn_out, rlogits,
       topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, ybuf, hdense, fcin, am_part, gtok, props,
       committed, ncommitted, hpend, total;
-  int hist_ld, max_chunks, am_blocks;
+  int hist_ld, am_blocks;
 };
 
 Layout make_layout(const ocrdec_config& c, int am_blocks) {
@@ -124,12 +124,11 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   const size_t F = std::max(c.dense_ffn, c.draft_ffn);
   const size_t nslot = K + S;
   L.hist_ld = c.kv_capacity + 8;
-  L.max_chunks = (c.kv_capacity + kAttnChunk - 1) / kAttnChunk;
   L.am_blocks = am_blocks;
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.status = take(256 + sizeof(TraceRec) * kTraceCap);  // status word + timeline trace
-  L.counters = take(sizeof(int) * (2 * B * H + 16));
+  L.counters = take(sizeof(int) * (16 + 2 * kWorkSlots));
   L.tile_ctr = take(sizeof(int) * kSplitMaxTiles);
   L.slots = take(sizeof(SlotState) * B);
   L.rows = take(sizeof(PassRows));
@@ -143,7 +142,6 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.x = take(4 * R * d);
   L.xd = take(4 * R * d);
   L.q = take(4 * R * d);
-  L.part = take(4 * R * H * L.max_chunks * (Dh + 2));
   L.attn_out = take(2 * R * d);
   L.rlogits = take(4 * R * E);
   L.topk_ids = take(4 * R * K);
@@ -181,7 +179,7 @@ cudaError_t max_carveout(K kernel) {
 
 cudaError_t prepare_kernels_now() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       2 * kAttnChunk * 128 * 2);
+                                       (int)attn_smem_bytes(kAttnMaxDh));
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
   if (e == cudaSuccess) e = max_carveout(attention_kernel);
   if (e == cudaSuccess) e = max_carveout(route_kernel);
@@ -238,10 +236,22 @@ struct ocrdec_ctx {
   template <class T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
   int* status() const { return at<int>(L.status); }
-  int* attn_counters(int which) const { return at<int>(L.counters) + which * cfg.max_batch * cfg.n_heads; }
-  int* am_counter(int which) const { return at<int>(L.counters) + 2 * cfg.max_batch * cfg.n_heads + which; }
+  int* am_counter(int which) const { return at<int>(L.counters) + which; }
   // misc[0] = routed experts touched by verifier MoE layers, misc[1] = such layer passes
-  int* misc() const { return at<int>(L.counters) + 2 * cfg.max_batch * cfg.n_heads + 8; }
+  int* misc() const { return at<int>(L.counters) + 8; }
+  // GEMV work counters, handed out round-robin so that launches next to each
+  // other in a stream (which may overlap under programmatic dependent launch)
+  // never share one; each launch's last CTA zeroes its pair
+  mutable int work_next = 0;
+  int* next_work() const {
+    int* w = at<int>(L.counters) + 16 + 2 * work_next;
+    work_next = (work_next + 1) % kWorkSlots;
+    return w;
+  }
+  cudaError_t gemv(GemvLaunch& g, const LaunchCfg& lc) const {
+    g.s.work = next_work();
+    return launch_gemv(g, lc);
+  }
   SlotState* slots() const { return at<SlotState>(L.slots); }
   PassRows* rows() const { return at<PassRows>(L.rows); }
   int* hist() const { return at<int>(L.hist); }
@@ -277,7 +287,6 @@ struct BlockIO {
   bf16* kc;            // K cache of this block, slot 0 (layer offset applied)
   bf16* vc;
   long long slot_stride;
-  int* attn_counters;
 };
 
 // A GEMV launch over one dense matrix.
@@ -311,7 +320,7 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   g.epi = EpiKind::QKV;
   g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
                          m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
-  CK(launch_gemv(g, lc));
+  CK(c->gemv(g, lc));
 
   AttnParams a{};
   a.q = c->at<float>(c->L.q);
@@ -325,20 +334,17 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   a.slot_row0 = rows->slot_row0;
   a.slot_nrows = rows->slot_nrows;
   a.row_pos = rows->pos;
-  a.part = c->at<float>(c->L.part);
-  a.max_chunks = c->L.max_chunks;
-  a.counters = io.attn_counters;
   a.out = c->at<bf16>(c->L.attn_out);
   a.status = c->status();
-  CK(launch_ex(attention_kernel, dim3(c->L.max_chunks, m.n_heads, m.max_batch), dim3(kAttnThreads),
-               (size_t)2 * kAttnChunk * m.head_dim * 2, lc, a));
+  CK(launch_cluster_ex(attention_kernel, dim3(kAttnSplit, m.n_heads, m.max_batch), dim3(kAttnThreads),
+               attn_smem_bytes(m.head_dim), lc, kAttnSplit, a));
 
   GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax, kTagOProj);
   o.src = SrcKind::Bf16;
   o.bf = SrcBf16::Params{c->at<bf16>(c->L.attn_out), m.d_model, 1, nullptr};
   o.epi = EpiKind::StoreAdd;
   o.store = EpiStore<false>::Params{io.x, m.d_model, 1, nullptr};
-  CK(launch_gemv(o, lc));
+  CK(c->gemv(o, lc));
   return OCRDEC_OK;
 }
 
@@ -353,14 +359,14 @@ int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16
   g.norm = SrcNorm::Params{x, m.d_model, nullptr, norm, m.rms_eps};
   g.epi = EpiKind::SwiGLU;
   g.swiglu = EpiSwiGLU::Params{h, F, 1};
-  CK(launch_gemv(g, lc));
+  CK(c->gemv(g, lc));
 
   GemvLaunch dn = dense_launch(c, w_down, 0, &rows->n, 0, rmax, kTagDenseDown);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{h, F, 1, nullptr};
   dn.epi = EpiKind::StoreAdd;
   dn.store = EpiStore<false>::Params{x, m.d_model, 1, nullptr};
-  CK(launch_gemv(dn, lc));
+  CK(c->gemv(dn, lc));
   return OCRDEC_OK;
 }
 
@@ -394,7 +400,7 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   r.epi = EpiKind::Route;
   r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
   r.route = rp;
-  CK(launch_gemv(r, lc));
+  CK(c->gemv(r, lc));
 
   auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half, int tag) {
     GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax, tag);
@@ -415,14 +421,14 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   gu.epi = EpiKind::SwiGLU;
   gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot};
-  CK(launch_gemv(gu, lc));
+  CK(c->gemv(gu, lc));
 
   GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0, kTagExpDown);
   dn.src = SrcKind::Bf16;
   dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot, nullptr};
   dn.epi = EpiKind::Store;
   dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
-  CK(launch_gemv(dn, lc));
+  CK(c->gemv(dn, lc));
 
   CombineParams cp{x, c->at<float>(c->L.ybuf), rp.gates, &rows->n, m.d_model, m.top_k, m.n_shared, c->status()};
   CK(launch_ex(combine_kernel, dim3((kRmax * m.d_model + 255) / 256), dim3(256), 0, lc, cp));
@@ -436,7 +442,7 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerW& w = c->layers[l];
     BlockIO io{c->at<float>(c->L.x), c->at<bf16>(c->L.kvk) + l * layer_elems, c->at<bf16>(c->L.kvv) + l * layer_elems,
-               layer_elems * m.n_layers, c->attn_counters(0)};
+               layer_elems * m.n_layers};
     int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
     if (st) return st;
     st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down) : moe_ffn(c, lc, rmax, w, count);
@@ -460,7 +466,7 @@ int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const 
   g.epi = EpiKind::Argmax;
   g.argmax = EpiArgmax::Params{tok, tok_stride, logits, c->at<float2>(c->L.am_part), nullptr};
   g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
-  CK(launch_gemv(g, lc));
+  CK(c->gemv(g, lc));
   return OCRDEC_OK;
 }
 
@@ -476,10 +482,10 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), 2 * m.d_model, 1, nullptr};
   fc.epi = EpiKind::Store;
   fc.store = EpiStore<false>::Params{xd, m.d_model, 1, nullptr};
-  CK(launch_gemv(fc, lc));
+  CK(c->gemv(fc, lc));
 
   const long long slot_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
-  BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems, c->attn_counters(1)};
+  BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems};
   if (kv_only) {
     GemvLaunch g = dense_launch(c, w.wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
     g.src = SrcKind::Norm;
@@ -487,7 +493,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
     g.epi = EpiKind::QKV;
     g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
                            m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
-    CK(launch_gemv(g, lc));
+    CK(c->gemv(g, lc));
     return OCRDEC_OK;
   }
   int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
@@ -557,7 +563,7 @@ int enqueue_verify(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, const int* 
   g.argmax = EpiArgmax::Params{c->at<int>(c->L.gtok), 1, c->dbg_logits, c->at<float2>(c->L.am_part), nullptr};
   g.accept = ap;
   g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
-  CK(launch_gemv(g, lc));
+  CK(c->gemv(g, lc));
   return OCRDEC_OK;
 }
 
@@ -1023,6 +1029,7 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
   gl.s.kparts = gemv_kparts(gl.s, 2 * sms);
   gl.s.part = reinterpret_cast<float*>(static_cast<char*>(scratch) + part_off);
   gl.s.tile_counter = reinterpret_cast<int*>(static_cast<char*>(scratch) + ctr_off);
+  gl.s.work = st + 12;
   gl.src = SrcKind::Norm;
   gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};
   gl.epi = EpiKind::Store;
@@ -1053,6 +1060,7 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   gl.s.rows_static = R;
   gl.s.status = st;
   gl.s.counter = st + 8;  // clear of the trace header (st[1], st[2])
+  gl.s.work = st + 12;
   gemv_plan(gl.s);
   gl.src = SrcKind::Norm;
   gl.norm = SrcNorm::Params{x, K, nullptr, static_cast<const bf16*>(g), eps};

@@ -66,13 +66,32 @@ struct GemvShape {
   float* part;          // [tiles][kparts][kNW * 32] partial sums
   int* tile_counter;    // [tiles], zero between launches
   int tag;              // timeline-trace tag of this launch
+  // dynamic work distribution: work[0] = next item to claim, work[1] = CTAs
+  // done claiming; the last CTA resets both (zero between launches)
+  int* work;
 };
 
+// Rows of one item: entry q = pass row | (output slot << 8).
 struct RowSet {
   int n;
-  int r[kRmax];
-  int slot[kRmax];
+  int e[kRmax];
+  __device__ __forceinline__ int r(int q) const { return e[q] & 0xff; }
+  __device__ __forceinline__ int slot(int q) const { return e[q] >> 8; }
+  __device__ __forceinline__ int r_sel(int q) const;     // runtime q
+  __device__ __forceinline__ int slot_sel(int q) const;
 };
+
+// a[i] for a runtime i without indexing the array (which would move it to
+// local memory): a chain of selects over the unrolled entries.
+template <int N>
+__device__ __forceinline__ int sel(const int (&a)[N], int i) {
+  int v = a[0];
+#pragma unroll
+  for (int k = 1; k < N; ++k) v = (i == k) ? a[k] : v;
+  return v;
+}
+__device__ __forceinline__ int RowSet::r_sel(int q) const { return sel(e, q) & 0xff; }
+__device__ __forceinline__ int RowSet::slot_sel(int q) const { return sel(e, q) >> 8; }
 
 __device__ __forceinline__ int pass_rows(const GemvShape& s) {
   int R = s.nrows ? *(volatile const int*)s.nrows : s.rows_static;
@@ -111,7 +130,7 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
     if (rs) {
       rs->n = R;
 #pragma unroll
-      for (int i = 0; i < kRmax; ++i) { rs->r[i] = i; rs->slot[i] = 0; }
+      for (int i = 0; i < kRmax; ++i) rs->e[i] = i;
     }
     return;
   }
@@ -124,11 +143,7 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
       n = n > kRmax ? kRmax : n;
       rs->n = n;
 #pragma unroll
-      for (int i = 0; i < kRmax; ++i) {
-        int v = i < n ? s.rowlist[off + i] : 0;
-        rs->r[i] = v & 0xff;
-        rs->slot[i] = v >> 8;
-      }
+      for (int i = 0; i < kRmax; ++i) rs->e[i] = i < n ? s.rowlist[off + i] : 0;
     }
   } else {
     int sh = e - s.n_experts;
@@ -137,7 +152,7 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
     if (rs) {
       rs->n = R;
 #pragma unroll
-      for (int i = 0; i < kRmax; ++i) { rs->r[i] = i; rs->slot[i] = s.top_k + sh; }
+      for (int i = 0; i < kRmax; ++i) rs->e[i] = i | ((s.top_k + sh) << 8);
     }
   }
 }
@@ -211,71 +226,101 @@ struct SrcNorm {
   static constexpr int kBytesPerElem = 4;
   static constexpr int kMaxPer = 16;     // elements per thread per row: K <= 16 * 256
 
-  // Called by all consumer threads after the dependency wait.  Thread t owns
-  // the float4 groups t, t + 256, ... of each row; a group of raw elements
-  // [4m, 4m + 4) is plane (m & 1) at offset (m >> 1) * 4 - contiguous in both
-  // layouts - so each group is read, scaled and written back as one float4.
-  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, uint64_t* xbar,
-                                  int* status, int tid) {
-    if (tid == 0) {
-      mbar_init(xbar, 1);
-      fence_mbar_init();
-      mbar_arrive_expect_tx(xbar, (uint32_t)(R * K * 4));
-      for (int r = 0; r < R; ++r)
-        bulk_g2s(xs + r * K, p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx, K * 4, xbar);
-    }
-    constexpr int kG = kMaxPer / 4;  // float4 groups per thread per row (K <= 4096)
-    const int ng = K / 4;
+  static constexpr int kG = kMaxPer / 4;  // float4 groups per thread per row (K <= 4096)
+  // Gains are weights: loaded before the dependency wait.
+  struct Pre {
     float4 g[kG];
+  };
+  __device__ static void pre_wait(const Params& p, int K, int tid, Pre& pre) {
+    const int ng = K / 4;
 #pragma unroll
     for (int j = 0; j < kG; ++j) {
       int m = tid + j * kConsumers;
       if (m < ng) {
         uint2 u = *reinterpret_cast<const uint2*>(p.gain + 4 * m);
-        g[j] = make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
+        pre.g[j] = make_float4(bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y));
       }
     }
-    named_sync(1, kConsumers);
+  }
+  // One thread, after the dependency wait: copy the R raw rows into xs.
+  __device__ static void issue(const Params& p, int K, int R, float* xs, uint64_t* xbar) {
+    if (R <= 0) return;
+    mbar_arrive_expect_tx(xbar, (uint32_t)(R * K * 4));
+    for (int r = 0; r < R; ++r)
+      bulk_g2s(xs + r * K, p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx, K * 4, xbar);
+  }
+
+  // All consumer threads.  Thread t owns the float4 groups t, t + 256, ... of
+  // each row; a group of raw elements [4m, 4m + 4) is plane (m & 1) at offset
+  // (m >> 1) * 4 - contiguous in both layouts - so each group is read, scaled
+  // and written back as one float4.  The sums of squares of all rows are formed
+  // together (one barrier); a row is rewritten in place only once every thread
+  // has read it, which the barrier after each row's reads guarantees.
+  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, uint64_t* xbar,
+                                  int* status, int tid, const Pre& pre) {
+    const int ng = K / 4;
     if (R > 0) mbar_wait(xbar, 0, status);
     const int lane = tid & 31, warp = tid >> 5;
     const int half = K / 2;
-    for (int r = 0; r < R; ++r) {
-      float* row = xs + r * K;
-      float4 v[kG];
-      float a = 0.f;
+    float a[kRmax];
+    float4 v[kG];
 #pragma unroll
-      for (int j = 0; j < kG; ++j) {
-        int m = tid + j * kConsumers;
-        if (m < ng) {
-          v[j] = reinterpret_cast<const float4*>(row)[m];
-          a = __fmaf_rn(v[j].x, v[j].x, a);
-          a = __fmaf_rn(v[j].y, v[j].y, a);
-          a = __fmaf_rn(v[j].z, v[j].z, a);
-          a = __fmaf_rn(v[j].w, v[j].w, a);
+    for (int r = 0; r < kRmax; ++r) {
+      a[r] = 0.f;
+      if (r < R) {
+        const float4* row = reinterpret_cast<const float4*>(xs + r * K);
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          int m = tid + j * kConsumers;
+          if (m < ng) {
+            float4 t = row[m];
+            if (r == 0) v[j] = t;
+            a[r] = __fmaf_rn(t.x, t.x, a[r]);
+            a[r] = __fmaf_rn(t.y, t.y, a[r]);
+            a[r] = __fmaf_rn(t.z, t.z, a[r]);
+            a[r] = __fmaf_rn(t.w, t.w, a[r]);
+          }
         }
       }
+    }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
-      if (lane == 0) red[r * kNW + warp] = a;
-      named_sync(1, kConsumers);  // every thread has read row r and posted its sum
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int r = 0; r < kRmax; ++r) a[r] = __fadd_rn(a[r], __shfl_xor_sync(0xffffffffu, a[r], o));
+    if (lane == 0)
+#pragma unroll
+      for (int r = 0; r < kRmax; ++r)
+        if (r < R) red[r * kNW + warp] = a[r];
+    named_sync(1, kConsumers);  // sums posted; row 0 read by every thread
+    for (int r = 0; r < R; ++r) {
       float ss = 0.f;
 #pragma unroll
       for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
       const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
+      float* row = xs + r * K;
 #pragma unroll
       for (int j = 0; j < kG; ++j) {
         int m = tid + j * kConsumers;
         if (m < ng) {
           float4 o;
-          o.x = round_bf(__fmul_rn(__fmul_rn(v[j].x, sc), g[j].x));
-          o.y = round_bf(__fmul_rn(__fmul_rn(v[j].y, sc), g[j].y));
-          o.z = round_bf(__fmul_rn(__fmul_rn(v[j].z, sc), g[j].z));
-          o.w = round_bf(__fmul_rn(__fmul_rn(v[j].w, sc), g[j].w));
+          o.x = round_bf(__fmul_rn(__fmul_rn(v[j].x, sc), pre.g[j].x));
+          o.y = round_bf(__fmul_rn(__fmul_rn(v[j].y, sc), pre.g[j].y));
+          o.z = round_bf(__fmul_rn(__fmul_rn(v[j].z, sc), pre.g[j].z));
+          o.w = round_bf(__fmul_rn(__fmul_rn(v[j].w, sc), pre.g[j].w));
           *reinterpret_cast<float4*>(row + (m & 1) * half + (m >> 1) * 4) = o;
         }
       }
+      if (r + 1 < R) {
+        const float4* nrow = reinterpret_cast<const float4*>(xs + (r + 1) * K);
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          int m = tid + j * kConsumers;
+          if (m < ng) v[j] = nrow[m];
+        }
+      }
+      named_sync(1, kConsumers);  // row r written; row r + 1 read by every thread
     }
-    named_sync(1, kConsumers);
+    if (R == 0) named_sync(1, kConsumers);
   }
 
   __device__ static Pairs8 chunk(const Params& p, const float* xs, const unsigned char* xstage, int K, int q, int r,
@@ -306,7 +351,10 @@ struct SrcBf16 {
   static constexpr bool kSmem = false;
   static constexpr bool kStaged = true;
   static constexpr int kBytesPerElem = 0;
-  __device__ static void prologue(const Params&, int, int, float*, float*, uint64_t*, int*, int) {}
+  struct Pre {};
+  __device__ static void pre_wait(const Params&, int, int, Pre&) {}
+  __device__ static void issue(const Params&, int, int, float*, uint64_t*) {}
+  __device__ static void prologue(const Params&, int, int, float*, float*, uint64_t*, int*, int, const Pre&) {}
   __device__ static const bf16* row_ptr(const Params& p, int r, int slot) {
     return p.x + (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
   }
@@ -324,7 +372,7 @@ struct SrcBf16 {
 struct WarpOut {
   float v;           // value for (local row i, row-set entry q) of this lane
   int i, q;          // i = lane >> 3, q = lane & 7
-  int n[kWarpRows];  // matrix row of each local row (may be >= N in a ragged tile)
+  int n;             // matrix row of local row i (may be >= N in a ragged tile)
 };
 
 // out[(row(r) * nslot + slot) * ld + n] = v   (or += v when kAdd)
@@ -339,10 +387,10 @@ struct EpiStore {
   __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
                                int lane) {
     if (o.q >= rs.n) return;
-    int nrow = o.n[o.i];
+    int nrow = o.n;
     if (nrow >= s.N) return;
-    int r = rs.r[o.q];
-    long long row = (long long)(p.row_dst ? p.row_dst[r] : r) * p.nslot + rs.slot[o.q];
+    int r = rs.r_sel(o.q);
+    long long row = (long long)(p.row_dst ? p.row_dst[r] : r) * p.nslot + rs.slot_sel(o.q);
     float* dst = p.y + row * p.ld + nrow;
     if (kAdd) *dst = __fadd_rn(*dst, o.v);
     else *dst = o.v;
@@ -364,8 +412,8 @@ struct EpiSwiGLU {
     if (o.i >= 2 || o.q >= rs.n) return;
     float gt = o.v;
     float act = __fdiv_rn(gt, __fadd_rn(1.f, expf(-gt)));
-    long long row = (long long)rs.r[o.q] * p.nslot + rs.slot[o.q];
-    p.h[row * p.ld + o.n[o.i]] = f2bf(__fmul_rn(act, up));
+    long long row = (long long)rs.r_sel(o.q) * p.nslot + rs.slot_sel(o.q);
+    p.h[row * p.ld + o.n] = f2bf(__fmul_rn(act, up));
   }
   __device__ static void finish(const Params&, const GemvShape&, int, int) {}
 };
@@ -389,11 +437,11 @@ struct EpiQKV {
     float b = __shfl_down_sync(0xffffffffu, o.v, 16);
     if (o.i >= 2 || o.q >= rs.n) return;
     float a = o.v;
-    int n = o.n[o.i];                  // row of the first half
+    int n = o.n;                  // row of the first half
     int blk = n / p.Dh;                // 0..3H-1 : q heads, k heads, v heads
     int dim = n - blk * p.Dh;          // < Dh/2
     int half = p.Dh / 2;
-    int r = rs.r[o.q];
+    int r = rs.r_sel(o.q);
     int pos = p.row_pos[r];
     if (blk < 2 * p.H) {
       float2 cs = p.rope[(long long)pos * half + dim];
@@ -434,10 +482,10 @@ struct EpiArgmax {
 
   __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs,
                                int lane) {
-    int nrow = o.n[o.i];
+    int nrow = o.n;
     bool valid = o.q < rs.n && nrow < s.N;
     if (p.logits && valid) {
-      int r = rs.r[o.q];
+      int r = rs.r_sel(o.q);
       p.logits[(long long)(p.row_dst ? p.row_dst[r] : r) * s.N + nrow] = o.v;
     }
     float bv = valid ? o.v : -INFINITY;
@@ -450,7 +498,7 @@ struct EpiArgmax {
     }
     if (lane < kRmax && lane < rs.n) {
       const int w = threadIdx.x >> 5;
-      const int r = rs.r[lane];
+      const int r = rs.r_sel(lane);
       float cv = best_v()[w * kRmax + r];
       int ci = best_i()[w * kRmax + r];
       if (bv > cv || (bv == cv && bi < ci)) {
@@ -568,7 +616,7 @@ __device__ __forceinline__ float consume_item(const GemvShape& s, const typename
       const unsigned char* stg = stages + st * stage_stride<Src>();
       Pairs8 xv[NR > 0 ? NR : 1];
 #pragma unroll
-      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, stg + kStageBytes, s.K, q, rs.r[q], rs.slot[q], c, lane);
+      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, stg + kStageBytes, s.K, q, rs.r(q), rs.slot(q), c, lane);
       const unsigned char* w_st = stg + lane * 16;
 #pragma unroll
       for (int i = 0; i < kWarpRows; ++i) {
@@ -628,11 +676,12 @@ __device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, con
 }
 
 template <int RG, class Src, class Epi>
-__global__ void __launch_bounds__(kGemvThreads, 2)
+__global__ void __maxnreg__(RG >= 8 ? 168 : 112)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem[];
   __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], xbar;
+  __shared__ int s_tag[kStages];  // item of the stage's slice (set with its first slice), -1 = end
   __shared__ float red_pro[kRmax * kNW];
   __shared__ int s_abort;
 
@@ -649,6 +698,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       mbar_init(&full_bar[i], Src::kStaged ? 2 : 1);
       mbar_init(&empty_bar[i], kNW);
     }
+    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -657,21 +707,18 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // ---------------- producer ----------------
     if (lane != 0) return;
     uint32_t it = 0;
-    // Dense weights do not depend on earlier kernels: start streaming the first
-    // stages before waiting for the previous kernel (programmatic dependent
-    // launch lets this overlap its tail).
-    int total = s.mats ? 0 : s.tiles_per_mat * s.kparts;
-    int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
-    int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
-    int item = start;
-    int sl = item < end ? item_pos(s, item).sl0 : 0;
     int R = 0;
     RowSet prs;  // rows of the current item (bf16 sources staged with the weights)
     int prs_m = -1;
+    auto stage_wait = [&](int st) {
+      // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
+      // stays uniform so the block always terminates
+      if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
+    };
     // Stage = weight box (one arrival with its transaction bytes) and, for a
     // staged bf16 source, the item's activation slice rows (a second arrival,
     // declared only after the dependency wait).
-    auto issue_w = [&](int m, int t, int slc) {
+    auto issue_w = [&](int item, int m, int t, int slc, bool first) {
       int ce;
       bool sh;
       mat_info(s, m, 0, &ce, &sh, nullptr);
@@ -679,9 +726,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       int r0, r1;
       tile_boxes(s, t, &r0, &r1);
       const int st = it % kStages;
-      // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
-      // stays uniform so the block always terminates
-      if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
+      stage_wait(st);
+      s_tag[st] = first ? item : -2;
       mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
       unsigned char* dst = stages + st * kStride;
       tma_load_box(dst, map, slc * kSlice, r0, ce, &full_bar[st]);
@@ -700,26 +746,40 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       unsigned char* dst = stages + st * kStride + kStageBytes;
       const int cols = min(kSlice, s.K - slc * kSlice);
       mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(prs.n * cols * 2));
-      for (int q = 0; q < prs.n; ++q)
-        bulk_g2s(dst + q * kXSliceBytes,
-                 SrcBf16::row_ptr(reinterpret_cast<const SrcBf16::Params&>(sp), prs.r[q], prs.slot[q]) + slc * kSlice,
-                 cols * 2, &full_bar[st]);
+#pragma unroll
+      for (int q = 0; q < kRmax; ++q)
+        if (q < prs.n)
+          bulk_g2s(dst + q * kXSliceBytes,
+                   SrcBf16::row_ptr(reinterpret_cast<const SrcBf16::Params&>(sp), prs.r(q), prs.slot(q)) + slc * kSlice,
+                   cols * 2, &full_bar[st]);
     };
-    // dense weights do not depend on earlier kernels: the first stages are
-    // requested before the dependency wait
-    int pre_item[kStages], pre_sl[kStages];
+    // items are claimed from the launch's work counter, so faster SMs take more
+    int total = s.mats ? 0 : s.tiles_per_mat * s.kparts;
+    // dense weights do not depend on earlier kernels: the stages of the CTA's
+    // first item are requested before the dependency wait (one item only, so
+    // that CTAs resident early do not take the work of those still arriving)
+    int pre_sl[kStages];
     int npre = 0;
+    int item = -1, sl = 0, sl_end = 0;
+    auto claim = [&]() {
+      item = atomicAdd(&s.work[0], 1);
+      if (item < total) {
+        ItemPos ip = item_pos(s, item);
+        sl = ip.sl0;
+        sl_end = ip.sl1;
+      }
+    };
+    bool claimed = false;  // item/sl hold a claimed item not yet fully issued
     if (!s.mats) {
-      for (; item < end && it < (uint32_t)kStages;) {
+      claim();
+      if (item < total) {
         const ItemPos ip = item_pos(s, item);
-        pre_item[npre] = item;
-        pre_sl[npre] = sl;
-        ++npre;
-        issue_w(0, ip.t, sl);
-        if (++sl == ip.sl1) {
-          ++item;
-          if (item < end) sl = item_pos(s, item).sl0;
+        while (sl < sl_end && it < (uint32_t)kStages) {
+          pre_sl[npre++] = sl;
+          issue_w(item, 0, ip.t, sl, sl == ip.sl0);
+          ++sl;
         }
+        claimed = sl < sl_end;
       }
     }
     pdl_wait();
@@ -727,28 +787,35 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     if (ok) {
       R = pass_rows(s);
       for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j]);
-      if (s.mats) {
-        total = *s.n_mats * s.tiles_per_mat;
-        start = (int)(((long long)blockIdx.x * total) / gridDim.x);
-        end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
-        item = start;
-        sl = 0;
-      }
-      for (; item < end;) {
+      if (s.mats) total = *s.n_mats * s.tiles_per_mat;
+      if (!claimed) claim();
+      while (item < total) {
         const ItemPos ip = item_pos(s, item);
         const uint32_t j = it;
-        issue_w(ip.m, ip.t, sl);
+        issue_w(item, ip.m, ip.t, sl, sl == ip.sl0);
         issue_x(j, ip.m, sl);
-        if (++sl == ip.sl1) {
-          ++item;
-          if (item < end) sl = item_pos(s, item).sl0;
-        }
+        if (++sl == sl_end) claim();
       }
     } else if (Src::kStaged) {
-      // aborting: complete the second arrival of every prefetched stage so the drain below can finish
+      // aborting: complete the second arrival of every prefetched stage
       for (int j = 0; j < npre; ++j) mbar_arrive(&full_bar[j]);
     }
-    (void)pre_item;
+    // end marker: a stage with no data
+    {
+      const int st = it % kStages;
+      stage_wait(st);
+      s_tag[st] = -1;
+      mbar_arrive(&full_bar[st]);
+      if (Src::kStaged) mbar_arrive(&full_bar[st]);
+      ++it;
+    }
+    // the last CTA done claiming resets the launch's counters
+    __threadfence();
+    if (atomicAdd(&s.work[1], 1) == (int)gridDim.x - 1) {
+      __threadfence();
+      s.work[0] = 0;
+      s.work[1] = 0;
+    }
     // drain: every issued copy has landed before the block can exit
     for (uint32_t j = (it > kStages ? it - kStages : 0); j < it; ++j)
       mbar_wait(&full_bar[j % kStages], (j / kStages) & 1, s.status);
@@ -756,25 +823,38 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   }
 
   // ---------------- consumers ----------------
+  typename Src::Pre pre;
+  Src::pre_wait(sp, s.K, tid, pre);
   pdl_wait();
   if (tid == 0) {
     tm.t0 = gtimer();
-    s_abort = status_bad(s.status);
+    const int ab = status_bad(s.status);
+    s_abort = ab;
+    if (!ab) Src::issue(sp, s.K, pass_rows(s), xs, &xbar);
   }
   named_sync(1, kConsumers);
-  if (s_abort) return;
+  if (s_abort) {
+    // consume the producer's stages up to its end marker so it can finish
+    uint32_t it = 0;
+    while (true) {
+      const int st = it % kStages;
+      mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
+      const int tag = s_tag[st];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
+      ++it;
+      if (tag == -1) break;
+    }
+    return;
+  }
   pdl_trigger();
 
   const int R = pass_rows(s);
-  const int n_mats = s.mats ? *s.n_mats : 1;
-  const int total = n_mats * s.tiles_per_mat * (s.mats ? 1 : s.kparts);
-  const int start = (int)(((long long)blockIdx.x * total) / gridDim.x);
-  const int end = (int)(((long long)(blockIdx.x + 1) * total) / gridDim.x);
   const int nch = s.K / 8;  // 16-byte chunks per row
   __shared__ int s_last_part;
 
   epi_init<Epi>(tid);
-  if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid);
+  if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid, pre);
   else named_sync(1, kConsumers);
   if (tid == 0) tm.t1 = gtimer();
 
@@ -787,7 +867,16 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
   for (int i = 0; i < kWarpRows; ++i) srow[i] = stage_row(paired, warp, i);
 
-  for (int item = start; item < end; ++item) {
+  while (true) {
+    const int st0 = it % kStages;
+    mbar_wait(&full_bar[st0], (it / kStages) & 1, s.status);
+    const int item = s_tag[st0];
+    if (item < 0) {  // end marker
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st0]);
+      ++it;
+      break;
+    }
     const ItemPos ip = item_pos(s, item);
     if (ip.m != cur_m) {
       mat_info(s, ip.m, R, &ce, &sh, &rs);
@@ -815,8 +904,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     o.q = lane & 7;
     int r0, r1;
     tile_boxes(s, ip.t, &r0, &r1);
-#pragma unroll
-    for (int i = 0; i < kWarpRows; ++i) o.n[i] = matrix_row(r0, r1, srow[i]);
+    o.n = matrix_row(r0, r1, sel(srow, o.i));
     Epi::apply(ep, s, o, rs, lane);
   }
   named_sync(1, kConsumers);

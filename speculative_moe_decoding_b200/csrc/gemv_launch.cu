@@ -12,9 +12,14 @@ void gemv_plan(GemvShape& s) {
 }
 
 int gemv_kparts(const GemvShape& s, int target_items) {
-  if (s.mats || s.tiles_per_mat >= target_items / 2 || s.ns < 2) return 1;
+  // Split only long, short matrices: a part posts partial sums, fences and
+  // counts, which costs about as much as streaming four slices, so parts are
+  // at least four slices long and only matrices too short to give every SM a
+  // tile are split.
+  constexpr int kMinSlicesPerPart = 4;
+  if (s.mats || s.tiles_per_mat >= 64 || s.ns < 2 * kMinSlicesPerPart) return 1;
   int want = (target_items + s.tiles_per_mat - 1) / s.tiles_per_mat;
-  want = std::min(want, s.ns);
+  want = std::min(want, (s.ns + kMinSlicesPerPart - 1) / kMinSlicesPerPart);
   const int spp = (s.ns + want - 1) / want;  // slices per part
   int kp = (s.ns + spp - 1) / spp;           // parts, all non-empty
   if ((long long)s.tiles_per_mat * kp * kNW * 32 > kSplitPartFloats || s.tiles_per_mat > kSplitMaxTiles) return 1;
@@ -89,9 +94,11 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
   size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
-  int grid = g.grid;
-  // two CTAs per SM (register-capped): the second hides the first's latencies
-  if (grid <= 0) grid = g.s.mats ? 2 * lc.num_sms : std::min(g.s.tiles_per_mat * g.s.kparts, 2 * lc.num_sms);
+  // two CTAs per SM (112 registers a thread) hide each other's latencies; the
+  // eight-row variant needs more registers and runs one CTA per SM
+  const int slots = (RG >= 8 ? 1 : 2) * lc.num_sms;
+  int grid = g.grid > 0 ? std::min(g.grid, slots) : slots;
+  if (!g.s.mats) grid = std::min(grid, g.s.tiles_per_mat * g.s.kparts);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
 }
 
@@ -109,6 +116,7 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
     return cudaErrorInvalidValue;
   if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
   if (g.s.kparts > 1 && (g.s.mats || !g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;
+  if (!g.s.work) return cudaErrorInvalidValue;
   if (g.src == SrcKind::Norm) {
     switch (g.epi) {
       case EpiKind::QKV: return launch_rg<SrcNorm, EpiQKV>(g, g.norm, g.qkv, lc);

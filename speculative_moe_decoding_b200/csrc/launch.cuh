@@ -30,6 +30,27 @@ cudaError_t launch_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// The same, with thread-block clusters of cluster_x CTAs along x.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_cluster_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, const LaunchCfg& lc,
+                      int cluster_x, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = lc.stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cluster_x;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = lc.pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 enum class SrcKind { Norm, Bf16 };
 enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, Route, ArgmaxAccept };
 
@@ -68,6 +89,7 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
 // largest size any launch uses (call outside stream capture, once per device).
 cudaError_t gemv_prepare();
 constexpr int kGemvMaxK = 4096;  // largest K of a normalised (shared-memory) source
+constexpr int kWorkSlots = 4;   // GEMV work-counter pairs cycled by a decoder context
 
 
 }  // namespace ocrdec

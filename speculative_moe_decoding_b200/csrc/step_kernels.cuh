@@ -35,6 +35,8 @@ struct PassRows {
 // to stream (shared experts first, then touched experts in ascending id).
 // One CTA, one warp per row.
 // ---------------------------------------------------------------------------
+constexpr int kMaxExperts = 128;
+
 struct RouteParams {
   const float* logits;  // [R][E]
   const int* nrows;
@@ -54,17 +56,21 @@ struct RouteParams {
 // over exactly those threads.
 template <class Sync>
 __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, Sync sync) {
+  __shared__ float s_p[kRmax][kMaxExperts];            // softmax probabilities
+  __shared__ unsigned char s_sel[kRmax][kMaxExperts];  // 1 if among the row's top-k
   __shared__ int s_ids[kRmax][8];
-  __shared__ int s_cnt[256];
-  __shared__ int s_off[256];
+  __shared__ int s_cnt[kMaxExperts];
+  __shared__ int s_off[kMaxExperts];
   const int lane = tid & 31, warp = tid >> 5;
   const int E = p.E, K = p.top_k;
+  // softmax of each row (warp per row; fixed-order sums)
   if (warp < R) {
     const float* lg = p.logits + warp * E;
-    float pe[8];  // E <= 256
+    constexpr int kPer = kMaxExperts / 32;
+    float pe[kPer];
     float m = -INFINITY;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kPer; ++i) {
       int e = lane + 32 * i;
       pe[i] = e < E ? lg[e] : -INFINITY;
       m = fmaxf(m, pe[i]);
@@ -73,7 +79,7 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     float sum = 0.f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < kPer; ++i) {
       int e = lane + 32 * i;
       pe[i] = e < E ? expf(__fsub_rn(pe[i], m)) : 0.f;
       sum = __fadd_rn(sum, pe[i]);
@@ -81,41 +87,35 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) sum = __fadd_rn(sum, __shfl_xor_sync(0xffffffffu, sum, o));
 #pragma unroll
-    for (int i = 0; i < 8; ++i) pe[i] = __fdiv_rn(pe[i], sum);
-    // top-k rounds: round s's winner (value, id) stays in lane s - no
-    // dynamically indexed arrays (they would live in local memory)
-    int my_id = 0x7fffffff;
-    float my_g = 0.f;
-    for (int s = 0; s < K; ++s) {
-      float bv = -1.f;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        int e = lane + 32 * i;
-        if (e < E && (pe[i] > bv || (pe[i] == bv && e < bi))) { bv = pe[i]; bi = e; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-        int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ov > bv || (ov == bv && oi < bi)) { bv = ov; bi = oi; }
-      }
-      if (lane == s) { my_id = bi; my_g = bv; }
-#pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (lane + 32 * i == bi) pe[i] = -2.f;  // taken
+    for (int i = 0; i < kPer; ++i) {
+      int e = lane + 32 * i;
+      if (e < E) s_p[warp][e] = __fdiv_rn(pe[i], sum);
     }
-    // slot order = ascending expert id: lane s < K moves to slot rank(s)
-    int rank = 0;
-    for (int t = 0; t < K; ++t) {
-      int other = __shfl_sync(0xffffffffu, my_id, t);
-      if (other < my_id) ++rank;
+  }
+  sync();
+  // top-k by rank: expert e of row r is selected when fewer than K experts beat
+  // it (larger probability, or equal probability and lower id)
+  for (int idx = tid; idx < R * E; idx += nthreads) {
+    const int r = idx / E, e = idx - r * E;
+    const float pv = s_p[r][e];
+    int beat = 0;
+    for (int f = 0; f < E; ++f) {
+      const float q = s_p[r][f];
+      beat += (q > pv) || (q == pv && f < e);
     }
-    if (lane < K) {
-      p.ids[warp * K + rank] = my_id;
-      p.gates[warp * K + rank] = my_g;
-      s_ids[warp][rank] = my_id;
-    }
+    s_sel[r][e] = beat < K;
+  }
+  sync();
+  // slot = rank of the expert id among the row's selected experts
+  for (int idx = tid; idx < R * E; idx += nthreads) {
+    const int r = idx / E, e = idx - r * E;
+    if (!s_sel[r][e]) continue;
+    int slot = 0;
+    for (int f = 0; f < e; ++f) slot += s_sel[r][f];
+    if (slot >= K) continue;  // only with NaN probabilities, which break the total order
+    p.ids[r * K + slot] = e;
+    p.gates[r * K + slot] = s_p[r][e];
+    s_ids[r][slot] = e;
   }
   sync();
   // bucketing: thread e counts its (row, slot) entries in row order

@@ -62,6 +62,7 @@ def test_config_validation(lib):
         dict(good, top_k=9),               # top_k > n_experts
         dict(good, shared_ffn=64),         # shared width must equal expert width
         dict(good, vocab=4095),            # vocab multiple of 8
+        dict(good, n_heads=8, head_dim=32),  # head_dim 64 or 128 only
     ]
     for bad in bad_cases:
         cfg = lib.make_config(bad, 3, 1, 256)
@@ -69,6 +70,8 @@ def test_config_validation(lib):
     cfg = lib.make_config(good, 4, 1, 256)  # max_k > 3
     assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
     cfg = lib.make_config(good, 3, 3, 256)  # batch * (k+1) rows beyond one pass
+    assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
+    cfg = lib.make_config(good, 3, 1, 8200)  # kv_capacity beyond 8192
     assert lib.ocrdec_create(ctypes.byref(cfg), ctypes.byref(ctx)) == lib.EINVAL
 
 
