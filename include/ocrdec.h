@@ -243,6 +243,35 @@ OCRDEC_API int ocrdec_op_lm_argmax(const void* dev_W, const float* dev_x, const 
 
 OCRDEC_API size_t ocrdec_op_scratch_bytes(void);
 
+/* The same final norm + LM head + greedy argmax as ocrdec_op_lm_argmax, for
+ * callers that may not allocate device memory and hold no scratch buffer of
+ * their own: for example a serving runtime whose memory pool owns all free
+ * device memory, or a caller inside an allocator callback, where a cudaMalloc
+ * would fail or re-enter the allocator.  It allocates nothing: its scratch is a
+ * fixed array of ocrdec_op_static_scratch_bytes() (64 KiB) in the library's own
+ * device image, one per device.
+ *
+ * The method's published description has no counterpart for this call; it is
+ * a deployment convenience around the kernel of ocrdec_op_lm_argmax.
+ *
+ * Arguments, layouts and results are those of ocrdec_op_lm_argmax (all device
+ * pointers, owned by the caller; the call only enqueues work on `stream`).
+ * The first call on a device, made with that device current, looks up the
+ * scratch's address (cudaGetSymbolAddress) and may load the module; make it
+ * before capturing any stream.  The scratch status words and counters are
+ * cleared on `stream` at every call.  The scratch is shared by every caller on
+ * a device: calls that overlap in time (other streams, other threads) race
+ * and give undefined results; serialise them.
+ *
+ * Returns OCRDEC_OK, OCRDEC_EINVAL (the argument checks of
+ * ocrdec_op_lm_argmax), OCRDEC_ENOMEM if this device needs more scratch than
+ * the fixed array holds (more than 509 SMs), or OCRDEC_ECUDA (no current
+ * device, symbol lookup or launch failed). */
+OCRDEC_API int ocrdec_op_lm_argmax_static(const void* dev_W, const float* dev_x, const void* dev_g, float eps,
+                                          int R, int N, int K, int32_t* dev_tok, float* dev_logits,
+                                          ocrdec_stream stream);
+OCRDEC_API size_t ocrdec_op_static_scratch_bytes(void);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1074,3 +1074,46 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
 }
 
 }  // extern "C"
+
+// ---- LM-head argmax on library-owned scratch ---------------------------------
+// Fixed scratch in the library's own device image, one copy per device.  Its
+// address is looked up once per device (cudaGetSymbolAddress) by the first
+// call made with that device current; later calls reuse it.  Nothing here
+// allocates device memory.
+namespace {
+constexpr size_t kStaticScratchBytes = 64 << 10;
+__device__ __align__(256) unsigned char g_static_scratch[kStaticScratchBytes];
+constexpr int kMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kMaxDevices] = {};
+}  // namespace
+
+extern "C" {
+
+size_t ocrdec_op_static_scratch_bytes(void) { return kStaticScratchBytes; }
+
+int ocrdec_op_lm_argmax_static(const void* W, const float* x, const void* g, float eps, int R, int N, int K,
+                               int32_t* tok, float* logits, ocrdec_stream stream) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return OCRDEC_ECUDA;
+  const int sms = device_sms();
+  if (sms <= 0) return OCRDEC_ECUDA;
+  size_t am_off;
+  op_scratch_layout(sms, &am_off, nullptr, nullptr);
+  // status words + one (value, index) partial per CTA and row; the CTA count is
+  // at most two per SM
+  if (am_off + sizeof(float2) * 2 * (size_t)sms * kRmax > kStaticScratchBytes) return OCRDEC_ENOMEM;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_static_scratch) != cudaSuccess || !p) return OCRDEC_ECUDA;
+      g_static_ptr[dev] = p;
+    }
+    scratch = g_static_ptr[dev];
+  }
+  return ocrdec_op_lm_argmax(W, x, g, eps, R, N, K, tok, logits, scratch, stream);
+}
+
+}  // extern "C"

@@ -76,6 +76,9 @@ ocrdec_strerror = _sig("ocrdec_strerror", ctypes.c_char_p, _i32)
 ocrdec_op_scratch_bytes = _sig("ocrdec_op_scratch_bytes", _sz)
 ocrdec_op_norm_gemv = _sig("ocrdec_op_norm_gemv", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp)
 ocrdec_op_lm_argmax = _sig("ocrdec_op_lm_argmax", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp, _vp, _vp, _vp)
+ocrdec_op_lm_argmax_static = _sig("ocrdec_op_lm_argmax_static", _i32, _vp, _vp, _vp, _f32, _i32, _i32, _i32, _vp,
+                                  _vp, _vp)
+ocrdec_op_static_scratch_bytes = _sig("ocrdec_op_static_scratch_bytes", _sz)
 
 
 class OcrdecError(RuntimeError):
@@ -284,3 +287,11 @@ def op_lm_argmax(W, x, g, eps, tok, logits, scratch, stream=None):
     N = W.shape[0]
     check(ocrdec_op_lm_argmax(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
                               _ptr(logits), scratch.data_ptr(), _stream(stream)), "ocrdec_op_lm_argmax")
+
+
+def op_lm_argmax_static(W, x, g, eps, tok, logits, stream=None):
+    """op_lm_argmax on the library's fixed per-device scratch (allocates nothing)."""
+    R, K = x.shape
+    N = W.shape[0]
+    check(ocrdec_op_lm_argmax_static(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
+                                     _ptr(logits), _stream(stream)), "ocrdec_op_lm_argmax_static")
