@@ -7,9 +7,10 @@
 //
 // The position axis is cut into fixed kAttnChunk-position chunks.  The
 // kAttnSplit CTAs of one cluster serve one (slot, head); CTA k takes chunks
-// k, k + kAttnSplit, ... in increasing order, streams each chunk's K and V
-// rows into a shared-memory ring with bulk copies, and keeps an online-softmax
-// state per row (running max M, sum L, unnormalised output O).  The CTAs then
+// k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time: it streams
+// their K and V rows into shared memory with bulk copies, scores them all,
+// and keeps an online-softmax state per row (running max M, sum L,
+// unnormalised output O) that is rescaled between such groups.  The CTAs then
 // merge their states through distributed shared memory, rank by rank, each CTA
 // producing Dh / kAttnSplit output dims.  Which CTA takes a chunk and the order
 // of every sum depend only on positions, so a row's result does not depend on
@@ -76,7 +77,7 @@ attention_kernel(const AttnParams p) {
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
   __shared__ float qs[kAttnRows][kAttnMaxDh];
-  __shared__ float sc[kAttnRows][kAttnChunk];
+  __shared__ float sc[kAttnRows][kAttnBufs * kAttnChunk];
   __shared__ float ored[kAttnWarps][kAttnRows][kAttnMaxDh];
   __shared__ float s_M[kAttnRows], s_L[kAttnRows], s_corr[kAttnRows];
   __shared__ float s_O[kAttnRows][kAttnMaxDh];
@@ -111,45 +112,47 @@ attention_kernel(const AttnParams p) {
   const int n_my = nch > k ? (nch - 1 - k) / kAttnSplit + 1 : 0;  // this CTA's chunks
   const long long head_base = (long long)b * p.slot_stride + (long long)h * p.cap * Dh;
 
-  auto issue = [&](int i) {  // chunk i of this CTA into ring buffer i % kAttnBufs
-    const int c = k + i * kAttnSplit;
-    const int p0 = c * kAttnChunk;
-    const int npos = min(kAttnChunk, maxpos + 1 - p0);
+  // chunk i of this CTA: position p0, valid positions npos, ring buffer i % kAttnBufs
+  auto chunk_p0 = [&](int i) { return (k + i * kAttnSplit) * kAttnChunk; };
+  auto chunk_npos = [&](int i) { return min(kAttnChunk, maxpos + 1 - chunk_p0(i)); };
+  auto issue = [&](int i) {
+    const int p0 = chunk_p0(i);
     const int buf = i % kAttnBufs;
     bf16* Ks = ring + (size_t)buf * 2 * kAttnChunk * Dh;
-    const uint32_t bytes = npos * Dh * 2;
+    const uint32_t bytes = chunk_npos(i) * Dh * 2;
     mbar_arrive_expect_tx(&bar[buf], 2 * bytes);
     bulk_g2s(Ks, p.kc + head_base + (long long)p0 * Dh, bytes, &bar[buf]);
     bulk_g2s(Ks + kAttnChunk * Dh, p.vc + head_base + (long long)p0 * Dh, bytes, &bar[buf]);
   };
-  auto old_chunk = [&](int i) { return (k + i * kAttnSplit + 1) * kAttnChunk <= minpos; };
+  auto old_chunk = [&](int i) { return chunk_p0(i) + kAttnChunk <= minpos; };
   const int n_first = min(n_my, kAttnBufs);
   if (tid == 0)
     for (int i = 0; i < n_first; ++i)
       if (old_chunk(i)) issue(i);
 
   pdl_wait();
-  TraceMarks tm;  // trace: wait returned, first chunk landed, local pass done
+  TraceMarks tm;  // trace: wait returned, first group landed, its softmax done
+  float qv[kAttnRows];
+#pragma unroll
+  for (int i = 0; i < kAttnRows; ++i)
+    qv[i] = (i < nr && tid < Dh) ? p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + tid] : 0.f;
   if (tid == 0) {
     tm.t0 = gtimer();
-    s_abort = status_bad(p.status);
+    const int ab = status_bad(p.status);
+    s_abort = ab;
+    if (!ab)
+      for (int i = 0; i < n_first; ++i)
+        if (!old_chunk(i)) issue(i);
   }
+  if (tid < Dh)
+#pragma unroll
+    for (int i = 0; i < kAttnRows; ++i) qs[i][tid] = qv[i];
   __syncthreads();
   const bool work = !s_abort && nr > 0;
   pdl_trigger();
 
-  if (work) {
-    if (tid == 0)
-      for (int i = 0; i < n_first; ++i)
-        if (!old_chunk(i)) issue(i);
-#pragma unroll
-    for (int i = 0; i < kAttnRows; ++i)
-      if (i < nr && tid < Dh) qs[i][tid] = p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + tid];
-    __syncthreads();
-  }
-
-  // per-warp output accumulators: warp w owns positions [w, w + 1) * kAttnWarpPos
-  // of each chunk, lane l dims [l*dpl, (l+1)*dpl)
+  // per-warp output accumulators: warp w owns offsets [w, w + 1) * kAttnWarpPos
+  // of every chunk, lane l dims [l*dpl, (l+1)*dpl)
   const int dpl = Dh / 32;  // 4 (Dh 128) or 2 (Dh 64)
   float o[kAttnRows][4];
 #pragma unroll
@@ -157,86 +160,89 @@ attention_kernel(const AttnParams p) {
 #pragma unroll
     for (int e = 0; e < 4; ++e) o[r][e] = 0.f;
 
-  const int g = lane >> 3, l8 = lane & 7;
+  const int g4 = lane >> 3, l8 = lane & 7;
   const int ndc = Dh / 8;  // 16-byte chunks per key row (8 or 16)
-  for (int i = 0; work && i < n_my; ++i) {
-    const int c = k + i * kAttnSplit;
-    const int p0 = c * kAttnChunk;
-    const int npos = min(kAttnChunk, maxpos + 1 - p0);
-    const int buf = i % kAttnBufs;
-    const bf16* Ks = ring + (size_t)buf * 2 * kAttnChunk * Dh;
-    const bf16* Vs = Ks + kAttnChunk * Dh;
-    mbar_wait(&bar[buf], (i / kAttnBufs) & 1, p.status);  // gives up with OCRDEC_ETIMEOUT; control flow stays uniform
-    if (tid == 0 && i == 0) tm.t1 = gtimer();
+  // Chunks are taken kAttnBufs at a time (a group); the online-softmax state
+  // is rescaled between groups.
+  for (int i0 = 0, grp = 0; work && i0 < n_my; i0 += kAttnBufs, ++grp) {
+    const int ni = min(kAttnBufs, n_my - i0);
+    for (int ii = 0; ii < ni; ++ii)
+      mbar_wait(&bar[ii], grp & 1, p.status);  // gives up with OCRDEC_ETIMEOUT; control flow stays uniform
+    if (tid == 0 && grp == 0) tm.t1 = gtimer();
 
-    // ---- scores: 4 groups of 8 lanes per warp, one position per group;
-    // lane l8 of a group owns the 16-byte dim-chunks l8 and l8 + 8 of a key row
+    // ---- scores: 4 groups of 8 lanes per warp, one position per lane group;
+    // lane l8 owns the 16-byte dim-chunks l8 and l8 + 8 of a key row
     for (int rb = 0; rb < nr; rb += 4) {
       float qr[4][16];
 #pragma unroll
-      for (int ii = 0; ii < 4; ++ii)
+      for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
           int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
-          qr[ii][e] = (rb + ii < nr && (e < 8 || l8 + 8 < ndc)) ? qs[rb + ii][d] : 0.f;
+          qr[q][e] = (rb + q < nr && (e < 8 || l8 + 8 < ndc)) ? qs[rb + q][d] : 0.f;
         }
-      for (int j0 = warp * kAttnWarpPos; j0 < (warp + 1) * kAttnWarpPos; j0 += 4) {
-        const int j = j0 + g;
-        float kv[16];
-        if (j < npos) {
-          float t[8];
-          unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + l8 * 8), t);
+      for (int ii = 0; ii < ni; ++ii) {
+        const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
+        const bf16* Ks = ring + (size_t)ii * 2 * kAttnChunk * Dh;
 #pragma unroll
-          for (int e = 0; e < 8; ++e) kv[e] = t[e];
-          if (l8 + 8 < ndc) {
-            unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + (l8 + 8) * 8), t);
+        for (int j0 = 0; j0 < kAttnWarpPos; j0 += 4) {
+          const int j = warp * kAttnWarpPos + j0 + g4;
+          float kv[16];
+          if (j < npos) {
+            float t[8];
+            unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + l8 * 8), t);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kv[8 + e] = t[e];
+            for (int e = 0; e < 8; ++e) kv[e] = t[e];
+            if (l8 + 8 < ndc) {
+              unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + (l8 + 8) * 8), t);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) kv[8 + e] = t[e];
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) kv[8 + e] = 0.f;
+            }
           } else {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) kv[8 + e] = 0.f;
+            for (int e = 0; e < 16; ++e) kv[e] = 0.f;
           }
-        } else {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) kv[e] = 0.f;
-        }
+          for (int q = 0; q < 4; ++q) {
+            float a = 0.f;
 #pragma unroll
-        for (int ii = 0; ii < 4; ++ii) {
-          float a = 0.f;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) a = __fmaf_rn(qr[ii][e], kv[e], a);
-          a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
-          a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
-          a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
-          const int r = rb + ii;
-          if (l8 == 0 && r < nr) {
-            const bool valid = j < npos && p0 + j <= s_pos[r];
-            sc[r][j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
+            for (int e = 0; e < 16; ++e) a = __fmaf_rn(qr[q][e], kv[e], a);
+            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
+            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
+            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
+            const int r = rb + q;
+            if (l8 == 0 && r < nr) {
+              const bool valid = j < npos && p0 + j <= s_pos[r];
+              sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
+            }
           }
         }
       }
     }
     __syncthreads();
 
-    // ---- online softmax update of each row (warp w takes row w) ----
+    // ---- online softmax update of each row over the group (warp w: row w).
+    // Invisible positions hold -inf and give exp(-inf) = 0 exactly, so a row's
+    // sums do not depend on how many chunks the group has. ----
+    const int nu = ni * kAttnChunk;
     for (int r = warp; r < nr; r += kAttnWarps) {
-      const int lim = min(s_pos[r] - p0 + 1, npos);  // visible positions of the row in the chunk
-      if (lim <= 0) {
-        for (int j = lane; j < kAttnChunk; j += 32) sc[r][j] = 0.f;
+      float m = -INFINITY;
+      for (int u = lane; u < nu; u += 32) m = fmaxf(m, sc[r][u]);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+      if (m == -INFINITY) {  // nothing visible to this row in the group
         if (lane == 0) s_corr[r] = 1.f;
         continue;
       }
-      float m = -INFINITY;
-      for (int j = lane; j < lim; j += 32) m = fmaxf(m, sc[r][j]);
-#pragma unroll
-      for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       const float Mold = s_M[r];
       const float Mn = fmaxf(Mold, m);
       float l = 0.f;
-      for (int j = lane; j < kAttnChunk; j += 32) {
-        float e = 0.f;
-        if (j < lim) e = expf(__fsub_rn(sc[r][j], Mn));
-        sc[r][j] = e;
+      for (int u = lane; u < nu; u += 32) {
+        const float e = expf(__fsub_rn(sc[r][u], Mn));
+        sc[r][u] = e;
         l = __fadd_rn(l, e);
       }
 #pragma unroll
@@ -250,24 +256,25 @@ attention_kernel(const AttnParams p) {
       }
     }
     __syncthreads();
-    if (tid == 0 && i == 0) tm.t2 = gtimer();
+    if (tid == 0 && grp == 0) tm.t2 = gtimer();
 
-    // ---- o = o * corr + sum_j p_j v_j over the warp's positions in order ----
-    {
-      int lim[kAttnRows];
+    // ---- o = o * corr + sum p_j v_j over the warp's offsets, chunk by chunk ----
 #pragma unroll
-      for (int r = 0; r < kAttnRows; ++r) {
-        lim[r] = r < nr ? min(s_pos[r] - p0 + 1, npos) : 0;
-        if (lim[r] > 0) {
-          const float cr = s_corr[r];
+    for (int r = 0; r < kAttnRows; ++r)
+      if (r < nr) {
+        const float cr = s_corr[r];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) o[r][e] = __fmul_rn(o[r][e], cr);
-        }
+        for (int e = 0; e < 4; ++e) o[r][e] = __fmul_rn(o[r][e], cr);
       }
-      const int jb = warp * kAttnWarpPos;
-#pragma unroll 2
+    for (int ii = 0; ii < ni; ++ii) {
+      const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
+      const bf16* Vs = ring + (size_t)ii * 2 * kAttnChunk * Dh + kAttnChunk * Dh;
+      int lim[kAttnRows];  // visible offsets of each row in this chunk
+#pragma unroll
+      for (int r = 0; r < kAttnRows; ++r) lim[r] = r < nr ? min(s_pos[r] - p0 + 1, npos) : 0;
+#pragma unroll
       for (int jj = 0; jj < kAttnWarpPos; ++jj) {
-        const int j = jb + jj;
+        const int j = warp * kAttnWarpPos + jj;
         if (j >= npos) break;
         float vv[4];
         if (dpl == 4) {
@@ -280,15 +287,16 @@ attention_kernel(const AttnParams p) {
 #pragma unroll
         for (int r = 0; r < kAttnRows; ++r) {
           if (j < lim[r]) {
-            const float pj = sc[r][j];
+            const float pj = sc[r][ii * kAttnChunk + j];
 #pragma unroll
             for (int e = 0; e < 4; ++e) o[r][e] = __fmaf_rn(pj, vv[e], o[r][e]);
           }
         }
       }
     }
-    __syncthreads();  // the chunk buffer and the scores are free again
-    if (tid == 0 && i + kAttnBufs < n_my) issue(i + kAttnBufs);
+    __syncthreads();  // ring buffers and scores are free again
+    if (tid == 0)
+      for (int ii = 0; ii < kAttnBufs && i0 + kAttnBufs + ii < n_my; ++ii) issue(i0 + kAttnBufs + ii);
   }
 
   // ---- this CTA's state: O = sum of the warp partials in warp order ----
@@ -318,9 +326,8 @@ attention_kernel(const AttnParams p) {
   // the CTAs' states in rank order ----
   if (work) {
     const int dpr = Dh / kAttnSplit;
-    const int t = tid;
-    if (t < nr * dpr) {
-      const int r = t / dpr, d = k * dpr + (t - r * dpr);
+    if (tid < nr * dpr) {
+      const int r = tid / dpr, d = k * dpr + (tid - r * dpr);
       // all remote loads are issued before any is used
       float Mk[kAttnSplit], Lk[kAttnSplit], Ok[kAttnSplit];
 #pragma unroll

@@ -242,12 +242,17 @@ struct SrcNorm {
       }
     }
   }
-  // One thread, after the dependency wait: copy the R raw rows into xs.
-  __device__ static void issue(const Params& p, int K, int R, float* xs, uint64_t* xbar) {
-    if (R <= 0) return;
-    mbar_arrive_expect_tx(xbar, (uint32_t)(R * K * 4));
-    for (int r = 0; r < R; ++r)
-      bulk_g2s(xs + r * K, p.x + (long long)(p.row_src ? p.row_src[r] : r) * p.ldx, K * 4, xbar);
+  // One thread, right after the dependency wait: copy Rc raw rows into xs.
+  // Rc is a bound known at launch (the pass's row count is read in parallel),
+  // so the copies wait on no other load; source rows are clamped to the
+  // kRmax-row buffers they index.
+  __device__ static void issue(const Params& p, int K, int Rc, float* xs, uint64_t* xbar) {
+    if (Rc <= 0) return;
+    mbar_arrive_expect_tx(xbar, (uint32_t)(Rc * K * 4));
+    for (int r = 0; r < Rc; ++r) {
+      const int src = p.row_src ? min(max(p.row_src[r], 0), kRmax - 1) : r;
+      bulk_g2s(xs + r * K, p.x + (long long)src * p.ldx, K * 4, xbar);
+    }
   }
 
   // All consumer threads.  Thread t owns the float4 groups t, t + 256, ... of
@@ -256,10 +261,10 @@ struct SrcNorm {
   // and written back as one float4.  The sums of squares of all rows are formed
   // together (one barrier); a row is rewritten in place only once every thread
   // has read it, which the barrier after each row's reads guarantees.
-  __device__ static void prologue(const Params& p, int K, int R, float* xs, float* red, uint64_t* xbar,
+  __device__ static void prologue(const Params& p, int K, int R, int Rc, float* xs, float* red, uint64_t* xbar,
                                   int* status, int tid, const Pre& pre) {
     const int ng = K / 4;
-    if (R > 0) mbar_wait(xbar, 0, status);
+    if (Rc > 0) mbar_wait(xbar, 0, status);
     const int lane = tid & 31, warp = tid >> 5;
     const int half = K / 2;
     float a[kRmax];
@@ -354,7 +359,7 @@ struct SrcBf16 {
   struct Pre {};
   __device__ static void pre_wait(const Params&, int, int, Pre&) {}
   __device__ static void issue(const Params&, int, int, float*, uint64_t*) {}
-  __device__ static void prologue(const Params&, int, int, float*, float*, uint64_t*, int*, int, const Pre&) {}
+  __device__ static void prologue(const Params&, int, int, int, float*, float*, uint64_t*, int*, int, const Pre&) {}
   __device__ static const bf16* row_ptr(const Params& p, int r, int slot) {
     return p.x + (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
   }
@@ -676,7 +681,7 @@ __device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, con
 }
 
 template <int RG, class Src, class Epi>
-__global__ void __maxnreg__(RG >= 8 ? 168 : 112)
+__global__ void __launch_bounds__(kGemvThreads, RG >= 8 ? 1 : 2)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem[];
@@ -785,7 +790,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     pdl_wait();
     const bool ok = !status_bad(s.status);
     if (ok) {
-      R = pass_rows(s);
+      R = min(pass_rows(s), RG);
       for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j]);
       if (s.mats) total = *s.n_mats * s.tiles_per_mat;
       if (!claimed) claim();
@@ -826,14 +831,17 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   typename Src::Pre pre;
   Src::pre_wait(sp, s.K, tid, pre);
   pdl_wait();
+  // rows copied for a normalised source: the pass bound of this variant (the
+  // engine's row buffers hold kRmax rows) or the exact static count
+  const int Rc = s.nrows ? min(RG, kRmax) : min(s.rows_static, kRmax);
   if (tid == 0) {
     tm.t0 = gtimer();
-    const int ab = status_bad(s.status);
-    s_abort = ab;
-    if (!ab) Src::issue(sp, s.K, pass_rows(s), xs, &xbar);
+    Src::issue(sp, s.K, Rc, xs, &xbar);
+    s_abort = status_bad(s.status);
   }
   named_sync(1, kConsumers);
   if (s_abort) {
+    if (Src::kSmem && tid == 0 && Rc > 0) mbar_wait(&xbar, 0, s.status);  // the row copies land first
     // consume the producer's stages up to its end marker so it can finish
     uint32_t it = 0;
     while (true) {
@@ -849,12 +857,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   }
   pdl_trigger();
 
-  const int R = pass_rows(s);
+  const int R = min(pass_rows(s), RG);
   const int nch = s.K / 8;  // 16-byte chunks per row
   __shared__ int s_last_part;
 
   epi_init<Epi>(tid);
-  if (Src::kSmem) Src::prologue(sp, s.K, R, xs, red_pro, &xbar, s.status, tid, pre);
+  if (Src::kSmem) Src::prologue(sp, s.K, R, Rc, xs, red_pro, &xbar, s.status, tid, pre);
   else named_sync(1, kConsumers);
   if (tid == 0) tm.t1 = gtimer();
 

@@ -94,7 +94,7 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
   size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
-  // two CTAs per SM (112 registers a thread) hide each other's latencies; the
+  // two CTAs per SM (96 registers a thread) hide each other's latencies; the
   // eight-row variant needs more registers and runs one CTA per SM
   const int slots = (RG >= 8 ? 1 : 2) * lc.num_sms;
   int grid = g.grid > 0 ? std::min(g.grid, slots) : slots;

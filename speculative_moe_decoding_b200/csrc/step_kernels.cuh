@@ -52,15 +52,13 @@ struct RouteParams {
   int* status;
 };
 
-// Routing of the R rows by nthreads cooperating threads; sync() is a barrier
-// over exactly those threads.
+// Routing of the R rows by nthreads (>= 32 * R) cooperating threads; sync()
+// is a barrier over exactly those threads.
 template <class Sync>
 __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, Sync sync) {
-  __shared__ float s_p[kRmax][kMaxExperts];            // softmax probabilities
-  __shared__ unsigned char s_sel[kRmax][kMaxExperts];  // 1 if among the row's top-k
-  __shared__ int s_ids[kRmax][8];
-  __shared__ int s_cnt[kMaxExperts];
-  __shared__ int s_off[kMaxExperts];
+  __shared__ float s_p[kRmax][kMaxExperts];             // softmax probabilities
+  __shared__ unsigned char s_sel[kRmax][kMaxExperts];   // 1 if among the row's top-k
+  __shared__ unsigned char s_slot[kRmax][kMaxExperts];  // slot of a selected expert, 0xff otherwise
   const int lane = tid & 31, warp = tid >> 5;
   const int E = p.E, K = p.top_k;
   // softmax of each row (warp per row; fixed-order sums)
@@ -106,33 +104,36 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
     s_sel[r][e] = beat < K;
   }
   sync();
-  // slot = rank of the expert id among the row's selected experts
-  for (int idx = tid; idx < R * E; idx += nthreads) {
-    const int r = idx / E, e = idx - r * E;
-    if (!s_sel[r][e]) continue;
-    int slot = 0;
-    for (int f = 0; f < e; ++f) slot += s_sel[r][f];
-    if (slot >= K) continue;  // only with NaN probabilities, which break the total order
-    p.ids[r * K + slot] = e;
-    p.gates[r * K + slot] = s_p[r][e];
-    s_ids[r][slot] = e;
+  // slots: the selected experts of a row in ascending id (warp per row, ballots)
+  if (warp < R) {
+    const int r = warp;
+    int base = 0;
+    for (int e0 = 0; e0 < E; e0 += 32) {
+      const int e = e0 + lane;
+      const bool sel = e < E && s_sel[r][e];
+      const unsigned m = __ballot_sync(0xffffffffu, sel);
+      const int slot = base + __popc(m & ((1u << lane) - 1u));
+      const bool ok = sel && slot < K;  // slot >= K only with NaN probabilities
+      if (ok) {
+        p.ids[r * K + slot] = e;
+        p.gates[r * K + slot] = s_p[r][e];
+      }
+      if (e < E) s_slot[r][e] = ok ? (unsigned char)slot : (unsigned char)0xff;
+      base += __popc(m);
+    }
   }
   sync();
-  // bucketing: thread e counts its (row, slot) entries in row order
-  for (int e = tid; e < E; e += nthreads) {
-    int n = 0;
-    for (int r = 0; r < R; ++r)
-      for (int s = 0; s < K; ++s) n += (s_ids[r][s] == e);
-    s_cnt[e] = n;
-  }
-  sync();
+  // bucketing by one warp: per-expert row counts, their exclusive prefix, the
+  // touched experts in ascending id after the shared ones, and each expert's
+  // (row, slot) entries in row order
   if (warp == 0) {
-    // exclusive prefix sum of the counts and of the touched flags, 8 experts per lane
     int base_c = 0, base_t = 0;
     for (int e0 = 0; e0 < E; e0 += 32) {
-      int e = e0 + lane;
-      int c = e < E ? s_cnt[e] : 0;
-      int t = c > 0;
+      const int e = e0 + lane;
+      int c = 0;
+      if (e < E)
+        for (int r = 0; r < R; ++r) c += s_slot[r][e] != 0xff;
+      const int t = c > 0;
       int ic = c, it = t;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -141,8 +142,14 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
         if (lane >= o) { ic += vc; it += vt; }
       }
       if (e < E) {
-        s_off[e] = base_c + ic - c;
+        int off = base_c + ic - c;
+        p.counts[e] = c;
+        p.offsets[e] = off;
         if (t) p.mats[p.S + base_t + it - 1] = e;
+        for (int r = 0; r < R; ++r) {
+          const int sl = s_slot[r][e];
+          if (sl != 0xff) p.rowlist[off++] = r | (sl << 8);
+        }
       }
       base_c += __shfl_sync(0xffffffffu, ic, 31);
       base_t += __shfl_sync(0xffffffffu, it, 31);
@@ -151,20 +158,10 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
     if (lane == 0) {
       *p.n_mats = p.S + base_t;
       if (p.touched) {
-        p.touched[0] += base_t;
-        p.touched[1] += 1;
+        atomicAdd(&p.touched[0], base_t);
+        atomicAdd(&p.touched[1], 1);
       }
     }
-  }
-  sync();
-  for (int e = tid; e < E; e += nthreads) {
-    int o = s_off[e];
-    p.counts[e] = s_cnt[e];
-    p.offsets[e] = o;
-    if (s_cnt[e] == 0) continue;
-    for (int r = 0; r < R; ++r)
-      for (int s = 0; s < K; ++s)
-        if (s_ids[r][s] == e) p.rowlist[o++] = r | (s << 8);
   }
 }
 
