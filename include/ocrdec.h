@@ -91,7 +91,8 @@ typedef struct {
 /* ---- setup ---------------------------------------------------------------- */
 
 /* Validates the config (positive sizes, n_heads*head_dim == d_model, head_dim
- * 64 or 128, sizes multiples of 8, top_k <= min(n_experts, 8), n_experts <= 128,
+ * 64 or 128, d_model <= 2048, d_model and the FFN widths multiples of 64,
+ * vocab a multiple of 8, top_k <= min(n_experts, 8), n_experts <= 128,
  * max_k <= 3, kv_capacity <= 8192).
  * *out receives a context that must be released with ocrdec_destroy. */
 OCRDEC_API int ocrdec_create(const ocrdec_config* cfg, ocrdec_ctx** out);
@@ -227,20 +228,31 @@ OCRDEC_API const char* ocrdec_strerror(int status);
 
 /* ---- single-kernel entry points (kernel-level parity tests) ----------------- */
 
-/* y[r][n] = sum_k W[n][k] * bf16(x[r][k] * inv_rms(x[r]) * g[k]) for r < R <= 8:
- * the RMSNorm-prologue GEMV used for Q/K/V, router, FFN inputs and LM head.
- * W bf16 [N][K], x float32 [R][K], g bf16 [K], y float32 [R][N].
- * dev_scratch: at least ocrdec_op_scratch_bytes() bytes. */
+/* RMSNorm followed by a linear map, the first step of every sub-layer of the
+ * decoder (pre-norm transformer block; the MoE router, Q/K/V and FFN inputs):
+ *   y[r][n] = sum_k W[n][k] * bf16(x[r][k] * rsqrt(mean_k x[r][k]^2 + eps) * g[k])
+ * for r < R, accumulated in float32 (bfloat16 operands, float32 products).
+ * Layouts (device pointers, owned by the caller): W bfloat16 [N][K] row-major
+ * (16-byte aligned), x float32 [R][K], g bfloat16 [K], y float32 [R][N].
+ * Sizes: 1 <= R <= 8, N >= 1, K a multiple of 64 with 64 <= K <= 2048.
+ * dev_scratch: ocrdec_op_scratch_bytes() bytes, 256-byte aligned; the call
+ * clears what it needs.  Asynchronous on `stream`.  Returns OCRDEC_OK,
+ * OCRDEC_EINVAL (sizes, alignment, NULL pointers) or OCRDEC_ECUDA (tensor
+ * map or launch failure); a device wait that gives up stores
+ * OCRDEC_ETIMEOUT in the first int of dev_scratch. */
 OCRDEC_API int ocrdec_op_norm_gemv(const void* dev_W, const float* dev_x, const void* dev_g, float eps,
                         int R, int N, int K, float* dev_y, void* dev_scratch, ocrdec_stream stream);
 
-/* Final norm + LM head + greedy argmax: tok[r] = argmax_n (W[n] . bf16(RMSNorm(x[r])))
- * with ties to the lower index; optional dev_logits[R][N] (float32) if non-NULL.
- * dev_scratch holds the per-block partial maxima. */
+/* Final RMSNorm, LM head and greedy argmax - the verifier's token choice in
+ * greedy speculative decoding: tok[r] = argmax_n (W[n] . bf16(RMSNorm(x[r]) * g))
+ * with ties to the lower index; if dev_logits is not NULL it also receives
+ * the float32 logits [R][N].  Layouts, sizes, scratch, stream and errors as
+ * for ocrdec_op_norm_gemv; dev_tok is int32 [R]. */
 OCRDEC_API int ocrdec_op_lm_argmax(const void* dev_W, const float* dev_x, const void* dev_g, float eps,
                         int R, int N, int K, int32_t* dev_tok, float* dev_logits,
                         void* dev_scratch, ocrdec_stream stream);
 
+/* Bytes of scratch the two single-kernel entry points need on the current device. */
 OCRDEC_API size_t ocrdec_op_scratch_bytes(void);
 
 /* The same final norm + LM head + greedy argmax as ocrdec_op_lm_argmax, for

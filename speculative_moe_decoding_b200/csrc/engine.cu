@@ -95,9 +95,10 @@ bool config_ok(const ocrdec_config* c) {
     if (v <= 0) return false;
   if (c->n_heads * c->head_dim != c->d_model) return false;
   if (c->head_dim != 64 && c->head_dim != 128) return false;
-  if (c->d_model % 8 || c->expert_ffn % 8 || c->draft_ffn % 8 || c->vocab % 8) return false;
+  // GEMV reduction dims are whole 64-column chunks; vocab rows need only 16-byte rows
+  if (c->d_model % kChunk || c->expert_ffn % kChunk || c->draft_ffn % kChunk || c->vocab % 8) return false;
   if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
-  if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % 8)) return false;
+  if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % kChunk)) return false;
   if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
   if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > kMaxExperts || c->top_k + c->n_shared > 127) return false;
   if (c->max_k < 0 || c->max_k > 3) return false;
@@ -1008,7 +1009,7 @@ size_t ocrdec_op_scratch_bytes(void) {
 
 int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps, int R, int N, int K, float* y,
                         void* scratch, ocrdec_stream stream) {
-  if (!W || !x || !g || !y || !scratch || R < 1 || R > kRmax || N < 1 || K < 8 || K % 8 || K > kGemvMaxK)
+  if (!W || !x || !g || !y || !scratch || R < 1 || R > kRmax || N < 1 || K < kChunk || K % kChunk || K > kGemvMaxK)
     return OCRDEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -1042,7 +1043,7 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
 
 int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps, int R, int N, int K, int32_t* tok,
                         float* logits, void* scratch, ocrdec_stream stream) {
-  if (!W || !x || !g || !tok || !scratch || R < 1 || R > kRmax || N < 1 || K < 8 || K % 8 || K > kGemvMaxK)
+  if (!W || !x || !g || !tok || !scratch || R < 1 || R > kRmax || N < 1 || K < kChunk || K % kChunk || K > kGemvMaxK)
     return OCRDEC_EINVAL;
   if ((reinterpret_cast<uintptr_t>(W) & 15) || (reinterpret_cast<uintptr_t>(scratch) & 255)) return OCRDEC_EINVAL;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

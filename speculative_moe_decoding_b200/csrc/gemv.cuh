@@ -2,24 +2,29 @@
 //
 // y[r][n] = sum_k W[n][k] * x[r][k] for the R <= kRmax rows of a pass.  The
 // work is HBM-bound: every weight byte is read once per pass.  The kernel is
-// built around the tensor-memory-access (TMA) unit:
-//   * one producer thread streams weight boxes of 32 rows x 256 columns
-//     (16 KB) into a kStages-deep shared-memory ring with
-//     cp.async.bulk.tensor (3-D tensor map: column, row, expert; no multicast),
-//     each stage completing an mbarrier by transaction bytes.  Columns past K
-//     and rows past N arrive zero-filled, so ragged shapes need no special case;
-//   * each of the kNW consumer warps owns 4 rows of every box: lane l handles
-//     the 16-byte chunk l of the 256-column slice for all 4 rows, with the
-//     matching activation chunk of every pass row loaded once per slice;
-//   * after the last slice a warp reduces its rows across lanes with a fixed
-//     transpose-reduce (xor 16, 8) and butterfly (xor 4, 2, 1), and runs the
-//     epilogue itself - no block-wide barrier per tile.
-// Every output's reduction order is fixed by K alone (slice order, lane, the
-// shuffle tree) - never by R, the row-group width or which rows share the
-// pass - which is what makes the speculative path bit-identical to k = 0.
+// built around the tensor-memory-access (TMA) unit and the tensor cores:
+//   * one producer thread streams weight tiles of 32 rows x 256 columns
+//     (16 KB, two 16-row boxes) into a kStages-deep shared-memory ring with
+//     cp.async.bulk.tensor (4-D tensor map: 64-column chunk, row, chunk index,
+//     expert; 128-byte swizzle; no multicast), each stage completing an
+//     mbarrier by transaction bytes.  Columns past K and rows past N arrive
+//     zero-filled, so ragged shapes need no special case;
+//   * each of the kNW consumer warps owns one 16-row box and one 64-column
+//     quarter of every slice and multiplies it with the pass rows on the
+//     tensor cores (mma m16n8k16, bfloat16 in, float32 accumulate; the up to
+//     8 pass rows are the 8 columns of B), so a 16 KB stage costs a warp four
+//     MMAs instead of hundreds of FMAs - at R = 4 the FMA version was
+//     issue-bound below the HBM roofline;
+//   * after the item's last slice the four column-quarter partials of every
+//     output are added in quarter order through shared memory and the warps
+//     run the epilogue.
+// Every output's reduction order is fixed by K alone (k16 steps, slices,
+// quarters) - never by R or by which rows share the pass: each MMA output
+// column depends on its own B column only.  That is what makes the
+// speculative path bit-identical to k = 0.
 //
-// Work items are (matrix, 32-row tile) pairs handed to CTAs in contiguous
-// ranges.  Dense mode has one matrix; expert mode walks a device-side list of
+// Work items are (matrix, 32-row tile) pairs claimed by CTAs from a per-launch
+// counter.  Dense mode has one matrix; expert mode walks a device-side list of
 // touched experts (shared experts first) so only the experts routed in this
 // pass are streamed.
 #pragma once
@@ -33,14 +38,17 @@ namespace ocrdec {
 constexpr int kNW = 8;                          // consumer warps
 constexpr int kConsumers = kNW * 32;            // consumer threads
 constexpr int kGemvThreads = kConsumers + 32;   // + producer warp
-constexpr int kWarpRows = 4;                    // weight rows per warp per tile
+constexpr int kWarpRows = 4;                    // output rows per warp in the epilogue
 constexpr int kTile = kNW * kWarpRows;          // 32 rows per tile
 constexpr int kSlice = 256;                     // columns per stage
+constexpr int kChunk = 64;                      // columns per 128-byte swizzled row of a box
 constexpr int kBoxRows = 16;                    // rows per TMA box (two boxes per stage)
-constexpr int kStageBytes = kTile * kSlice * 2; // 16 KB of weights per stage
+constexpr int kBoxBytes = kBoxRows * kSlice * 2;  // 8 KB: [4 chunks][16 rows][128 B]
+constexpr int kStageBytes = 2 * kBoxBytes;      // 16 KB of weights per stage
 constexpr int kStages = 4;
 constexpr int kRmax = 8;                        // rows per pass on the GEMV path
-constexpr int kXSliceBytes = kSlice * 2;        // one activation row of a staged bf16 slice (512 B)
+constexpr int kXStride = kSlice * 2 + 16;       // staged activation row (512 B + 16 B pad, ldmatrix-conflict-free)
+constexpr int kRedFloats = 2 * 4 * kTile * 8;   // quarter partials, double-buffered by item
 
 struct GemvShape {
   int N, K;
@@ -157,62 +165,45 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
   }
 }
 
-// 3-D tensor-map load: box (256 columns, 16 rows, 1 matrix) at (c0, row, mat).
-__device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, int c0, int row, int mat,
+
+// 4-D tensor-map load of one box: 4 chunks of 64 columns x 16 rows of matrix
+// `mat`, starting at column chunk c4 and row `row`; shared layout
+// [chunk][row][128 B] with the 128-byte swizzle.
+__device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, int c4, int row, int mat,
                                              uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(row), "r"(mat), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(c4), "r"(mat), "r"(smem_u32(bar))
       : "memory");
 }
 
-// ---- packed float pairs (Blackwell f32x2 FMA) -------------------------------
-typedef unsigned long long f2_t;
-__device__ __forceinline__ f2_t pk2(float lo, float hi) {
-  f2_t r;
-  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-  return r;
+// ---- tensor-core fragments ----------------------------------------------------
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
 }
-__device__ __forceinline__ float2 upk2(f2_t v) {
-  float2 f;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(f.x), "=f"(f.y) : "l"(v));
-  return f;
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t (&b)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(b[0]), "=r"(b[1]) : "r"(addr));
 }
-// acc.{x,y} = fma(a.{x,y}, b.{x,y}, acc.{x,y}), each rounded like a scalar fma
-__device__ __forceinline__ void ffma2(f2_t& acc, f2_t a, f2_t b) {
-  asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(acc) : "l"(a), "l"(b));
-}
-// a bfloat16 pair (low half = element 0) as a float pair
-__device__ __forceinline__ f2_t bf2_to_f2(uint32_t u) {
-  return pk2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
-}
-
-// The 8 elements of one 16-byte weight chunk, or of the matching activation
-// chunk, as 4 float pairs (0,1), (2,3), (4,5), (6,7).
-struct Pairs8 {
-  f2_t p[4];
-};
-
-__device__ __forceinline__ Pairs8 pairs_from_bf16(const uint4& u) {
-  Pairs8 r;
-  r.p[0] = bf2_to_f2(u.x);
-  r.p[1] = bf2_to_f2(u.y);
-  r.p[2] = bf2_to_f2(u.z);
-  r.p[3] = bf2_to_f2(u.w);
-  return r;
+// d += A (16x16, row) * B (16x8, col); bfloat16 in, float32 accumulate
+__device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
 // ---------------------------------------------------------------------------
-// activation sources: 16-byte chunk c16 of pass row r (slot for expert outputs)
+// activation sources: the B operand (row-set entry q = MMA column q)
 // ---------------------------------------------------------------------------
 
 // Rows of a float32 matrix, RMS-normalised, scaled by a gain vector and rounded
-// to bfloat16 (the GEMV input precision), kept as float32 in shared memory for
-// the whole kernel (K = model width).  The raw rows arrive by bulk copy; each
-// is then normalised in place into two planes: plane 0 holds elements
-// 8c..8c+3 of every 16-byte chunk c, plane 1 elements 8c+4..8c+7, so a lane's
-// two 16-byte loads are consecutive across the warp.
+// to bfloat16 (the GEMV input precision), kept in shared memory for the whole
+// kernel as bfloat16 rows of K + 8 elements (the pad makes the eight rows of
+// an ldmatrix fall in distinct banks).  Rows past R are zero.
 struct SrcNorm {
   struct Params {
     const float* x;
@@ -223,10 +214,9 @@ struct SrcNorm {
   };
   static constexpr bool kSmem = true;    // activations live in shared memory (prologue)
   static constexpr bool kStaged = false; // activations are not part of the weight stages
-  static constexpr int kBytesPerElem = 4;
-  static constexpr int kMaxPer = 16;     // elements per thread per row: K <= 16 * 256
+  static constexpr int kG = 2;           // float4 groups per thread per row: K <= 2048
+  __host__ __device__ static constexpr size_t smem_bytes(int K) { return (size_t)kRmax * (K + 8) * 2; }
 
-  static constexpr int kG = kMaxPer / 4;  // float4 groups per thread per row (K <= 4096)
   // Gains are weights: loaded before the dependency wait.
   struct Pre {
     float4 g[kG];
@@ -242,110 +232,93 @@ struct SrcNorm {
       }
     }
   }
-  // One thread, right after the dependency wait: copy Rc raw rows into xs.
-  // Rc is a bound known at launch (the pass's row count is read in parallel),
-  // so the copies wait on no other load; source rows are clamped to the
-  // kRmax-row buffers they index.
-  __device__ static void issue(const Params& p, int K, int Rc, float* xs, uint64_t* xbar) {
-    if (Rc <= 0) return;
-    mbar_arrive_expect_tx(xbar, (uint32_t)(Rc * K * 4));
-    for (int r = 0; r < Rc; ++r) {
-      const int src = p.row_src ? min(max(p.row_src[r], 0), kRmax - 1) : r;
-      bulk_g2s(xs + r * K, p.x + (long long)src * p.ldx, K * 4, xbar);
-    }
-  }
 
-  // All consumer threads.  Thread t owns the float4 groups t, t + 256, ... of
-  // each row; a group of raw elements [4m, 4m + 4) is plane (m & 1) at offset
-  // (m >> 1) * 4 - contiguous in both layouts - so each group is read, scaled
-  // and written back as one float4.  The sums of squares of all rows are formed
-  // together (one barrier); a row is rewritten in place only once every thread
-  // has read it, which the barrier after each row's reads guarantees.
-  __device__ static void prologue(const Params& p, int K, int R, int Rc, float* xs, float* red, uint64_t* xbar,
-                                  int* status, int tid, const Pre& pre) {
-    const int ng = K / 4;
-    if (Rc > 0) mbar_wait(xbar, 0, status);
+  // All consumer threads, after the dependency wait.  Thread t owns the float4
+  // groups t, t + 256 of each row, read straight from L2 (the rows were just
+  // written by the previous kernel); rows go four at a time: sums of squares,
+  // one barrier, then the scaled bfloat16 values.
+  __device__ static void prologue(const Params& p, int K, int R, unsigned char* xsm, float* red, int tid,
+                                  const Pre& pre) {
+    bf16* xb = reinterpret_cast<bf16*>(xsm);
+    const int ld = K + 8, ng = K / 4;
     const int lane = tid & 31, warp = tid >> 5;
-    const int half = K / 2;
-    float a[kRmax];
-    float4 v[kG];
+    for (int rb = 0; rb < kRmax; rb += 4) {
+      if (rb >= R) {  // zero rows: MMA columns past R stay finite
 #pragma unroll
-    for (int r = 0; r < kRmax; ++r) {
-      a[r] = 0.f;
-      if (r < R) {
-        const float4* row = reinterpret_cast<const float4*>(xs + r * K);
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+          for (int j = 0; j < kG; ++j) {
+            int m = tid + j * kConsumers;
+            if (m < ng) *reinterpret_cast<uint2*>(xb + (rb + rr) * ld + 4 * m) = make_uint2(0u, 0u);
+          }
+        continue;
+      }
+      float4 v[4][kG];
+      float a[4];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = rb + rr;
+        a[rr] = 0.f;
+        const int src = r < R ? (p.row_src ? min(max(p.row_src[r], 0), kRmax - 1) : r) : 0;
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          int m = tid + j * kConsumers;
+          v[rr][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r < R && m < ng) v[rr][j] = __ldcg(reinterpret_cast<const float4*>(p.x + (long long)src * p.ldx) + m);
+        }
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          a[rr] = __fmaf_rn(v[rr][j].x, v[rr][j].x, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].y, v[rr][j].y, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].z, v[rr][j].z, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].w, v[rr][j].w, a[rr]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) a[rr] = __fadd_rn(a[rr], __shfl_xor_sync(0xffffffffu, a[rr], o));
+      if (lane == 0)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) red[(rb + rr) * kNW + warp] = a[rr];
+      named_sync(1, kConsumers);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = rb + rr;
+        float sc = 0.f;
+        if (r < R) {
+          float ss = 0.f;
+#pragma unroll
+          for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
+          sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
+        }
 #pragma unroll
         for (int j = 0; j < kG; ++j) {
           int m = tid + j * kConsumers;
           if (m < ng) {
-            float4 t = row[m];
-            if (r == 0) v[j] = t;
-            a[r] = __fmaf_rn(t.x, t.x, a[r]);
-            a[r] = __fmaf_rn(t.y, t.y, a[r]);
-            a[r] = __fmaf_rn(t.z, t.z, a[r]);
-            a[r] = __fmaf_rn(t.w, t.w, a[r]);
+            uint2 o;
+            o.x = pack2(__fmul_rn(__fmul_rn(v[rr][j].x, sc), pre.g[j].x), __fmul_rn(__fmul_rn(v[rr][j].y, sc), pre.g[j].y));
+            o.y = pack2(__fmul_rn(__fmul_rn(v[rr][j].z, sc), pre.g[j].z), __fmul_rn(__fmul_rn(v[rr][j].w, sc), pre.g[j].w));
+            *reinterpret_cast<uint2*>(xb + r * ld + 4 * m) = o;
           }
         }
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1)
-#pragma unroll
-      for (int r = 0; r < kRmax; ++r) a[r] = __fadd_rn(a[r], __shfl_xor_sync(0xffffffffu, a[r], o));
-    if (lane == 0)
-#pragma unroll
-      for (int r = 0; r < kRmax; ++r)
-        if (r < R) red[r * kNW + warp] = a[r];
-    named_sync(1, kConsumers);  // sums posted; row 0 read by every thread
-    for (int r = 0; r < R; ++r) {
-      float ss = 0.f;
-#pragma unroll
-      for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
-      const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
-      float* row = xs + r * K;
-#pragma unroll
-      for (int j = 0; j < kG; ++j) {
-        int m = tid + j * kConsumers;
-        if (m < ng) {
-          float4 o;
-          o.x = round_bf(__fmul_rn(__fmul_rn(v[j].x, sc), pre.g[j].x));
-          o.y = round_bf(__fmul_rn(__fmul_rn(v[j].y, sc), pre.g[j].y));
-          o.z = round_bf(__fmul_rn(__fmul_rn(v[j].z, sc), pre.g[j].z));
-          o.w = round_bf(__fmul_rn(__fmul_rn(v[j].w, sc), pre.g[j].w));
-          *reinterpret_cast<float4*>(row + (m & 1) * half + (m >> 1) * 4) = o;
-        }
-      }
-      if (r + 1 < R) {
-        const float4* nrow = reinterpret_cast<const float4*>(xs + (r + 1) * K);
-#pragma unroll
-        for (int j = 0; j < kG; ++j) {
-          int m = tid + j * kConsumers;
-          if (m < ng) v[j] = nrow[m];
-        }
-      }
-      named_sync(1, kConsumers);  // row r written; row r + 1 read by every thread
-    }
-    if (R == 0) named_sync(1, kConsumers);
+    named_sync(1, kConsumers);
   }
 
-  __device__ static Pairs8 chunk(const Params& p, const float* xs, const unsigned char* xstage, int K, int q, int r,
-                                 int slot, int c16, int lane) {
-    const float* base = xs + r * K + c16 * 4;
-    float4 lo = *reinterpret_cast<const float4*>(base);
-    float4 hi = *reinterpret_cast<const float4*>(base + K / 2);
-    Pairs8 o;
-    o.p[0] = pk2(lo.x, lo.y);
-    o.p[1] = pk2(lo.z, lo.w);
-    o.p[2] = pk2(hi.x, hi.y);
-    o.p[3] = pk2(hi.z, hi.w);
-    return o;
+  // Shared address of B-fragment row data for ldmatrix.x2: row-set entry q of
+  // this lane (lane & 7), column k0 (+8 for lanes 8..15) of the slice start.
+  __device__ static uint32_t b_base(const unsigned char* xsm, const unsigned char* stage_x, int K, int row, int lane) {
+    return smem_u32(xsm) + (uint32_t)(row * (K + 8) + ((lane >> 3) & 1) * 8) * 2;
   }
+  __device__ static uint32_t b_slice(int slc) { return (uint32_t)slc * kSlice * 2; }
 };
 
 // Rows of a bfloat16 matrix in global memory: row (row_src[r] * nslot + slot).
 // The producer copies each slice of the item's rows into the stage next to the
-// weight box (row-set entry q at offset q * 512 B), so consumers read them from
-// shared memory.
+// weight boxes (row-set entry q at offset q * kXStride), so consumers read them
+// from shared memory.
 struct SrcBf16 {
   struct Params {
     const bf16* x;
@@ -355,18 +328,17 @@ struct SrcBf16 {
   };
   static constexpr bool kSmem = false;
   static constexpr bool kStaged = true;
-  static constexpr int kBytesPerElem = 0;
+  __host__ __device__ static constexpr size_t smem_bytes(int) { return 0; }
   struct Pre {};
   __device__ static void pre_wait(const Params&, int, int, Pre&) {}
-  __device__ static void issue(const Params&, int, int, float*, uint64_t*) {}
-  __device__ static void prologue(const Params&, int, int, int, float*, float*, uint64_t*, int*, int, const Pre&) {}
+  __device__ static void prologue(const Params&, int, int, unsigned char*, float*, int, const Pre&) {}
   __device__ static const bf16* row_ptr(const Params& p, int r, int slot) {
     return p.x + (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
   }
-  __device__ static Pairs8 chunk(const Params& p, const float*, const unsigned char* xstage, int K, int q, int r,
-                                 int slot, int c16, int lane) {
-    return pairs_from_bf16(*reinterpret_cast<const uint4*>(xstage + q * kXSliceBytes + lane * 16));
+  __device__ static uint32_t b_base(const unsigned char*, const unsigned char* stage_x, int, int, int lane) {
+    return smem_u32(stage_x) + (uint32_t)((lane & 7) * kXStride + ((lane >> 3) & 1) * 16);
   }
+  __device__ static uint32_t b_slice(int) { return 0; }
 };
 
 // ---------------------------------------------------------------------------
@@ -568,10 +540,6 @@ __device__ __forceinline__ void epi_init<EpiArgmax>(int tid) { EpiArgmax::init(t
 // the kernel
 // ---------------------------------------------------------------------------
 
-// Streams the tiles of one work item through the ring and returns the warp's
-// reduced values: lane L = 8 i + q gets local row i (0..3) for row-set entry q.
-// NR = live rows of the item (row-set entries 0..NR-1); the arithmetic of a
-// row does not depend on NR.
 // Work item -> (matrix, tile, slice range).  Dense mode may split a tile's
 // slices into s.kparts parts (items tile * kparts + part).
 struct ItemPos {
@@ -597,96 +565,28 @@ __device__ __forceinline__ ItemPos item_pos(const GemvShape& s, int item) {
   return ip;
 }
 
+
 template <class Src>
 constexpr int stage_stride() {
-  return kStageBytes + (Src::kStaged ? kRmax * kXSliceBytes : 0);
+  // weights, then (staged sources) the slice rows; 1 KB-aligned for the swizzle
+  return Src::kStaged ? (kStageBytes + kRmax * kXStride + 1023) / 1024 * 1024 : kStageBytes;
 }
 
-template <int NR, class Src>
-__device__ __forceinline__ float consume_item(const GemvShape& s, const typename Src::Params& sp, const float* xs,
-                                              const unsigned char* stages, uint64_t* full_bar, uint64_t* empty_bar,
-                                              uint32_t& it, const RowSet& rs, const int (&srow)[kWarpRows],
-                                              int nch, int lane, int sl0, int sl1) {
-  f2_t acc[kWarpRows][NR > 0 ? NR : 1];
-#pragma unroll
-  for (int i = 0; i < kWarpRows; ++i)
-#pragma unroll
-    for (int q = 0; q < (NR > 0 ? NR : 1); ++q) acc[i][q] = 0ull;
-
-  for (int sl = sl0; sl < sl1; ++sl, ++it) {
-    const int st = it % kStages;
-    mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
-    const int c = sl * 32 + lane;  // this lane's 16-byte chunk of the row
-    if (NR > 0 && c < nch) {
-      const unsigned char* stg = stages + st * stage_stride<Src>();
-      Pairs8 xv[NR > 0 ? NR : 1];
-#pragma unroll
-      for (int q = 0; q < NR; ++q) xv[q] = Src::chunk(sp, xs, stg + kStageBytes, s.K, q, rs.r(q), rs.slot(q), c, lane);
-      const unsigned char* w_st = stg + lane * 16;
-#pragma unroll
-      for (int i = 0; i < kWarpRows; ++i) {
-        Pairs8 wv = pairs_from_bf16(*reinterpret_cast<const uint4*>(w_st + srow[i] * (kSlice * 2)));
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-#pragma unroll
-          for (int q = 0; q < NR; ++q) ffma2(acc[i][q], wv.p[e], xv[q].p[e]);
-      }
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty_bar[st]);
-  }
-
-  // per lane: even + odd partial; then transpose over lane bits 4, 3 and a
-  // butterfly over bits 2..0, after which lane L holds local row L >> 3
-  float out = 0.f;
-#pragma unroll
-  for (int q = 0; q < NR; ++q) {
-    float r4[kWarpRows];
-#pragma unroll
-    for (int i = 0; i < kWarpRows; ++i) {
-      float2 t = upk2(acc[i][q]);
-      r4[i] = __fadd_rn(t.x, t.y);
-    }
-    const bool up16 = lane & 16;
-    float a0 = __fadd_rn(up16 ? r4[2] : r4[0], __shfl_xor_sync(0xffffffffu, up16 ? r4[0] : r4[2], 16));
-    float a1 = __fadd_rn(up16 ? r4[3] : r4[1], __shfl_xor_sync(0xffffffffu, up16 ? r4[1] : r4[3], 16));
-    const bool up8 = lane & 8;
-    float b = __fadd_rn(up8 ? a1 : a0, __shfl_xor_sync(0xffffffffu, up8 ? a0 : a1, 8));
-    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 4));
-    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 2));
-    b = __fadd_rn(b, __shfl_xor_sync(0xffffffffu, b, 1));
-    if ((lane & 7) == q) out = b;
-  }
-  return out;
-}
-
-template <int RG, class Src>
-__device__ __forceinline__ float consume_dispatch(int n, const GemvShape& s, const typename Src::Params& sp,
-                                                  const float* xs, const unsigned char* stages, uint64_t* full_bar,
-                                                  uint64_t* empty_bar, uint32_t& it, const RowSet& rs,
-                                                  const int (&srow)[kWarpRows], int nch, int lane, int sl0,
-                                                  int sl1) {
-#define OCRDEC_CONSUME(NRV) \
-  consume_item<NRV, Src>(s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane, sl0, sl1)
-  if (n <= 0) return OCRDEC_CONSUME(0);
-  if (n == 1 || RG == 1) return OCRDEC_CONSUME(1);
-  if (n == 2 || RG == 2) return OCRDEC_CONSUME((RG >= 2 ? 2 : 1));
-  if (n == 3) return OCRDEC_CONSUME((RG >= 3 ? 3 : 1));
-  if (n == 4 || RG == 4) return OCRDEC_CONSUME((RG >= 4 ? 4 : 1));
-  if (n == 5) return OCRDEC_CONSUME((RG >= 5 ? 5 : 1));
-  if (n == 6) return OCRDEC_CONSUME((RG >= 6 ? 6 : 1));
-  if (n == 7) return OCRDEC_CONSUME((RG >= 7 ? 7 : 1));
-  return OCRDEC_CONSUME((RG >= 8 ? 8 : 1));
-#undef OCRDEC_CONSUME
+// Dynamic shared memory of one CTA: 1 KB alignment slack, the ring, the
+// source's rows and the quarter partials.
+template <class Src>
+constexpr size_t gemv_smem_bytes(int K) {
+  return 1024 + (size_t)kStages * stage_stride<Src>() + Src::smem_bytes(K) + kRedFloats * 4;
 }
 
 template <int RG, class Src, class Epi>
-__global__ void __launch_bounds__(kGemvThreads, RG >= 8 ? 1 : 2)
+__global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
-  extern __shared__ __align__(1024) unsigned char smem[];
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], xbar;
-  __shared__ int s_tag[kStages];  // item of the stage's slice (set with its first slice), -1 = end
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ int s_tag[kStages];               // item of the stage's slice (set with its first slice), -1 = end
+  __shared__ int s_rs[kStages][kRmax + 1];     // expert mode: the item's row set (n, entries), with its first slice
   __shared__ float red_pro[kRmax * kNW];
   __shared__ int s_abort;
 
@@ -694,8 +594,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int warp = tid >> 5, lane = tid & 31;
   TraceMarks tm;  // trace (consumer thread 0): wait returned, prologue done, main loop done
   constexpr int kStride = stage_stride<Src>();
-  unsigned char* stages = smem;
-  float* xs = reinterpret_cast<float*>(smem + kStages * kStride);
+  // the 128-byte swizzle repeats every 1 KB: the ring starts on a 1 KB boundary
+  unsigned char* stages = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  unsigned char* xsm = stages + kStages * kStride;
+  float* red = reinterpret_cast<float*>(xsm + Src::smem_bytes(s.K));
   const bool paired = s.pair_half != 0;
 
   if (tid == 0) {
@@ -703,7 +605,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       mbar_init(&full_bar[i], Src::kStaged ? 2 : 1);
       mbar_init(&empty_bar[i], kNW);
     }
-    mbar_init(&xbar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -713,16 +614,24 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     if (lane != 0) return;
     uint32_t it = 0;
     int R = 0;
-    RowSet prs;  // rows of the current item (bf16 sources staged with the weights)
+    RowSet prs;  // rows of the current item (expert mode / staged sources)
     int prs_m = -1;
     auto stage_wait = [&](int st) {
       // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
       // stays uniform so the block always terminates
       if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
     };
-    // Stage = weight box (one arrival with its transaction bytes) and, for a
-    // staged bf16 source, the item's activation slice rows (a second arrival,
-    // declared only after the dependency wait).
+    auto rows_of = [&](int m) {
+      if (m != prs_m) {
+        int ce;
+        bool sh;
+        mat_info(s, m, R, &ce, &sh, &prs);
+        prs_m = m;
+      }
+    };
+    // Stage = two weight boxes (one arrival with their transaction bytes) and,
+    // for a staged bf16 source, the item's activation slice rows (a second
+    // arrival, declared only after the dependency wait).
     auto issue_w = [&](int item, int m, int t, int slc, bool first) {
       int ce;
       bool sh;
@@ -733,20 +642,21 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       const int st = it % kStages;
       stage_wait(st);
       s_tag[st] = first ? item : -2;
+      if (first && s.mats) {
+        rows_of(m);
+        s_rs[st][0] = prs.n;
+#pragma unroll
+        for (int q = 0; q < kRmax; ++q) s_rs[st][1 + q] = prs.e[q];
+      }
       mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
       unsigned char* dst = stages + st * kStride;
-      tma_load_box(dst, map, slc * kSlice, r0, ce, &full_bar[st]);
-      tma_load_box(dst + kStageBytes / 2, map, slc * kSlice, r1, ce, &full_bar[st]);
+      tma_load_box(dst, map, slc * (kSlice / kChunk), r0, ce, &full_bar[st]);
+      tma_load_box(dst + kBoxBytes, map, slc * (kSlice / kChunk), r1, ce, &full_bar[st]);
       ++it;
     };
     auto issue_x = [&](uint32_t j, int m, int slc) {
       if (!Src::kStaged) return;
-      if (m != prs_m) {
-        int ce;
-        bool sh;
-        mat_info(s, m, R, &ce, &sh, &prs);
-        prs_m = m;
-      }
+      rows_of(m);
       const int st = j % kStages;
       unsigned char* dst = stages + st * kStride + kStageBytes;
       const int cols = min(kSlice, s.K - slc * kSlice);
@@ -754,7 +664,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
       for (int q = 0; q < kRmax; ++q)
         if (q < prs.n)
-          bulk_g2s(dst + q * kXSliceBytes,
+          bulk_g2s(dst + q * kXStride,
                    SrcBf16::row_ptr(reinterpret_cast<const SrcBf16::Params&>(sp), prs.r(q), prs.slot(q)) + slc * kSlice,
                    cols * 2, &full_bar[st]);
     };
@@ -831,17 +741,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   typename Src::Pre pre;
   Src::pre_wait(sp, s.K, tid, pre);
   pdl_wait();
-  // rows copied for a normalised source: the pass bound of this variant (the
-  // engine's row buffers hold kRmax rows) or the exact static count
-  const int Rc = s.nrows ? min(RG, kRmax) : min(s.rows_static, kRmax);
   if (tid == 0) {
     tm.t0 = gtimer();
-    Src::issue(sp, s.K, Rc, xs, &xbar);
     s_abort = status_bad(s.status);
   }
   named_sync(1, kConsumers);
   if (s_abort) {
-    if (Src::kSmem && tid == 0 && Rc > 0) mbar_wait(&xbar, 0, s.status);  // the row copies land first
     // consume the producer's stages up to its end marker so it can finish
     uint32_t it = 0;
     while (true) {
@@ -858,22 +763,30 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   pdl_trigger();
 
   const int R = min(pass_rows(s), RG);
-  const int nch = s.K / 8;  // 16-byte chunks per row
   __shared__ int s_last_part;
 
   epi_init<Epi>(tid);
-  if (Src::kSmem) Src::prologue(sp, s.K, R, Rc, xs, red_pro, &xbar, s.status, tid, pre);
-  else named_sync(1, kConsumers);
+  Src::prologue(sp, s.K, R, xsm, red_pro, tid, pre);
+  if (!Src::kSmem) named_sync(1, kConsumers);
   if (tid == 0) tm.t1 = gtimer();
 
+  // this warp's share of every stage: box g (16 rows), column quarter kq
+  const int g = warp & 1, kq = warp >> 1;
+  const int nchunks = s.K / kChunk;
+  // A fragments (ldmatrix.x4): lane -> row (lane & 7) + 8 * bit 3, chunk +1 for lanes 16..31
+  const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8;
+  const uint32_t a_off = (uint32_t)(g * kBoxBytes + kq * (kBoxRows * 128) + a_row * 128);
+  const int a_sw = a_row & 7, a_hi = lane >> 4;
+  // epilogue mapping: lane L = 8 i + q takes local row i, row-set entry q
+  const int ep_i = lane >> 3, ep_q = lane & 7;
+  const int ep_srow = stage_row(paired, warp, ep_i);
+
   uint32_t it = 0;
-  int cur_m = -1;
+  int nitem = 0;
   RowSet rs;
-  int ce = 0;
-  bool sh = false;
-  int srow[kWarpRows];
+  rs.n = R;
 #pragma unroll
-  for (int i = 0; i < kWarpRows; ++i) srow[i] = stage_row(paired, warp, i);
+  for (int q = 0; q < kRmax; ++q) rs.e[q] = q;
 
   while (true) {
     const int st0 = it % kStages;
@@ -886,13 +799,46 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       break;
     }
     const ItemPos ip = item_pos(s, item);
-    if (ip.m != cur_m) {
-      mat_info(s, ip.m, R, &ce, &sh, &rs);
-      cur_m = ip.m;
+    if (s.mats) {
+      rs.n = s_rs[st0][0];
+#pragma unroll
+      for (int q = 0; q < kRmax; ++q) rs.e[q] = s_rs[st0][1 + q];
     }
+    // B rows of this lane: row-set entry (lane & 7)
+    const int brow = rs.r_sel(lane & 7);
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int sl = ip.sl0; sl < ip.sl1; ++sl, ++it) {
+      const int st = it % kStages;
+      mbar_wait(&full_bar[st], (it / kStages) & 1, s.status);
+      if (sl * (kSlice / kChunk) + kq < nchunks) {
+        const unsigned char* stg = stages + st * kStride;
+        const uint32_t a_base = smem_u32(stg) + a_off;
+        const uint32_t b_addr = Src::b_base(xsm, stg + kStageBytes, s.K, brow, lane) + Src::b_slice(sl) +
+                                (uint32_t)kq * kChunk * 2;
+#pragma unroll
+        for (int k16 = 0; k16 < kChunk / 16; ++k16) {
+          uint32_t a[4], b[2];
+          ldsm_x4(a_base + (uint32_t)((((2 * k16 + a_hi) ^ a_sw)) << 4), a);
+          ldsm_x2(b_addr + k16 * 32, b);
+          mma_bf16(d, a, b);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty_bar[st]);
+    }
+    // quarter partials -> shared, then every output adds its quarters in order
+    float* rb = red + (nitem & 1) * (4 * kTile * 8);
+    ++nitem;
+    {
+      const int r = g * kBoxRows + (lane >> 2), c = 2 * (lane & 3);
+      *reinterpret_cast<float2*>(rb + (kq * kTile + r) * 8 + c) = make_float2(d[0], d[1]);
+      *reinterpret_cast<float2*>(rb + (kq * kTile + r + 8) * 8 + c) = make_float2(d[2], d[3]);
+    }
+    named_sync(1, kConsumers);
     WarpOut o;
-    o.v = consume_dispatch<RG, Src>(rs.n, s, sp, xs, stages, full_bar, empty_bar, it, rs, srow, nch, lane, ip.sl0,
-                                    ip.sl1);
+    o.v = __fadd_rn(__fadd_rn(__fadd_rn(rb[(0 * kTile + ep_srow) * 8 + ep_q], rb[(1 * kTile + ep_srow) * 8 + ep_q]),
+                              rb[(2 * kTile + ep_srow) * 8 + ep_q]),
+                    rb[(3 * kTile + ep_srow) * 8 + ep_q]);
     if (s.kparts > 1) {
       // post this part; the tile's last part adds all parts in part order
       float* pt = s.part + ((long long)ip.t * s.kparts) * (kNW * 32);
@@ -908,11 +854,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       o.v = v;
       if (tid == 0) s.tile_counter[ip.t] = 0;
     }
-    o.i = lane >> 3;
-    o.q = lane & 7;
+    o.i = ep_i;
+    o.q = ep_q;
     int r0, r1;
     tile_boxes(s, ip.t, &r0, &r1);
-    o.n = matrix_row(r0, r1, sel(srow, o.i));
+    o.n = matrix_row(r0, r1, ep_srow);
     Epi::apply(ep, s, o, rs, lane);
   }
   named_sync(1, kConsumers);

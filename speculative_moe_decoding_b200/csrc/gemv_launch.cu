@@ -39,20 +39,24 @@ cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap
     if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
     fn = reinterpret_cast<EncodeTiledFn>(p);
   }
-  if ((reinterpret_cast<uintptr_t>(base) & 15) || K % 8 || K <= 0 || N <= 0 || E <= 0) return cudaErrorInvalidValue;
-  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)E};
-  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)K * 2 * N};
-  cuuint32_t box[3] = {kSlice, kBoxRows, 1};
-  cuuint32_t estr[3] = {1, 1, 1};
-  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
-                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+  // 4-D view of the [E][N][K] bfloat16 array: (64-column chunk, row, chunk
+  // index, matrix); a box is 4 chunks x 16 rows, stored with the 128-byte
+  // swizzle that makes the consumers' ldmatrix reads conflict-free
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || K % kChunk || K <= 0 || N <= 0 || E <= 0)
+    return cudaErrorInvalidValue;
+  cuuint64_t dims[4] = {(cuuint64_t)kChunk, (cuuint64_t)N, (cuuint64_t)(K / kChunk), (cuuint64_t)E};
+  cuuint64_t strides[3] = {(cuuint64_t)K * 2, (cuuint64_t)kChunk * 2, (cuuint64_t)K * 2 * N};
+  cuuint32_t box[4] = {kChunk, kBoxRows, kSlice / kChunk, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
 template <class Src>
 static size_t smem_max() {
-  return (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * kGemvMaxK * Src::kBytesPerElem;
+  return gemv_smem_bytes<Src>(kGemvMaxK);
 }
 
 template <int RG, class Src, class Epi>
@@ -93,10 +97,9 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
                               const LaunchCfg& lc) {
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
-  size_t smem = (size_t)kStages * stage_stride<Src>() + (size_t)kRmax * g.s.K * Src::kBytesPerElem;
-  // two CTAs per SM (96 registers a thread) hide each other's latencies; the
-  // eight-row variant needs more registers and runs one CTA per SM
-  const int slots = (RG >= 8 ? 1 : 2) * lc.num_sms;
+  const size_t smem = gemv_smem_bytes<Src>(g.s.K);
+  // two CTAs per SM hide each other's latencies
+  const int slots = 2 * lc.num_sms;
   int grid = g.grid > 0 ? std::min(g.grid, slots) : slots;
   if (!g.s.mats) grid = std::min(grid, g.s.tiles_per_mat * g.s.kparts);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
@@ -112,7 +115,7 @@ static cudaError_t launch_rg(const GemvLaunch& g, const typename Src::Params& sp
 }
 
 cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
-  if (g.s.K % 8 || (g.s.pair_half && (g.s.pair_half % kBoxRows || g.s.N % (2 * g.s.pair_half))))
+  if (g.s.K % kChunk || (g.s.pair_half && (g.s.pair_half % kBoxRows || g.s.N % (2 * g.s.pair_half))))
     return cudaErrorInvalidValue;
   if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
   if (g.s.kparts > 1 && (g.s.mats || !g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;

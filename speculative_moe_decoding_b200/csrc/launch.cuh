@@ -88,7 +88,7 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
 // Raises the dynamic shared-memory limit of every GEMV instantiation to the
 // largest size any launch uses (call outside stream capture, once per device).
 cudaError_t gemv_prepare();
-constexpr int kGemvMaxK = 4096;  // largest K of a normalised (shared-memory) source
+constexpr int kGemvMaxK = 2048;  // largest K of a normalised (shared-memory) source
 constexpr int kWorkSlots = 4;   // GEMV work-counter pairs cycled by a decoder context
 
 

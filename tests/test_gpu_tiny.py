@@ -55,7 +55,9 @@ def _bf16(a):
     return O.bf16_bits_to_f32(synth.f32_to_bf16_bits(a))
 
 
-@pytest.mark.parametrize("R,N,K", [(1, 72, 256), (3, 1280, 1280), (8, 64, 4000), (4, 3840, 1280)])
+# K = 2048 is the largest normalised width; K = 1984 ends in a slice of three
+# 64-column chunks; N values that are not multiples of 32 leave ragged tiles
+@pytest.mark.parametrize("R,N,K", [(1, 72, 256), (3, 1280, 1280), (8, 64, 2048), (4, 3840, 1280), (5, 100, 1984)])
 def test_op_norm_gemv(R, N, K):
     import torch
     from speculative_moe_decoding_b200 import build

@@ -87,3 +87,12 @@ def test_calls_before_setup_fail_cleanly(lib):
         assert lib.ocrdec_strerror(lib.ECAPACITY) == b"KV capacity exceeded"
     finally:
         lib.ocrdec_destroy(ctx)
+
+
+def test_op_argument_checks(lib):
+    """The single-kernel entry points reject widths that are not whole 64-column
+    chunks or exceed 2048, and row counts outside 1..8, before touching the GPU."""
+    p = ctypes.c_void_p(256)  # never dereferenced: validation comes first
+    for R, N, K in [(1, 64, 4000), (1, 64, 1000), (0, 64, 256), (9, 64, 256), (1, 0, 256), (1, 64, 32)]:
+        assert lib.ocrdec_op_norm_gemv(p, p, p, ctypes.c_float(1e-6), R, N, K, p, p, None) == lib.EINVAL
+        assert lib.ocrdec_op_lm_argmax(p, p, p, ctypes.c_float(1e-6), R, N, K, p, None, p, None) == lib.EINVAL
