@@ -96,7 +96,7 @@ attention_kernel(const AttnParams p) {
   // finished before the kernel this one follows
   const int r0 = p.slot_row0[b];
   const int nr = max(0, min(p.slot_nrows[b], kAttnRows));
-  if (tid < nr) s_pos[tid] = p.row_pos[r0 + tid];
+  if (tid < kAttnRows) s_pos[tid] = tid < nr ? p.row_pos[r0 + tid] : -1;  // -1: sees nothing
   if (tid < kAttnRows) {
     s_M[tid] = -INFINITY;
     s_L[tid] = 0.f;
@@ -144,9 +144,9 @@ attention_kernel(const AttnParams p) {
       for (int i = 0; i < n_first; ++i)
         if (!old_chunk(i)) issue(i);
   }
-  if (tid < Dh)
+  if (tid < kAttnMaxDh)
 #pragma unroll
-    for (int i = 0; i < kAttnRows; ++i) qs[i][tid] = qv[i];
+    for (int i = 0; i < kAttnRows; ++i) qs[i][tid] = tid < Dh ? qv[i] : 0.f;
   __syncthreads();
   const bool work = !s_abort && nr > 0;
   pdl_trigger();
@@ -178,8 +178,8 @@ attention_kernel(const AttnParams p) {
       for (int q = 0; q < 4; ++q)
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
-          qr[q][e] = (rb + q < nr && (e < 8 || l8 + 8 < ndc)) ? qs[rb + q][d] : 0.f;
+          const int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
+          qr[q][e] = qs[rb + q][d];  // rows past nr and dims past Dh hold zeros
         }
       for (int ii = 0; ii < ni; ++ii) {
         const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
@@ -213,11 +213,9 @@ attention_kernel(const AttnParams p) {
             a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
             a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
             a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
-            const int r = rb + q;
-            if (l8 == 0 && r < nr) {
-              const bool valid = j < npos && p0 + j <= s_pos[r];
-              sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
-            }
+            const int r = rb + q;  // < kAttnRows; rows past nr have position -1
+            const bool valid = j < npos && p0 + j <= s_pos[r];
+            if (l8 == 0) sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
           }
         }
       }
@@ -234,6 +232,7 @@ attention_kernel(const AttnParams p) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       if (m == -INFINITY) {  // nothing visible to this row in the group
+        for (int u = lane; u < nu; u += 32) sc[r][u] = 0.f;
         if (lane == 0) s_corr[r] = 1.f;
         continue;
       }
@@ -267,11 +266,8 @@ attention_kernel(const AttnParams p) {
         for (int e = 0; e < 4; ++e) o[r][e] = __fmul_rn(o[r][e], cr);
       }
     for (int ii = 0; ii < ni; ++ii) {
-      const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
+      const int npos = chunk_npos(i0 + ii);
       const bf16* Vs = ring + (size_t)ii * 2 * kAttnChunk * Dh + kAttnChunk * Dh;
-      int lim[kAttnRows];  // visible offsets of each row in this chunk
-#pragma unroll
-      for (int r = 0; r < kAttnRows; ++r) lim[r] = r < nr ? min(s_pos[r] - p0 + 1, npos) : 0;
 #pragma unroll
       for (int jj = 0; jj < kAttnWarpPos; ++jj) {
         const int j = warp * kAttnWarpPos + jj;
@@ -284,14 +280,16 @@ attention_kernel(const AttnParams p) {
           uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + j * Dh + lane * 2);
           vv[0] = bf_lo(u); vv[1] = bf_hi(u); vv[2] = 0.f; vv[3] = 0.f;
         }
+        // positions a row does not see have p = 0 exactly and add nothing;
+        // the loads are unconditional so they issue together
+        float pj[kAttnRows];
 #pragma unroll
-        for (int r = 0; r < kAttnRows; ++r) {
-          if (j < lim[r]) {
-            const float pj = sc[r][ii * kAttnChunk + j];
+        for (int r = 0; r < kAttnRows; ++r) pj[r] = sc[r][ii * kAttnChunk + j];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) o[r][e] = __fmaf_rn(pj, vv[e], o[r][e]);
-          }
-        }
+        for (int r = 0; r < kAttnRows; ++r)
+          if (r < nr)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o[r][e] = __fmaf_rn(pj[r], vv[e], o[r][e]);
       }
     }
     __syncthreads();  // ring buffers and scores are free again

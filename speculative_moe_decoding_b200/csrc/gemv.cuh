@@ -509,17 +509,53 @@ struct EpiArgmax {
     named_sync(1, kConsumers);
     if (!last) return false;
     __threadfence();
-    if (tid < R) {
-      float bv = -INFINITY;
-      int bi = 0x7fffffff;
-      const volatile float2* part = p.partial;
-      for (int b = 0; b < (int)gridDim.x; ++b) {
-        float ev = part[b * kRmax + tid].x;
-        int ei = __float_as_int(part[b * kRmax + tid].y);
-        if (ev > bv || (ev == bv && ei < bi)) { bv = ev; bi = ei; }
+    // every consumer thread takes the partials b = tid, tid + 256, ... of each
+    // row (all loads in flight together); then warps, then the 8 warp results.
+    // (value, lower index) is a total order, so the grouping cannot change it.
+    __shared__ float m_v[kNW][kRmax];
+    __shared__ int m_i[kNW][kRmax];
+    const int lane = tid & 31, warp = tid >> 5;
+    float bv[kRmax];
+    int bi[kRmax];
+#pragma unroll
+    for (int r = 0; r < kRmax; ++r) {
+      bv[r] = -INFINITY;
+      bi[r] = 0x7fffffff;
+    }
+    for (int b = tid; b < (int)gridDim.x; b += kConsumers) {
+      float2 e[kRmax];
+#pragma unroll
+      for (int r = 0; r < kRmax; ++r)
+        if (r < R) e[r] = __ldcg(p.partial + b * kRmax + r);
+#pragma unroll
+      for (int r = 0; r < kRmax; ++r)
+        if (r < R) {
+          const int ei = __float_as_int(e[r].y);
+          if (e[r].x > bv[r] || (e[r].x == bv[r] && ei < bi[r])) { bv[r] = e[r].x; bi[r] = ei; }
+        }
+    }
+#pragma unroll
+    for (int r = 0; r < kRmax; ++r) {
+      if (r >= R) break;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xffffffffu, bv[r], o);
+        const int oi = __shfl_xor_sync(0xffffffffu, bi[r], o);
+        if (ov > bv[r] || (ov == bv[r] && oi < bi[r])) { bv[r] = ov; bi[r] = oi; }
       }
-      p.tok[(p.row_dst ? p.row_dst[tid] : tid) * p.tok_stride] = bi;
-      s_tok[tid] = bi;
+      if (lane == 0) {
+        m_v[warp][r] = bv[r];
+        m_i[warp][r] = bi[r];
+      }
+    }
+    named_sync(1, kConsumers);
+    if (tid < R) {
+      float v = m_v[0][tid];
+      int i = m_i[0][tid];
+      for (int w = 1; w < kNW; ++w)
+        if (m_v[w][tid] > v || (m_v[w][tid] == v && m_i[w][tid] < i)) { v = m_v[w][tid]; i = m_i[w][tid]; }
+      p.tok[(p.row_dst ? p.row_dst[tid] : tid) * p.tok_stride] = i;
+      s_tok[tid] = i;
     }
     if (tid == 0) *s.counter = 0;
     return true;
