@@ -1,5 +1,5 @@
 // Decode attention over a contiguous per-slot KV cache, split over a
-// thread-block cluster.
+// thread-block cluster, with both contractions on the tensor cores.
 //
 // For pass row r (slot b, position pos_r) and head h:
 //   out[r][h] = softmax_j(q_r . k_j / sqrt(Dh)) v_j over positions j = 0..pos_r
@@ -7,19 +7,28 @@
 //
 // The position axis is cut into fixed kAttnChunk-position chunks.  The
 // kAttnSplit CTAs of one cluster serve one (slot, head); CTA k takes chunks
-// k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time: it streams
-// their K and V rows into shared memory with bulk copies, scores them all,
-// and keeps an online-softmax state per row (running max M, sum L,
-// unnormalised output O) that is rescaled between such groups.  The CTAs then
-// merge their states through distributed shared memory, rank by rank, each CTA
-// producing Dh / kAttnSplit output dims.  Which CTA takes a chunk and the order
-// of every sum depend only on positions, so a row's result does not depend on
-// the other rows of the pass.
+// k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time (a group):
+//   * TMA brings each chunk's K and V rows into shared memory (5-D tensor map
+//     over the cache, 128-byte swizzle, no multicast);
+//   * scores S[j][r] = K[j] . q_r as m16n8k16 MMAs (positions x rows, the up
+//     to 8 pass rows are the 8 MMA columns); q is split into bfloat16 high and
+//     low parts, so the products carry float32-level precision;
+//   * an online softmax per row (running max M, sum L) over the group;
+//   * O[d][r] += V[j][d] P[r][j] as MMAs on V transposed (ldmatrix .trans),
+//     P again split into bfloat16 high and low parts; each warp owns 16 dims.
+// The CTAs then merge their (M, L, O) states through distributed shared
+// memory in rank order, each CTA producing Dh / kAttnSplit output dims.
+// Which CTA takes a chunk and the order of every sum depend only on positions
+// (an MMA column depends on its own row's data only; positions a row does not
+// see carry p = 0 exactly), so a row's result does not depend on the other
+// rows of the pass.
 //
 // Chunks that lie wholly below the pass's first new position are not written
 // by the kernel before this one (which writes the pass rows' keys and values),
 // so their copies are issued before the dependency wait.
 #pragma once
+
+#include <cuda.h>
 
 #include "common.cuh"
 
@@ -27,21 +36,24 @@ namespace ocrdec {
 
 constexpr int kAttnChunk = 64;
 constexpr int kAttnSplit = 8;    // CTAs per (slot, head): one cluster
-constexpr int kAttnBufs = 3;     // K/V chunk ring per CTA
+constexpr int kAttnBufs = 3;     // K/V chunks per group (ring)
 constexpr int kTagAttention = 40;
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
-constexpr int kAttnWarpPos = kAttnChunk / kAttnWarps;  // positions of a chunk per warp
-constexpr int kAttnRows = 8;     // rows of one slot in a pass
+constexpr int kAttnRows = 8;     // rows of one slot in a pass (MMA columns)
 constexpr int kAttnMaxDh = 128;
+constexpr int kAttnQLd = kAttnMaxDh + 8;                // bf16 q row (+16 B: conflict-free ldmatrix)
+constexpr int kAttnPLd = kAttnBufs * kAttnChunk + 8;    // bf16 P row
+constexpr int kAttnChunkBytes = kAttnChunk * kAttnMaxDh * 2;  // K (or V) of one chunk: [half][pos][128 B]
 
-constexpr size_t attn_smem_bytes(int Dh) { return (size_t)kAttnBufs * 2 * kAttnChunk * Dh * 2; }
+// K and V of every chunk in the ring, plus 1 KB of alignment slack (the
+// 128-byte swizzle repeats every 1 KB).
+constexpr size_t attn_smem_bytes(int) { return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes; }
 
 struct AttnParams {
   const float* q;          // [R][H*Dh]
-  const bf16* kc;          // this layer, slot 0: [H][cap][Dh]
-  const bf16* vc;
-  long long slot_stride;   // elements between slots
+  int layer;               // cache layer index (map coordinate slot * n_layers + layer)
+  int n_layers;            // layers in the cache (1 for the draft cache)
   int cap, H, Dh;          // Dh 64 or 128
   float scale;             // 1/sqrt(Dh)
   const int* slot_row0;    // [B] first pass row of each slot
@@ -70,15 +82,53 @@ __device__ __forceinline__ const T* cluster_map(const T* p, uint32_t rank) {
   return reinterpret_cast<const T*>(r);
 }
 
-__global__ void __launch_bounds__(kAttnThreads)
-attention_kernel(const AttnParams p) {
-  extern __shared__ __align__(128) unsigned char smem[];
+// 5-D tensor-map load of one chunk of K or V: 64 columns x 64 positions x
+// Dh/64 halves at (position p0, head h, cache plane pl) -> [half][pos][128 B].
+__device__ __forceinline__ void tma_load_kv(void* dst, const CUtensorMap* map, int p0, int h, int pl, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.5d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5, %6}], [%7];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(p0), "r"(0), "r"(h), "r"(pl), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void attn_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void attn_ldsm_x4_t(uint32_t addr, uint32_t (&a)[4]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+               : "r"(addr));
+}
+__device__ __forceinline__ void attn_ldsm_x2(uint32_t addr, uint32_t (&b)[2]) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0, %1}, [%2];" : "=r"(b[0]), "=r"(b[1]) : "r"(addr));
+}
+__device__ __forceinline__ void attn_mma(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// Shared address of the 16-byte unit `u` (0..7) of position `pos`, half `hf`
+// of a swizzled chunk tile.
+__device__ __forceinline__ uint32_t kv_addr(uint32_t base, int hf, int pos, int u) {
+  return base + (uint32_t)(hf * kAttnChunk * 128 + pos * 128 + ((u ^ (pos & 7)) << 4));
+}
+
+__global__ void __launch_bounds__(kAttnThreads, 1)
+attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                 const AttnParams p) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar[kAttnBufs];
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
-  __shared__ float qs[kAttnRows][kAttnMaxDh];
-  __shared__ float sc[kAttnRows][kAttnBufs * kAttnChunk];
-  __shared__ float ored[kAttnWarps][kAttnRows][kAttnMaxDh];
+  __shared__ __align__(16) bf16 s_q[2][kAttnRows][kAttnQLd];   // q high / low parts
+  __shared__ __align__(16) bf16 s_p[2][kAttnRows][kAttnPLd];   // P high / low parts
+  __shared__ float sc[kAttnRows][kAttnBufs * kAttnChunk];      // scores
   __shared__ float s_M[kAttnRows], s_L[kAttnRows], s_corr[kAttnRows];
   __shared__ float s_O[kAttnRows][kAttnMaxDh];
 
@@ -86,7 +136,8 @@ attention_kernel(const AttnParams p) {
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int Dh = p.Dh;
-  bf16* ring = reinterpret_cast<bf16*>(smem);
+  unsigned char* ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
+  const uint32_t ring_s = smem_u32(ring);
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBufs; ++i) mbar_init(&bar[i], 1);
@@ -96,8 +147,8 @@ attention_kernel(const AttnParams p) {
   // finished before the kernel this one follows
   const int r0 = p.slot_row0[b];
   const int nr = max(0, min(p.slot_nrows[b], kAttnRows));
-  if (tid < kAttnRows) s_pos[tid] = tid < nr ? p.row_pos[r0 + tid] : -1;  // -1: sees nothing
   if (tid < kAttnRows) {
+    s_pos[tid] = tid < nr ? p.row_pos[r0 + tid] : -1;  // -1: sees nothing
     s_M[tid] = -INFINITY;
     s_L[tid] = 0.f;
   }
@@ -110,19 +161,17 @@ attention_kernel(const AttnParams p) {
   maxpos = min(maxpos, p.cap - 1);
   const int nch = maxpos >= 0 ? maxpos / kAttnChunk + 1 : 0;  // chunks of the slot
   const int n_my = nch > k ? (nch - 1 - k) / kAttnSplit + 1 : 0;  // this CTA's chunks
-  const long long head_base = (long long)b * p.slot_stride + (long long)h * p.cap * Dh;
+  const int plane = b * p.n_layers + p.layer;
 
   // chunk i of this CTA: position p0, valid positions npos, ring buffer i % kAttnBufs
   auto chunk_p0 = [&](int i) { return (k + i * kAttnSplit) * kAttnChunk; };
   auto chunk_npos = [&](int i) { return min(kAttnChunk, maxpos + 1 - chunk_p0(i)); };
   auto issue = [&](int i) {
-    const int p0 = chunk_p0(i);
     const int buf = i % kAttnBufs;
-    bf16* Ks = ring + (size_t)buf * 2 * kAttnChunk * Dh;
-    const uint32_t bytes = chunk_npos(i) * Dh * 2;
-    mbar_arrive_expect_tx(&bar[buf], 2 * bytes);
-    bulk_g2s(Ks, p.kc + head_base + (long long)p0 * Dh, bytes, &bar[buf]);
-    bulk_g2s(Ks + kAttnChunk * Dh, p.vc + head_base + (long long)p0 * Dh, bytes, &bar[buf]);
+    unsigned char* kd = ring + (size_t)buf * 2 * kAttnChunkBytes;
+    mbar_arrive_expect_tx(&bar[buf], (uint32_t)(2 * kAttnChunk * Dh * 2));
+    tma_load_kv(kd, &tm_k, chunk_p0(i), h, plane, &bar[buf]);
+    tma_load_kv(kd + kAttnChunkBytes, &tm_v, chunk_p0(i), h, plane, &bar[buf]);
   };
   auto old_chunk = [&](int i) { return chunk_p0(i) + kAttnChunk <= minpos; };
   const int n_first = min(n_my, kAttnBufs);
@@ -146,85 +195,56 @@ attention_kernel(const AttnParams p) {
   }
   if (tid < kAttnMaxDh)
 #pragma unroll
-    for (int i = 0; i < kAttnRows; ++i) qs[i][tid] = tid < Dh ? qv[i] : 0.f;
+    for (int i = 0; i < kAttnRows; ++i) {  // q = hi + lo, both bfloat16; zeros past nr and Dh
+      const bf16 hi = f2bf(qv[i]);
+      s_q[0][i][tid] = hi;
+      s_q[1][i][tid] = f2bf(__fsub_rn(qv[i], bf2f(hi)));
+    }
   __syncthreads();
   const bool work = !s_abort && nr > 0;
   pdl_trigger();
 
-  // per-warp output accumulators: warp w owns offsets [w, w + 1) * kAttnWarpPos
-  // of every chunk, lane l dims [l*dpl, (l+1)*dpl)
-  const int dpl = Dh / 32;  // 4 (Dh 128) or 2 (Dh 64)
-  float o[kAttnRows][4];
-#pragma unroll
-  for (int r = 0; r < kAttnRows; ++r)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) o[r][e] = 0.f;
+  // PV accumulators: warp w owns dims [16w, 16w + 16) (MMA m) for all 8 rows
+  // (MMA n): o0 (dim 16w + lane/4, row 2(lane%4)), o1 (row + 1), o2/o3 (dim + 8)
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool pv_warp = warp * 16 < Dh;
+  // fragment lane roles
+  const int fr_row = (lane & 7) + ((lane >> 3) & 1) * 8;   // ldmatrix.x4 row within a 16-row tile
+  const int fr_hi = lane >> 4;                             // second 16-byte unit for lanes 16..31
+  const int b_n = lane & 7, b_k8 = ((lane >> 3) & 1) * 8;  // ldmatrix.x2: MMA column and k offset
 
-  const int g4 = lane >> 3, l8 = lane & 7;
-  const int ndc = Dh / 8;  // 16-byte chunks per key row (8 or 16)
-  // Chunks are taken kAttnBufs at a time (a group); the online-softmax state
-  // is rescaled between groups.
   for (int i0 = 0, grp = 0; work && i0 < n_my; i0 += kAttnBufs, ++grp) {
     const int ni = min(kAttnBufs, n_my - i0);
     for (int ii = 0; ii < ni; ++ii)
       mbar_wait(&bar[ii], grp & 1, p.status);  // gives up with OCRDEC_ETIMEOUT; control flow stays uniform
     if (tid == 0 && grp == 0) tm.t1 = gtimer();
 
-    // ---- scores: 4 groups of 8 lanes per warp, one position per lane group;
-    // lane l8 owns the 16-byte dim-chunks l8 and l8 + 8 of a key row
-    for (int rb = 0; rb < nr; rb += 4) {
-      float qr[4][16];
+    // ---- scores: 16-position tiles t = warp, warp + 8, ... of the group ----
+    for (int t = warp; t < ni * (kAttnChunk / 16); t += kAttnWarps) {
+      const int ii = t / (kAttnChunk / 16), pt = (t % (kAttnChunk / 16)) * 16;
+      const uint32_t kb = ring_s + (uint32_t)(ii * 2 * kAttnChunkBytes);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < Dh / 16; ++s) {
+        uint32_t a[4], bh[2], bl[2];
+        attn_ldsm_x4(kv_addr(kb, s >> 2, pt + fr_row, (s & 3) * 2 + fr_hi), a);
+        attn_ldsm_x2(smem_u32(&s_q[0][b_n][s * 16 + b_k8]), bh);
+        attn_ldsm_x2(smem_u32(&s_q[1][b_n][s * 16 + b_k8]), bl);
+        attn_mma(d, a, bh);
+        attn_mma(d, a, bl);
+      }
+      const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
 #pragma unroll
-      for (int q = 0; q < 4; ++q)
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int d = (e < 8 ? l8 * 8 + e : (l8 + 8) * 8 + (e - 8));
-          qr[q][e] = qs[rb + q][d];  // rows past nr and dims past Dh hold zeros
-        }
-      for (int ii = 0; ii < ni; ++ii) {
-        const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
-        const bf16* Ks = ring + (size_t)ii * 2 * kAttnChunk * Dh;
-#pragma unroll
-        for (int j0 = 0; j0 < kAttnWarpPos; j0 += 4) {
-          const int j = warp * kAttnWarpPos + j0 + g4;
-          float kv[16];
-          if (j < npos) {
-            float t[8];
-            unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + l8 * 8), t);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) kv[e] = t[e];
-            if (l8 + 8 < ndc) {
-              unpack8(*reinterpret_cast<const uint4*>(Ks + j * Dh + (l8 + 8) * 8), t);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) kv[8 + e] = t[e];
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) kv[8 + e] = 0.f;
-            }
-          } else {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) kv[e] = 0.f;
-          }
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            float a = 0.f;
-#pragma unroll
-            for (int e = 0; e < 16; ++e) a = __fmaf_rn(qr[q][e], kv[e], a);
-            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 4));
-            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
-            a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
-            const int r = rb + q;  // < kAttnRows; rows past nr have position -1
-            const bool valid = j < npos && p0 + j <= s_pos[r];
-            if (l8 == 0) sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(a, p.scale) : -INFINITY;
-          }
-        }
+      for (int e = 0; e < 4; ++e) {
+        const int j = pt + (lane >> 2) + (e >> 1) * 8;  // position in the chunk
+        const int r = 2 * (lane & 3) + (e & 1);         // row
+        const bool valid = j < npos && p0 + j <= s_pos[r];
+        sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(d[e], p.scale) : -INFINITY;
       }
     }
     __syncthreads();
 
     // ---- online softmax update of each row over the group (warp w: row w).
-    // Invisible positions hold -inf and give exp(-inf) = 0 exactly, so a row's
-    // sums do not depend on how many chunks the group has. ----
+    // Invisible positions hold -inf and give exp(-inf) = 0 exactly. ----
     const int nu = ni * kAttnChunk;
     for (int r = warp; r < nr; r += kAttnWarps) {
       float m = -INFINITY;
@@ -232,7 +252,10 @@ attention_kernel(const AttnParams p) {
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
       if (m == -INFINITY) {  // nothing visible to this row in the group
-        for (int u = lane; u < nu; u += 32) sc[r][u] = 0.f;
+        for (int u = lane; u < nu; u += 32) {
+          s_p[0][r][u] = f2bf(0.f);
+          s_p[1][r][u] = f2bf(0.f);
+        }
         if (lane == 0) s_corr[r] = 1.f;
         continue;
       }
@@ -241,7 +264,9 @@ attention_kernel(const AttnParams p) {
       float l = 0.f;
       for (int u = lane; u < nu; u += 32) {
         const float e = expf(__fsub_rn(sc[r][u], Mn));
-        sc[r][u] = e;
+        const bf16 hi = f2bf(e);
+        s_p[0][r][u] = hi;
+        s_p[1][r][u] = f2bf(__fsub_rn(e, bf2f(hi)));
         l = __fadd_rn(l, e);
       }
 #pragma unroll
@@ -257,61 +282,47 @@ attention_kernel(const AttnParams p) {
     __syncthreads();
     if (tid == 0 && grp == 0) tm.t2 = gtimer();
 
-    // ---- o = o * corr + sum p_j v_j over the warp's offsets, chunk by chunk ----
+    // ---- O = O * corr + V^T P^T over the group's positions ----
+    if (pv_warp) {
+      const int c0 = 2 * (lane & 3);
+      const float cr0 = c0 < nr ? s_corr[c0] : 1.f, cr1 = c0 + 1 < nr ? s_corr[c0 + 1] : 1.f;
+      o[0] = __fmul_rn(o[0], cr0);
+      o[1] = __fmul_rn(o[1], cr1);
+      o[2] = __fmul_rn(o[2], cr0);
+      o[3] = __fmul_rn(o[3], cr1);
+      const int hf = (warp * 16) / 64, u0 = ((warp * 16) % 64) / 8;
+      for (int ii = 0; ii < ni; ++ii) {
+        const uint32_t vb = ring_s + (uint32_t)(ii * 2 * kAttnChunkBytes + kAttnChunkBytes);
 #pragma unroll
-    for (int r = 0; r < kAttnRows; ++r)
-      if (r < nr) {
-        const float cr = s_corr[r];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) o[r][e] = __fmul_rn(o[r][e], cr);
-      }
-    for (int ii = 0; ii < ni; ++ii) {
-      const int npos = chunk_npos(i0 + ii);
-      const bf16* Vs = ring + (size_t)ii * 2 * kAttnChunk * Dh + kAttnChunk * Dh;
-#pragma unroll
-      for (int jj = 0; jj < kAttnWarpPos; ++jj) {
-        const int j = warp * kAttnWarpPos + jj;
-        if (j >= npos) break;
-        float vv[4];
-        if (dpl == 4) {
-          uint2 u = *reinterpret_cast<const uint2*>(Vs + j * Dh + lane * 4);
-          vv[0] = bf_lo(u.x); vv[1] = bf_hi(u.x); vv[2] = bf_lo(u.y); vv[3] = bf_hi(u.y);
-        } else {
-          uint32_t u = *reinterpret_cast<const uint32_t*>(Vs + j * Dh + lane * 2);
-          vv[0] = bf_lo(u); vv[1] = bf_hi(u); vv[2] = 0.f; vv[3] = 0.f;
+        for (int s = 0; s < kAttnChunk / 16; ++s) {
+          // A = V^T (16 dims x 16 positions) from the stored [pos][dim] tile:
+          // lanes 0-7 pos 0-7 dims 0-7, 8-15 pos 0-7 dims 8-15, 16-23 pos 8-15
+          // dims 0-7, 24-31 pos 8-15 dims 8-15
+          const int pos = s * 16 + (lane & 7) + (lane >> 4) * 8;
+          const int u = u0 + ((lane >> 3) & 1);
+          uint32_t a[4], bh[2], bl[2];
+          attn_ldsm_x4_t(kv_addr(vb, hf, pos, u), a);
+          const int pc = ii * kAttnChunk + s * 16 + b_k8;
+          attn_ldsm_x2(smem_u32(&s_p[0][b_n][pc]), bh);
+          attn_ldsm_x2(smem_u32(&s_p[1][b_n][pc]), bl);
+          attn_mma(o, a, bh);
+          attn_mma(o, a, bl);
         }
-        // positions a row does not see have p = 0 exactly and add nothing;
-        // the loads are unconditional so they issue together
-        float pj[kAttnRows];
-#pragma unroll
-        for (int r = 0; r < kAttnRows; ++r) pj[r] = sc[r][ii * kAttnChunk + j];
-#pragma unroll
-        for (int r = 0; r < kAttnRows; ++r)
-          if (r < nr)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) o[r][e] = __fmaf_rn(pj[r], vv[e], o[r][e]);
       }
     }
-    __syncthreads();  // ring buffers and scores are free again
+    __syncthreads();  // ring buffers, scores and probabilities are free again
     if (tid == 0)
       for (int ii = 0; ii < kAttnBufs && i0 + kAttnBufs + ii < n_my; ++ii) issue(i0 + kAttnBufs + ii);
   }
 
-  // ---- this CTA's state: O = sum of the warp partials in warp order ----
+  // ---- this CTA's state: every warp holds the final O of its 16 dims ----
   if (work) {
-#pragma unroll
-    for (int r = 0; r < kAttnRows; ++r)
-      if (r < nr)
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          if (e < dpl) ored[warp][r][lane * dpl + e] = o[r][e];
-    __syncthreads();
-    for (int idx = tid; idx < nr * Dh; idx += kAttnThreads) {
-      const int r = idx / Dh, d = idx - r * Dh;
-      float v = ored[0][r][d];
-#pragma unroll
-      for (int w = 1; w < kAttnWarps; ++w) v = __fadd_rn(v, ored[w][r][d]);
-      s_O[r][d] = v;
+    if (pv_warp) {
+      const int dm = warp * 16 + (lane >> 2), c0 = 2 * (lane & 3);
+      s_O[c0][dm] = o[0];
+      s_O[c0 + 1][dm] = o[1];
+      s_O[c0][dm + 8] = o[2];
+      s_O[c0 + 1][dm + 8] = o[3];
     }
   } else if (s_abort && tid == 0) {
     // copies issued before the dependency wait land before the CTA exits

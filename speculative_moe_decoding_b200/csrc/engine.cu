@@ -233,6 +233,7 @@ struct ocrdec_ctx {
   float* dbg_hidden = nullptr;
   float* dbg_logits = nullptr;
   float* dbg_draft_logits = nullptr;
+  CUtensorMap kv_map[4];  // verifier K, V; draft K, V (encoded when the workspace is bound)
 
   template <class T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
@@ -288,6 +289,9 @@ struct BlockIO {
   bf16* kc;            // K cache of this block, slot 0 (layer offset applied)
   bf16* vc;
   long long slot_stride;
+  const CUtensorMap* tk;  // tensor maps over the whole K / V cache
+  const CUtensorMap* tv;
+  int layer, n_layers;    // this block's layer in the cache
 };
 
 // A GEMV launch over one dense matrix.
@@ -325,9 +329,8 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
 
   AttnParams a{};
   a.q = c->at<float>(c->L.q);
-  a.kc = io.kc;
-  a.vc = io.vc;
-  a.slot_stride = io.slot_stride;
+  a.layer = io.layer;
+  a.n_layers = io.n_layers;
   a.cap = m.kv_capacity;
   a.H = m.n_heads;
   a.Dh = m.head_dim;
@@ -338,7 +341,7 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   a.out = c->at<bf16>(c->L.attn_out);
   a.status = c->status();
   CK(launch_cluster_ex(attention_kernel, dim3(kAttnSplit, m.n_heads, m.max_batch), dim3(kAttnThreads),
-               attn_smem_bytes(m.head_dim), lc, kAttnSplit, a));
+                       attn_smem_bytes(m.head_dim), lc, kAttnSplit, *io.tk, *io.tv, a));
 
   GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax, kTagOProj);
   o.src = SrcKind::Bf16;
@@ -443,7 +446,7 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
   for (int l = 0; l < m.n_layers; ++l) {
     const LayerW& w = c->layers[l];
     BlockIO io{c->at<float>(c->L.x), c->at<bf16>(c->L.kvk) + l * layer_elems, c->at<bf16>(c->L.kvv) + l * layer_elems,
-               layer_elems * m.n_layers};
+               layer_elems * m.n_layers, &c->kv_map[0], &c->kv_map[1], l, m.n_layers};
     int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
     if (st) return st;
     st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down) : moe_ffn(c, lc, rmax, w, count);
@@ -486,7 +489,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   CK(c->gemv(fc, lc));
 
   const long long slot_elems = (long long)m.n_heads * m.kv_capacity * m.head_dim;
-  BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems};
+  BlockIO io{xd, c->at<bf16>(c->L.dkvk), c->at<bf16>(c->L.dkvv), slot_elems, &c->kv_map[2], &c->kv_map[3], 0, 1};
   if (kv_only) {
     GemvLaunch g = dense_launch(c, w.wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
     g.src = SrcKind::Norm;
@@ -663,8 +666,17 @@ int ocrdec_bind_workspace(ocrdec_ctx* c, void* ws, size_t bytes, ocrdec_stream s
   c->ws = static_cast<char*>(ws);
   c->drop_graphs();
   CK(prepare_kernels());
-  // status, counters, slots, rows and token history start at zero
+  // status, counters, slots, rows and token history start at zero; so do the
+  // KV caches, whose unwritten positions attention reads (with weight 0)
   CK(cudaMemsetAsync(c->ws, 0, c->L.rope, s));
+  CK(cudaMemsetAsync(c->ws + c->L.kvk, 0, c->L.x - c->L.kvk, s));
+  {
+    const ocrdec_config& mc = c->cfg;
+    const int B = mc.max_batch;
+    const void* bases[4] = {c->ws + c->L.kvk, c->ws + c->L.kvv, c->ws + c->L.dkvk, c->ws + c->L.dkvv};
+    for (int i = 0; i < 4; ++i)
+      CK(encode_kv_map(bases[i], mc.head_dim, mc.kv_capacity, mc.n_heads, i < 2 ? B * mc.n_layers : B, &c->kv_map[i]));
+  }
   const ocrdec_config& m = c->cfg;
   long long n = (long long)m.kv_capacity * (m.head_dim / 2);
   rope_table_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(c->at<float2>(c->L.rope), m.kv_capacity, m.head_dim,

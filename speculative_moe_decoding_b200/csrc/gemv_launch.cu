@@ -54,6 +54,32 @@ cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 5-D view of a KV cache [planes][H][cap][Dh] (planes = slots x layers):
+// (64-column chunk, position, chunk index, head, plane); a box is one
+// 64-position chunk of one head, stored [chunk][position][128 B] with the
+// 128-byte swizzle.
+cudaError_t encode_kv_map(const void* base, int Dh, int cap, int H, int planes, CUtensorMap* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || Dh % 64 || cap <= 0 || H <= 0 || planes <= 0)
+    return cudaErrorInvalidValue;
+  const cuuint64_t row = (cuuint64_t)Dh * 2;
+  cuuint64_t dims[5] = {64, (cuuint64_t)cap, (cuuint64_t)(Dh / 64), (cuuint64_t)H, (cuuint64_t)planes};
+  cuuint64_t strides[4] = {row, 128, row * cap, row * cap * H};
+  cuuint32_t box[5] = {64, 64, (cuuint32_t)(Dh / 64), 1, 1};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <class Src>
 static size_t smem_max() {
   return gemv_smem_bytes<Src>(kGemvMaxK);
