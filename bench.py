@@ -169,6 +169,29 @@ def reference_arm(args, dims):
 
 # ---- our arm --------------------------------------------------------------------
 
+def profiled_traffic(name):
+    """DRAM bytes per launch recorded in a profiles/ summary, if the kernel
+    sources it lists still hash to the recorded value (else None)."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", name)
+    if not os.path.exists(path):
+        return None
+    fields = {}
+    for line in open(path):
+        if ":" in line and line.startswith("    "):
+            key, _, val = line.strip().partition(":")
+            fields[key.strip()] = val.strip()
+    try:
+        h = hashlib.sha256()
+        for f in fields["source_files"].split():
+            h.update(open(os.path.join(ROOT, f), "rb").read())
+        if h.hexdigest() != fields["source_sha256"]:
+            return None
+        return int(fields["traffic_bytes_per_launch"])
+    except (KeyError, OSError, ValueError):
+        return None
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -325,26 +348,29 @@ def main():
     xr = torch.randn((R, dims.d_model), dtype=torch.float32, device="cuda")
     tok = torch.empty(R, dtype=torch.int32, device="cuda")
     scratch = ocrdec.op_scratch()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
     ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)  # one-time kernel set-up
     torch.cuda.synchronize()
+    # LM_BACK_TO_BACK launches in one graph: each streams the whole 331 MB head,
+    # more than L2 holds, so no launch finds its weights in cache
+    LM_BACK_TO_BACK = 10
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
+        for _ in range(LM_BACK_TO_BACK):
+            ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
     times = []
-    for i in range(23):
-        flush.fill_(i & 0xff)
+    for i in range(8):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         graph.replay()
         b.record(stream)
         torch.cuda.synchronize()
         if i >= 3:
-            times.append(a.elapsed_time(b))
+            times.append(a.elapsed_time(b) / LM_BACK_TO_BACK)
     del graph
     lm_ms = float(np.mean(times))
     lm_bytes = dims.vocab * dims.d_model * 2 + R * dims.d_model * 4 + dims.d_model * 2
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
+    lm_traffic = profiled_traffic("lm_head_argmax_r4.md")
 
     # ---- end to end through host buffers ----
     e2e = None
@@ -401,11 +427,15 @@ def main():
                               "dependency_aware_frac_of_measured_peak": dep_b / (step_ms / 1000) / 1e9 / peak_gbs},
             "roofline": {"kernel": "lm_head_argmax (final RMSNorm + 129,280 x 1280 GEMV + argmax, k+1 rows)",
                          "bound": "hbm", "achieved": lm_gbs, "peak": peak_gbs, "unit": "GB/s",
-                         "frac": lm_gbs / peak_gbs, "traffic": None, "peak_source": peak_src,
+                         "frac": lm_gbs / peak_gbs, "traffic": lm_traffic, "peak_source": peak_src,
                          "launch_ms": lm_ms, "bytes_per_launch": lm_bytes,
-                         "timing": "same kernel instantiation as in the step, launched alone through ocrdec_op_lm_argmax "
-                                   "replayed from a CUDA graph, L2 flushed before each launch, CUDA events on the "
-                                   "launching stream"},
+                         "timing": "same kernel instantiation as in the verify pass, launched through "
+                                   "ocrdec_op_lm_argmax: 10 launches back to back in one CUDA graph (each streams "
+                                   "331 MB > L2), CUDA events on the launching stream, mean of 5 replays; each "
+                                   "launch includes the op's 64-byte scratch memset",
+                         "traffic_source": "profiles/lm_head_argmax_r4.md (ncu dram__bytes_read.sum + "
+                                           "dram__bytes_write.sum, one launch; null if the kernel sources changed "
+                                           "since)"},
             "timeline": timeline,
             "gpu_launches": kernels * args.steps,
             "kernels_per_step": kernels,
