@@ -91,7 +91,8 @@ typedef struct {
 /* ---- setup ---------------------------------------------------------------- */
 
 /* Validates the config (positive sizes, n_heads*head_dim == d_model, head_dim
- * 64 or 128, d_model <= 2048, d_model and the FFN widths multiples of 64,
+ * 64 or 128, n_heads <= 16, d_model <= 2048 and a multiple of 128, the FFN
+ * widths multiples of 64,
  * vocab a multiple of 8, top_k <= min(n_experts, 8), n_experts <= 128,
  * max_k <= 3, kv_capacity <= 8192).
  * *out receives a context that must be released with ocrdec_destroy. */
@@ -176,6 +177,8 @@ OCRDEC_API int ocrdec_set_forced_acceptance(ocrdec_ctx* ctx, const int32_t* dev_
 
 /* Sticky device status (ocrdec_status); synchronises `stream` to read it. */
 OCRDEC_API int ocrdec_get_status(ocrdec_ctx* ctx, int32_t* host_status, ocrdec_stream stream);
+/* Clears the sticky status and the device's internal arrival counters (which
+ * a launch that gave up part-way may leave inconsistent), on `stream`. */
 OCRDEC_API int ocrdec_clear_status(ocrdec_ctx* ctx, ocrdec_stream stream);
 /* Synchronises `stream` and copies the slot's counters. */
 OCRDEC_API int ocrdec_get_slot_stats(ocrdec_ctx* ctx, int slot, ocrdec_slot_stats* host_stats, ocrdec_stream stream);
@@ -210,11 +213,11 @@ OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* 
  * loop, epilogue/finish; attention: first K/V chunk landed, its softmax done,
  * end (after the cluster merge); routing: one phase.  ocrdec_read_trace copies
  * up to max_records records to host memory and sets *n to the number recorded
- * (synchronises `stream`).  Tags: 1 QKV, 2 O-proj, 3 router+routing, 4 expert
+ * (synchronises `stream`).  Tags: 1 QKV, 3 router+routing, 4 expert
  * gate/up, 5 expert down, 6 dense gate/up, 7 dense down, 8 verify LM head +
- * acceptance, 9 draft LM head, 10 draft input fc, 40 attention (41 for cluster
- * rank 0), 42 verify setup, 43 draft setup, 44 MoE combine, 45 routing step of
- * the router's last CTA. */
+ * acceptance, 9 draft LM head, 10 draft input fc, 40 attention with the
+ * output projection (41 for cluster rank 0), 42 verify setup, 43 draft setup,
+ * 44 MoE combine, 45 routing step of the router's last CTA. */
 OCRDEC_API int ocrdec_set_trace(ocrdec_ctx* ctx, int enable, ocrdec_stream stream);
 OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_records, int32_t* n,
                                  ocrdec_stream stream);

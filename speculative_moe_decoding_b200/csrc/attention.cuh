@@ -17,7 +17,14 @@
 //   * O[d][r] += V[j][d] P[r][j] as MMAs on V transposed (ldmatrix .trans),
 //     P again split into bfloat16 high and low parts; each warp owns 16 dims.
 // The CTAs then merge their (M, L, O) states through distributed shared
-// memory in rank order, each CTA producing Dh / kAttnSplit output dims.
+// memory in rank order, each CTA producing Dh / kAttnSplit output dims of the
+// head and storing them into every CTA of the cluster.
+//
+// The output projection is folded in: CTA k multiplies the head's output by
+// its block of W_o (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; the
+// block arrives by TMA before the dependency wait) and writes the partial sums
+// per head; the last of the H heads to finish a row block adds the partials
+// in head order to the residual stream.
 // Which CTA takes a chunk and the order of every sum depend only on positions
 // (an MMA column depends on its own row's data only; positions a row does not
 // see carry p = 0 exactly), so a row's result does not depend on the other
@@ -42,13 +49,18 @@ constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int kAttnRows = 8;     // rows of one slot in a pass (MMA columns)
 constexpr int kAttnMaxDh = 128;
+constexpr int kAttnMaxHeads = 16;  // heads summed by the fused output projection
 constexpr int kAttnQLd = kAttnMaxDh + 8;                // bf16 q row (+16 B: conflict-free ldmatrix)
 constexpr int kAttnPLd = kAttnBufs * kAttnChunk + 8;    // bf16 P row
 constexpr int kAttnChunkBytes = kAttnChunk * kAttnMaxDh * 2;  // K (or V) of one chunk: [half][pos][128 B]
 
 // K and V of every chunk in the ring, plus 1 KB of alignment slack (the
 // 128-byte swizzle repeats every 1 KB).
-constexpr size_t attn_smem_bytes(int) { return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes; }
+// Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
+// every 1 KB), the K/V ring, and the CTA's W_o block (d / kAttnSplit rows x Dh).
+constexpr size_t attn_smem_bytes(int d, int Dh) {
+  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + (size_t)(d / kAttnSplit) * Dh * 2;
+}
 
 struct AttnParams {
   const float* q;          // [R][H*Dh]
@@ -59,7 +71,10 @@ struct AttnParams {
   const int* slot_row0;    // [B] first pass row of each slot
   const int* slot_nrows;   // [B] rows of each slot in this pass
   const int* row_pos;      // [R]
-  bf16* out;               // [R][H*Dh]
+  float* x;                // residual rows [R][d] (+= the projected attention output)
+  float* yp;               // [H][kRmax][d] per-head partial projections
+  int* cnt;                // [B][kAttnSplit] arrivals per row block, zero between launches
+  int d;                   // model width (= H * Dh), a multiple of 16 * kAttnSplit
   int* status;
 };
 
@@ -92,6 +107,16 @@ __device__ __forceinline__ void tma_load_kv(void* dst, const CUtensorMap* map, i
       : "memory");
 }
 
+// 3-D tensor-map load of a W_o block: 64 columns x nb rows x Dh/64 chunks at
+// (row r0, column chunk c0) -> [chunk][row][128 B].
+__device__ __forceinline__ void tma_load_wo(void* dst, const CUtensorMap* map, int r0, int c0, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(r0), "r"(c0), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ void attn_ldsm_x4(uint32_t addr, uint32_t (&a)[4]) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
                : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
@@ -121,9 +146,11 @@ __device__ __forceinline__ uint32_t kv_addr(uint32_t base, int hf, int pos, int 
 
 __global__ void __launch_bounds__(kAttnThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                 const AttnParams p) {
+                 const __grid_constant__ CUtensorMap tm_wo, const AttnParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bar[kAttnBufs];
+  __shared__ __align__(8) uint64_t bar[kAttnBufs], wo_bar;
+  __shared__ __align__(16) bf16 s_head[kAttnRows][kAttnQLd];  // the head's merged output (bf16)
+  __shared__ int s_last;
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
   __shared__ __align__(16) bf16 s_q[2][kAttnRows][kAttnQLd];   // q high / low parts
@@ -138,10 +165,16 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const int Dh = p.Dh;
   unsigned char* ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t ring_s = smem_u32(ring);
+  unsigned char* wo_s = ring + (size_t)kAttnBufs * 2 * kAttnChunkBytes;  // [Dh/64][nb rows][128 B]
+  const int nb = p.d / kAttnSplit;  // W_o rows of this CTA
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBufs; ++i) mbar_init(&bar[i], 1);
+    mbar_init(&wo_bar, 1);
     fence_mbar_init();
+    // the W_o block is a weight: requested before anything else
+    mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2));
+    tma_load_wo(wo_s, &tm_wo, k * nb, h * (Dh / 64), &wo_bar);
   }
   // pass rows and positions are written by the pass's setup kernel, which
   // finished before the kernel this one follows
@@ -331,8 +364,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   }
   cluster_sync_all();  // every CTA's state is visible to the cluster
 
-  // ---- merge: CTA k writes dims [k*dpr, (k+1)*dpr) of every row, combining
-  // the CTAs' states in rank order ----
+  // ---- merge: CTA k forms dims [k*dpr, (k+1)*dpr) of every row, combining
+  // the CTAs' states in rank order, and stores them (bf16) into the head
+  // output of every CTA of the cluster ----
   if (work) {
     const int dpr = Dh / kAttnSplit;
     if (tid < nr * dpr) {
@@ -355,10 +389,80 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         L = __fmaf_rn(Lk[q], f, L);
         O = __fmaf_rn(Ok[q], f, O);
       }
-      p.out[(long long)(r0 + r) * p.H * Dh + h * Dh + d] = f2bf(__fdiv_rn(O, L));
+      const bf16 ov = f2bf(__fdiv_rn(O, L));
+#pragma unroll
+      for (int q = 0; q < kAttnSplit; ++q) *const_cast<bf16*>(cluster_map(&s_head[r][d], q)) = ov;
+    } else if (tid < kAttnRows * dpr) {  // rows past nr: zeros (MMA columns stay finite)
+      const int r = tid / dpr, d = k * dpr + (tid - r * dpr);
+#pragma unroll
+      for (int q = 0; q < kAttnSplit; ++q) *const_cast<bf16*>(cluster_map(&s_head[r][d], q)) = f2bf(0.f);
     }
   }
-  cluster_sync_all();  // no CTA leaves while another may still read its state
+  cluster_sync_all();  // every CTA holds the whole head output; no remote access follows
+
+  // ---- output projection of this head, rows [k*nb, (k+1)*nb) of W_o:
+  // yp[h][row][n] = sum_d W_o[n][h*Dh + d] * head[row][d] (MMAs: n x rows) ----
+  if (work) {
+    mbar_wait(&wo_bar, 0, p.status);
+    const uint32_t wb = smem_u32(wo_s);
+    for (int t = warp; t < nb / 16; t += kAttnWarps) {
+      float d4[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int s = 0; s < Dh / 16; ++s) {
+        uint32_t a[4], bb[2];
+        const int row = t * 16 + fr_row, u = (s & 3) * 2 + fr_hi;
+        attn_ldsm_x4(wb + (uint32_t)((s >> 2) * nb * 128 + row * 128 + ((u ^ (row & 7)) << 4)), a);
+        attn_ldsm_x2(smem_u32(&s_head[b_n][s * 16 + b_k8]), bb);
+        attn_mma(d4, a, bb);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int n = k * nb + t * 16 + (lane >> 2) + (e >> 1) * 8;
+        const int r = 2 * (lane & 3) + (e & 1);
+        if (r < nr) p.yp[((long long)h * kAttnRows + r0 + r) * p.d + n] = d4[e];
+      }
+    }
+    // the last head to finish this row block adds the heads' partials in
+    // head order to the residual stream.  The block's residual values are
+    // read first (no kernel writes them meanwhile), so the tail after the
+    // arrival count is one round of loads.
+    constexpr int kPer = kAttnRows * 256 / kAttnThreads;  // elements per thread: nr * nb <= 8 * 256
+    float xv[kPer];
+#pragma unroll
+    for (int i = 0; i < kPer; ++i) {
+      const int idx = tid + i * kAttnThreads;
+      xv[i] = 0.f;
+      if (idx < nr * nb) {
+        const int r = idx / nb, n = k * nb + (idx - r * nb);
+        xv[i] = __ldcg(p.x + (long long)(r0 + r) * p.d + n);
+      }
+    }
+    __threadfence();
+    __syncthreads();
+    if (tid == 0) s_last = atomicAdd(&p.cnt[b * kAttnSplit + k], 1) == p.H - 1;
+    __syncthreads();
+    if (s_last) {
+      __threadfence();
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int idx = tid + i * kAttnThreads;
+        if (idx >= nr * nb) break;
+        const int r = idx / nb, n = k * nb + (idx - r * nb);
+        const float* yr = p.yp + (long long)(r0 + r) * p.d + n;
+        float y[kAttnMaxHeads];
+#pragma unroll
+        for (int hh = 0; hh < kAttnMaxHeads; ++hh)
+          if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * p.d);
+        float v = 0.f;
+#pragma unroll
+        for (int hh = 0; hh < kAttnMaxHeads; ++hh)
+          if (hh < p.H) v = __fadd_rn(v, y[hh]);
+        p.x[(long long)(r0 + r) * p.d + n] = __fadd_rn(xv[i], v);
+      }
+      if (tid == 0) p.cnt[b * kAttnSplit + k] = 0;
+    }
+  } else if (tid == 0) {
+    mbar_wait(&wo_bar, 0, p.status);  // the W_o copy lands before the CTA exits
+  }
   if (tid == 0 && work && n_my > 0) trace_end(p.status, k == 0 ? kTagAttention + 1 : kTagAttention, tm);
 }
 

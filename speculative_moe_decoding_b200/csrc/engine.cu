@@ -29,7 +29,8 @@ constexpr int kPrefillChunk = kRmax;  // context rows per prefill pass
 struct Mat {
   const bf16* p = nullptr;
   int N = 0, K = 0, E = 1;
-  CUtensorMap map;
+  CUtensorMap map;       // GEMV tiles
+  CUtensorMap map_attn;  // W_o only: the attention kernel's per-(head, row block) boxes
 };
 
 struct LayerW {
@@ -104,6 +105,8 @@ bool config_ok(const ocrdec_config* c) {
   if (c->max_k < 0 || c->max_k > 3) return false;
   if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
   if (c->d_model > kGemvMaxK) return false;  // shared-memory copy of the normalised rows
+  // attention's fused output projection: d / 8 rows of W_o per CTA, whole 16-row MMA tiles, one TMA box
+  if (c->d_model % (16 * kAttnSplit) || c->d_model / kAttnSplit > 256 || c->n_heads > kAttnMaxHeads) return false;
   if (c->kv_capacity > 8192) return false;  // documented limit of the C ABI
   if (!(c->rms_eps > 0.f) || !(c->rope_theta > 1.f)) return false;
   return true;
@@ -112,7 +115,7 @@ bool config_ok(const ocrdec_config* c) {
 size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, part, attn_out, rlogits,
+  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp, rlogits,
       topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, ybuf, hdense, fcin, am_part, gtok, props,
       committed, ncommitted, hpend, total;
   int hist_ld, am_blocks;
@@ -129,7 +132,7 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   size_t o = 0;
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.status = take(256 + sizeof(TraceRec) * kTraceCap);  // status word + timeline trace
-  L.counters = take(sizeof(int) * (16 + 2 * kWorkSlots));
+  L.counters = take(sizeof(int) * (16 + 2 * kWorkSlots + kRmax * kAttnSplit));
   L.tile_ctr = take(sizeof(int) * kSplitMaxTiles);
   L.slots = take(sizeof(SlotState) * B);
   L.rows = take(sizeof(PassRows));
@@ -143,7 +146,7 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.x = take(4 * R * d);
   L.xd = take(4 * R * d);
   L.q = take(4 * R * d);
-  L.attn_out = take(2 * R * d);
+  L.yp = take(4 * H * kRmax * d);  // per-head output projections
   L.rlogits = take(4 * R * E);
   L.topk_ids = take(4 * R * K);
   L.topk_gates = take(4 * R * K);
@@ -180,7 +183,7 @@ cudaError_t max_carveout(K kernel) {
 
 cudaError_t prepare_kernels_now() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)attn_smem_bytes(kAttnMaxDh));
+                                       (int)attn_smem_bytes(kGemvMaxK, kAttnMaxDh));
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
   if (e == cudaSuccess) e = max_carveout(attention_kernel);
   if (e == cudaSuccess) e = max_carveout(route_kernel);
@@ -241,6 +244,8 @@ struct ocrdec_ctx {
   int* am_counter(int which) const { return at<int>(L.counters) + which; }
   // misc[0] = routed experts touched by verifier MoE layers, misc[1] = such layer passes
   int* misc() const { return at<int>(L.counters) + 8; }
+  // attention / output-projection arrivals per (slot, row block)
+  int* attn_counters() const { return at<int>(L.counters) + 16 + 2 * kWorkSlots; }
   // GEMV work counters, handed out round-robin so that launches next to each
   // other in a stream (which may overlap under programmatic dependent launch)
   // never share one; each launch's last CTA zeroes its pair
@@ -338,17 +343,14 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   a.slot_row0 = rows->slot_row0;
   a.slot_nrows = rows->slot_nrows;
   a.row_pos = rows->pos;
-  a.out = c->at<bf16>(c->L.attn_out);
+  a.x = io.x;
+  a.yp = c->at<float>(c->L.yp);
+  a.cnt = c->attn_counters();
+  a.d = m.d_model;
   a.status = c->status();
+  // attention and the output projection (x += attn . W_o^T) in one launch
   CK(launch_cluster_ex(attention_kernel, dim3(kAttnSplit, m.n_heads, m.max_batch), dim3(kAttnThreads),
-                       attn_smem_bytes(m.head_dim), lc, kAttnSplit, *io.tk, *io.tv, a));
-
-  GemvLaunch o = dense_launch(c, wo, 0, &rows->n, 0, rmax, kTagOProj);
-  o.src = SrcKind::Bf16;
-  o.bf = SrcBf16::Params{c->at<bf16>(c->L.attn_out), m.d_model, 1, nullptr};
-  o.epi = EpiKind::StoreAdd;
-  o.store = EpiStore<false>::Params{io.x, m.d_model, 1, nullptr};
-  CK(c->gemv(o, lc));
+                       attn_smem_bytes(m.d_model, m.head_dim), lc, kAttnSplit, *io.tk, *io.tv, wo.map_attn, a));
   return OCRDEC_OK;
 }
 
@@ -705,6 +707,7 @@ int ocrdec_load_weights(ocrdec_ctx* c, const void* const* ptrs, int n) {
     L.attn_norm = W(i++);
     ok &= make_mat(L.wqkv, W(i++), 3 * d, d, 1);
     ok &= make_mat(L.wo, W(i++), d, d, 1);
+    ok &= encode_oproj_map(L.wo.p, d, m.head_dim, &L.wo.map_attn) == cudaSuccess;
     L.ffn_norm = W(i++);
     L.dense = l < m.n_dense_first;
     if (L.dense) {
@@ -733,6 +736,7 @@ int ocrdec_load_weights(ocrdec_ctx* c, const void* const* ptrs, int n) {
   dw.attn_norm = W(i++);
   ok &= make_mat(dw.wqkv, W(i++), 3 * d, d, 1);
   ok &= make_mat(dw.wo, W(i++), d, d, 1);
+  ok &= encode_oproj_map(dw.wo.p, d, m.head_dim, &dw.wo.map_attn) == cudaSuccess;
   dw.ffn_norm = W(i++);
   ok &= make_mat(dw.w_gu, W(i++), 2 * m.draft_ffn, d, 1);
   ok &= make_mat(dw.w_down, W(i++), d, m.draft_ffn, 1);
@@ -912,7 +916,12 @@ int ocrdec_get_status(ocrdec_ctx* c, int32_t* host_status, ocrdec_stream stream)
 int ocrdec_clear_status(ocrdec_ctx* c, ocrdec_stream stream) {
   if (!c) return OCRDEC_EINVAL;
   if (!c->ws) return OCRDEC_ESTATE;
-  CK(cudaMemsetAsync(c->status(), 0, sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  CK(cudaMemsetAsync(c->status(), 0, sizeof(int), s));
+  // arrival counters that an aborted launch may have left part-way
+  CK(cudaMemsetAsync(c->am_counter(0), 0, 8 * sizeof(int), s));
+  CK(cudaMemsetAsync(c->at<int>(c->L.counters) + 16, 0, (2 * kWorkSlots + kRmax * kAttnSplit) * sizeof(int), s));
+  CK(cudaMemsetAsync(c->at<int>(c->L.tile_ctr), 0, kSplitMaxTiles * sizeof(int), s));
   return OCRDEC_OK;
 }
 

@@ -80,6 +80,29 @@ cudaError_t encode_kv_map(const void* base, int Dh, int cap, int H, int planes, 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// 3-D view of W_o [d][d] for the attention kernel's output projection:
+// (64-column chunk, row, chunk index); a box is one CTA's block, d/8 rows x the
+// head's Dh columns, stored [chunk][row][128 B] with the 128-byte swizzle.
+cudaError_t encode_oproj_map(const void* base, int d, int Dh, CUtensorMap* out) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !p) return cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  if ((reinterpret_cast<uintptr_t>(base) & 15) || d % 64 || Dh % 64 || d / 8 > 256 || d % 8) return cudaErrorInvalidValue;
+  cuuint64_t dims[3] = {64, (cuuint64_t)d, (cuuint64_t)(d / 64)};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, 128};
+  cuuint32_t box[3] = {64, (cuuint32_t)(d / 8), (cuuint32_t)(Dh / 64)};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(out, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 template <class Src>
 static size_t smem_max() {
   return gemv_smem_bytes<Src>(kGemvMaxK);

@@ -83,6 +83,7 @@ constexpr int kSplitPartFloats = 1 << 19;  // partial-sum buffer (floats) shared
 constexpr int kSplitMaxTiles = 4096;       // per-tile counters
 // 3-D tensor map (columns K, rows N, matrices E) of a bfloat16 weight array with
 // the GEMV's 256 x 16 box; base 16-byte aligned.
+cudaError_t encode_oproj_map(const void* base, int d, int Dh, CUtensorMap* out);
 cudaError_t encode_kv_map(const void* base, int Dh, int cap, int H, int planes, CUtensorMap* out);
 cudaError_t encode_weight_map(const void* base, int K, int N, int E, CUtensorMap* out);
 cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
