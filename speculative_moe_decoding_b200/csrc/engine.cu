@@ -2,10 +2,11 @@
 //
 // Host side only orders launches; every step of the decode path runs in the
 // kernels of gemv.cuh, attention.cuh and step_kernels.cuh.  One verifier pass
-// per layer is: Q/K/V GEMV (+RoPE, KV append) -> split-K attention -> O-proj
-// GEMV (+residual) -> [dense SwiGLU up/down | router GEMV -> softmax/top-k and
-// bucketing -> expert gate/up GEMV over the touched experts -> expert down
-// GEMV -> combine].  Then final norm + LM head + argmax, then acceptance.
+// per layer is: Q/K/V GEMV (+RoPE, KV append) -> attention with the output
+// projection (+residual) -> [dense SwiGLU up/down | router GEMV (+softmax,
+// top-k and bucketing in its last CTA) -> expert gate/up GEMV over the touched
+// experts -> expert down GEMV -> combine].  Then final norm + LM head + argmax
+// with acceptance in its last CTA.
 #include <cmath>
 #include <cstring>
 #include <map>

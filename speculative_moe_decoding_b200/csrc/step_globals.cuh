@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(256) accept_kernel(const AcceptParams p) {
   __syncthreads();
   if (s_abort) return;
   pdl_trigger();
-  accept_rows(p, p.g, tid, 256, BlockSync{});
+  accept_rows(p, p.g, tid, 256, BlockSync{}, true);
 }
 
 __global__ void force_kernel(const ForceParams p) {

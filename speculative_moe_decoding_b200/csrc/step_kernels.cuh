@@ -36,6 +36,7 @@ struct PassRows {
 // One CTA, one warp per row.
 // ---------------------------------------------------------------------------
 constexpr int kMaxExperts = 128;
+constexpr int kMaxK = 3;  // draft tokens per step
 
 struct RouteParams {
   const float* logits;  // [R][E]
@@ -276,30 +277,41 @@ struct AcceptParams {
 
 // Greedy acceptance of every slot given the verifier tokens g (in shared or
 // global memory) by nthreads cooperating threads; sync() spans exactly them.
+// Thread b < B reads its slot's proposals and state before using any of them.
+// copy_hidden: also copy the verifier residual rows of each slot into hpend
+// (callers that copy them elsewhere pass false).
 template <class Sync>
-__device__ void accept_rows(const AcceptParams& p, const int* g_all, int tid, int nthreads, Sync sync) {
+__device__ void accept_rows(const AcceptParams& p, const int* g_all, int tid, int nthreads, Sync sync,
+                            bool copy_hidden) {
   __shared__ int s_a[kRmax];
   const int K1 = p.k + 1;
   if (tid < p.B) {
     const int b = tid;
     const int* g = g_all + b * K1;
+    int prop[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) prop[j] = j < p.k ? p.proposals[b * p.k + j] : -1;
+    SlotState* sp = p.slots + b;
+    const SlotState st = *sp;
     int a = 0;
-    while (a < p.k && p.proposals[b * p.k + a] == g[a]) ++a;
-    SlotState& st = p.slots[b];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j)
+      if (a == j && j < p.k && prop[j] == g[j]) a = j + 1;
     const int n = st.kv_len;
     for (int i = 0; i <= p.k; ++i) p.committed[b * K1 + i] = i <= a ? g[i] : -1;
     for (int i = 0; i <= a; ++i) p.hist[b * p.hist_ld + n + 1 + i] = g[i];
     p.n_committed[b] = a + 1;
-    st.kv_len = n + a + 1;
-    st.n_generated += a + 1;
-    st.bonus = g[a];
-    st.steps += 1;
-    st.tau_sum += a + 1;
-    st.hist[a] += 1;
-    st.pending = a + 1;
-    st.pend_pos = n;
+    sp->kv_len = n + a + 1;
+    sp->n_generated = st.n_generated + a + 1;
+    sp->bonus = g[a];
+    sp->steps = st.steps + 1;
+    sp->tau_sum = st.tau_sum + a + 1;
+    sp->hist[a] = st.hist[a] + 1;
+    sp->pending = a + 1;
+    sp->pend_pos = n;
     s_a[b] = a;
   }
+  if (!copy_hidden) return;
   sync();
   for (int b = 0; b < p.B; ++b)
     for (int idx = tid; idx < (s_a[b] + 1) * p.d; idx += nthreads) {
@@ -307,8 +319,6 @@ __device__ void accept_rows(const AcceptParams& p, const int* g_all, int tid, in
       p.hpend[((long long)b * (p.max_k + 1) + i) * p.d + n] = p.x[(long long)(b * K1 + i) * p.d + n];
     }
 }
-
-
 
 // Forced acceptance (benchmark harness): proposal for target t = kv_len + j.
 struct ForceParams {
