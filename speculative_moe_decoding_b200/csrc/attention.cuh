@@ -18,7 +18,8 @@
 //     P again split into bfloat16 high and low parts; each warp owns 16 dims.
 // The CTAs then merge their (M, L, O) states through distributed shared
 // memory in rank order, each CTA producing Dh / kAttnSplit output dims of the
-// head and storing them into every CTA of the cluster.
+// head and storing them (as bf16 high and low parts) into every CTA of the
+// cluster.
 //
 // The output projection is folded in: CTA k multiplies the head's output by
 // its block of W_o (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; the
@@ -149,7 +150,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                  const __grid_constant__ CUtensorMap tm_wo, const AttnParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   __shared__ __align__(8) uint64_t bar[kAttnBufs], wo_bar;
-  __shared__ __align__(16) bf16 s_head[kAttnRows][kAttnQLd];  // the head's merged output (bf16)
+  __shared__ __align__(16) bf16 s_head[2][kAttnRows][kAttnQLd];  // the head's merged output, high / low parts
   __shared__ int s_last;
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
@@ -389,13 +390,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         L = __fmaf_rn(Lk[q], f, L);
         O = __fmaf_rn(Ok[q], f, O);
       }
-      const bf16 ov = f2bf(__fdiv_rn(O, L));
+      const float ov = __fdiv_rn(O, L);
+      const bf16 hi = f2bf(ov), lo = f2bf(__fsub_rn(ov, bf2f(hi)));
 #pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) *const_cast<bf16*>(cluster_map(&s_head[r][d], q)) = ov;
+      for (int q = 0; q < kAttnSplit; ++q) {
+        *const_cast<bf16*>(cluster_map(&s_head[0][r][d], q)) = hi;
+        *const_cast<bf16*>(cluster_map(&s_head[1][r][d], q)) = lo;
+      }
     } else if (tid < kAttnRows * dpr) {  // rows past nr: zeros (MMA columns stay finite)
       const int r = tid / dpr, d = k * dpr + (tid - r * dpr);
 #pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) *const_cast<bf16*>(cluster_map(&s_head[r][d], q)) = f2bf(0.f);
+      for (int q = 0; q < kAttnSplit; ++q) {
+        *const_cast<bf16*>(cluster_map(&s_head[0][r][d], q)) = f2bf(0.f);
+        *const_cast<bf16*>(cluster_map(&s_head[1][r][d], q)) = f2bf(0.f);
+      }
     }
   }
   cluster_sync_all();  // every CTA holds the whole head output; no remote access follows
@@ -408,11 +416,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     for (int t = warp; t < nb / 16; t += kAttnWarps) {
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
       for (int s = 0; s < Dh / 16; ++s) {
-        uint32_t a[4], bb[2];
+        uint32_t a[4], bh[2], bl[2];
         const int row = t * 16 + fr_row, u = (s & 3) * 2 + fr_hi;
         attn_ldsm_x4(wb + (uint32_t)((s >> 2) * nb * 128 + row * 128 + ((u ^ (row & 7)) << 4)), a);
-        attn_ldsm_x2(smem_u32(&s_head[b_n][s * 16 + b_k8]), bb);
-        attn_mma(d4, a, bb);
+        attn_ldsm_x2(smem_u32(&s_head[0][b_n][s * 16 + b_k8]), bh);
+        attn_ldsm_x2(smem_u32(&s_head[1][b_n][s * 16 + b_k8]), bl);
+        attn_mma(d4, a, bh);
+        attn_mma(d4, a, bl);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {

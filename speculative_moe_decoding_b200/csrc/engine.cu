@@ -117,7 +117,8 @@ size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
   size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp, rlogits,
-      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, ybuf, hdense, fcin, am_part, gtok, props,
+      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
+      am_part, gtok, props,
       committed, ncommitted, hpend, total;
   int hist_ld, am_blocks;
 };
@@ -157,9 +158,12 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.mats = take(4 * (E + S));
   L.n_mats = take(4);
   L.hbuf = take(2 * R * nslot * f);
+  L.hbuf_lo = take(2 * R * nslot * f);
   L.ybuf = take(4 * R * nslot * d);
   L.hdense = take(2 * R * F);
+  L.hdense_lo = take(2 * R * F);
   L.fcin = take(2 * R * 2 * d);
+  L.fcin_lo = take(2 * R * 2 * d);
   L.am_part = take(sizeof(float2) * am_blocks * kRmax);
   L.gtok = take(4 * R);
   L.props = take(4 * B * 4);
@@ -365,12 +369,12 @@ int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16
   g.src = SrcKind::Norm;
   g.norm = SrcNorm::Params{x, m.d_model, nullptr, norm, m.rms_eps};
   g.epi = EpiKind::SwiGLU;
-  g.swiglu = EpiSwiGLU::Params{h, F, 1};
+  g.swiglu = EpiSwiGLU::Params{h, c->at<bf16>(c->L.hdense_lo), F, 1};
   CK(c->gemv(g, lc));
 
   GemvLaunch dn = dense_launch(c, w_down, 0, &rows->n, 0, rmax, kTagDenseDown);
   dn.src = SrcKind::Bf16;
-  dn.bf = SrcBf16::Params{h, F, 1, nullptr};
+  dn.bf = SrcBf16::Params{h, c->at<bf16>(c->L.hdense_lo), F, 1, nullptr};
   dn.epi = EpiKind::StoreAdd;
   dn.store = EpiStore<false>::Params{x, m.d_model, 1, nullptr};
   CK(c->gemv(dn, lc));
@@ -427,12 +431,12 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   gu.src = SrcKind::Norm;
   gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   gu.epi = EpiKind::SwiGLU;
-  gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot};
+  gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), c->at<bf16>(c->L.hbuf_lo), m.expert_ffn, nslot};
   CK(c->gemv(gu, lc));
 
   GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0, kTagExpDown);
   dn.src = SrcKind::Bf16;
-  dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), m.expert_ffn, nslot, nullptr};
+  dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), c->at<bf16>(c->L.hbuf_lo), m.expert_ffn, nslot, nullptr};
   dn.epi = EpiKind::Store;
   dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
   CK(c->gemv(dn, lc));
@@ -486,7 +490,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   float* xd = c->at<float>(c->L.xd);
   GemvLaunch fc = dense_launch(c, w.fc, 0, &rows->n, 0, rmax, kTagFC);
   fc.src = SrcKind::Bf16;
-  fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), 2 * m.d_model, 1, nullptr};
+  fc.bf = SrcBf16::Params{c->at<bf16>(c->L.fcin), c->at<bf16>(c->L.fcin_lo), 2 * m.d_model, 1, nullptr};
   fc.epi = EpiKind::Store;
   fc.store = EpiStore<false>::Params{xd, m.d_model, 1, nullptr};
   CK(c->gemv(fc, lc));
@@ -532,6 +536,7 @@ int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) 
     dp.g_h = c->dw.norm_h;
     dp.g_e = c->dw.norm_e;
     dp.fcin = c->at<bf16>(c->L.fcin);
+    dp.fcin_lo = c->at<bf16>(c->L.fcin_lo);
     dp.rows = c->rows();
     dp.rows_prev = c->rows();
     dp.status = c->status();
@@ -792,6 +797,8 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
       dp.g_h = c->dw.norm_h;
       dp.g_e = c->dw.norm_e;
       dp.fcin = c->at<bf16>(c->L.fcin);
+      dp.fcin_lo = c->at<bf16>(c->L.fcin_lo);
+    dp.fcin_lo = c->at<bf16>(c->L.fcin_lo);
       dp.rows = c->rows();
       dp.rows_prev = c->rows();
       dp.status = c->status();

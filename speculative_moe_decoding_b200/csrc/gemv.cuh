@@ -196,14 +196,30 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// Four floats as high and low bfloat16 parts (high = bf16(f), low = bf16(f - high)).
+__device__ __forceinline__ void split_bf16x4(float f0, float f1, float f2, float f3, uint2& hi, uint2& lo) {
+  const bf16 h0 = f2bf(f0), h1 = f2bf(f1), h2 = f2bf(f2), h3 = f2bf(f3);
+  hi.x = (uint32_t)__bfloat16_as_ushort(h0) | ((uint32_t)__bfloat16_as_ushort(h1) << 16);
+  hi.y = (uint32_t)__bfloat16_as_ushort(h2) | ((uint32_t)__bfloat16_as_ushort(h3) << 16);
+  lo.x = pack2(__fsub_rn(f0, bf2f(h0)), __fsub_rn(f1, bf2f(h1)));
+  lo.y = pack2(__fsub_rn(f2, bf2f(h2)), __fsub_rn(f3, bf2f(h3)));
+}
+
 // ---------------------------------------------------------------------------
 // activation sources: the B operand (row-set entry q = MMA column q)
 // ---------------------------------------------------------------------------
 
-// Rows of a float32 matrix, RMS-normalised, scaled by a gain vector and rounded
-// to bfloat16 (the GEMV input precision), kept in shared memory for the whole
-// kernel as bfloat16 rows of K + 8 elements (the pad makes the eight rows of
-// an ldmatrix fall in distinct banks).  Rows past R are zero.
+// Activations enter the MMAs as two bfloat16 parts, high = bf16(v) and
+// low = bf16(v - high), each multiplied with the weights and accumulated in
+// float32: the products carry float32-level precision of v (the only bfloat16
+// rounding left on the path is the weights' own).  Rows of a source: RG
+// high rows, then RG low rows; MMA column q >= RG reads row q % RG (its result
+// is never used).
+
+// Rows of a float32 matrix, RMS-normalised and scaled by a gain vector, kept in
+// shared memory for the whole kernel as high / low bfloat16 rows of K + 8
+// elements (the pad makes the eight rows of an ldmatrix fall in distinct
+// banks).
 struct SrcNorm {
   struct Params {
     const float* x;
@@ -215,7 +231,7 @@ struct SrcNorm {
   static constexpr bool kSmem = true;    // activations live in shared memory (prologue)
   static constexpr bool kStaged = false; // activations are not part of the weight stages
   static constexpr int kG = 2;           // float4 groups per thread per row: K <= 2048
-  __host__ __device__ static constexpr size_t smem_bytes(int K) { return (size_t)kRmax * (K + 8) * 2; }
+  __host__ __device__ static constexpr size_t smem_bytes(int K, int RG) { return (size_t)2 * RG * (K + 8) * 2; }
 
   // Gains are weights: loaded before the dependency wait.
   struct Pre {
@@ -236,23 +252,15 @@ struct SrcNorm {
   // All consumer threads, after the dependency wait.  Thread t owns the float4
   // groups t, t + 256 of each row, read straight from L2 (the rows were just
   // written by the previous kernel); rows go four at a time: sums of squares,
-  // one barrier, then the scaled bfloat16 values.
+  // one barrier, then the scaled values as high and low parts.
+  template <int RG>
   __device__ static void prologue(const Params& p, int K, int R, unsigned char* xsm, float* red, int tid,
                                   const Pre& pre) {
-    bf16* xb = reinterpret_cast<bf16*>(xsm);
+    bf16* xh = reinterpret_cast<bf16*>(xsm);
     const int ld = K + 8, ng = K / 4;
+    bf16* xl = xh + RG * ld;
     const int lane = tid & 31, warp = tid >> 5;
-    for (int rb = 0; rb < kRmax; rb += 4) {
-      if (rb >= R) {  // zero rows: MMA columns past R stay finite
-#pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
-#pragma unroll
-          for (int j = 0; j < kG; ++j) {
-            int m = tid + j * kConsumers;
-            if (m < ng) *reinterpret_cast<uint2*>(xb + (rb + rr) * ld + 4 * m) = make_uint2(0u, 0u);
-          }
-        continue;
-      }
+    for (int rb = 0; rb < R; rb += 4) {
       float4 v[4][kG];
       float a[4];
 #pragma unroll
@@ -285,21 +293,23 @@ struct SrcNorm {
 #pragma unroll
       for (int rr = 0; rr < 4; ++rr) {
         const int r = rb + rr;
-        float sc = 0.f;
-        if (r < R) {
-          float ss = 0.f;
+        if (r >= R) break;
+        float ss = 0.f;
 #pragma unroll
-          for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
-          sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
-        }
+        for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
+        const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)K), p.eps));
 #pragma unroll
         for (int j = 0; j < kG; ++j) {
           int m = tid + j * kConsumers;
           if (m < ng) {
-            uint2 o;
-            o.x = pack2(__fmul_rn(__fmul_rn(v[rr][j].x, sc), pre.g[j].x), __fmul_rn(__fmul_rn(v[rr][j].y, sc), pre.g[j].y));
-            o.y = pack2(__fmul_rn(__fmul_rn(v[rr][j].z, sc), pre.g[j].z), __fmul_rn(__fmul_rn(v[rr][j].w, sc), pre.g[j].w));
-            *reinterpret_cast<uint2*>(xb + r * ld + 4 * m) = o;
+            const float f0 = __fmul_rn(__fmul_rn(v[rr][j].x, sc), pre.g[j].x);
+            const float f1 = __fmul_rn(__fmul_rn(v[rr][j].y, sc), pre.g[j].y);
+            const float f2 = __fmul_rn(__fmul_rn(v[rr][j].z, sc), pre.g[j].z);
+            const float f3 = __fmul_rn(__fmul_rn(v[rr][j].w, sc), pre.g[j].w);
+            uint2 hi, lo;
+            split_bf16x4(f0, f1, f2, f3, hi, lo);
+            *reinterpret_cast<uint2*>(xh + r * ld + 4 * m) = hi;
+            *reinterpret_cast<uint2*>(xl + r * ld + 4 * m) = lo;
           }
         }
       }
@@ -307,37 +317,45 @@ struct SrcNorm {
     named_sync(1, kConsumers);
   }
 
-  // Shared address of B-fragment row data for ldmatrix.x2: row-set entry q of
-  // this lane (lane & 7), column k0 (+8 for lanes 8..15) of the slice start.
+  // Shared address of the high B-fragment row data for ldmatrix.x2: row `row`
+  // of this lane (lane & 7), column k0 (+8 for lanes 8..15) of the slice start;
+  // the low part is lo_offset bytes further.
   __device__ static uint32_t b_base(const unsigned char* xsm, const unsigned char* stage_x, int K, int row, int lane) {
     return smem_u32(xsm) + (uint32_t)(row * (K + 8) + ((lane >> 3) & 1) * 8) * 2;
   }
+  template <int RG>
+  __device__ static uint32_t lo_offset(int K) { return (uint32_t)(RG * (K + 8) * 2); }
   __device__ static uint32_t b_slice(int slc) { return (uint32_t)slc * kSlice * 2; }
 };
 
-// Rows of a bfloat16 matrix in global memory: row (row_src[r] * nslot + slot).
-// The producer copies each slice of the item's rows into the stage next to the
-// weight boxes (row-set entry q at offset q * kXStride), so consumers read them
-// from shared memory.
+// Rows of a bfloat16 matrix pair (high, low parts) in global memory: row
+// (row_src[r] * nslot + slot).  The producer copies each slice of the item's
+// rows into the stage next to the weight boxes (row-set entry q at slot q, its
+// low part at slot RG + q, kXStride apart), so consumers read them from shared
+// memory.
 struct SrcBf16 {
   struct Params {
-    const bf16* x;
+    const bf16* x;       // high parts
+    const bf16* x_lo;    // low parts (same layout)
     long long ld;
     int nslot;
     const int* row_src;
   };
   static constexpr bool kSmem = false;
   static constexpr bool kStaged = true;
-  __host__ __device__ static constexpr size_t smem_bytes(int) { return 0; }
+  __host__ __device__ static constexpr size_t smem_bytes(int, int) { return 0; }
   struct Pre {};
   __device__ static void pre_wait(const Params&, int, int, Pre&) {}
+  template <int RG>
   __device__ static void prologue(const Params&, int, int, unsigned char*, float*, int, const Pre&) {}
-  __device__ static const bf16* row_ptr(const Params& p, int r, int slot) {
-    return p.x + (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
+  __device__ static long long row_off(const Params& p, int r, int slot) {
+    return (long long)((p.row_src ? p.row_src[r] : r) * p.nslot + slot) * p.ld;
   }
-  __device__ static uint32_t b_base(const unsigned char*, const unsigned char* stage_x, int, int, int lane) {
-    return smem_u32(stage_x) + (uint32_t)((lane & 7) * kXStride + ((lane >> 3) & 1) * 16);
+  __device__ static uint32_t b_base(const unsigned char*, const unsigned char* stage_x, int, int row, int lane) {
+    return smem_u32(stage_x) + (uint32_t)(row * kXStride + ((lane >> 3) & 1) * 16);
   }
+  template <int RG>
+  __device__ static uint32_t lo_offset(int) { return (uint32_t)(RG * kXStride); }
   __device__ static uint32_t b_slice(int) { return 0; }
 };
 
@@ -376,10 +394,11 @@ struct EpiStore {
 };
 
 // SwiGLU on paired tiles (gate row n, up row n + pair_half):
-// h[(r * nslot + slot) * ld + n] = bf16(silu(gate) * up)
+// h[(r * nslot + slot) * ld + n] = silu(gate) * up, as high and low bfloat16 parts
 struct EpiSwiGLU {
   struct Params {
-    bf16* h;
+    bf16* h;      // high parts
+    bf16* h_lo;   // low parts (the next GEMV's second operand)
     long long ld;
     int nslot;
   };
@@ -390,7 +409,10 @@ struct EpiSwiGLU {
     float gt = o.v;
     float act = __fdiv_rn(gt, __fadd_rn(1.f, expf(-gt)));
     long long row = (long long)rs.r_sel(o.q) * p.nslot + rs.slot_sel(o.q);
-    p.h[row * p.ld + o.n] = f2bf(__fmul_rn(act, up));
+    const float hv = __fmul_rn(act, up);
+    const bf16 hi = f2bf(hv);
+    p.h[row * p.ld + o.n] = hi;
+    p.h_lo[row * p.ld + o.n] = f2bf(__fsub_rn(hv, bf2f(hi)));
   }
   __device__ static void finish(const Params&, const GemvShape&, int, int) {}
 };
@@ -602,17 +624,18 @@ __device__ __forceinline__ ItemPos item_pos(const GemvShape& s, int item) {
 }
 
 
-template <class Src>
+template <class Src, int RG>
 constexpr int stage_stride() {
-  // weights, then (staged sources) the slice rows; 1 KB-aligned for the swizzle
-  return Src::kStaged ? (kStageBytes + kRmax * kXStride + 1023) / 1024 * 1024 : kStageBytes;
+  // weights, then (staged sources) the slice rows, high and low; 1 KB-aligned
+  // for the swizzle
+  return Src::kStaged ? (kStageBytes + 2 * RG * kXStride + 1023) / 1024 * 1024 : kStageBytes;
 }
 
 // Dynamic shared memory of one CTA: 1 KB alignment slack, the ring, the
 // source's rows and the quarter partials.
-template <class Src>
+template <class Src, int RG>
 constexpr size_t gemv_smem_bytes(int K) {
-  return 1024 + (size_t)kStages * stage_stride<Src>() + Src::smem_bytes(K) + kRedFloats * 4;
+  return 1024 + (size_t)kStages * stage_stride<Src, RG>() + Src::smem_bytes(K, RG) + kRedFloats * 4;
 }
 
 template <int RG, class Src, class Epi>
@@ -629,11 +652,11 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
   TraceMarks tm;  // trace (consumer thread 0): wait returned, prologue done, main loop done
-  constexpr int kStride = stage_stride<Src>();
+  constexpr int kStride = stage_stride<Src, RG>();
   // the 128-byte swizzle repeats every 1 KB: the ring starts on a 1 KB boundary
   unsigned char* stages = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   unsigned char* xsm = stages + kStages * kStride;
-  float* red = reinterpret_cast<float*>(xsm + Src::smem_bytes(s.K));
+  float* red = reinterpret_cast<float*>(xsm + Src::smem_bytes(s.K, RG));
   const bool paired = s.pair_half != 0;
 
   if (tid == 0) {
@@ -696,13 +719,16 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       const int st = j % kStages;
       unsigned char* dst = stages + st * kStride + kStageBytes;
       const int cols = min(kSlice, s.K - slc * kSlice);
-      mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(prs.n * cols * 2));
+      const int nq = min(prs.n, RG);
+      mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(2 * nq * cols * 2));
+      const SrcBf16::Params& bp = reinterpret_cast<const SrcBf16::Params&>(sp);
 #pragma unroll
-      for (int q = 0; q < kRmax; ++q)
-        if (q < prs.n)
-          bulk_g2s(dst + q * kXStride,
-                   SrcBf16::row_ptr(reinterpret_cast<const SrcBf16::Params&>(sp), prs.r(q), prs.slot(q)) + slc * kSlice,
-                   cols * 2, &full_bar[st]);
+      for (int q = 0; q < RG; ++q)
+        if (q < nq) {
+          const long long off = SrcBf16::row_off(bp, prs.r(q), prs.slot(q)) + slc * kSlice;
+          bulk_g2s(dst + q * kXStride, bp.x + off, cols * 2, &full_bar[st]);
+          bulk_g2s(dst + (RG + q) * kXStride, bp.x_lo + off, cols * 2, &full_bar[st]);
+        }
     };
     // items are claimed from the launch's work counter, so faster SMs take more
     int total = s.mats ? 0 : s.tiles_per_mat * s.kparts;
@@ -802,7 +828,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   __shared__ int s_last_part;
 
   epi_init<Epi>(tid);
-  Src::prologue(sp, s.K, R, xsm, red_pro, tid, pre);
+  Src::template prologue<RG>(sp, s.K, R, xsm, red_pro, tid, pre);
   if (!Src::kSmem) named_sync(1, kConsumers);
   if (tid == 0) tm.t1 = gtimer();
 
@@ -840,8 +866,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 #pragma unroll
       for (int q = 0; q < kRmax; ++q) rs.e[q] = s_rs[st0][1 + q];
     }
-    // B rows of this lane: row-set entry (lane & 7)
-    const int brow = rs.r_sel(lane & 7);
+    // B rows of this lane: row-set entry (lane & 7); columns past RG reuse row q % RG
+    const int bq = (lane & 7) % RG;
+    const int brow = Src::kStaged ? bq : rs.r_sel(bq);
+    const uint32_t b_lo = Src::template lo_offset<RG>(s.K);
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     for (int sl = ip.sl0; sl < ip.sl1; ++sl, ++it) {
       const int st = it % kStages;
@@ -853,10 +881,12 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
                                 (uint32_t)kq * kChunk * 2;
 #pragma unroll
         for (int k16 = 0; k16 < kChunk / 16; ++k16) {
-          uint32_t a[4], b[2];
+          uint32_t a[4], bh[2], bl[2];
           ldsm_x4(a_base + (uint32_t)((((2 * k16 + a_hi) ^ a_sw)) << 4), a);
-          ldsm_x2(b_addr + k16 * 32, b);
-          mma_bf16(d, a, b);
+          ldsm_x2(b_addr + k16 * 32, bh);
+          ldsm_x2(b_addr + b_lo + k16 * 32, bl);
+          mma_bf16(d, a, bh);
+          mma_bf16(d, a, bl);
         }
       }
       __syncwarp();

@@ -103,15 +103,10 @@ cudaError_t encode_oproj_map(const void* base, int d, int Dh, CUtensorMap* out) 
   return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
-template <class Src>
-static size_t smem_max() {
-  return gemv_smem_bytes<Src>(kGemvMaxK);
-}
-
 template <int RG, class Src, class Epi>
 static cudaError_t configure_one() {
   cudaError_t e = cudaFuncSetAttribute(gemv_kernel<RG, Src, Epi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)smem_max<Src>());
+                                       (int)gemv_smem_bytes<Src, RG>(kGemvMaxK));
   // every kernel of the library asks for the same (maximal) shared-memory
   // carveout, so consecutive kernels never wait for an SM reconfiguration
   if (e == cudaSuccess)
@@ -146,9 +141,13 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
                               const LaunchCfg& lc) {
   auto kern = gemv_kernel<RG, Src, Epi>;
   if (Src::kSmem && g.s.K > kGemvMaxK) return cudaErrorInvalidValue;
-  const size_t smem = gemv_smem_bytes<Src>(g.s.K);
-  // two CTAs per SM hide each other's latencies
-  const int slots = 2 * lc.num_sms;
+  const size_t smem = gemv_smem_bytes<Src, RG>(g.s.K);
+  // as many CTAs per SM as fit (two for the common shapes: they hide each
+  // other's latencies)
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kGemvThreads, smem) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
+  const int slots = std::min(per_sm, 2) * lc.num_sms;
   int grid = g.grid > 0 ? std::min(g.grid, slots) : slots;
   if (!g.s.mats) grid = std::min(grid, g.s.tiles_per_mat * g.s.kparts);
   return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);

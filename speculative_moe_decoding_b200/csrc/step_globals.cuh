@@ -211,7 +211,7 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
     pr.last_row[b] = p.mode == 2 ? p.n - 1 : (nrows > 0 ? row0 + nrows - 1 : 0);
   }
   __syncthreads();
-  // fcin[r] = [bf16(RMSNorm(h_r) * g_h) ; bf16(RMSNorm(e_r) * g_e)]: all 256
+  // fcin[r] = [RMSNorm(h_r) * g_h ; RMSNorm(e_r) * g_e] as high / low bf16 parts: all 256
   // threads per row, the sums of every row reduced in one round
   const int d = p.d;
   const int nrow = pr.n;
@@ -269,8 +269,13 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
 #pragma unroll 4
     for (int n = tid; n < d; n += 256) {
       float e = ev ? ev[n] : bf2f(eb[n]);
-      p.fcin[(long long)r * 2 * d + n] = f2bf(__fmul_rn(__fmul_rn(h[n], ch), bf2f(p.g_h[n])));
-      p.fcin[(long long)r * 2 * d + d + n] = f2bf(__fmul_rn(__fmul_rn(e, ce), bf2f(p.g_e[n])));
+      const float zh = __fmul_rn(__fmul_rn(h[n], ch), bf2f(p.g_h[n]));
+      const float ze = __fmul_rn(__fmul_rn(e, ce), bf2f(p.g_e[n]));
+      const bf16 hh = f2bf(zh), he = f2bf(ze);
+      p.fcin[(long long)r * 2 * d + n] = hh;
+      p.fcin[(long long)r * 2 * d + d + n] = he;
+      p.fcin_lo[(long long)r * 2 * d + n] = f2bf(__fsub_rn(zh, bf2f(hh)));
+      p.fcin_lo[(long long)r * 2 * d + d + n] = f2bf(__fsub_rn(ze, bf2f(he)));
     }
   }
   // publish the row metadata

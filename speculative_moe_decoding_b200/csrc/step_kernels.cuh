@@ -250,7 +250,8 @@ struct DraftSetupParams {
   const bf16* embed;
   const bf16* g_h;
   const bf16* g_e;
-  bf16* fcin;            // [R][2d]
+  bf16* fcin;            // [R][2d] high parts
+  bf16* fcin_lo;         // [R][2d] low parts
   PassRows* rows;        // written
   const PassRows* rows_prev;  // mode 1: rows of the previous recursion (last_row)
   int* status;
