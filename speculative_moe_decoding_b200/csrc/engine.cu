@@ -435,7 +435,8 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   CK(c->gemv(gu, lc));
 
   GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0, kTagExpDown);
-  dn.src = SrcKind::Bf16;
+  // the rows of an expert item are copied once per item when they are short
+  dn.src = m.expert_ffn <= SrcBf16Item::kMaxK ? SrcKind::Bf16Item : SrcKind::Bf16;
   dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), c->at<bf16>(c->L.hbuf_lo), m.expert_ffn, nslot, nullptr};
   dn.epi = EpiKind::Store;
   dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};

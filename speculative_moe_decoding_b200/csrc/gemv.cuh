@@ -359,6 +359,41 @@ struct SrcBf16 {
   __device__ static uint32_t b_slice(int) { return 0; }
 };
 
+// The same rows, copied once per work item instead of once per stage: at an
+// item's first stage the producer copies the item's whole rows (high and low
+// parts, K + 8 elements apart) into one of two item buffers, so a stage
+// carries only weights.  Consumers release a buffer (x_empty barrier) after
+// the item's last stage.  For short rows (K <= 1024): the expert down
+// projections, whose per-stage copies made the producer thread the bottleneck.
+struct SrcBf16Item {
+  typedef SrcBf16::Params Params;
+  static constexpr bool kSmem = false;
+  static constexpr bool kStaged = true;   // activations arrive with the stages (second arrival)
+  static constexpr bool kItemX = true;
+  static constexpr int kMaxK = 1024;
+  __host__ __device__ static constexpr size_t buf_bytes(int K, int RG) { return (size_t)2 * RG * (K + 8) * 2; }
+  __host__ __device__ static constexpr size_t smem_bytes(int K, int RG) { return 2 * buf_bytes(K, RG); }
+  struct Pre {};
+  __device__ static void pre_wait(const Params&, int, int, Pre&) {}
+  template <int RG>
+  __device__ static void prologue(const Params&, int, int, unsigned char*, float*, int, const Pre&) {}
+  __device__ static uint32_t b_base(const unsigned char* xbuf, const unsigned char*, int K, int row, int lane) {
+    return smem_u32(xbuf) + (uint32_t)(row * (K + 8) + ((lane >> 3) & 1) * 8) * 2;
+  }
+  template <int RG>
+  __device__ static uint32_t lo_offset(int K) { return (uint32_t)(RG * (K + 8) * 2); }
+  __device__ static uint32_t b_slice(int slc) { return (uint32_t)slc * kSlice * 2; }
+};
+
+template <class Src>
+struct ItemX {
+  static constexpr bool value = false;
+};
+template <>
+struct ItemX<SrcBf16Item> {
+  static constexpr bool value = true;
+};
+
 // ---------------------------------------------------------------------------
 // epilogues: run by one warp on its 4 reduced rows.  Lane L = 8 i + q holds
 // (in v) the result of local row i for pass-row slot q of the item's row set.
@@ -628,7 +663,7 @@ template <class Src, int RG>
 constexpr int stage_stride() {
   // weights, then (staged sources) the slice rows, high and low; 1 KB-aligned
   // for the swizzle
-  return Src::kStaged ? (kStageBytes + 2 * RG * kXStride + 1023) / 1024 * 1024 : kStageBytes;
+  return Src::kStaged && !ItemX<Src>::value ? (kStageBytes + 2 * RG * kXStride + 1023) / 1024 * 1024 : kStageBytes;
 }
 
 // Dynamic shared memory of one CTA: 1 KB alignment slack, the ring, the
@@ -643,7 +678,7 @@ __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
             const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], x_empty[2];
   __shared__ int s_tag[kStages];               // item of the stage's slice (set with its first slice), -1 = end
   __shared__ int s_rs[kStages][kRmax + 1];     // expert mode: the item's row set (n, entries), with its first slice
   __shared__ float red_pro[kRmax * kNW];
@@ -664,6 +699,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       mbar_init(&full_bar[i], Src::kStaged ? 2 : 1);
       mbar_init(&empty_bar[i], kNW);
     }
+    mbar_init(&x_empty[0], kNW);
+    mbar_init(&x_empty[1], kNW);
     fence_mbar_init();
   }
   __syncthreads();
@@ -713,10 +750,34 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       tma_load_box(dst + kBoxBytes, map, slc * (kSlice / kChunk), r1, ce, &full_bar[st]);
       ++it;
     };
-    auto issue_x = [&](uint32_t j, int m, int slc) {
+    uint32_t xitems = 0;  // item buffers handed out (item-resident sources)
+    auto issue_x = [&](uint32_t j, int m, int slc, bool first) {
       if (!Src::kStaged) return;
       rows_of(m);
       const int st = j % kStages;
+      if (ItemX<Src>::value) {
+        if (!first) {  // the item's rows came with its first stage
+          mbar_arrive(&full_bar[st]);
+          return;
+        }
+        const int xb = xitems & 1;
+        const uint32_t use = xitems >> 1;
+        if (use > 0) mbar_wait(&x_empty[xb], (use - 1) & 1, s.status);  // consumers are done with it
+        ++xitems;
+        const int nq = min(prs.n, RG);
+        const int ld = s.K + 8;
+        unsigned char* xb_dst = xsm + xb * SrcBf16Item::buf_bytes(s.K, RG);
+        mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(2 * nq * s.K * 2));
+        const SrcBf16::Params& bp = reinterpret_cast<const SrcBf16::Params&>(sp);
+#pragma unroll
+        for (int q = 0; q < RG; ++q)
+          if (q < nq) {
+            const long long off = SrcBf16::row_off(bp, prs.r(q), prs.slot(q));
+            bulk_g2s(xb_dst + (size_t)q * ld * 2, bp.x + off, s.K * 2, &full_bar[st]);
+            bulk_g2s(xb_dst + (size_t)(RG + q) * ld * 2, bp.x_lo + off, s.K * 2, &full_bar[st]);
+          }
+        return;
+      }
       unsigned char* dst = stages + st * kStride + kStageBytes;
       const int cols = min(kSlice, s.K - slc * kSlice);
       const int nq = min(prs.n, RG);
@@ -736,6 +797,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     // first item are requested before the dependency wait (one item only, so
     // that CTAs resident early do not take the work of those still arriving)
     int pre_sl[kStages];
+    bool pre_first[kStages];
     int npre = 0;
     int item = -1, sl = 0, sl_end = 0;
     auto claim = [&]() {
@@ -752,6 +814,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       if (item < total) {
         const ItemPos ip = item_pos(s, item);
         while (sl < sl_end && it < (uint32_t)kStages) {
+          pre_first[npre] = sl == ip.sl0;
           pre_sl[npre++] = sl;
           issue_w(item, 0, ip.t, sl, sl == ip.sl0);
           ++sl;
@@ -763,14 +826,14 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     const bool ok = !status_bad(s.status);
     if (ok) {
       R = min(pass_rows(s), RG);
-      for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j]);
+      for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j], pre_first[j]);
       if (s.mats) total = *s.n_mats * s.tiles_per_mat;
       if (!claimed) claim();
       while (item < total) {
         const ItemPos ip = item_pos(s, item);
         const uint32_t j = it;
         issue_w(item, ip.m, ip.t, sl, sl == ip.sl0);
-        issue_x(j, ip.m, sl);
+        issue_x(j, ip.m, sl, sl == ip.sl0);
         if (++sl == sl_end) claim();
       }
     } else if (Src::kStaged) {
@@ -877,7 +940,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       if (sl * (kSlice / kChunk) + kq < nchunks) {
         const unsigned char* stg = stages + st * kStride;
         const uint32_t a_base = smem_u32(stg) + a_off;
-        const uint32_t b_addr = Src::b_base(xsm, stg + kStageBytes, s.K, brow, lane) + Src::b_slice(sl) +
+        const unsigned char* xsrc = ItemX<Src>::value ? xsm + (nitem & 1) * SrcBf16Item::buf_bytes(s.K, RG) : xsm;
+        const uint32_t b_addr = Src::b_base(xsrc, stg + kStageBytes, s.K, brow, lane) + Src::b_slice(sl) +
                                 (uint32_t)kq * kChunk * 2;
 #pragma unroll
         for (int k16 = 0; k16 < kChunk / 16; ++k16) {
@@ -892,6 +956,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
+    if (ItemX<Src>::value && lane == 0) mbar_arrive(&x_empty[nitem & 1]);  // the item's rows are no longer read
     // quarter partials -> shared, then every output adds its quarters in order
     float* rb = red + (nitem & 1) * (4 * kTile * 8);
     ++nitem;

@@ -133,6 +133,7 @@ cudaError_t gemv_prepare() {
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmaxAccept>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<true>>();
+  if (e == cudaSuccess) e = configure_rg<SrcBf16Item, EpiStore<false>>();
   return e;
 }
 
@@ -184,6 +185,10 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
       }
       default: return cudaErrorInvalidValue;
     }
+  }
+  if (g.src == SrcKind::Bf16Item) {
+    if (g.s.K > SrcBf16Item::kMaxK || g.epi != EpiKind::Store) return cudaErrorInvalidValue;
+    return launch_rg<SrcBf16Item, EpiStore<false>>(g, g.bf, g.store, lc);
   }
   switch (g.epi) {
     case EpiKind::Store: return launch_rg<SrcBf16, EpiStore<false>>(g, g.bf, g.store, lc);

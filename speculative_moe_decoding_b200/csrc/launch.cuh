@@ -51,7 +51,7 @@ cudaError_t launch_cluster_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-enum class SrcKind { Norm, Bf16 };
+enum class SrcKind { Norm, Bf16, Bf16Item };
 enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, Route, ArgmaxAccept };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.
