@@ -110,11 +110,13 @@ __device__ __forceinline__ void tma_load_kv(void* dst, const CUtensorMap* map, i
 
 // 3-D tensor-map load of a W_o block: 64 columns x nb rows x Dh/64 chunks at
 // (row r0, column chunk c0) -> [chunk][row][128 B].
+// The weights are read once per pass: evict-first in L2.
 __device__ __forceinline__ void tma_load_wo(void* dst, const CUtensorMap* map, int r0, int c0, uint64_t* bar) {
   asm volatile(
-      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(r0), "r"(c0), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4}], [%5], %6;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(r0), "r"(c0), "r"(smem_u32(bar)),
+      "l"(l2_evict_first_policy())
       : "memory");
 }
 

@@ -114,6 +114,15 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* s
 }
 
 // ---- bulk copy global -> shared (TMA unit, no multicast) ------------------
+// L2 policy for data read once per step (weights): their lines are the first
+// to be evicted, so the step's reused data - KV caches, activations, kernel
+// code - stays in L2 while gigabytes of weights stream past.
+__device__ __forceinline__ uint64_t l2_evict_first_policy() {
+  uint64_t pol;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(pol));
+  return pol;
+}
+
 // dst, src 16-byte aligned; bytes a multiple of 16.
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(

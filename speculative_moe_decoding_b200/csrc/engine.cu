@@ -195,6 +195,9 @@ cudaError_t prepare_kernels_now() {
   if (e == cudaSuccess) e = max_carveout(combine_kernel);
   if (e == cudaSuccess) e = max_carveout(verify_setup_kernel);
   if (e == cudaSuccess) e = max_carveout(prefill_setup_kernel);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(draft_setup_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)draft_setup_smem_bytes(kGemvMaxK));
   if (e == cudaSuccess) e = max_carveout(draft_setup_kernel);
   if (e == cudaSuccess) e = max_carveout(accept_kernel);
   if (e == cudaSuccess) e = max_carveout(force_kernel);
@@ -541,7 +544,7 @@ int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) 
     dp.rows = c->rows();
     dp.rows_prev = c->rows();
     dp.status = c->status();
-    CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
+    CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), draft_setup_smem_bytes(m.d_model), lc, dp));
     int rmax = j == 1 ? std::min(kRmax, B * (m.max_k + 1)) : B;
     int st = draft_block(c, lc, rmax, false, props + (j - 1), k, j);
     if (st) return st;
@@ -764,7 +767,6 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
   if ((n_visual > 0 && !visual) || (n_prompt > 0 && !prompt)) return OCRDEC_EINVAL;
   if (C + m.max_k + 2 > m.kv_capacity) return OCRDEC_ECAPACITY;
   LaunchCfg lc = c->lc(reinterpret_cast<cudaStream_t>(stream));
-  int last_p0 = 0;
   for (int p0 = 0; p0 < C; p0 += kPrefillChunk) {
     const int n = std::min(kPrefillChunk, C - p0);
     PrefillSetupParams ps{slot, p0, n, n_visual, m.vocab, n_prompt, visual, prompt, c->embed, m.d_model,
@@ -776,7 +778,6 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
       st = lm_head(c, lc, 1, c->at<float>(c->L.x), c->final_norm, c->rows()->last_row, nullptr, 1,
                    c->at<int>(c->L.gtok), 1, nullptr, 0);
       if (st) return st;
-      last_p0 = p0;
     }
     const int q1 = std::min(p0 + n, C - 1);
     if (q1 > p0) {
@@ -811,7 +812,7 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
                                first_token, c->status()};
         CK(launch_ex(prefill_finish_kernel, dim3(1), dim3(256), 0, lc, pf));
       }
-      CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), 0, lc, dp));
+      CK(launch_ex(draft_setup_kernel, dim3(1), dim3(256), draft_setup_smem_bytes(m.d_model), lc, dp));
       st = draft_block(c, lc, q1 - p0, true, nullptr, 0, 0);
       if (st) return st;
     } else if (p0 + n == C) {
@@ -821,7 +822,6 @@ int ocrdec_prefill(ocrdec_ctx* c, int slot, const float* visual, int n_visual, c
       CK(launch_ex(prefill_finish_kernel, dim3(1), dim3(256), 0, lc, pf));
     }
   }
-  (void)last_p0;
   return OCRDEC_OK;
 }
 

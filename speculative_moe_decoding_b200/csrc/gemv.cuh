@@ -170,11 +170,11 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
 // `mat`, starting at column chunk c4 and row `row`; shared layout
 // [chunk][row][128 B] with the 128-byte swizzle.
 __device__ __forceinline__ void tma_load_box(void* dst, const CUtensorMap* map, int c4, int row, int mat,
-                                             uint64_t* bar) {
+                                             uint64_t* bar, uint64_t policy) {
   asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(c4), "r"(mat), "r"(smem_u32(bar))
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(0), "r"(row), "r"(c4), "r"(mat), "r"(smem_u32(bar)), "l"(policy)
       : "memory");
 }
 
@@ -712,6 +712,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     int R = 0;
     RowSet prs;  // rows of the current item (expert mode / staged sources)
     int prs_m = -1;
+    const uint64_t wpol = l2_evict_first_policy();  // weights are read once per pass
     auto stage_wait = [&](int st) {
       // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
       // stays uniform so the block always terminates
@@ -746,8 +747,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       }
       mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
       unsigned char* dst = stages + st * kStride;
-      tma_load_box(dst, map, slc * (kSlice / kChunk), r0, ce, &full_bar[st]);
-      tma_load_box(dst + kBoxBytes, map, slc * (kSlice / kChunk), r1, ce, &full_bar[st]);
+      tma_load_box(dst, map, slc * (kSlice / kChunk), r0, ce, &full_bar[st], wpol);
+      tma_load_box(dst + kBoxBytes, map, slc * (kSlice / kChunk), r1, ce, &full_bar[st], wpol);
       ++it;
     };
     uint32_t xitems = 0;  // item buffers handed out (item-resident sources)

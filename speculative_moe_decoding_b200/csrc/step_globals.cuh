@@ -52,16 +52,21 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   __shared__ int s_bad;
   const int tid = threadIdx.x;
   const int K1 = p.k + 1, R = p.B * K1;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
   pdl_wait();
   TraceMarks tm;
   if (tid == 0) tm.t0 = gtimer();
-  if (tid == 0) s_bad = status_bad(p.status);
-  __syncthreads();
-  if (s_bad) return;
+  // the status, slot state and proposals are read together
+  int kv = 0, t = 0;
   if (tid < R) {
     const int b = tid / K1, i = tid - b * K1;
-    const int kv = p.slots[b].kv_len;
-    int t = i == 0 ? p.slots[b].bonus : p.proposals[b * p.k + i - 1];
+    kv = p.slots[b].kv_len;
+    t = i == 0 ? p.slots[b].bonus : p.proposals[b * p.k + i - 1];
+  }
+  if (tid == 0 && status_bad(p.status)) s_bad = 1;
+  if (tid < R) {
+    const int b = tid / K1, i = tid - b * K1;
     if (kv + K1 > p.cap) {
       set_status(p.status, OCRDEC_ECAPACITY);
       s_bad = 1;
@@ -89,14 +94,28 @@ __global__ void __launch_bounds__(256) verify_setup_kernel(const VerifySetupPara
   __syncthreads();
   if (s_bad) return;
   pdl_trigger();
-  // embedding gather: every row's loads are issued before any is consumed
+  // embedding gather, 8 columns per load: every load is issued before any
+  // store (R * d / 8 <= 8 * 256)
+  const int per_row = p.d / 8, total = R * per_row;
+  uint4 v[8];
 #pragma unroll
-  for (int r = 0; r < kRmax; ++r) {
-    if (r >= R) break;
-    const bf16* e = p.embed + (long long)s_tok[r] * p.d;
-    float* xr = p.x + (long long)r * p.d;
-#pragma unroll 8
-    for (int n = tid; n < p.d; n += 256) xr[n] = bf2f(e[n]);
+  for (int i = 0; i < 8; ++i) {
+    const int idx = tid + 256 * i;
+    if (idx < total) {
+      const int r = idx / per_row, c = idx - r * per_row;
+      v[i] = ld_nc_v4(p.embed + (long long)s_tok[r] * p.d + c * 8);
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int idx = tid + 256 * i;
+    if (idx < total) {
+      const int r = idx / per_row, c = idx - r * per_row;
+      const bf16* b = reinterpret_cast<const bf16*>(&v[i]);
+      float4* xr = reinterpret_cast<float4*>(p.x + (long long)r * p.d + c * 8);
+      xr[0] = make_float4(bf2f(b[0]), bf2f(b[1]), bf2f(b[2]), bf2f(b[3]));
+      xr[1] = make_float4(bf2f(b[4]), bf2f(b[5]), bf2f(b[6]), bf2f(b[7]));
+    }
   }
   if (tid == 0) trace_end(p.status, 42, tm);
 }
@@ -145,14 +164,32 @@ __global__ void __launch_bounds__(256) prefill_setup_kernel(const PrefillSetupPa
   }
 }
 
+// The draft's input rows (DraftSetupParams).  The gains, each row's hidden
+// state and its token embedding arrive in shared memory by bulk copies (the
+// gains before the grid dependency wait); warp r then normalises row r.
 __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams p) {
+  extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ int s_bad;
   __shared__ PassRows pr;
-  __shared__ int s_pend[kRmax], s_ppos[kRmax], s_kv[kRmax], s_prev_last[kRmax];
+  __shared__ int s_pend[kRmax], s_ppos[kRmax], s_kv[kRmax], s_prev_last[kRmax], s_dtok[kRmax];
+  __shared__ uint64_t bars[2];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int d = p.d;
+  bf16* sg = reinterpret_cast<bf16*>(dsm);                  // [2][d] g_h, g_e
+  float* sh_rows = reinterpret_cast<float*>(dsm + 4 * d);  // [kRmax][d] hidden rows
+  bf16* se_rows = reinterpret_cast<bf16*>(sh_rows + kRmax * d);  // [kRmax][d] embedding rows
+  if (tid == 0) {
+    mbar_init(&bars[0], 1);
+    mbar_init(&bars[1], 1);
+    fence_mbar_init();
+    mbar_arrive_expect_tx(&bars[0], 4 * d);
+    bulk_g2s(sg, p.g_h, 2 * d, &bars[0]);
+    bulk_g2s(sg + d, p.g_e, 2 * d, &bars[0]);
+  }
   pdl_wait();
   TraceMarks tm;
   if (tid == 0) tm.t0 = gtimer();
+  // status, slot state, previous draft tokens and rows: one round of loads
   if (tid == 0) s_bad = status_bad(p.status);
   if (tid < kRmax) {
     const bool live = tid < p.B;
@@ -160,9 +197,13 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
     s_ppos[tid] = live && p.mode == 0 ? p.slots[tid].pend_pos : 0;
     s_kv[tid] = live && p.mode == 1 ? p.slots[tid].kv_len : 0;
     s_prev_last[tid] = p.mode == 1 ? p.rows_prev->last_row[tid] : 0;
+    s_dtok[tid] = live && p.mode == 1 ? p.dtok[tid * p.dtok_stride] : 0;
   }
   __syncthreads();
-  if (s_bad) return;
+  if (s_bad) {
+    if (tid == 0) mbar_wait(&bars[0], 0, p.status);  // the gains' copy lands before exit
+    return;
+  }
   pdl_trigger();
   // row metadata: thread r < kRmax fills row r; thread kRmax + b the per-slot fields
   if (tid < kRmax) {
@@ -178,7 +219,7 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
       if (slot >= 0) tok = p.hist[slot * p.hist_ld + pos + 1];
     } else if (p.mode == 1) {
       n = p.B;
-      if (r < p.B) { slot = r; pos = s_kv[r] + p.j - 2; tok = p.dtok[r * p.dtok_stride]; }
+      if (r < p.B) { slot = r; pos = s_kv[r] + p.j - 2; tok = s_dtok[r]; }
     } else {
       n = p.n;
       if (r < p.n) {
@@ -211,73 +252,64 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
     pr.last_row[b] = p.mode == 2 ? p.n - 1 : (nrows > 0 ? row0 + nrows - 1 : 0);
   }
   __syncthreads();
-  // fcin[r] = [RMSNorm(h_r) * g_h ; RMSNorm(e_r) * g_e] as high / low bf16 parts: all 256
-  // threads per row, the sums of every row reduced in one round
-  const int d = p.d;
-  const int nrow = pr.n;
-  __shared__ float red[8][kRmax][2];
-  __shared__ const float* s_h[kRmax];
-  __shared__ const float* s_ev[kRmax];
-  __shared__ const bf16* s_eb[kRmax];
-  if (tid < nrow) {
-    const int r = tid, b = pr.slot[r];
-    const float* h;
-    if (p.mode == 0) h = p.hpend + ((long long)b * (p.max_k + 1) + (r - pr.slot_row0[b])) * d;
-    else if (p.mode == 1) h = p.xd + (long long)s_prev_last[b] * d;
-    else h = p.xv + (long long)r * d;
-    const int tok = pr.tok[r];
-    s_h[r] = h;
-    s_ev[r] = (p.mode == 2 && tok < 0) ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
-    s_eb[r] = p.embed + (long long)(tok < 0 ? 0 : tok) * d;
+  const int nrow = min(pr.n, kRmax);
+  // one thread requests every row: the hidden state (float) and the token
+  // embedding (bf16); a visual vector (prefill) is read in place
+  if (tid == 0) {
+    uint32_t bytes = 0;
+    for (int r = 0; r < nrow; ++r) bytes += 4 * d + (pr.tok[r] < 0 ? 0 : 2 * d);
+    mbar_arrive_expect_tx(&bars[1], bytes);
+    for (int r = 0; r < nrow; ++r) {
+      const int b = pr.slot[r], tok = pr.tok[r];
+      const float* h;
+      if (p.mode == 0) h = p.hpend + ((long long)b * (p.max_k + 1) + (r - pr.slot_row0[b])) * d;
+      else if (p.mode == 1) h = p.xd + (long long)s_prev_last[b] * d;
+      else h = p.xv + (long long)r * d;
+      bulk_g2s(sh_rows + r * d, h, 4 * d, &bars[1]);
+      if (tok >= 0) bulk_g2s(se_rows + r * d, p.embed + (long long)tok * d, 2 * d, &bars[1]);
+    }
+    tm.t1 = gtimer();
   }
-  __syncthreads();
-  float sh[kRmax], se[kRmax];
-#pragma unroll
-  for (int r = 0; r < kRmax; ++r) {
-    sh[r] = 0.f;
-    se[r] = 0.f;
-    if (r < nrow) {
-      const float* h = s_h[r];
-      const float* ev = s_ev[r];
-      const bf16* eb = s_eb[r];
-#pragma unroll 4
-      for (int n = tid; n < d; n += 256) {
-        float hv = h[n];
-        float e = ev ? ev[n] : bf2f(eb[n]);
-        sh[r] = __fmaf_rn(hv, hv, sh[r]);
-        se[r] = __fmaf_rn(e, e, se[r]);
-      }
+  mbar_wait(&bars[0], 0, p.status);
+  mbar_wait(&bars[1], 0, p.status);
+  // fcin[r] as high / low bf16 parts; warp r normalises row r
+  if (warp < nrow) {
+    const int r = warp, tok = pr.tok[r];
+    const float* hr = sh_rows + r * d;
+    const bf16* er = se_rows + r * d;
+    const float* ev = tok < 0 ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
+    float sh = 0.f, se = 0.f;
+    for (int n = lane; n < d; n += 32) {
+      const float hv = hr[n];
+      const float e = ev ? ev[n] : bf2f(er[n]);
+      sh = __fmaf_rn(hv, hv, sh);
+      se = __fmaf_rn(e, e, se);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      sh[r] = __fadd_rn(sh[r], __shfl_xor_sync(0xffffffffu, sh[r], o));
-      se[r] = __fadd_rn(se[r], __shfl_xor_sync(0xffffffffu, se[r], o));
+      sh = __fadd_rn(sh, __shfl_xor_sync(0xffffffffu, sh, o));
+      se = __fadd_rn(se, __shfl_xor_sync(0xffffffffu, se, o));
     }
-    if (lane == 0) { red[warp][r][0] = sh[r]; red[warp][r][1] = se[r]; }
-  }
-  __syncthreads();
+    const float ch = rsqrtf(__fadd_rn(__fdiv_rn(sh, (float)d), p.eps));
+    const float ce = rsqrtf(__fadd_rn(__fdiv_rn(se, (float)d), p.eps));
+    bf16* hi = p.fcin + (long long)r * 2 * d;
+    bf16* lo = p.fcin_lo + (long long)r * 2 * d;
+    for (int n = 2 * lane; n < 2 * d; n += 64) {  // column pairs of [h ; e]
+      float z[2];
 #pragma unroll
-  for (int r = 0; r < kRmax; ++r) {
-    if (r >= nrow) break;
-    float a = 0.f, c = 0.f;
-    for (int w = 0; w < 8; ++w) { a = __fadd_rn(a, red[w][r][0]); c = __fadd_rn(c, red[w][r][1]); }
-    const float ch = rsqrtf(__fadd_rn(__fdiv_rn(a, (float)d), p.eps));
-    const float ce = rsqrtf(__fadd_rn(__fdiv_rn(c, (float)d), p.eps));
-    const float* h = s_h[r];
-    const float* ev = s_ev[r];
-    const bf16* eb = s_eb[r];
-#pragma unroll 4
-    for (int n = tid; n < d; n += 256) {
-      float e = ev ? ev[n] : bf2f(eb[n]);
-      const float zh = __fmul_rn(__fmul_rn(h[n], ch), bf2f(p.g_h[n]));
-      const float ze = __fmul_rn(__fmul_rn(e, ce), bf2f(p.g_e[n]));
-      const bf16 hh = f2bf(zh), he = f2bf(ze);
-      p.fcin[(long long)r * 2 * d + n] = hh;
-      p.fcin[(long long)r * 2 * d + d + n] = he;
-      p.fcin_lo[(long long)r * 2 * d + n] = f2bf(__fsub_rn(zh, bf2f(hh)));
-      p.fcin_lo[(long long)r * 2 * d + d + n] = f2bf(__fsub_rn(ze, bf2f(he)));
+      for (int t = 0; t < 2; ++t) {
+        const int c = n + t;
+        z[t] = c < d ? __fmul_rn(__fmul_rn(hr[c], ch), bf2f(sg[c]))
+                     : __fmul_rn(__fmul_rn(ev ? ev[c - d] : bf2f(er[c - d]), ce), bf2f(sg[c]));
+      }
+      const __nv_bfloat162 zh = __floats2bfloat162_rn(z[0], z[1]);
+      const __nv_bfloat162 zl = __floats2bfloat162_rn(__fsub_rn(z[0], __low2float(zh)),
+                                                       __fsub_rn(z[1], __high2float(zh)));
+      *reinterpret_cast<__nv_bfloat162*>(hi + n) = zh;
+      *reinterpret_cast<__nv_bfloat162*>(lo + n) = zl;
     }
   }
+  if (tid == 0) tm.t2 = gtimer();
   // publish the row metadata
   int* dst = reinterpret_cast<int*>(p.rows);
   const int* src = reinterpret_cast<const int*>(&pr);

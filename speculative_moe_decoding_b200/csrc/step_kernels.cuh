@@ -57,14 +57,14 @@ struct RouteParams {
 // is a barrier over exactly those threads.
 template <class Sync>
 __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, Sync sync) {
-  __shared__ float s_p[kRmax][kMaxExperts];             // softmax probabilities
-  __shared__ unsigned char s_sel[kRmax][kMaxExperts];   // 1 if among the row's top-k
-  __shared__ unsigned char s_slot[kRmax][kMaxExperts];  // slot of a selected expert, 0xff otherwise
+  __shared__ __align__(16) float s_p[kRmax][kMaxExperts];  // softmax probabilities, -1 past E
+  __shared__ unsigned char s_slot[kRmax][kMaxExperts];      // slot of a selected expert, 0xff otherwise
   const int lane = tid & 31, warp = tid >> 5;
   const int E = p.E, K = p.top_k;
-  // softmax of each row (warp per row; fixed-order sums)
+  // warp r: softmax of row r (fixed-order sums), top-k by rank and the slots
   if (warp < R) {
-    const float* lg = p.logits + warp * E;
+    const int r = warp;
+    const float* lg = p.logits + r * E;
     constexpr int kPer = kMaxExperts / 32;
     float pe[kPer];
     float m = -INFINITY;
@@ -88,39 +88,40 @@ __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, S
 #pragma unroll
     for (int i = 0; i < kPer; ++i) {
       int e = lane + 32 * i;
-      if (e < E) s_p[warp][e] = __fdiv_rn(pe[i], sum);
+      pe[i] = e < E ? __fdiv_rn(pe[i], sum) : -1.f;
+      s_p[r][e] = pe[i];
     }
-  }
-  sync();
-  // top-k by rank: expert e of row r is selected when fewer than K experts beat
-  // it (larger probability, or equal probability and lower id)
-  for (int idx = tid; idx < R * E; idx += nthreads) {
-    const int r = idx / E, e = idx - r * E;
-    const float pv = s_p[r][e];
-    int beat = 0;
-    for (int f = 0; f < E; ++f) {
-      const float q = s_p[r][f];
-      beat += (q > pv) || (q == pv && f < e);
-    }
-    s_sel[r][e] = beat < K;
-  }
-  sync();
-  // slots: the selected experts of a row in ascending id (warp per row, ballots)
-  if (warp < R) {
-    const int r = warp;
+    __syncwarp();
+    // expert e is selected when fewer than K experts beat it (larger
+    // probability, or equal probability and lower id)
+    const float4* row4 = reinterpret_cast<const float4*>(s_p[r]);
+    const int E4 = (E + 3) >> 2;
     int base = 0;
-    for (int e0 = 0; e0 < E; e0 += 32) {
-      const int e = e0 + lane;
-      const bool sel = e < E && s_sel[r][e];
-      const unsigned m = __ballot_sync(0xffffffffu, sel);
-      const int slot = base + __popc(m & ((1u << lane) - 1u));
+#pragma unroll 1
+    for (int i = 0; 32 * i < E; ++i) {
+      const int e = lane + 32 * i;
+      const float pv = s_p[r][e];
+      int beat = 0;
+#pragma unroll 4
+      for (int j = 0; j < E4; ++j) {
+        const float4 q = row4[j];
+        const int f = 4 * j;
+        beat += (q.x > pv) || (q.x == pv && f < e);
+        beat += (q.y > pv) || (q.y == pv && f + 1 < e);
+        beat += (q.z > pv) || (q.z == pv && f + 2 < e);
+        beat += (q.w > pv) || (q.w == pv && f + 3 < e);
+      }
+      // slots: the selected experts in ascending id
+      const bool sel = e < E && beat < K;
+      const unsigned msk = __ballot_sync(0xffffffffu, sel);
+      const int slot = base + __popc(msk & ((1u << lane) - 1u));
       const bool ok = sel && slot < K;  // slot >= K only with NaN probabilities
       if (ok) {
         p.ids[r * K + slot] = e;
-        p.gates[r * K + slot] = s_p[r][e];
+        p.gates[r * K + slot] = pv;
       }
       if (e < E) s_slot[r][e] = ok ? (unsigned char)slot : (unsigned char)0xff;
-      base += __popc(m);
+      base += __popc(msk);
     }
   }
   sync();
@@ -223,7 +224,8 @@ struct PrefillSetupParams {
 
 
 
-// Draft input rows: fcin[r] = [bf16(RMSNorm(h_r) * g_h) ; bf16(RMSNorm(e_r) * g_e)]
+// Draft input rows: fcin[r] = [RMSNorm(h_r) * g_h ; RMSNorm(e_r) * g_e] as high and
+// low bf16 parts (fcin, fcin_lo), at most kRmax rows,
 // where (h_r, e_r, pos_r) come from one of three row sources:
 //   mode 0 (recursion 1): the pending pairs of each slot - verifier hidden
 //          hpend[b][i] and the embedding of the committed token at pos+1;
@@ -231,6 +233,9 @@ struct PrefillSetupParams {
 //          the embedding of draft token dtok[b], at kv_len + j - 2;
 //   mode 2 (prefill): verifier hidden x[p - p0] and the next context input
 //          (visual vector or prompt embedding) for pairs p in [p0, p0 + n).
+// Dynamic shared memory of draft_setup_kernel: gains, hidden rows, embedding rows.
+constexpr size_t draft_setup_smem_bytes(int d) { return (size_t)d * (4 + kRmax * 4 + kRmax * 2); }
+
 struct DraftSetupParams {
   int mode, B, j, d, max_k;
   float eps;
