@@ -166,7 +166,8 @@ __global__ void __launch_bounds__(256) prefill_setup_kernel(const PrefillSetupPa
 
 // The draft's input rows (DraftSetupParams).  The gains, each row's hidden
 // state and its token embedding arrive in shared memory by bulk copies (the
-// gains before the grid dependency wait); warp r then normalises row r.
+// gains before the grid dependency wait); the whole block then normalises
+// each row.
 __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams p) {
   extern __shared__ __align__(128) unsigned char dsm[];
   __shared__ int s_bad;
@@ -268,46 +269,60 @@ __global__ void __launch_bounds__(256) draft_setup_kernel(const DraftSetupParams
       bulk_g2s(sh_rows + r * d, h, 4 * d, &bars[1]);
       if (tok >= 0) bulk_g2s(se_rows + r * d, p.embed + (long long)tok * d, 2 * d, &bars[1]);
     }
-    tm.t1 = gtimer();
   }
   mbar_wait(&bars[0], 0, p.status);
   mbar_wait(&bars[1], 0, p.status);
-  // fcin[r] as high / low bf16 parts; warp r normalises row r
-  if (warp < nrow) {
-    const int r = warp, tok = pr.tok[r];
+  if (tid == 0) tm.t1 = gtimer();
+  // fcin[r] as high / low bf16 parts, all 256 threads on every row: sums of
+  // squares (thread, then warp, then the 8 warps in order), then the outputs
+  __shared__ float red[kRmax][8][2];
+  __shared__ float s_scale[kRmax][2];
+  for (int r = 0; r < nrow; ++r) {
     const float* hr = sh_rows + r * d;
     const bf16* er = se_rows + r * d;
-    const float* ev = tok < 0 ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
-    float sh = 0.f, se = 0.f;
-    for (int n = lane; n < d; n += 32) {
+    const float* ev = pr.tok[r] < 0 ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
+    float a = 0.f, c = 0.f;
+    for (int n = tid; n < d; n += 256) {
       const float hv = hr[n];
       const float e = ev ? ev[n] : bf2f(er[n]);
-      sh = __fmaf_rn(hv, hv, sh);
-      se = __fmaf_rn(e, e, se);
+      a = __fmaf_rn(hv, hv, a);
+      c = __fmaf_rn(e, e, c);
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) {
-      sh = __fadd_rn(sh, __shfl_xor_sync(0xffffffffu, sh, o));
-      se = __fadd_rn(se, __shfl_xor_sync(0xffffffffu, se, o));
+      a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, o));
+      c = __fadd_rn(c, __shfl_xor_sync(0xffffffffu, c, o));
     }
-    const float ch = rsqrtf(__fadd_rn(__fdiv_rn(sh, (float)d), p.eps));
-    const float ce = rsqrtf(__fadd_rn(__fdiv_rn(se, (float)d), p.eps));
-    bf16* hi = p.fcin + (long long)r * 2 * d;
-    bf16* lo = p.fcin_lo + (long long)r * 2 * d;
-    for (int n = 2 * lane; n < 2 * d; n += 64) {  // column pairs of [h ; e]
-      float z[2];
+    if (lane == 0) {
+      red[r][warp][0] = a;
+      red[r][warp][1] = c;
+    }
+  }
+  __syncthreads();
+  if (tid < 2 * nrow) {
+    const int r = tid >> 1, w = tid & 1;
+    float v = 0.f;
+    for (int q = 0; q < 8; ++q) v = __fadd_rn(v, red[r][q][w]);
+    s_scale[r][w] = rsqrtf(__fadd_rn(__fdiv_rn(v, (float)d), p.eps));
+  }
+  __syncthreads();
+  for (int idx = tid; idx < nrow * d; idx += 256) {  // column pairs of [h ; e]
+    const int r = idx / d, n = 2 * (idx - r * d);
+    const float* hr = sh_rows + r * d;
+    const bf16* er = se_rows + r * d;
+    const float* ev = pr.tok[r] < 0 ? p.visual + (long long)(pr.pos[r] + 1) * d : nullptr;
+    float z[2];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int c = n + t;
-        z[t] = c < d ? __fmul_rn(__fmul_rn(hr[c], ch), bf2f(sg[c]))
-                     : __fmul_rn(__fmul_rn(ev ? ev[c - d] : bf2f(er[c - d]), ce), bf2f(sg[c]));
-      }
-      const __nv_bfloat162 zh = __floats2bfloat162_rn(z[0], z[1]);
-      const __nv_bfloat162 zl = __floats2bfloat162_rn(__fsub_rn(z[0], __low2float(zh)),
-                                                       __fsub_rn(z[1], __high2float(zh)));
-      *reinterpret_cast<__nv_bfloat162*>(hi + n) = zh;
-      *reinterpret_cast<__nv_bfloat162*>(lo + n) = zl;
+    for (int t = 0; t < 2; ++t) {
+      const int cidx = n + t;
+      z[t] = cidx < d ? __fmul_rn(__fmul_rn(hr[cidx], s_scale[r][0]), bf2f(sg[cidx]))
+                      : __fmul_rn(__fmul_rn(ev ? ev[cidx - d] : bf2f(er[cidx - d]), s_scale[r][1]), bf2f(sg[cidx]));
     }
+    const __nv_bfloat162 zh = __floats2bfloat162_rn(z[0], z[1]);
+    const __nv_bfloat162 zl = __floats2bfloat162_rn(__fsub_rn(z[0], __low2float(zh)),
+                                                     __fsub_rn(z[1], __high2float(zh)));
+    *reinterpret_cast<__nv_bfloat162*>(p.fcin + (long long)r * 2 * d + n) = zh;
+    *reinterpret_cast<__nv_bfloat162*>(p.fcin_lo + (long long)r * 2 * d + n) = zl;
   }
   if (tid == 0) tm.t2 = gtimer();
   // publish the row metadata
