@@ -39,6 +39,7 @@
 #include <cuda.h>
 
 #include "common.cuh"
+#include "route.cuh"
 
 namespace ocrdec {
 
@@ -59,8 +60,17 @@ constexpr int kAttnChunkBytes = kAttnChunk * kAttnMaxDh * 2;  // K (or V) of one
 // 128-byte swizzle repeats every 1 KB).
 // Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
 // every 1 KB), the K/V ring, and the CTA's W_o block (d / kAttnSplit rows x Dh).
-constexpr size_t attn_smem_bytes(int d, int Dh) {
-  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + (size_t)(d / kAttnSplit) * Dh * 2;
+static_assert(kAttnSplit == kRouteParts, "router partials: one per attention row block");
+
+// Router block of a CTA (MoE layers): W_r rows (E rounded up to 16, zero
+// padded) x the CTA's d / kAttnSplit columns, rows padded by 16 bytes, then the
+// FFN RMSNorm gains of those columns.
+constexpr size_t attn_router_bytes(int d, int E) {
+  return E > 0 ? ((size_t)(E + 15) / 16 * 16 * (d / kAttnSplit + 8) + d / kAttnSplit) * 2 : 0;
+}
+
+constexpr size_t attn_smem_bytes(int d, int Dh, int E) {
+  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + (size_t)(d / kAttnSplit) * Dh * 2 + attn_router_bytes(d, E);
 }
 
 struct AttnParams {
@@ -76,6 +86,11 @@ struct AttnParams {
   float* yp;               // [H][kRmax][d] per-head partial projections
   int* cnt;                // [B][kAttnSplit] arrivals per row block, zero between launches
   int d;                   // model width (= H * Dh), a multiple of 16 * kAttnSplit
+  // MoE layers: the router partials of the updated residual rows (see route.cuh)
+  const bf16* wr;          // W_r [E][d], or nullptr (dense FFN layer)
+  const bf16* g_ffn;       // FFN RMSNorm gains [d]
+  float* rpart;            // [rows][kRouteParts][kRouteLd]
+  int E;
   int* status;
 };
 
@@ -170,15 +185,25 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const uint32_t ring_s = smem_u32(ring);
   unsigned char* wo_s = ring + (size_t)kAttnBufs * 2 * kAttnChunkBytes;  // [Dh/64][nb rows][128 B]
   const int nb = p.d / kAttnSplit;  // W_o rows of this CTA
+  const int E16 = p.wr ? (p.E + 15) / 16 * 16 : 0;
+  const int ldw = nb + 8;
+  bf16* s_wr = reinterpret_cast<bf16*>(wo_s + (size_t)nb * Dh * 2);  // [E16][ldw]
+  bf16* s_gr = s_wr + (size_t)E16 * ldw;                                // [nb]
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBufs; ++i) mbar_init(&bar[i], 1);
     mbar_init(&wo_bar, 1);
     fence_mbar_init();
-    // the W_o block is a weight: requested before anything else
-    mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2));
+    // the W_o block (and the router block) are weights: requested before anything else
+    mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2 + (p.wr ? (p.E + 1) * nb * 2 : 0)));
     tma_load_wo(wo_s, &tm_wo, k * nb, h * (Dh / 64), &wo_bar);
+    if (p.wr) {
+      for (int e = 0; e < p.E; ++e)
+        bulk_g2s(s_wr + (size_t)e * ldw, p.wr + (size_t)e * p.d + k * nb, nb * 2, &wo_bar);
+      bulk_g2s(s_gr, p.g_ffn + k * nb, nb * 2, &wo_bar);
+    }
   }
+  for (int i = p.E * ldw + tid; i < E16 * ldw; i += kAttnThreads) s_wr[i] = f2bf(0.f);  // padding rows
   // pass rows and positions are written by the pass's setup kernel, which
   // finished before the kernel this one follows
   const int r0 = p.slot_row0[b];
@@ -454,23 +479,68 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     __syncthreads();
     if (s_last) {
       __threadfence();
+      // MoE layers: u = g * x (new residual) as bf16 high and low parts and
+      // x itself go to the (now free) K/V ring for the router partials
+      bf16* su = reinterpret_cast<bf16*>(ring);                                    // [2][kAttnRows][ldw]
+      float* sx = reinterpret_cast<float*>(ring + (size_t)2 * kAttnRows * ldw * 2);  // [kAttnRows][nb]
 #pragma unroll
       for (int i = 0; i < kPer; ++i) {
         const int idx = tid + i * kAttnThreads;
-        if (idx >= nr * nb) break;
-        const int r = idx / nb, n = k * nb + (idx - r * nb);
-        const float* yr = p.yp + (long long)(r0 + r) * p.d + n;
-        float y[kAttnMaxHeads];
+        if (idx >= kAttnRows * nb) break;
+        const int r = idx / nb, nl = idx - r * nb, n = k * nb + nl;
+        float xn = 0.f;
+        if (r < nr) {
+          const float* yr = p.yp + (long long)(r0 + r) * p.d + n;
+          float y[kAttnMaxHeads];
 #pragma unroll
-        for (int hh = 0; hh < kAttnMaxHeads; ++hh)
-          if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * p.d);
-        float v = 0.f;
+          for (int hh = 0; hh < kAttnMaxHeads; ++hh)
+            if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * p.d);
+          float v = 0.f;
 #pragma unroll
-        for (int hh = 0; hh < kAttnMaxHeads; ++hh)
-          if (hh < p.H) v = __fadd_rn(v, y[hh]);
-        p.x[(long long)(r0 + r) * p.d + n] = __fadd_rn(xv[i], v);
+          for (int hh = 0; hh < kAttnMaxHeads; ++hh)
+            if (hh < p.H) v = __fadd_rn(v, y[hh]);
+          xn = __fadd_rn(xv[i], v);
+          p.x[(long long)(r0 + r) * p.d + n] = xn;
+        }
+        if (p.wr) {
+          const float u = __fmul_rn(xn, bf2f(s_gr[nl]));
+          const bf16 hi = f2bf(u);
+          su[r * ldw + nl] = hi;
+          su[(kAttnRows + r) * ldw + nl] = f2bf(__fsub_rn(u, bf2f(hi)));
+          sx[r * nb + nl] = xn;
+        }
       }
       if (tid == 0) p.cnt[b * kAttnSplit + k] = 0;
+      if (p.wr) {
+        __syncthreads();
+        float* rp = p.rpart + (size_t)r0 * kRouteParts * kRouteLd + k * kRouteLd;
+        // each row's sum of squares over the block (warp w: row w, fixed order)
+        if (warp < nr) {
+          float a = 0.f;
+          for (int nl = lane; nl < nb; nl += 32) a = __fmaf_rn(sx[warp * nb + nl], sx[warp * nb + nl], a);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, off));
+          if (lane == 0) rp[(size_t)warp * kRouteParts * kRouteLd + kMaxExperts] = a;
+        }
+        // dot products of the block's W_r columns with u (experts x rows MMAs)
+        for (int t = warp; t < E16 / 16; t += kAttnWarps) {
+          float d4[4] = {0.f, 0.f, 0.f, 0.f};
+          for (int s = 0; s < nb / 16; ++s) {
+            uint32_t a[4], bh[2], bl[2];
+            attn_ldsm_x4(smem_u32(s_wr + (size_t)(t * 16 + fr_row) * ldw + s * 16 + fr_hi * 8), a);
+            attn_ldsm_x2(smem_u32(su + b_n * ldw + s * 16 + b_k8), bh);
+            attn_ldsm_x2(smem_u32(su + (kAttnRows + b_n) * ldw + s * 16 + b_k8), bl);
+            attn_mma(d4, a, bh);
+            attn_mma(d4, a, bl);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int e = t * 16 + (lane >> 2) + (q >> 1) * 8;
+            const int r = 2 * (lane & 3) + (q & 1);
+            if (e < p.E && r < nr) rp[(size_t)r * kRouteParts * kRouteLd + e] = d4[q];
+          }
+        }
+      }
     }
   } else if (tid == 0) {
     mbar_wait(&wo_bar, 0, p.status);  // the W_o copy lands before the CTA exits

@@ -18,6 +18,7 @@ typedef __nv_bfloat16 bf16;
 // Upper bound of try_wait rounds before a wait is declared stuck.  Each round
 // suspends for up to the hardware's time slice, so this is well above a second.
 constexpr uint32_t kSpinLimit = 1u << 24;
+constexpr int kRmax = 8;  // rows per pass (pass rows are the 8 MMA columns)
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

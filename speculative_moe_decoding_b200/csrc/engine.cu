@@ -102,7 +102,8 @@ bool config_ok(const ocrdec_config* c) {
   if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
   if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % kChunk)) return false;
   if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
-  if (c->top_k > c->n_experts || c->top_k > 8 || c->n_experts > kMaxExperts || c->top_k + c->n_shared > 127) return false;
+  if (c->top_k > c->n_experts || c->top_k > kMaxTopK || c->n_experts > kMaxExperts || c->n_shared > kMaxShared)
+    return false;
   if (c->max_k < 0 || c->max_k > 3) return false;
   if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
   if (c->d_model > kGemvMaxK) return false;  // shared-memory copy of the normalised rows
@@ -116,8 +117,8 @@ bool config_ok(const ocrdec_config* c) {
 size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp, rlogits,
-      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
+  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp,
+      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, rpart, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
       am_part, gtok, props,
       committed, ncommitted, hpend, total;
   int hist_ld, am_blocks;
@@ -149,7 +150,7 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.xd = take(4 * R * d);
   L.q = take(4 * R * d);
   L.yp = take(4 * H * kRmax * d);  // per-head output projections
-  L.rlogits = take(4 * R * E);
+  L.rpart = take(4 * R * kRouteParts * kRouteLd);
   L.topk_ids = take(4 * R * K);
   L.topk_gates = take(4 * R * K);
   L.counts = take(4 * E);
@@ -188,10 +189,9 @@ cudaError_t max_carveout(K kernel) {
 
 cudaError_t prepare_kernels_now() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)attn_smem_bytes(kGemvMaxK, kAttnMaxDh));
+                                       (int)attn_smem_bytes(kGemvMaxK, kAttnMaxDh, kMaxExperts));
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
   if (e == cudaSuccess) e = max_carveout(attention_kernel);
-  if (e == cudaSuccess) e = max_carveout(route_kernel);
   if (e == cudaSuccess) e = max_carveout(combine_kernel);
   if (e == cudaSuccess) e = max_carveout(verify_setup_kernel);
   if (e == cudaSuccess) e = max_carveout(prefill_setup_kernel);
@@ -328,8 +328,10 @@ GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* n
   return g;
 }
 
+// router / ffn_norm: a MoE layer's router and FFN norm gains (the attention
+// kernel then also writes the router partials), or nullptr.
 int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* attn_norm, const Mat& wqkv,
-                   const Mat& wo, const BlockIO& io) {
+                   const Mat& wo, const BlockIO& io, const bf16* router = nullptr, const bf16* ffn_norm = nullptr) {
   const ocrdec_config& m = c->cfg;
   PassRows* rows = c->rows();
   GemvLaunch g = dense_launch(c, wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
@@ -355,10 +357,15 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   a.yp = c->at<float>(c->L.yp);
   a.cnt = c->attn_counters();
   a.d = m.d_model;
+  a.wr = router;
+  a.g_ffn = ffn_norm;
+  a.rpart = c->at<float>(c->L.rpart);
+  a.E = m.n_experts;
   a.status = c->status();
   // attention and the output projection (x += attn . W_o^T) in one launch
   CK(launch_cluster_ex(attention_kernel, dim3(kAttnSplit, m.n_heads, m.max_batch), dim3(kAttnThreads),
-                       attn_smem_bytes(m.d_model, m.head_dim), lc, kAttnSplit, *io.tk, *io.tv, wo.map_attn, a));
+                       attn_smem_bytes(m.d_model, m.head_dim, router ? m.n_experts : 0), lc, kAttnSplit, *io.tk,
+                       *io.tv, wo.map_attn, a));
   return OCRDEC_OK;
 }
 
@@ -390,47 +397,29 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   float* x = c->at<float>(c->L.x);
   const int nslot = m.top_k + m.n_shared;
 
-  RouteParams rp{};
-  rp.logits = c->at<float>(c->L.rlogits);
-  rp.nrows = &rows->n;
-  rp.E = m.n_experts;
-  rp.top_k = m.top_k;
-  rp.S = m.n_shared;
-  rp.ids = c->at<int>(c->L.topk_ids);
-  rp.gates = c->at<float>(c->L.topk_gates);
-  rp.counts = c->at<int>(c->L.counts);
-  rp.offsets = c->at<int>(c->L.offsets);
-  rp.rowlist = c->at<int>(c->L.rowlist);
-  rp.mats = c->at<int>(c->L.mats);
-  rp.n_mats = c->at<int>(c->L.n_mats);
-  rp.touched = count ? c->misc() : nullptr;
-  rp.status = c->status();
-
-  // router logits + (last CTA) softmax / top-k / bucketing
-  GemvLaunch r = dense_launch(c, w.router, 0, &rows->n, 0, rmax, kTagRouter);
-  r.s.counter = c->am_counter(2);
-  r.src = SrcKind::Norm;
-  r.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
-  r.epi = EpiKind::Route;
-  r.store = EpiStore<false>::Params{c->at<float>(c->L.rlogits), m.n_experts, 1, nullptr};
-  r.route = rp;
-  CK(c->gemv(r, lc));
-
   auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half, int tag) {
     GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax, tag);
     g.s.kparts = 1;
     g.tm_sh = shared.map;
     g.s.n_experts = m.n_experts;
     g.s.top_k = m.top_k;
-    g.s.mats = rp.mats;
-    g.s.n_mats = rp.n_mats;
-    g.s.counts = rp.counts;
-    g.s.offsets = rp.offsets;
-    g.s.rowlist = rp.rowlist;
+    g.s.n_shared = m.n_shared;
+    g.s.mats = c->at<int>(c->L.mats);
+    g.s.n_mats = c->at<int>(c->L.n_mats);
+    g.s.counts = c->at<int>(c->L.counts);
+    g.s.offsets = c->at<int>(c->L.offsets);
+    g.s.rowlist = c->at<int>(c->L.rowlist);
     return g;
   };
 
+  // gate/up: every CTA routes the pass from the attention kernel's router
+  // partials (CTA 0 stores the tables, ids and gates)
   GemvLaunch gu = expert_launch(w.exp_gu, w.sh_gu, m.expert_ffn, kTagExpGU);
+  gu.s.rpart = c->at<float>(c->L.rpart);
+  gu.s.rms_eps = m.rms_eps;
+  gu.s.ids = c->at<int>(c->L.topk_ids);
+  gu.s.gates = c->at<float>(c->L.topk_gates);
+  gu.s.touched = count ? c->misc() : nullptr;
   gu.src = SrcKind::Norm;
   gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
   gu.epi = EpiKind::SwiGLU;
@@ -445,7 +434,8 @@ int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool 
   dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
   CK(c->gemv(dn, lc));
 
-  CombineParams cp{x, c->at<float>(c->L.ybuf), rp.gates, &rows->n, m.d_model, m.top_k, m.n_shared, c->status()};
+  CombineParams cp{x, c->at<float>(c->L.ybuf), c->at<float>(c->L.topk_gates), &rows->n, m.d_model, m.top_k,
+                   m.n_shared, c->status()};
   CK(launch_ex(combine_kernel, dim3((kRmax * m.d_model + 255) / 256), dim3(256), 0, lc, cp));
   return OCRDEC_OK;
 }
@@ -458,7 +448,8 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
     const LayerW& w = c->layers[l];
     BlockIO io{c->at<float>(c->L.x), c->at<bf16>(c->L.kvk) + l * layer_elems, c->at<bf16>(c->L.kvv) + l * layer_elems,
                layer_elems * m.n_layers, &c->kv_map[0], &c->kv_map[1], l, m.n_layers};
-    int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
+    int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io, w.dense ? nullptr : w.router.p,
+                            w.ffn_norm);
     if (st) return st;
     st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down) : moe_ffn(c, lc, rmax, w, count);
     if (st) return st;

@@ -1,44 +1,11 @@
-// GEMV epilogues that finish a pass step in the GEMV's last CTA: routing after
-// the router logits, greedy acceptance after the verifier's LM-head argmax.
-// Each saves one launch per use.
+// GEMV epilogue that finishes a pass step in the GEMV's last CTA: greedy
+// acceptance after the verifier's LM-head argmax (saves one launch per step).
 #pragma once
 
 #include "gemv.cuh"
 #include "step_kernels.cuh"
 
 namespace ocrdec {
-
-struct ConsumerSync {
-  __device__ void operator()() const { named_sync(1, kConsumers); }
-};
-
-// Router logits (stored like EpiStore), then - in the last CTA to finish -
-// softmax, top-k and bucketing of every row.
-struct EpiRoute {
-  struct Params {
-    EpiStore<false>::Params store;
-    RouteParams route;
-  };
-  __device__ static void apply(const Params& p, const GemvShape& s, const WarpOut& o, const RowSet& rs, int lane) {
-    EpiStore<false>::apply(p.store, s, o, rs, lane);
-  }
-  __device__ static void finish(const Params& p, const GemvShape& s, int R, int tid) {
-    __shared__ int last;
-    __threadfence();
-    named_sync(1, kConsumers);
-    if (tid == 0) last = (atomicAdd(s.counter, 1) == (int)gridDim.x - 1);
-    named_sync(1, kConsumers);
-    if (!last) return;
-    TraceMarks tm;
-    if (tid == 0) tm.t0 = gtimer();
-    __threadfence();
-    route_rows(p.route, R, tid, kConsumers, ConsumerSync{});
-    if (tid == 0) {
-      *s.counter = 0;
-      trace_end(s.status, 45, tm);  // the routing step alone
-    }
-  }
-};
 
 // LM-head argmax, then - in the last CTA - acceptance, commit and rollback.
 struct EpiArgmaxAccept {
@@ -65,7 +32,7 @@ struct EpiArgmaxAccept {
     }
     if (!EpiArgmax::merge(p.am, s, R, tid, s_tok)) return;
     named_sync(1, kConsumers);
-    accept_rows(p.accept, s_tok, tid, kConsumers, ConsumerSync{}, false);
+    accept_rows(p.accept, s_tok, tid, kConsumers, ConsumerBarrier{}, false);
   }
 };
 

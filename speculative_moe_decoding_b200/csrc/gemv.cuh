@@ -8,13 +8,15 @@
 //     cp.async.bulk.tensor (4-D tensor map: 64-column chunk, row, chunk index,
 //     expert; 128-byte swizzle; no multicast), each stage completing an
 //     mbarrier by transaction bytes.  Columns past K and rows past N arrive
-//     zero-filled, so ragged shapes need no special case;
+//     zero-filled, so ragged shapes need no special case.  The boxes carry
+//     an L2 evict-first policy: weights are read once per pass, and the
+//     pass's reused data (KV caches, activations, code) should stay in L2;
 //   * each of the kNW consumer warps owns one 16-row box and one 64-column
 //     quarter of every slice and multiplies it with the pass rows on the
 //     tensor cores (mma m16n8k16, bfloat16 in, float32 accumulate; the up to
-//     8 pass rows are the 8 columns of B), so a 16 KB stage costs a warp four
-//     MMAs instead of hundreds of FMAs - at R = 4 the FMA version was
-//     issue-bound below the HBM roofline;
+//     8 pass rows are the 8 columns of B, each as a bfloat16 high and low
+//     part), so a 16 KB stage costs a warp eight MMAs instead of hundreds of
+//     FMAs - at R = 4 the FMA version was issue-bound below the HBM roofline;
 //   * after the item's last slice the four column-quarter partials of every
 //     output are added in quarter order through shared memory and the warps
 //     run the epilogue.
@@ -24,14 +26,17 @@
 // speculative path bit-identical to k = 0.
 //
 // Work items are (matrix, 32-row tile) pairs claimed by CTAs from a per-launch
-// counter.  Dense mode has one matrix; expert mode walks a device-side list of
-// touched experts (shared experts first) so only the experts routed in this
-// pass are streamed.
+// counter.  Dense mode has one matrix; expert mode walks the list of touched
+// experts (shared experts first) so only the experts routed in this pass are
+// streamed.  Its routing tables live in shared memory: copied from memory, or
+// (expert gate/up) computed in every CTA from the attention kernel's router
+// partials.
 #pragma once
 
 #include <cuda.h>
 
 #include "common.cuh"
+#include "route.cuh"
 
 namespace ocrdec {
 
@@ -46,9 +51,13 @@ constexpr int kBoxRows = 16;                    // rows per TMA box (two boxes p
 constexpr int kBoxBytes = kBoxRows * kSlice * 2;  // 8 KB: [4 chunks][16 rows][128 B]
 constexpr int kStageBytes = 2 * kBoxBytes;      // 16 KB of weights per stage
 constexpr int kStages = 4;
-constexpr int kRmax = 8;                        // rows per pass on the GEMV path
 constexpr int kXStride = kSlice * 2 + 16;       // staged activation row (512 B + 16 B pad, ldmatrix-conflict-free)
 constexpr int kRedFloats = 2 * 4 * kTile * 8;   // quarter partials, double-buffered by item
+
+// Barrier over the consumer warps only (the producer warp does not take part).
+struct ConsumerBarrier {
+  __device__ void operator()() const { named_sync(1, kConsumers); }
+};
 
 struct GemvShape {
   int N, K;
@@ -77,6 +86,17 @@ struct GemvShape {
   // dynamic work distribution: work[0] = next item to claim, work[1] = CTAs
   // done claiming; the last CTA resets both (zero between launches)
   int* work;
+  // expert mode: the routing tables (mats, n_mats, counts, offsets, rowlist)
+  // are copied into shared memory before any item is claimed.  With rpart set
+  // (expert gate/up), every CTA instead routes the pass itself from the
+  // attention kernel's router partials, and CTA 0 stores the tables, ids and
+  // gates for the kernels that follow.
+  const float* rpart;   // [rows][kRouteParts][kRouteLd]
+  int n_shared;
+  float rms_eps;
+  int* ids;             // [rows][top_k]
+  float* gates;         // [rows][top_k]
+  int* touched;         // optional: [0] += routed experts touched, [1] += 1
 };
 
 // Rows of one item: entry q = pass row | (output slot << 8).
@@ -130,8 +150,8 @@ __device__ __forceinline__ int matrix_row(int r0, int r1, int srow) {
   return srow < kBoxRows ? r0 + srow : r1 + (srow - kBoxRows);
 }
 
-__device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* coord_e, bool* shared,
-                                         RowSet* rs) {
+__device__ __forceinline__ void mat_info(const GemvShape& s, const RouteTables& rt, int m, int R, int* coord_e,
+                                         bool* shared, RowSet* rs) {
   if (!s.mats) {
     *coord_e = 0;
     *shared = false;
@@ -142,16 +162,16 @@ __device__ __forceinline__ void mat_info(const GemvShape& s, int m, int R, int* 
     }
     return;
   }
-  int e = s.mats[m];
+  int e = rt.mats[m];
   if (e < s.n_experts) {
     *coord_e = e;
     *shared = false;
     if (rs) {
-      int n = s.counts[e], off = s.offsets[e];
+      int n = rt.counts[e], off = rt.offsets[e];
       n = n > kRmax ? kRmax : n;
       rs->n = n;
 #pragma unroll
-      for (int i = 0; i < kRmax; ++i) rs->e[i] = i < n ? s.rowlist[off + i] : 0;
+      for (int i = 0; i < kRmax; ++i) rs->e[i] = i < n ? rt.rowlist[off + i] : 0;
     }
   } else {
     int sh = e - s.n_experts;
@@ -673,6 +693,95 @@ constexpr size_t gemv_smem_bytes(int K) {
   return 1024 + (size_t)kStages * stage_stride<Src, RG>() + Src::smem_bytes(K, RG) + kRedFloats * 4;
 }
 
+// Epilogues whose expert-mode launches may route the pass themselves.
+template <class Epi>
+struct EpiRoutes {
+  static constexpr bool value = false;
+};
+template <>
+struct EpiRoutes<EpiSwiGLU> {
+  static constexpr bool value = true;
+};
+
+// Expert mode: the routing tables of the pass from memory (written by an
+// earlier kernel) into shared memory; all loads are independent.
+__device__ __forceinline__ void load_tables(const GemvShape& s, int R, int tid, RouteTables& rt) {
+  const int E = s.n_experts;
+  if (tid == 0) rt.n_mats = *s.n_mats;
+  for (int i = tid; i < s.n_shared + E; i += kConsumers) rt.mats[i] = s.mats[i];
+  for (int e = tid; e < E; e += kConsumers) {
+    rt.counts[e] = s.counts[e];
+    rt.offsets[e] = s.offsets[e];
+  }
+  for (int i = tid; i < R * s.top_k; i += kConsumers) rt.rowlist[i] = s.rowlist[i];
+}
+
+// Expert gate/up: every CTA routes the pass.  The router logits of row r are
+// assembled from the attention kernel's partials in a fixed order:
+//   logit[r][e] = (sum_k dot[r][k][e]) * rsqrt((sum_k ss[r][k]) / d + eps)
+// - the RMSNorm scale applied after the row-block dot products of W_r with
+// g * x (the gain g folded in by the attention kernel).  Every CTA computes
+// the same tables; CTA 0 also stores them, with the ids and gates, for the
+// down projection and the combine.
+static __device__ __forceinline__ void route_in_cta(const GemvShape& s, int R, int tid, RouteTables& rt) {
+  __shared__ float s_lg[kRmax * kMaxExperts];
+  __shared__ int s_ids[kRmax * kMaxTopK];
+  __shared__ float s_gates[kRmax * kMaxTopK];
+  const int E = s.n_experts;
+  for (int idx = tid; idx < R * E; idx += kConsumers) {
+    const int r = idx / E, e = idx - r * E;
+    const float* pr = s.rpart + (size_t)r * kRouteParts * kRouteLd;
+    float dk[kRouteParts], sk[kRouteParts];
+#pragma unroll
+    for (int k = 0; k < kRouteParts; ++k) {
+      dk[k] = __ldcg(pr + k * kRouteLd + e);
+      sk[k] = __ldcg(pr + k * kRouteLd + kMaxExperts);
+    }
+    float dot = 0.f, ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < kRouteParts; ++k) {
+      dot = __fadd_rn(dot, dk[k]);
+      ss = __fadd_rn(ss, sk[k]);
+    }
+    s_lg[idx] = __fmul_rn(dot, rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)s.K), s.rms_eps)));
+  }
+  named_sync(1, kConsumers);
+  RouteParams p{};
+  p.logits = s_lg;
+  p.E = E;
+  p.top_k = s.top_k;
+  p.S = s.n_shared;
+  p.ids = s_ids;
+  p.gates = s_gates;
+  p.counts = rt.counts;
+  p.offsets = rt.offsets;
+  p.rowlist = rt.rowlist;
+  p.mats = rt.mats;
+  p.n_mats = &rt.n_mats;
+  route_rows(p, R, tid, kConsumers, ConsumerBarrier{});
+  named_sync(1, kConsumers);
+  if (blockIdx.x == 0) {
+    const int K = s.top_k;
+    if (tid == 0) {
+      *const_cast<int*>(s.n_mats) = rt.n_mats;
+      if (s.touched) {
+        atomicAdd(&s.touched[0], rt.n_mats - s.n_shared);
+        atomicAdd(&s.touched[1], 1);
+      }
+    }
+    for (int i = tid; i < s.n_shared + E; i += kConsumers) const_cast<int*>(s.mats)[i] = rt.mats[i];
+    for (int e = tid; e < E; e += kConsumers) {
+      const_cast<int*>(s.counts)[e] = rt.counts[e];
+      const_cast<int*>(s.offsets)[e] = rt.offsets[e];
+    }
+    for (int i = tid; i < R * K; i += kConsumers) {
+      const_cast<int*>(s.rowlist)[i] = rt.rowlist[i];
+      s.ids[i] = s_ids[i];
+      s.gates[i] = s_gates[i];
+    }
+  }
+}
+
 template <int RG, class Src, class Epi>
 __global__ void __launch_bounds__(kGemvThreads, 2)
 gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
@@ -683,6 +792,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   __shared__ int s_rs[kStages][kRmax + 1];     // expert mode: the item's row set (n, entries), with its first slice
   __shared__ float red_pro[kRmax * kNW];
   __shared__ int s_abort;
+  __shared__ RouteTables s_rt;                 // expert mode: the pass's routing tables
+  __shared__ __align__(8) uint64_t tab_bar;    // consumers -> producer: s_rt is ready
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -701,6 +812,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     }
     mbar_init(&x_empty[0], kNW);
     mbar_init(&x_empty[1], kNW);
+    mbar_init(&tab_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -722,7 +834,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       if (m != prs_m) {
         int ce;
         bool sh;
-        mat_info(s, m, R, &ce, &sh, &prs);
+        mat_info(s, s_rt, m, R, &ce, &sh, &prs);
         prs_m = m;
       }
     };
@@ -732,7 +844,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     auto issue_w = [&](int item, int m, int t, int slc, bool first) {
       int ce;
       bool sh;
-      mat_info(s, m, 0, &ce, &sh, nullptr);
+      mat_info(s, s_rt, m, 0, &ce, &sh, nullptr);
       const CUtensorMap* map = sh ? &tm_sh : &tm_w;
       int r0, r1;
       tile_boxes(s, t, &r0, &r1);
@@ -828,7 +940,8 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     if (ok) {
       R = min(pass_rows(s), RG);
       for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j], pre_first[j]);
-      if (s.mats) total = *s.n_mats * s.tiles_per_mat;
+      // expert mode: the item list is known once the consumers have the tables
+      if (s.mats) total = mbar_wait(&tab_bar, 0, s.status) ? s_rt.n_mats * s.tiles_per_mat : 0;
       if (!claimed) claim();
       while (item < total) {
         const ItemPos ip = item_pos(s, item);
@@ -873,6 +986,10 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   }
   named_sync(1, kConsumers);
   if (s_abort) {
+    if (s.mats && tid == 0) {  // no items
+      s_rt.n_mats = 0;
+      mbar_arrive(&tab_bar);
+    }
     // consume the producer's stages up to its end marker so it can finish
     uint32_t it = 0;
     while (true) {
@@ -890,6 +1007,16 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int R = min(pass_rows(s), RG);
   __shared__ int s_last_part;
+  if (s.mats) {
+    if constexpr (EpiRoutes<Epi>::value) {
+      if (s.rpart) route_in_cta(s, R, tid, s_rt);
+      else load_tables(s, R, tid, s_rt);
+    } else {
+      load_tables(s, R, tid, s_rt);
+    }
+    named_sync(1, kConsumers);
+    if (tid == 0) mbar_arrive(&tab_bar);  // releases the tables to the producer
+  }
 
   epi_init<Epi>(tid);
   Src::template prologue<RG>(sp, s.K, R, xsm, red_pro, tid, pre);

@@ -129,7 +129,6 @@ cudaError_t gemv_prepare() {
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiSwiGLU>();
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmax>();
-  if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiRoute>();
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmaxAccept>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<true>>();
@@ -175,10 +174,6 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
       case EpiKind::Store: return launch_rg<SrcNorm, EpiStore<false>>(g, g.norm, g.store, lc);
       case EpiKind::SwiGLU: return launch_rg<SrcNorm, EpiSwiGLU>(g, g.norm, g.swiglu, lc);
       case EpiKind::Argmax: return launch_rg<SrcNorm, EpiArgmax>(g, g.norm, g.argmax, lc);
-      case EpiKind::Route: {
-        EpiRoute::Params ep{g.store, g.route};
-        return launch_rg<SrcNorm, EpiRoute>(g, g.norm, ep, lc);
-      }
       case EpiKind::ArgmaxAccept: {
         EpiArgmaxAccept::Params ep{g.argmax, g.accept};
         return launch_rg<SrcNorm, EpiArgmaxAccept>(g, g.norm, ep, lc);

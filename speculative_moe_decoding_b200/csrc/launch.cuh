@@ -52,7 +52,7 @@ cudaError_t launch_cluster_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
 }
 
 enum class SrcKind { Norm, Bf16, Bf16Item };
-enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, Route, ArgmaxAccept };
+enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, ArgmaxAccept };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.
 struct GemvLaunch {
@@ -67,7 +67,6 @@ struct GemvLaunch {
   EpiSwiGLU::Params swiglu{};
   EpiQKV::Params qkv{};
   EpiArgmax::Params argmax{};
-  RouteParams route{};    // EpiKind::Route (with store)
   AcceptParams accept{};  // EpiKind::ArgmaxAccept (with argmax)
   int rows_bound = kRmax;  // static bound on rows of one work item (selects the row-group width)
   int grid = 0;            // 0: derived from the work and the SM count

@@ -1,21 +1,10 @@
 // The stand-alone kernels of the decode step (launched by the engine only):
-// pass setup, routing, combine, acceptance, forced proposals, RoPE table.
+// pass setup, combine, acceptance, forced proposals, RoPE table.
 #pragma once
 
 #include "step_kernels.cuh"
 
 namespace ocrdec {
-
-__global__ void __launch_bounds__(256) route_kernel(const RouteParams p) {
-  __shared__ int s_abort;
-  const int tid = threadIdx.x;
-  pdl_wait();
-  if (tid == 0) s_abort = status_bad(p.status);
-  __syncthreads();
-  if (s_abort) return;
-  pdl_trigger();
-  route_rows(p, min(*p.nrows, kRmax), tid, 256, BlockSync{});
-}
 
 __global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
   pdl_wait();

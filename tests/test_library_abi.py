@@ -65,6 +65,8 @@ def test_config_validation(lib):
         dict(good, n_heads=8, head_dim=32),  # head_dim 64 or 128 only
         dict(good, d_model=2048, n_heads=32),  # at most 16 heads
         dict(good, d_model=192, n_heads=3),    # d_model a multiple of 128
+        dict(good, n_experts=65),          # routed experts beyond the router block
+        dict(good, n_shared=9),            # shared experts beyond the routing tables
     ]
     for bad in bad_cases:
         cfg = lib.make_config(bad, 3, 1, 256)
