@@ -1,12 +1,12 @@
 // The decode-step engine behind the C ABI of include/ocrdec.h.
 //
 // Host side only orders launches; every step of the decode path runs in the
-// kernels of gemv.cuh, attention.cuh and step_kernels.cuh.  One verifier pass
-// per layer is: Q/K/V GEMV (+RoPE, KV append) -> attention with the output
-// projection (+residual) -> [dense SwiGLU up/down | router GEMV (+softmax,
-// top-k and bucketing in its last CTA) -> expert gate/up GEMV over the touched
-// experts -> expert down GEMV -> combine].  Then final norm + LM head + argmax
-// with acceptance in its last CTA.
+// kernels of gemv.cuh, attention.cuh, route.cuh and step_kernels.cuh.  One
+// verifier pass per layer is: Q/K/V GEMV (+RoPE, KV append) -> attention with
+// the output projection (+residual; in MoE layers also the router partials)
+// -> [dense SwiGLU up/down | expert gate/up GEMV that first routes the pass in
+// every CTA, over the touched experts -> expert down GEMV -> combine].  Then
+// final norm + LM head + argmax with acceptance in its last CTA.
 #include <cmath>
 #include <cstring>
 #include <map>
@@ -293,7 +293,7 @@ namespace {
 
 // Timeline-trace tags of the launches (ocrdec_read_trace).
 enum Tag {
-  kTagQKV = 1, kTagOProj = 2, kTagRouter = 3, kTagExpGU = 4, kTagExpDown = 5, kTagDenseGU = 6, kTagDenseDown = 7,
+  kTagQKV = 1, kTagExpGU = 4, kTagExpDown = 5, kTagDenseGU = 6, kTagDenseDown = 7,
   kTagLMVerify = 8, kTagLMDraft = 9, kTagFC = 10
 };
 
