@@ -1,7 +1,7 @@
-// Small kernels of the decode step: router softmax/top-k with expert
-// bucketing, the MoE combine, pass setup (embedding gather, row metadata,
-// draft inputs), greedy acceptance with commit and rollback, the benchmark's
-// forced-acceptance override, and the RoPE table.
+// Small kernels of the decode step: the MoE combine, pass setup (embedding
+// gather, row metadata, draft inputs), greedy acceptance with commit and
+// rollback, the benchmark's forced-acceptance override, and the RoPE table.
+// (Routing is in route.cuh.)
 #pragma once
 
 #include "common.cuh"
