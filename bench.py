@@ -111,12 +111,15 @@ class ClockSampler:
 ORACLE_SAMPLE = dict(n_visual=32, n_prompt=8, n_ref=16)
 
 
-def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.0):
-    """Times the oracle's speculative decode (forced acceptance, draft running)
-    on a bounded sample: the decode of the first n_ref tokens after a short
-    context, repeated (each repetition from a fresh prefill, not timed) until
-    about budget_s of timed decode has run; returns (tokens/s, description,
-    threads, steps, seconds)."""
+def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.0, threads=None):
+    """Times the oracle's speculative decode (forced acceptance, draft running;
+    k = 0: plain greedy decode) on a bounded sample: the decode of the first
+    n_ref tokens after a short context, repeated (each repetition from a fresh
+    prefill, not timed) until about budget_s of timed decode has run.
+    threads limits the BLAS threads of the timed part (None: all cores).
+    Returns (tokens/s, description, threads, steps, seconds)."""
+    from contextlib import nullcontext
+
     from oracle import decoder as O
     w = synth.WORKLOADS["full_spec"]
     orc = O.Oracle(dims.as_dict(), bits)
@@ -131,30 +134,51 @@ def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.
         return O.forced_proposals({p: ref.get(p, 0) for p in range(s.kv_len, s.kv_len + k + 1)}, s.kv_len, k,
                                   tab.u, tab.r, tab.p, dims.vocab)
 
-    dt = 0.0
-    steps = toks = reps = 0
-    while dt < budget_s:
-        st = O.prefill(orc, inp.visual, inp.prompt)
-        t0 = time.perf_counter()
-        while st.n_generated < ORACLE_SAMPLE["n_ref"] - k - 1:
-            before = st.n_generated
-            props = O.draft_propose(orc, st, k)
-            props = proposer(st)
-            O.verify_commit(orc, st, props)
-            toks += st.n_generated - before
-            steps += 1
-        dt += time.perf_counter() - t0
-        reps += 1
     try:
         import threadpoolctl
-        threads = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
-    except Exception:
-        threads = 1
-    desc = (f"oracle spec decode k={k}, forced acceptance, draft running; context {C} rows "
+    except ImportError:
+        threadpoolctl = None
+    limiter = threadpoolctl.threadpool_limits(threads) if (threads and threadpoolctl) else nullcontext()
+    dt = 0.0
+    steps = toks = reps = 0
+    used = 1
+    with limiter:
+        if threadpoolctl:
+            used = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
+        while dt < budget_s:
+            st = O.prefill(orc, inp.visual, inp.prompt)
+            t0 = time.perf_counter()
+            while st.n_generated < ORACLE_SAMPLE["n_ref"] - k - 1:
+                before = st.n_generated
+                if k > 0:
+                    O.draft_propose(orc, st, k)  # the draft runs; the forced stream decides
+                    props = proposer(st)
+                else:
+                    props = []
+                O.verify_commit(orc, st, props)
+                toks += st.n_generated - before
+                steps += 1
+            dt += time.perf_counter() - t0
+            reps += 1
+    mode = f"spec decode k={k}, forced acceptance, draft running" if k > 0 else "greedy decode (k=0)"
+    desc = (f"oracle {mode}; context {C} rows "
             f"({ORACLE_SAMPLE['n_visual']} visual + {ORACLE_SAMPLE['n_prompt']} prompt) instead of 288; "
             f"{reps} repetitions of the first {ORACLE_SAMPLE['n_ref'] - k - 1} tokens: {steps} steps, "
-            f"{toks} tokens in {dt:.1f} s")
-    return toks / dt, desc, threads, steps, dt
+            f"{toks} tokens in {dt:.1f} s, {used} BLAS thread(s)")
+    return toks / dt, desc, used, steps, dt
+
+
+def oracle_variants(dims: synth.ModelDims, k: int, bits, budget_s: float = 6.0):
+    """The oracle at k = 0 on all cores and at k on one BLAS thread (shorter
+    samples, reported beside the main CPU baseline); never fails the bench."""
+    out = []
+    for kk, th in ((0, None), (k, 1)):
+        try:
+            tps, desc, used, _, _ = run_oracle_sample(dims, kk, bits, budget_s=budget_s, threads=th)
+            out.append({"k": kk, "threads": used, "value": tps, "unit": "tokens/s", "sample": desc})
+        except Exception as e:  # diagnostics only
+            out.append({"k": kk, "threads": th, "value": None, "error": repr(e)})
+    return out
 
 
 def reference_arm(args, dims):
@@ -412,6 +436,8 @@ def main():
                    "host_cpus": os.cpu_count()}
         except MemoryError as e:
             cpu = {"value": None, "unit": "tokens/s", "cores": None, "kind": "oracle", "sample": f"failed: {e}"}
+        if cpu is not None and cpu["value"] is not None:
+            cpu["variants"] = oracle_variants(dims, k, bits)
 
     if rank == 0:
         line = {
