@@ -415,17 +415,24 @@ def main():
         g_before = dec.stats(0).n_generated
         barrier()
         torch.cuda.synchronize()
+        lat = []  # per-step latency as the host sees it (launch, copy-out, sync)
         t0 = time.perf_counter()
+        tp = t0
         for _ in range(args.steps):
             dec.step_host(1, k, hc, hn)
-        t1 = time.perf_counter()
+            tn = time.perf_counter()
+            lat.append(tn - tp)
+            tp = tn
+        t1 = tp
         barrier()
         e2e_tok = dec.stats(0).n_generated - g_before
         e2e_s = max_over_ranks(t1 - t0)
         e2e = {"value": sum_over_ranks(e2e_tok) / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
                "d2h_bytes_per_step": 4 * (k + 2),
                "note": "ocrdec_step_host per step: graph launch, D2H of committed tokens + count, stream sync; "
-                       "the step has no per-step host input (state lives on the device)"}
+                       "the step has no per-step host input (state lives on the device)",
+               "step_latency_ms": {"mean": 1000 * float(np.mean(lat)), "p50": 1000 * float(np.percentile(lat, 50)),
+                                   "p99": 1000 * float(np.percentile(lat, 99)), "rank": rank}}
 
     # ---- CPU baseline (rank 0, N = 1) ----
     cpu = None
