@@ -92,7 +92,25 @@ WORKLOADS: Dict[str, Workload] = {
     "full_spec": Workload("full_spec", FULL, 1, 101, 256, 32, 1085, (1, 2, 3), stream_seed=202),
     # dynamic-resolution long context: 256 + 100 x 9 visual + 64 prompt, 4096 tokens, k = 3
     "full_long": Workload("full_long", FULL, 1, 103, 1156, 64, 4096, (3,), stream_seed=203),
+    # batched serving, 32 concurrent sequences at k = 1 (p = 0.83), finished
+    # sequences refilled; per-sequence visual counts and lengths from
+    # make_batch_sequences (n_visual / n_generate here are the means)
+    "full_batch32": Workload("full_batch32", FULL, 1, 104, 706, 32, 1085, (1,), stream_seed=204,
+                             accept_p=(0.83,), batch=32),
 }
+
+
+def make_batch_sequences(seed: int, n: int) -> Tuple[np.ndarray, np.ndarray]:
+    """Shapes of n sequences of the batched-serving workload: visual count
+    256 + 100 u with u uniform on 0..9 (dynamic resolution), and an output
+    length drawn lognormal with sigma 0.5 and mean 1,085 (mu = ln 1085 -
+    sigma^2 / 2), rounded to an integer in [1, 4096]."""
+    rng = np.random.default_rng([seed, 4])
+    u = rng.integers(0, 10, n)
+    sigma = 0.5
+    mu = np.log(1085.0) - sigma * sigma / 2
+    lengths = np.clip(np.rint(rng.lognormal(mu, sigma, n)), 1, 4096).astype(np.int64)
+    return (256 + 100 * u).astype(np.int64), lengths
 
 
 def manifest(m: ModelDims) -> List[Tuple[str, Tuple[int, ...]]]:

@@ -94,3 +94,19 @@ def test_forced_miss_is_uniform_over_other_tokens():
     assert seen[3] == 0
     others = seen[np.arange(V) != 3]
     assert others.min() > 0.9 * others.mean() and others.max() < 1.1 * others.mean()
+
+
+def test_batch_workload_shapes():
+    """The batched-serving stand-in: lengths lognormal with mean 1,085 capped at
+    4,096, visual counts 256 + 100 n with n uniform on 0..9."""
+    from speculative_moe_decoding_b200 import synth
+    vis, lengths = synth.make_batch_sequences(synth.WORKLOADS["full_batch32"].input_seed, 40000)
+    assert lengths.min() >= 1 and lengths.max() <= 4096
+    assert abs(lengths.mean() - 1085) < 0.01 * 1085
+    # lognormal: the median is exp(mu) = 1085 * exp(-sigma^2 / 2)
+    assert abs(np.median(lengths) - 1085 * np.exp(-0.125)) < 0.02 * 1085
+    assert set(np.unique(vis)) == {256 + 100 * n for n in range(10)}
+    counts = np.bincount((vis - 256) // 100, minlength=10)
+    assert counts.min() > 0.9 * len(vis) / 10
+    again = synth.make_batch_sequences(synth.WORKLOADS["full_batch32"].input_seed, 40000)
+    assert np.array_equal(again[1], lengths)
