@@ -25,7 +25,11 @@
 // its block of W_o (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; the
 // block arrives by TMA before the dependency wait) and writes the partial sums
 // per head; the last of the H heads to finish a row block adds the partials
-// in head order to the residual stream.
+// in head order to the residual stream.  In MoE layers that last arriver also
+// writes the block's router partials (route.cuh): the dot products of its
+// columns of W_r with g * x (g the FFN RMSNorm gains, x the new residual, as
+// bf16 high and low parts, on the tensor cores) and the block's sum of
+// squares of x; the expert gate/up GEMV finishes the router logits from them.
 // Which CTA takes a chunk and the order of every sum depend only on positions
 // (an MMA column depends on its own row's data only; positions a row does not
 // see carry p = 0 exactly), so a row's result does not depend on the other
