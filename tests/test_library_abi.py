@@ -67,6 +67,13 @@ def test_config_validation(lib):
         dict(good, d_model=192, n_heads=3),    # d_model a multiple of 128
         dict(good, n_experts=65),          # routed experts beyond the router block
         dict(good, n_shared=9),            # shared experts beyond the routing tables
+        dict(good, top_k=0),               # sizes must be positive
+        dict(good, d_model=2176, n_heads=17),  # d_model beyond 2048 (and > 16 heads)
+        dict(good, n_dense_first=3),       # more dense layers than layers
+        dict(good, n_dense_first=1, dense_ffn=100),  # dense width a multiple of 64
+        dict(good, expert_ffn=96, shared_ffn=96),    # expert width a multiple of 64
+        dict(good, rms_eps=0.0),           # eps must be positive
+        dict(good, rope_theta=1.0),        # theta must exceed 1
     ]
     for bad in bad_cases:
         cfg = lib.make_config(bad, 3, 1, 256)
