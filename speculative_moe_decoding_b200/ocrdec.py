@@ -275,23 +275,70 @@ def op_scratch(device="cuda"):
     return torch.zeros(ocrdec_op_scratch_bytes(), dtype=torch.uint8, device=device)
 
 
-def op_norm_gemv(W, x, g, eps, y, scratch, stream=None):
+def _need(t, name, dtypes, shape=None, cuda=True):
+    """Argument checks before a pointer crosses the ABI: a torch tensor of one
+    of the dtypes, the given shape, contiguous and (cuda) on a CUDA device."""
+    import torch
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch tensor, got {type(t).__name__}")
+    if t.dtype not in dtypes:
+        raise ValueError(f"{name}: dtype {t.dtype}, expected one of {', '.join(map(str, dtypes))}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+    if cuda and not t.is_cuda:
+        raise ValueError(f"{name}: must be a CUDA tensor")
+
+
+def _bf16_types():
+    import torch
+    return (torch.bfloat16, torch.int16) + ((torch.uint16,) if hasattr(torch, "uint16") else ())
+
+
+def _op_args(W, x, g, out_name, out, out_dtypes, scratch=None, logits=None):
+    """Types and shapes of every argument first, then their devices."""
+    import torch
+    _need(x, "x", (torch.float32,), cuda=False)
+    if x.dim() != 2:
+        raise ValueError(f"x: expected [R, K], got shape {tuple(x.shape)}")
     R, K = x.shape
+    if not isinstance(W, torch.Tensor) or W.dim() != 2:
+        raise ValueError("W: expected a [N, K] tensor")
     N = W.shape[0]
+    _need(W, "W", _bf16_types(), (N, K), cuda=False)
+    _need(g, "g", _bf16_types(), (K,), cuda=False)
+    _need(out, out_name, out_dtypes, (R, N) if out_name == "y" else (R,), cuda=False)
+    named = [("x", x), ("W", W), ("g", g), (out_name, out)]
+    if logits is not None:
+        _need(logits, "logits", (torch.float32,), (R, N), cuda=False)
+        named.append(("logits", logits))
+    if scratch is not None:
+        _need(scratch, "scratch", (torch.uint8,), cuda=False)
+        named.append(("scratch", scratch))
+    for name, t in named:
+        if not t.is_cuda:
+            raise ValueError(f"{name}: must be a CUDA tensor")
+    return R, N, K
+
+
+def op_norm_gemv(W, x, g, eps, y, scratch, stream=None):
+    import torch
+    R, N, K = _op_args(W, x, g, "y", y, (torch.float32,), scratch)
     check(ocrdec_op_norm_gemv(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, y.data_ptr(),
                               scratch.data_ptr(), _stream(stream)), "ocrdec_op_norm_gemv")
 
 
 def op_lm_argmax(W, x, g, eps, tok, logits, scratch, stream=None):
-    R, K = x.shape
-    N = W.shape[0]
+    import torch
+    R, N, K = _op_args(W, x, g, "tok", tok, (torch.int32,), scratch, logits)
     check(ocrdec_op_lm_argmax(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
                               _ptr(logits), scratch.data_ptr(), _stream(stream)), "ocrdec_op_lm_argmax")
 
 
 def op_lm_argmax_static(W, x, g, eps, tok, logits, stream=None):
     """op_lm_argmax on the library's fixed per-device scratch (allocates nothing)."""
-    R, K = x.shape
-    N = W.shape[0]
+    import torch
+    R, N, K = _op_args(W, x, g, "tok", tok, (torch.int32,), None, logits)
     check(ocrdec_op_lm_argmax_static(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
                                      _ptr(logits), _stream(stream)), "ocrdec_op_lm_argmax_static")

@@ -107,3 +107,29 @@ def test_op_argument_checks(lib):
     for R, N, K in [(1, 64, 4000), (1, 64, 1000), (0, 64, 256), (9, 64, 256), (1, 0, 256), (1, 64, 32)]:
         assert lib.ocrdec_op_norm_gemv(p, p, p, ctypes.c_float(1e-6), R, N, K, p, p, None) == lib.EINVAL
         assert lib.ocrdec_op_lm_argmax(p, p, p, ctypes.c_float(1e-6), R, N, K, p, None, p, None) == lib.EINVAL
+
+
+def test_binding_checks_op_arguments_before_the_abi():
+    """The op wrappers reject wrong dtypes, shapes and layouts (and host
+    tensors) before a pointer crosses the ABI."""
+    import torch
+    from speculative_moe_decoding_b200 import ocrdec
+    W = torch.zeros(64, 256, dtype=torch.int16)
+    x = torch.zeros(2, 256)
+    g = torch.zeros(256, dtype=torch.bfloat16)
+    y = torch.zeros(2, 64)
+    tok = torch.zeros(2, dtype=torch.int32)
+    sc = torch.zeros(16, dtype=torch.uint8)
+    bad = [
+        (lambda: ocrdec.op_norm_gemv(W.float(), x, g, 1e-6, y, sc), "W: dtype"),
+        (lambda: ocrdec.op_norm_gemv(W, x.double(), g, 1e-6, y, sc), "x: dtype"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g[:128], 1e-6, y, sc), "g: shape"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, y[:, :32].contiguous(), sc), "y: shape"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, torch.zeros(64, 2).t(), sc), "y: must be contiguous"),
+        (lambda: ocrdec.op_lm_argmax(W, x, g, 1e-6, tok.long(), None, sc), "tok: dtype"),
+        (lambda: ocrdec.op_lm_argmax_static(W, x, g, 1e-6, tok, torch.zeros(2, 63)), "logits: shape"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, y, sc), "must be a CUDA tensor"),
+    ]
+    for call, msg in bad:
+        with pytest.raises(ValueError, match=msg):
+            call()
