@@ -176,6 +176,11 @@ class Decoder:
     def prefill(self, slot: int, visual, prompt, stream=None):
         """visual: float32 CUDA tensor [n_visual, d]; prompt: int32 CUDA tensor.  Returns a 1-element
         int32 CUDA tensor holding the first generated token."""
+        torch = self.torch
+        if visual is not None:
+            _need(visual, "visual", (torch.float32,), (int(visual.shape[0]), int(self.dims["d_model"])))
+        if prompt is not None:
+            _need(prompt, "prompt", (torch.int32,), (int(prompt.numel()),))
         out = self._i32(1)
         check(ocrdec_prefill(self.ctx, slot, _ptr(visual), int(visual.shape[0]) if visual is not None else 0,
                              _ptr(prompt), int(prompt.shape[0]) if prompt is not None else 0, out.data_ptr(),
