@@ -341,3 +341,81 @@ def test_attention_two_keys_is_logistic_in_scaled_score_gap():
         gap = float(q.astype(np.float64) @ (K[0] - K[1]).astype(np.float64)) / np.sqrt(dh)
         np.testing.assert_allclose(out[0], scipy.special.expit(gap), rtol=1e-5)
         np.testing.assert_allclose(out[0] + out[1], 1.0, rtol=1e-6)
+
+
+# ---------------------------------------------------------------- RoPE frequencies
+def _pair_rotation_matrix(dh, angles):
+    """Block rotation of the rotate-half layout, built entry by entry: dims i
+    and i + dh/2 form plane i, turned by angles[i] (a counter-clockwise turn of
+    the column vector (a, b))."""
+    half = dh // 2
+    M = np.zeros((dh, dh), np.float64)
+    for i in range(half):
+        c, s = np.cos(angles[i]), np.sin(angles[i])
+        M[i, i], M[i, i + half] = c, -s
+        M[i + half, i], M[i + half, i + half] = s, c
+    return M
+
+
+@pytest.mark.parametrize("dh", [4, 8, 128])
+def test_rope_pair_frequencies_follow_the_inverse_power_schedule(dh):
+    """Plane i at position p turns by p * theta^(-2i/dh), theta = 10^6 (model
+    specification table, RoPE row).  At dh = 4 the second plane turns by
+    p * 10^-3 radians; a schedule theta^(-i/dh), a different theta or swapped
+    halves all give other angles and fail."""
+    spec = _read_kv(os.path.join(GOLDEN, "model_spec.txt"))
+    theta = spec["rope_theta"]
+    assert theta == 1e6
+    half = dh // 2
+    rng = np.random.default_rng(dh)
+    v = rng.standard_normal(dh).astype(np.float32)
+    for p in (1, 7, 250, 4095):
+        # the frequencies written out for the small cases
+        if dh == 4:
+            want_ang = [p * 1.0, p * 1e-3]
+        elif dh == 8:
+            want_ang = [p * 1.0, p * 10 ** -1.5, p * 1e-3, p * 10 ** -4.5]
+        else:
+            want_ang = [p * 10.0 ** (-6.0 * 2 * i / dh) for i in range(half)]
+        c, s = O.rope_cos_sin(p, dh, theta)
+        np.testing.assert_allclose(c, np.cos(want_ang), atol=1e-7)
+        np.testing.assert_allclose(s, np.sin(want_ang), atol=1e-7)
+        got = O.apply_rope(v, p, theta)
+        want = _pair_rotation_matrix(dh, want_ang) @ v.astype(np.float64)
+        np.testing.assert_allclose(got, want, rtol=1e-5, atol=1e-5)
+
+
+def test_rope_dh4_second_plane_turns_by_a_thousandth_per_position():
+    """Direct reading at dh = 4: unit vector on dim 1 (plane 1's first axis)
+    goes to (cos(p/1000), sin(p/1000)) on dims (1, 3)."""
+    for p in (1, 500, 3141):
+        e1 = np.array([0.0, 1.0, 0.0, 0.0], np.float32)
+        r = O.apply_rope(e1, p, 1e6)
+        np.testing.assert_allclose(r, [0.0, np.cos(p * 1e-3), 0.0, np.sin(p * 1e-3)], atol=1e-6)
+
+
+# ---------------------------------------------------------------- argmax margin
+def test_top2_margin_hand_built_logits():
+    """The gap between the largest and second-largest logit: the quantity the
+    teacher-forced token comparison is gated on (margin < 0.1 is exempt)."""
+    cases = [
+        ([1.0, 3.0, 2.0], 1.0),           # max in the middle
+        ([9.0, 1.0, 2.0], 7.0),           # max at index 0
+        ([0.5, 0.25, 4.0], 3.5),          # max at the last index
+        ([5.0, 5.0, 1.0], 0.0),           # tie at the top
+        ([2.0, 7.0, 7.0, 7.0], 0.0),      # three-way tie
+        ([-1.0, -5.0, -3.0], 2.0),        # all negative
+        ([0.0, 0.125], 0.125),            # two entries
+        ([3.0, 3.0 - 2 ** -20, -1e9], 2 ** -20),  # tiny gap, float32-exact
+    ]
+    for logits, want in cases:
+        got = O.top2_margin(np.array(logits, np.float32))
+        assert got == want, (logits, got, want)
+    # invariant under a permutation and a common shift; never negative
+    rng = np.random.default_rng(12)
+    z = rng.standard_normal(4096).astype(np.float32)
+    m = O.top2_margin(z)
+    srt = np.sort(z)
+    assert m == float(srt[-1] - srt[-2]) and m >= 0
+    assert O.top2_margin(rng.permutation(z)) == m
+    np.testing.assert_allclose(O.top2_margin(z + np.float32(10.0)), m, atol=2e-6)
