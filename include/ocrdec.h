@@ -34,6 +34,16 @@
  *     length in to out outputs.  Weights are bfloat16, 16-byte aligned.
  *   - Sequences live in slots 0..max_batch-1.  Batched calls operate on
  *     slots 0..batch-1.
+ *
+ * Names against the planned interface of this step (create / workspace /
+ * load_weights / prefill / draft / verify_commit / step graph / status /
+ * debug taps): the captured whole-step call is ocrdec_step (planned name
+ * ocrdec_step_graph); the parity taps are set with ocrdec_set_debug_taps
+ * (planned ocrdec_debug_taps) and ocrdec_set_draft_taps; batched calls take
+ * the slot range 0..batch-1 instead of a device array of slot ids, because
+ * every pass is laid out slot-major on the device; the expert path has one
+ * mode (the weight-streaming GEMV of up to 8 rows per pass), so the config
+ * has no expert-path field.
  */
 #ifndef OCRDEC_H
 #define OCRDEC_H
@@ -90,7 +100,12 @@ typedef struct {
 
 /* ---- setup ---------------------------------------------------------------- */
 
-/* Validates the config (positive sizes, n_heads*head_dim == d_model, head_dim
+/* The model: the specification table of the news article "jina-ocr-v1:
+ * faster document parsing on low-budget GPUs" (and the tahou.com item's
+ * "model core parameters" table): 12 layers, d = 1280, 64 routed + 2 shared
+ * experts, top-6, vocabulary 129,280, RoPE theta = 10^6; the head layout and
+ * FFN widths are free parameters of the config.
+ * Validates the config (positive sizes, n_heads*head_dim == d_model, head_dim
  * 64 or 128, n_heads <= 16, d_model <= 2048 and a multiple of 128, the FFN
  * widths multiples of 64,
  * vocab a multiple of 8, top_k <= min(n_experts, 8), n_experts <= 64,
@@ -99,7 +114,10 @@ typedef struct {
 OCRDEC_API int ocrdec_create(const ocrdec_config* cfg, ocrdec_ctx** out);
 OCRDEC_API void ocrdec_destroy(ocrdec_ctx* ctx);
 
-/* Number of weight tensors and the shape of tensor `index` in manifest order:
+/* The tensors of the decoder and its draft block (news article, "Model and
+ * training": a DeepSeek-style MoE decoder and one FastMTP dense block; model
+ * page "jina-ocr-v1", architecture paragraph).
+ * Number of weight tensors and the shape of tensor `index` in manifest order:
  * embed[V][d]; per layer: attn_norm[d], wqkv[3d][d] (rows q | k | v, head-major),
  * wo[d][d], ffn_norm[d], then for a dense layer w_gate_up[2F][d] (gate rows then
  * up rows), w_down[d][F], and for a MoE layer router[E][d],
@@ -125,7 +143,11 @@ OCRDEC_API int ocrdec_load_weights(ocrdec_ctx* ctx, const void* const* host_dev_
 
 /* ---- the decode path -------------------------------------------------------- */
 
-/* Context of one sequence: n_visual visual embeddings (float32 [n_visual][d],
+/* Prefill (news article, figure caption of the architecture and "Model and
+ * training": the decoder reads 256 + 100n visual tokens from the vision
+ * encoder, then the text prompt; model page: up to 1,156 visual tokens per
+ * page in Gundam mode).
+ * Context of one sequence: n_visual visual embeddings (float32 [n_visual][d],
  * standing in for the vision encoder output) then n_prompt tokens, at
  * positions 0..C-1.  Runs the verifier over the context and the draft block
  * over the context pairs, writes the first generated token (argmax at C-1) to
@@ -135,14 +157,23 @@ OCRDEC_API int ocrdec_prefill(ocrdec_ctx* ctx, int slot, const float* dev_visual
                    const int32_t* dev_prompt, int n_prompt, int32_t* dev_first_token,
                    ocrdec_stream stream);
 
-/* FastMTP draft for slots 0..batch-1: recursion 1 runs the shared block on the
+/* The FastMTP draft (news article, "Model and training": ONE shared dense
+ * block applied recursively for K = 3 prediction steps; "Getting started":
+ * recursive hidden-state feedback, mtp_recursive=True; model page, FastMTP
+ * paragraph).
+ * Draft for slots 0..batch-1: recursion 1 runs the shared block on the
  * pairs committed by the previous verify (verifier hidden at p, token at p+1),
  * recursions 2..k feed the block's own output hidden with the previous draft
  * token; each recursion ends with the tied LM head's argmax.  Writes
  * dev_proposals[batch][k].  1 <= k <= max_k. */
 OCRDEC_API int ocrdec_draft(ocrdec_ctx* ctx, int batch, int k, int32_t* dev_proposals, ocrdec_stream stream);
 
-/* Verifier pass over [bonus, proposals[b][0..k-1]] at positions kv_len..kv_len+k
+/* Greedy verification (news article, "Model and training": the verifier
+ * checks the proposals greedily and keeps the longest prefix on which draft
+ * and verifier agree, plus the verifier's own next token; model page: the
+ * output is bit-identical to plain autoregressive decoding; "L4 speculative
+ * decoding" analysis: tau counts the committed tokens including that bonus).
+ * Verifier pass over [bonus, proposals[b][0..k-1]] at positions kv_len..kv_len+k
  * for slots 0..batch-1, then greedy acceptance: a = length of the longest prefix
  * with proposals[b][j] == argmax at row j; commits rows' argmax 0..a (a+1 tokens),
  * sets kv_len += a+1 (the rejected rows' KV entries become dead), and stores
@@ -152,19 +183,26 @@ OCRDEC_API int ocrdec_draft(ocrdec_ctx* ctx, int batch, int k, int32_t* dev_prop
 OCRDEC_API int ocrdec_verify_commit(ocrdec_ctx* ctx, int batch, int k, const int32_t* dev_proposals,
                          int32_t* dev_committed, int32_t* dev_n_committed, ocrdec_stream stream);
 
-/* One whole step (draft when k > 0, the forced-acceptance override when set,
+/* The step as one replayed CUDA graph (news article, "L4 speculative
+ * decoding" table: graph mode against eager mode, 158.3 against 42.7 tokens/s
+ * at k = 0 - launch overhead is the lever at batch 1).
+ * One whole step (draft when k > 0, the forced-acceptance override when set,
  * verify and commit), launched as a CUDA graph captured on first use for each
  * (batch, k, output pointers).  Same outputs as ocrdec_verify_commit. */
 OCRDEC_API int ocrdec_step(ocrdec_ctx* ctx, int batch, int k, int32_t* dev_committed,
                 int32_t* dev_n_committed, ocrdec_stream stream);
 
-/* Same step for callers holding host buffers: copies the results back into
+/* The same passage as ocrdec_step.
+ * Same step for callers holding host buffers: copies the results back into
  * host_committed[batch][k+1] / host_n_committed[batch] and synchronises the
  * stream before returning. */
 OCRDEC_API int ocrdec_step_host(ocrdec_ctx* ctx, int batch, int k, int32_t* host_committed,
                      int32_t* host_n_committed, ocrdec_stream stream);
 
-/* Benchmark acceptance model (not part of the method): after the draft runs,
+/* Benchmark acceptance model (not part of the method; its per-depth hit
+ * probabilities 0.83 / 0.69 / 0.58 reproduce the acceptance and tau columns of
+ * the news article's "L4 speculative decoding" table, and 0.83 is the
+ * mubeitech.com interpretation's first-draft hit rate): after the draft runs,
  * its proposal for target position t at depth j (1-based) is replaced by
  * dev_ref[t] when dev_u[t*max_k + j-1] < p[j-1], and otherwise by the token
  * dev_alt[t*max_k + j-1] of the vocabulary with dev_ref[t] removed.  dev_ref
@@ -282,7 +320,8 @@ OCRDEC_API size_t ocrdec_op_scratch_bytes(void);
  *
  * Returns OCRDEC_OK, OCRDEC_EINVAL (the argument checks of
  * ocrdec_op_lm_argmax), OCRDEC_ENOMEM if this device needs more scratch than
- * the fixed array holds (more than 509 SMs), or OCRDEC_ECUDA (no current
+ * the fixed array holds (more than 510 SMs: 256 + 128 bytes per SM must fit
+ * in 64 KiB), or OCRDEC_ECUDA (no current
  * device, symbol lookup or launch failed). */
 OCRDEC_API int ocrdec_op_lm_argmax_static(const void* dev_W, const float* dev_x, const void* dev_g, float eps,
                                           int R, int N, int K, int32_t* dev_tok, float* dev_logits,

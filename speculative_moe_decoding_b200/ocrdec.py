@@ -181,6 +181,9 @@ class Decoder:
             _need(visual, "visual", (torch.float32,), (int(visual.shape[0]), int(self.dims["d_model"])))
         if prompt is not None:
             _need(prompt, "prompt", (torch.int32,), (int(prompt.numel()),))
+        for name, t in (("visual", visual), ("prompt", prompt)):
+            if t is not None and t.device != self.workspace.device:
+                raise ValueError(f"{name}: on {t.device}, but the decoder lives on {self.workspace.device}")
         out = self._i32(1)
         check(ocrdec_prefill(self.ctx, slot, _ptr(visual), int(visual.shape[0]) if visual is not None else 0,
                              _ptr(prompt), int(prompt.shape[0]) if prompt is not None else 0, out.data_ptr(),
@@ -302,7 +305,8 @@ def _bf16_types():
 
 
 def _op_args(W, x, g, out_name, out, out_dtypes, scratch=None, logits=None):
-    """Types and shapes of every argument first, then their devices."""
+    """Types and shapes of every argument first, then the scratch size, then
+    that all tensors share one CUDA device.  Returns (R, N, K, device)."""
     import torch
     _need(x, "x", (torch.float32,), cuda=False)
     if x.dim() != 2:
@@ -320,30 +324,41 @@ def _op_args(W, x, g, out_name, out, out_dtypes, scratch=None, logits=None):
         named.append(("logits", logits))
     if scratch is not None:
         _need(scratch, "scratch", (torch.uint8,), cuda=False)
+        # the kernels write status words, counters and partials across the
+        # whole documented scratch size; the C side cannot see the length
+        need = int(ocrdec_op_scratch_bytes())
+        if scratch.numel() < need:
+            raise ValueError(f"scratch: {scratch.numel()} bytes, need at least {need} (op_scratch() allocates it)")
         named.append(("scratch", scratch))
+    for name, t in named:
+        if t.device != x.device:
+            raise ValueError(f"{name}: on {t.device}, but x is on {x.device}; all tensors must share one device")
     for name, t in named:
         if not t.is_cuda:
             raise ValueError(f"{name}: must be a CUDA tensor")
-    return R, N, K
+    return R, N, K, x.device
 
 
 def op_norm_gemv(W, x, g, eps, y, scratch, stream=None):
     import torch
-    R, N, K = _op_args(W, x, g, "y", y, (torch.float32,), scratch)
-    check(ocrdec_op_norm_gemv(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, y.data_ptr(),
-                              scratch.data_ptr(), _stream(stream)), "ocrdec_op_norm_gemv")
+    R, N, K, dev = _op_args(W, x, g, "y", y, (torch.float32,), scratch)
+    with torch.cuda.device(dev):  # the kernel runs on the tensors' device
+        check(ocrdec_op_norm_gemv(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, y.data_ptr(),
+                                  scratch.data_ptr(), _stream(stream)), "ocrdec_op_norm_gemv")
 
 
 def op_lm_argmax(W, x, g, eps, tok, logits, scratch, stream=None):
     import torch
-    R, N, K = _op_args(W, x, g, "tok", tok, (torch.int32,), scratch, logits)
-    check(ocrdec_op_lm_argmax(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
-                              _ptr(logits), scratch.data_ptr(), _stream(stream)), "ocrdec_op_lm_argmax")
+    R, N, K, dev = _op_args(W, x, g, "tok", tok, (torch.int32,), scratch, logits)
+    with torch.cuda.device(dev):
+        check(ocrdec_op_lm_argmax(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
+                                  _ptr(logits), scratch.data_ptr(), _stream(stream)), "ocrdec_op_lm_argmax")
 
 
 def op_lm_argmax_static(W, x, g, eps, tok, logits, stream=None):
     """op_lm_argmax on the library's fixed per-device scratch (allocates nothing)."""
     import torch
-    R, N, K = _op_args(W, x, g, "tok", tok, (torch.int32,), None, logits)
-    check(ocrdec_op_lm_argmax_static(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
-                                     _ptr(logits), _stream(stream)), "ocrdec_op_lm_argmax_static")
+    R, N, K, dev = _op_args(W, x, g, "tok", tok, (torch.int32,), None, logits)
+    with torch.cuda.device(dev):  # the scratch used is the one of this device
+        check(ocrdec_op_lm_argmax_static(W.data_ptr(), x.data_ptr(), g.data_ptr(), eps, R, N, K, tok.data_ptr(),
+                                         _ptr(logits), _stream(stream)), "ocrdec_op_lm_argmax_static")

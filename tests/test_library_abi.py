@@ -119,7 +119,8 @@ def test_binding_checks_op_arguments_before_the_abi():
     g = torch.zeros(256, dtype=torch.bfloat16)
     y = torch.zeros(2, 64)
     tok = torch.zeros(2, dtype=torch.int32)
-    sc = torch.zeros(16, dtype=torch.uint8)
+    sc = torch.zeros(ocrdec.ocrdec_op_scratch_bytes(), dtype=torch.uint8)
+    small = torch.zeros(16, dtype=torch.uint8)
     bad = [
         (lambda: ocrdec.op_norm_gemv(W.float(), x, g, 1e-6, y, sc), "W: dtype"),
         (lambda: ocrdec.op_norm_gemv(W, x.double(), g, 1e-6, y, sc), "x: dtype"),
@@ -128,6 +129,11 @@ def test_binding_checks_op_arguments_before_the_abi():
         (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, torch.zeros(64, 2).t(), sc), "y: must be contiguous"),
         (lambda: ocrdec.op_lm_argmax(W, x, g, 1e-6, tok.long(), None, sc), "tok: dtype"),
         (lambda: ocrdec.op_lm_argmax_static(W, x, g, 1e-6, tok, torch.zeros(2, 63)), "logits: shape"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, y, small), "scratch: 16 bytes, need at least"),
+        (lambda: ocrdec.op_lm_argmax(W, x, g, 1e-6, tok, None, small), "scratch: 16 bytes, need at least"),
+        (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, y.to("meta"), sc), "y: on meta, but x is on cpu"),
+        (lambda: ocrdec.op_lm_argmax(W.to("meta"), x, g, 1e-6, tok, None, sc), "W: on meta"),
+        (lambda: ocrdec.op_lm_argmax_static(W, x, g, 1e-6, tok, torch.zeros(2, 64, device="meta")), "logits: on meta"),
         (lambda: ocrdec.op_norm_gemv(W, x, g, 1e-6, y, sc), "must be a CUDA tensor"),
     ]
     for call, msg in bad:
