@@ -224,12 +224,42 @@ def profiled_traffic(name):
         return None
 
 
+def _peak():
+    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(peaks_path):
+        pk = json.load(open(peaks_path))
+        return float(pk["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, STREAM-style copy)"
+    return 6650.0, "fallback (6.65 TB/s, earlier measurement on this pool)"
+
+
+def _graph_time_ms(torch, stream, enqueue, n_inner, replays=8, skip=3):
+    """Mean time of one of n_inner back-to-back enqueues captured in one CUDA
+    graph: CUDA events on the launching stream around each replay."""
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        for _ in range(n_inner):
+            enqueue()
+    times = []
+    for i in range(replays):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        graph.replay()
+        b.record(stream)
+        torch.cuda.synchronize()
+        if i >= skip:
+            times.append(a.elapsed_time(b) / n_inner)
+    del graph
+    return float(np.mean(times))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=390)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--k", type=int, default=3)
+    ap.add_argument("--workload", default="full_spec", choices=["full_spec", "full_long"],
+                    help="full_spec: 256 + 32 context, 1,085 tokens; full_long: 1,156 + 64 context, 4,096 tokens")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-only", action="store_true", help="skip e2e and the CPU baseline (for ncu)")
@@ -257,13 +287,17 @@ def main():
     build.build()
     from speculative_moe_decoding_b200 import ocrdec
 
-    wl = synth.WORKLOADS["full_spec"]
+    wl = synth.WORKLOADS[args.workload]
     k = args.k
     bits, _ = synth.make_weights(dims, wl.weight_seed)
     names = [n for n, _ in synth.manifest(dims)]
-    n_steps_total = args.warmup + args.steps
     C = wl.n_visual + wl.n_prompt
-    n_ref = n_steps_total * (k + 1) + 16
+    tau_exp = metrics.expected_tau(wl.accept_p[:k]) if k > 0 else 1.0
+    # the timed steps sit in the middle of the workload's decode (mean KV
+    # length of the whole decode); the steps before them only position it
+    t_timed = args.steps * tau_exp
+    start_tok = int(max(1, wl.n_generate / 2 - t_timed / 2 - args.warmup * tau_exp))
+    n_ref = max(wl.n_generate, start_tok + int((args.warmup + args.steps) * (k + 1))) + 64
     cap = C + n_ref + 16
     dec = ocrdec.Decoder(dims.as_dict(), bits, names, max_k=3, max_batch=1, kv_capacity=cap)
     inp = synth.make_inputs(dims, wl.input_seed, wl.n_visual, wl.n_prompt, index=rank)
@@ -289,22 +323,20 @@ def main():
         torch.distributed.all_reduce(t)
         return float(t.item())
 
-    # ---- k = 0 reference run (also the plain greedy baseline) ----
+    def advance(kk, n_tokens):
+        """Untimed steps until the slot has generated at least n_tokens."""
+        while True:
+            g = dec.stats(0).n_generated
+            if g >= n_tokens:
+                return
+            for _ in range(max(1, min(64, int((n_tokens - g) / max(1.0, tau_exp if kk else 1.0))))):
+                dec.step(1, kk)
+
+    # ---- k = 0 greedy decode: the reference history of the forced stream ----
     dec.set_forced_acceptance(None, None, None, ())
     dec.prefill(0, vis, prm)
-    n0_steps = n_ref - 1
-    for _ in range(args.warmup):
-        dec.step(1, 0)
+    advance(0, n_ref)
     torch.cuda.synchronize()
-    g0 = dec.stats(0).n_generated
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(n0_steps - args.warmup):
-        dec.step(1, 0)
-    e1.record(stream)
-    torch.cuda.synchronize()
-    k0_ms = e0.elapsed_time(e1)
-    k0_tokens = dec.stats(0).n_generated - g0
     assert dec.status() == 0, dec.status()
     ref_hist = dec.history(0, 0, C + n_ref).clone()
 
@@ -314,6 +346,7 @@ def main():
     r_t = torch.from_numpy(tab.r).cuda()
     dec.set_forced_acceptance(ref_hist, u_t, r_t, tab.p)
     dec.prefill(0, vis, prm)
+    advance(k, start_tok)
     for _ in range(args.warmup):
         dec.step(1, k)
     torch.cuda.synchronize()
@@ -324,6 +357,7 @@ def main():
     time.sleep(0.3)
     barrier()
     torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.nvtx.range_push("timed_steps")
     e0.record(stream)
     for _ in range(args.steps):
@@ -352,10 +386,26 @@ def main():
     kv_mid = C + (st0.n_generated + st1.n_generated) / 2
     union_b, dep_b = step_bytes(dims, k, U, kv_mid)
 
+    # ---- k = 0 over the same token range, same kernels ----
+    dec.set_forced_acceptance(None, None, None, ())
+    dec.prefill(0, vis, prm)
+    advance(0, st0.n_generated)
+    torch.cuda.synchronize()
+    n0 = st1.n_generated - st0.n_generated
+    e0.record(stream)
+    for _ in range(n0):
+        dec.step(1, 0)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    k0_ms = e0.elapsed_time(e1)
+    k0_tps = n0 / (k0_ms / 1000.0)
+    assert dec.status() == 0, dec.status()
+
     # ---- device timeline of a few more steps (outside the timed region) ----
     timeline = None
     if args.trace > 0:
         from speculative_moe_decoding_b200 import timeline as tl
+        dec.set_forced_acceptance(ref_hist, u_t, r_t, tab.p)
         dec.set_trace(True)
         for _ in range(args.trace):
             dec.step(1, k)
@@ -368,13 +418,24 @@ def main():
         if rank == 0:
             print(tl.format_summary(timeline), file=sys.stderr)
 
-    # ---- dominant kernel: LM head + argmax over k+1 rows, timed alone ----
-    import math
-    peaks_path = os.path.join(ROOT, "MEASURED_PEAKS.json")
-    peak_gbs, peak_src = 6650.0, "fallback"
-    if os.path.exists(peaks_path):
-        peak_gbs, peak_src = float(json.load(open(peaks_path))["hbm_gbs"]), "measured"
+    peak_gbs, peak_src = _peak()
     R = k + 1
+    # ---- dominant kernel: the MoE FFN of the 11 MoE layers, replayed on the
+    # last verify pass's rows and routing, each layer's weights once ----
+    dec.set_forced_acceptance(ref_hist, u_t, r_t, tab.p)
+    dec.step(1, k)  # a k-row verify pass leaves its rows and router partials
+    torch.cuda.synchronize()
+    dec.reset_counters()
+    n_moe = dims.n_layers - dims.n_dense_first
+    moe_ms = _graph_time_ms(torch, stream, lambda: dec.replay_moe_ffn(1, k, dims.n_dense_first, n_moe), 1) / n_moe
+    torch.cuda.synchronize()
+    mt, mp = dec.counters()
+    U_moe = mt / max(1, mp)
+    expert_bytes = 3 * dims.d_model * dims.expert_ffn * 2
+    moe_bytes = (U_moe + dims.n_shared) * expert_bytes + 2 * R * dims.d_model * 4
+    moe_gbs = moe_bytes / (moe_ms / 1000.0) / 1e9
+
+    # ---- LM head + argmax over k+1 rows, timed alone ----
     lm_w = dec.weights[names.index("lm_head")]
     g_w = dec.weights[names.index("final_norm")]
     xr = torch.randn((R, dims.d_model), dtype=torch.float32, device="cuda")
@@ -382,66 +443,77 @@ def main():
     scratch = ocrdec.op_scratch()
     ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)  # one-time kernel set-up
     torch.cuda.synchronize()
-    # LM_BACK_TO_BACK launches in one graph: each streams the whole 331 MB head,
-    # more than L2 holds, so no launch finds its weights in cache
-    LM_BACK_TO_BACK = 10
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(graph):
-        for _ in range(LM_BACK_TO_BACK):
-            ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None, scratch)
-    times = []
-    for i in range(8):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        graph.replay()
-        b.record(stream)
-        torch.cuda.synchronize()
-        if i >= 3:
-            times.append(a.elapsed_time(b) / LM_BACK_TO_BACK)
-    del graph
-    lm_ms = float(np.mean(times))
+    # 10 launches back to back: each streams the whole 331 MB head, more than
+    # L2 holds, so no launch finds its weights in cache
+    lm_ms = _graph_time_ms(torch, stream, lambda: ocrdec.op_lm_argmax(lm_w, xr, g_w, dims.rms_eps, tok, None,
+                                                                       scratch), 10)
     lm_bytes = dims.vocab * dims.d_model * 2 + R * dims.d_model * 4 + dims.d_model * 2
     lm_gbs = lm_bytes / (lm_ms / 1000.0) / 1e9
-    lm_traffic = profiled_traffic("lm_head_argmax_r4.md")
 
-    # ---- end to end through host buffers ----
+    # ---- end to end: whole requests through the C ABI from host buffers ----
     e2e = None
     if not args.profile_only:
-        # result buffers in pinned host memory (a copy into pageable memory is
-        # staged and synchronous); numpy views keep the call's signature
+        pin = lambda t: t.pin_memory()
         try:
-            pinned = (torch.zeros(k + 1, dtype=torch.int32).pin_memory(),
-                      torch.zeros(1, dtype=torch.int32).pin_memory())
-            hc, hn = pinned[0].numpy(), pinned[1].numpy()
+            vis_h, prm_h = pin(torch.from_numpy(inp.visual)), pin(torch.from_numpy(inp.prompt))
+            hc_t = pin(torch.zeros(k + 1, dtype=torch.int32))
+            hn_t = pin(torch.zeros(1, dtype=torch.int32))
+            hf_t = pin(torch.zeros(1, dtype=torch.int32))
+            pinned = True
         except Exception:  # no pinned memory: pageable buffers (the note says which)
-            pinned = None
-            hc = np.zeros(k + 1, np.int32)
-            hn = np.zeros(1, np.int32)
-        dec.prefill(0, vis, prm)
-        for _ in range(args.warmup):
-            dec.step_host(1, k, hc, hn)
-        g_before = dec.stats(0).n_generated
+            vis_h, prm_h = torch.from_numpy(inp.visual), torch.from_numpy(inp.prompt)
+            hc_t, hn_t, hf_t = (torch.zeros(k + 1, dtype=torch.int32), torch.zeros(1, dtype=torch.int32),
+                                torch.zeros(1, dtype=torch.int32))
+            pinned = False
+        hc, hn = hc_t.numpy(), hn_t.numpy()
+        vis_d, prm_d = torch.empty_like(vis), torch.empty_like(prm)
+        dec.set_forced_acceptance(ref_hist, u_t, r_t, tab.p)
+
+        def request():
+            """One page: inputs host -> device, prefill, decode to n_generate
+            tokens with the committed tokens read back after every step (what
+            a streaming client receives).  Returns (tokens, steps, prefill s)."""
+            vis_d.copy_(vis_h, non_blocking=True)
+            prm_d.copy_(prm_h, non_blocking=True)
+            first = dec.prefill(0, vis_d, prm_d)
+            hf_t.copy_(first, non_blocking=True)
+            stream.synchronize()
+            t_pf = time.perf_counter()
+            got, n_st = 1, 0
+            while got < wl.n_generate:
+                dec.step_host(1, k, hc, hn)
+                got += int(hn[0])
+                n_st += 1
+            return got, n_st, t_pf
+
+        request()  # warm-up request
         barrier()
         torch.cuda.synchronize()
-        lat = []  # per-step latency as the host sees it (launch, copy-out, sync)
+        n_req = 2 if wl.n_generate <= 2048 else 1
         t0 = time.perf_counter()
-        tp = t0
-        for _ in range(args.steps):
-            dec.step_host(1, k, hc, hn)
-            tn = time.perf_counter()
-            lat.append(tn - tp)
-            tp = tn
-        t1 = tp
+        tot = nst = 0
+        pf = 0.0
+        for _ in range(n_req):
+            ts = time.perf_counter()
+            got, n_st, t_pf = request()
+            pf += t_pf - ts
+            tot += got
+            nst += n_st
+        t1 = time.perf_counter()
         barrier()
-        e2e_tok = dec.stats(0).n_generated - g_before
         e2e_s = max_over_ranks(t1 - t0)
-        e2e = {"value": sum_over_ranks(e2e_tok) / e2e_s, "unit": "tokens/s", "h2d_bytes_per_step": 0,
-               "d2h_bytes_per_step": 4 * (k + 2),
-               "note": "ocrdec_step_host per step: graph launch, D2H of committed tokens + count into "
-                       + ("pinned" if pinned is not None else "pageable") + " host memory, stream sync; "
-                       "the step has no per-step host input (state lives on the device)",
-               "step_latency_ms": {"mean": 1000 * float(np.mean(lat)), "p50": 1000 * float(np.percentile(lat, 50)),
-                                   "p99": 1000 * float(np.percentile(lat, 99)), "rank": rank}}
+        h2d_req = inp.visual.nbytes + inp.prompt.nbytes
+        d2h_req = 4 + nst / n_req * 4 * (k + 2)
+        e2e = {"value": sum_over_ranks(tot) / e2e_s, "unit": "tokens/s",
+               "h2d_bytes_per_step": h2d_req / (nst / n_req), "d2h_bytes_per_step": d2h_req / (nst / n_req),
+               "h2d_bytes_per_request": h2d_req, "d2h_bytes_per_request": d2h_req,
+               "requests": n_req, "tokens_per_request": tot / n_req, "steps_per_request": nst / n_req,
+               "prefill_ms": 1000 * pf / n_req, "request_ms": 1000 * (t1 - t0) / n_req,
+               "note": f"whole requests through the C ABI, wall clock: H2D of the page's {wl.n_visual} visual "
+                       f"rows (float32) and {wl.n_prompt} prompt tokens from "
+                       + ("pinned" if pinned else "pageable") + " host memory, ocrdec_prefill, then "
+                       "ocrdec_step_host until n_generate tokens (each step copies its committed tokens and "
+                       "count back and synchronises); per-step bytes are the request's bytes over its steps"}
 
     # ---- CPU baseline (rank 0, N = 1) ----
     cpu = None
@@ -456,36 +528,48 @@ def main():
             cpu["variants"] = oracle_variants(dims, k, bits)
 
     if rank == 0:
+        moe_traffic = profiled_traffic("moe_ffn_full_spec_k3.md")
         line = {
             "metric": "accepted tokens/sec (speculative decode step, batch 1)",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "full_spec", "k": k, "batch": 1, "context": f"{wl.n_visual} visual + {wl.n_prompt} prompt",
+            "config": {"workload": args.workload, "k": k, "batch": 1,
+                       "context": f"{wl.n_visual} visual + {wl.n_prompt} prompt", "n_generate": wl.n_generate,
+                       "timed_tokens": [int(st0.n_generated), int(st1.n_generated)],
+                       "timed_kv_mean": kv_mid,
                        "model": "12L d1280 64+2 experts top6 V129280 + FastMTP block", "parallelism": f"replicas x{world}",
                        "l2": "inputs larger than L2 (each step streams ~3.5 GB of weights, L2 is 126 MB)",
                        "acceptance_model": list(tab.p), "graph": True},
             "tau": tau, "acceptance": metrics.acceptance_rate(tau, k) if k else None,
             "lossless_vs_k0": lossless,
-            "k0": {"tokens_per_s": k0_tokens / (k0_ms / 1000.0), "ms_per_step": k0_ms / max(1, n0_steps - args.warmup)},
-            "speedup_vs_k0": value / world / (k0_tokens / (k0_ms / 1000.0)),
-            "step_roofline": {"union_bytes": union_b, "dependency_aware_bytes": dep_b,
-                              "touched_routed_experts_per_layer": U,
-                              "union_GBps": union_b / (step_ms / 1000) / 1e9,
-                              "frac_of_8TBps": union_b / (step_ms / 1000) / 8e12,
-                              "frac_of_measured_peak": union_b / (step_ms / 1000) / 1e9 / peak_gbs,
-                              "dependency_aware_frac_of_measured_peak": dep_b / (step_ms / 1000) / 1e9 / peak_gbs},
-            "roofline": {"kernel": "lm_head_argmax (final RMSNorm + 129,280 x 1280 GEMV + argmax, k+1 rows)",
-                         "bound": "hbm", "achieved": lm_gbs, "peak": peak_gbs, "unit": "GB/s",
-                         "frac": lm_gbs / peak_gbs, "traffic": lm_traffic, "peak_source": peak_src,
-                         "launch_ms": lm_ms, "bytes_per_launch": lm_bytes,
-                         "timing": "same kernel instantiation as in the verify pass, launched through "
-                                   "ocrdec_op_lm_argmax: 10 launches back to back in one CUDA graph (each streams "
-                                   "331 MB > L2), CUDA events on the launching stream, mean of 5 replays; each "
-                                   "launch includes the op's 64-byte scratch memset",
-                         "traffic_source": "profiles/lm_head_argmax_r4.md (ncu dram__bytes_read.sum + "
-                                           "dram__bytes_write.sum, one launch; null if the kernel sources changed "
-                                           "since)"},
+            "k0": {"tokens_per_s": k0_tps, "ms_per_step": k0_ms / max(1, n0)},
+            "speedup_vs_k0": value / world / k0_tps,
+            "roofline": {"kernel": "MoE FFN of one layer (routing in every CTA, shared + touched routed experts "
+                                   "gate/up and down, combine)",
+                         "bound": "hbm", "achieved": moe_gbs, "peak": peak_gbs, "unit": "GB/s",
+                         "frac": moe_gbs / peak_gbs, "traffic": moe_traffic, "peak_source": peak_src,
+                         "launch_ms": moe_ms, "bytes_per_launch": moe_bytes,
+                         "touched_routed_experts": U_moe,
+                         "timing": f"ocrdec_replay_moe_ffn over the {n_moe} MoE layers on the last k+1-row verify "
+                                   "pass's routing, captured in one CUDA graph (each layer's expert weights once, "
+                                   "~1 GB > L2), CUDA events on the launching stream around each replay, mean of 5 "
+                                   "replays divided by the layers; bytes = (touched routed + shared experts) x "
+                                   "3 x 1280 x 896 x 2 B + the rows' residual read and write",
+                         "lm_head": {"kernel": "final RMSNorm + 129,280 x 1280 LM head GEMV + argmax, k+1 rows "
+                                               "(ocrdec_op_lm_argmax, the verify head's GEMV and merge without the "
+                                               "acceptance epilogue)",
+                                     "achieved": lm_gbs, "frac": lm_gbs / peak_gbs, "launch_ms": lm_ms,
+                                     "bytes_per_launch": lm_bytes,
+                                     "traffic": profiled_traffic("lm_head_argmax_r4.md")},
+                         "step": {"union_bytes": union_b, "dependency_aware_bytes": dep_b,
+                                  "touched_routed_experts_per_layer": U, "tau": tau,
+                                  "k0_tokens_per_s": k0_tps, "ms_per_step": step_ms,
+                                  "union_GBps": union_b / (step_ms / 1000) / 1e9,
+                                  "union_frac": union_b / (step_ms / 1000) / 1e9 / peak_gbs,
+                                  "union_frac_of_8TBps": union_b / (step_ms / 1000) / 8e12,
+                                  "dependency_aware_frac": dep_b / (step_ms / 1000) / 1e9 / peak_gbs,
+                                  "target_union_frac": 0.60}},
             "timeline": timeline,
             "gpu_launches": kernels * args.steps,
             "kernels_per_step": kernels,
@@ -497,6 +581,9 @@ def main():
     dec.close()
     if world > 1:
         torch.distributed.destroy_process_group()
+    if not lossless:
+        print("bench: the speculative output differs from the k = 0 output", file=sys.stderr)
+        return 3
     return 0
 
 

@@ -262,6 +262,19 @@ OCRDEC_API int ocrdec_set_trace(ocrdec_ctx* ctx, int enable, ocrdec_stream strea
 OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_records, int32_t* n,
                                  ocrdec_stream stream);
 
+/* Timing hook (diagnostics, not part of the decode path): enqueues again the
+ * MoE FFN sub-layer - routing, shared and routed experts, combine - of
+ * verifier layers first_layer .. first_layer + n_layers - 1, with the launches
+ * of a (batch, k) verify pass, on the pass rows and router partials the last
+ * verifier pass (which must have been a (batch, k) pass) left in the
+ * workspace, so that the MoE kernels can be timed alone (CUDA events, graph
+ * capture) on their real routing.  The workspace's residual rows are updated in place: call it
+ * only between steps; the next step recomputes everything it reads.  The
+ * routed experts touched are added to the ocrdec_get_counters counters.
+ * first_layer must be a MoE layer (>= n_dense_first). */
+OCRDEC_API int ocrdec_replay_moe_ffn(ocrdec_ctx* ctx, int batch, int k, int first_layer, int n_layers,
+                                     ocrdec_stream stream);
+
 /* Parity tap for the draft: when set, recursion j (1-based) of every draft
  * also writes its LM-head logits to dev_logits[j-1][slot][V] (float32,
  * max_k * max_batch * V entries).  NULL switches it off. */

@@ -993,6 +993,21 @@ int ocrdec_read_trace(ocrdec_ctx* c, void* host_records, int max_records, int32_
   return OCRDEC_OK;
 }
 
+int ocrdec_replay_moe_ffn(ocrdec_ctx* c, int batch, int k, int first_layer, int n_layers, ocrdec_stream stream) {
+  int st = check_ready(c);
+  if (st) return st;
+  if ((st = check_bk(c, batch, k))) return st;
+  const ocrdec_config& m = c->cfg;
+  if (first_layer < m.n_dense_first || n_layers < 1 || first_layer + n_layers > m.n_layers) return OCRDEC_EINVAL;
+  const LaunchCfg lc = c->lc(reinterpret_cast<cudaStream_t>(stream));
+  // the same launches (row bound batch * (k + 1)) as the verify pass of a step
+  for (int l = first_layer; l < first_layer + n_layers; ++l) {
+    st = moe_ffn(c, lc, batch * (k + 1), c->layers[l], true);
+    if (st) return st;
+  }
+  return OCRDEC_OK;
+}
+
 int ocrdec_set_draft_taps(ocrdec_ctx* c, float* logits) {
   if (!c) return OCRDEC_EINVAL;
   c->dbg_draft_logits = logits;

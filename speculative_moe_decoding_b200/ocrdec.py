@@ -68,6 +68,7 @@ ocrdec_step_kernel_count = _sig("ocrdec_step_kernel_count", _i32, _vp, _i32, _i3
 ocrdec_set_debug_taps = _sig("ocrdec_set_debug_taps", _i32, _vp, _vp, _vp)
 ocrdec_set_draft_taps = _sig("ocrdec_set_draft_taps", _i32, _vp, _vp)
 ocrdec_set_trace = _sig("ocrdec_set_trace", _i32, _vp, _i32, _vp)
+ocrdec_replay_moe_ffn = _sig("ocrdec_replay_moe_ffn", _i32, _vp, _i32, _i32, _i32, _i32, _vp)
 ocrdec_read_trace = _sig("ocrdec_read_trace", _i32, _vp, _vp, _i32, ctypes.POINTER(_i32), _vp)
 
 TRACE_DTYPE = np.dtype([("t0", "<u8"), ("d1", "<u4"), ("d2", "<u4"), ("dt", "<u4"), ("tag", "<u2"),
@@ -267,6 +268,12 @@ class Decoder:
         check(ocrdec_read_trace(self.ctx, buf.ctypes.data, max_records, ctypes.byref(n), _stream(stream)),
               "ocrdec_read_trace")
         return buf[:min(n.value, max_records)]
+
+    def replay_moe_ffn(self, batch: int, k: int, first_layer: int, n_layers: int, stream=None):
+        """Timing hook: the MoE FFN kernels of verifier layers first_layer.. again, on the last
+        (batch, k) pass's rows and routing."""
+        check(ocrdec_replay_moe_ffn(self.ctx, batch, k, first_layer, n_layers, _stream(stream)),
+              "ocrdec_replay_moe_ffn")
 
     def set_draft_taps(self, logits=None):
         self._dtaps = logits

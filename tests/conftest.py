@@ -25,3 +25,12 @@ def tiny_inputs():
     from speculative_moe_decoding_b200 import synth
     w = synth.WORKLOADS["tiny"]
     return synth.make_inputs(synth.TINY, w.input_seed, w.n_visual, w.n_prompt)
+
+
+@pytest.fixture(scope="session")
+def full_bits():
+    """bf16 weight bits of the full-size model (the benchmark's seed), made once
+    per session and shared by the full-size GPU tests."""
+    from speculative_moe_decoding_b200 import synth
+    bits, _ = synth.make_weights(synth.FULL, synth.WORKLOADS["full_spec"].weight_seed)
+    return bits

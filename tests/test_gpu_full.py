@@ -20,12 +20,6 @@ LOGIT_ABS = 5e-2
 MARGIN = 0.1
 
 
-@pytest.fixture(scope="module")
-def full_bits():
-    bits, _ = synth.make_weights(synth.FULL, synth.WORKLOADS["full_spec"].weight_seed)
-    return bits
-
-
 def test_full_model_matches_oracle(full_bits):
     import torch
     m = synth.FULL
