@@ -102,6 +102,8 @@ bool config_ok(const ocrdec_config* c) {
   if (c->n_dense_first < 0 || c->n_dense_first > c->n_layers) return false;
   if (c->n_dense_first > 0 && (c->dense_ffn <= 0 || c->dense_ffn % kChunk)) return false;
   if (c->n_shared < 0 || c->shared_ffn != c->expert_ffn) return false;
+  // MoE layers: the down projection's rows of one item are copied whole (<= 1024 columns)
+  if (c->n_dense_first < c->n_layers && c->expert_ffn > 1024) return false;
   if (c->top_k > c->n_experts || c->top_k > kMaxTopK || c->n_experts > kMaxExperts || c->n_shared > kMaxShared)
     return false;
   if (c->max_k < 0 || c->max_k > 3) return false;
@@ -117,7 +119,7 @@ bool config_ok(const ocrdec_config* c) {
 size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
-  size_t status, counters, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp,
+  size_t status, counters, moe_ctr, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp,
       topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, rpart, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
       am_part, gtok, props,
       committed, ncommitted, hpend, total;
@@ -136,6 +138,7 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   auto take = [&](size_t bytes) { size_t at = o; o = align_up(o + bytes); return at; };
   L.status = take(256 + sizeof(TraceRec) * kTraceCap);  // status word + timeline trace
   L.counters = take(sizeof(int) * (16 + 2 * kWorkSlots + kRmax * kAttnSplit));
+  L.moe_ctr = take(sizeof(int) * kMoeCtrInts);
   L.tile_ctr = take(sizeof(int) * kSplitMaxTiles);
   L.slots = take(sizeof(SlotState) * B);
   L.rows = take(sizeof(PassRows));
@@ -202,6 +205,8 @@ cudaError_t prepare_kernels_now() {
   if (e == cudaSuccess) e = max_carveout(accept_kernel);
   if (e == cudaSuccess) e = max_carveout(force_kernel);
   if (e == cudaSuccess) e = max_carveout(prefill_finish_kernel);
+  if (e != cudaSuccess) return e;
+  e = moe_prepare();
   if (e != cudaSuccess) return e;
   return gemv_prepare();
 }
@@ -393,50 +398,32 @@ int dense_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, float* x, const bf16
 
 int moe_ffn(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const LayerW& w, bool count) {
   const ocrdec_config& m = c->cfg;
-  PassRows* rows = c->rows();
-  float* x = c->at<float>(c->L.x);
-  const int nslot = m.top_k + m.n_shared;
-
-  auto expert_launch = [&](const Mat& routed, const Mat& shared, int pair_half, int tag) {
-    GemvLaunch g = dense_launch(c, routed, pair_half, &rows->n, 0, rmax, tag);
-    g.s.kparts = 1;
-    g.tm_sh = shared.map;
-    g.s.n_experts = m.n_experts;
-    g.s.top_k = m.top_k;
-    g.s.n_shared = m.n_shared;
-    g.s.mats = c->at<int>(c->L.mats);
-    g.s.n_mats = c->at<int>(c->L.n_mats);
-    g.s.counts = c->at<int>(c->L.counts);
-    g.s.offsets = c->at<int>(c->L.offsets);
-    g.s.rowlist = c->at<int>(c->L.rowlist);
-    return g;
-  };
-
-  // gate/up: every CTA routes the pass from the attention kernel's router
-  // partials (CTA 0 stores the tables, ids and gates)
-  GemvLaunch gu = expert_launch(w.exp_gu, w.sh_gu, m.expert_ffn, kTagExpGU);
-  gu.s.rpart = c->at<float>(c->L.rpart);
-  gu.s.rms_eps = m.rms_eps;
-  gu.s.ids = c->at<int>(c->L.topk_ids);
-  gu.s.gates = c->at<float>(c->L.topk_gates);
-  gu.s.touched = count ? c->misc() : nullptr;
-  gu.src = SrcKind::Norm;
-  gu.norm = SrcNorm::Params{x, m.d_model, nullptr, w.ffn_norm, m.rms_eps};
-  gu.epi = EpiKind::SwiGLU;
-  gu.swiglu = EpiSwiGLU::Params{c->at<bf16>(c->L.hbuf), c->at<bf16>(c->L.hbuf_lo), m.expert_ffn, nslot};
-  CK(c->gemv(gu, lc));
-
-  GemvLaunch dn = expert_launch(w.exp_down, w.sh_down, 0, kTagExpDown);
-  // the rows of an expert item are copied once per item when they are short
-  dn.src = m.expert_ffn <= SrcBf16Item::kMaxK ? SrcKind::Bf16Item : SrcKind::Bf16;
-  dn.bf = SrcBf16::Params{c->at<bf16>(c->L.hbuf), c->at<bf16>(c->L.hbuf_lo), m.expert_ffn, nslot, nullptr};
-  dn.epi = EpiKind::Store;
-  dn.store = EpiStore<false>::Params{c->at<float>(c->L.ybuf), m.d_model, nslot, nullptr};
-  CK(c->gemv(dn, lc));
-
-  CombineParams cp{x, c->at<float>(c->L.ybuf), c->at<float>(c->L.topk_gates), &rows->n, m.d_model, m.top_k,
-                   m.n_shared, c->status()};
-  CK(launch_ex(combine_kernel, dim3((kRmax * m.d_model + 255) / 256), dim3(256), 0, lc, cp));
+  // routing, shared + routed experts and the combine: one persistent kernel
+  MoeLaunch g;
+  g.tm_gu = w.exp_gu.map;
+  g.tm_sgu = w.sh_gu.map;
+  g.tm_dn = w.exp_down.map;
+  g.tm_sdn = w.sh_down.map;
+  MoeParams& p = g.p;
+  p.d = m.d_model;
+  p.f = m.expert_ffn;
+  p.E = m.n_experts;
+  p.S = m.n_shared;
+  p.top_k = m.top_k;
+  p.tiles_gu = m.expert_ffn / kBoxRows;
+  p.tiles_dn = m.d_model / kTile;
+  p.eps = m.rms_eps;
+  p.x = c->at<float>(c->L.x);
+  p.nrows = &c->rows()->n;
+  p.gain = w.ffn_norm;
+  p.rpart = c->at<float>(c->L.rpart);
+  p.h = c->at<bf16>(c->L.hbuf);
+  p.h_lo = c->at<bf16>(c->L.hbuf_lo);
+  p.y = c->at<float>(c->L.ybuf);
+  p.ctr = c->at<int>(c->L.moe_ctr);
+  p.touched = count ? c->misc() : nullptr;
+  p.status = c->status();
+  CK(launch_moe(g, rmax, lc));
   return OCRDEC_OK;
 }
 
@@ -922,6 +909,7 @@ int ocrdec_clear_status(ocrdec_ctx* c, ocrdec_stream stream) {
   CK(cudaMemsetAsync(c->am_counter(0), 0, 8 * sizeof(int), s));
   CK(cudaMemsetAsync(c->at<int>(c->L.counters) + 16, 0, (2 * kWorkSlots + kRmax * kAttnSplit) * sizeof(int), s));
   CK(cudaMemsetAsync(c->at<int>(c->L.tile_ctr), 0, kSplitMaxTiles * sizeof(int), s));
+  CK(cudaMemsetAsync(c->at<int>(c->L.moe_ctr), 0, kMoeCtrInts * sizeof(int), s));
   return OCRDEC_OK;
 }
 

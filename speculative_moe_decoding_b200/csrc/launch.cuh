@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include "fused_epi.cuh"
+#include "moe.cuh"
 
 namespace ocrdec {
 
@@ -90,6 +91,15 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc);
 // largest size any launch uses (call outside stream capture, once per device).
 cudaError_t gemv_prepare();
 constexpr int kGemvMaxK = 2048;  // largest K of a normalised (shared-memory) source
+
+// One launch of the MoE FFN kernel (moe.cuh): routed / shared gate-up and
+// down tensor maps and the parameters.
+struct MoeLaunch {
+  CUtensorMap tm_gu, tm_sgu, tm_dn, tm_sdn;
+  MoeParams p{};
+};
+cudaError_t launch_moe(const MoeLaunch& g, int rows_bound, const LaunchCfg& lc);
+cudaError_t moe_prepare();
 constexpr int kWorkSlots = 4;   // GEMV work-counter pairs cycled by a decoder context
 
 
