@@ -40,13 +40,13 @@ cudaError_t launch_rg(const MoeLaunch& g, const LaunchCfg& lc) {
   p.nst = nst;
   const size_t smem = moe_smem_bytes(p.d, p.f, RG, nst);
   int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe_kernel<RG>, kGemvThreads, smem) != cudaSuccess ||
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe_kernel<RG>, kMoeThreads, smem) != cudaSuccess ||
       per_sm < 1)
     return cudaErrorInvalidConfiguration;
   // one CTA per SM: every CTA of the grid is resident at once (the combine
   // waits until all CTAs have read the residual)
   const int grid = lc.num_sms;
-  return launch_ex(moe_kernel<RG>, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_gu, g.tm_sgu, g.tm_dn, g.tm_sdn, p);
+  return launch_ex(moe_kernel<RG>, dim3(grid), dim3(kMoeThreads), smem, lc, g.tm_gu, g.tm_sgu, g.tm_dn, g.tm_sdn, p);
 }
 
 }  // namespace

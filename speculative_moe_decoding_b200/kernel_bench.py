@@ -2,6 +2,14 @@
 
     python -m speculative_moe_decoding_b200.kernel_bench --op lm_argmax --rows 4
     python -m speculative_moe_decoding_b200.kernel_bench --op norm_gemv --n 64 --k 1280 --rows 4
+    python -m speculative_moe_decoding_b200.kernel_bench --op moe --rows 4
+
+--op moe builds a two-layer decoder whose second layer is the full-size MoE
+layer (d = 1280, 64 routed + 2 shared experts of ffn 896, top-6; vocabulary
+4,096 to keep the model near 0.6 GB), decodes a few k = rows - 1 steps and then
+times that layer's MoE FFN alone (ocrdec_replay_moe_ffn on the last pass's
+routing).  With --eager the launches go straight to the stream (for ncu: the
+layer's launches are the 4th and later of the MoE kernel).
 
 Weights are random bf16 on the device (values do not matter for timing).  L2 is
 flushed (a 256 MB write) before every timed launch; times are CUDA events on the
@@ -20,7 +28,8 @@ from . import build
 
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--op", choices=["lm_argmax", "norm_gemv"], default="lm_argmax")
+    ap.add_argument("--op", choices=["lm_argmax", "norm_gemv", "moe"], default="lm_argmax")
+    ap.add_argument("--eager", action="store_true", help="moe: launch without a graph (ncu)")
     ap.add_argument("--n", type=int, default=129280)
     ap.add_argument("--k", type=int, default=1280)
     ap.add_argument("--rows", type=int, default=4)
@@ -29,6 +38,8 @@ def main():
     ap.add_argument("--no-flush", action="store_true")
     a = ap.parse_args()
     build.build()
+    if a.op == "moe":
+        return moe(a)
     from . import ocrdec
     torch.manual_seed(0)
     W = (torch.randn(a.n, a.k, device="cuda") * 0.02).to(torch.bfloat16)
@@ -66,6 +77,60 @@ def main():
     nbytes = a.n * a.k * 2 + a.rows * a.k * 4
     print(json.dumps({"op": a.op, "n": a.n, "k": a.k, "rows": a.rows, "mean_us": ms * 1e3,
                       "min_us": min(times) * 1e3, "GBps": nbytes / (ms / 1e3) / 1e9}))
+
+
+def moe(a):
+    import numpy as np
+
+    from . import ocrdec, synth
+    m = synth.ModelDims(d_model=1280, n_layers=2, n_heads=10, head_dim=128, n_dense_first=1, n_experts=64,
+                        n_shared=2, top_k=6, expert_ffn=896, shared_ffn=896, dense_ffn=6848, draft_ffn=6848,
+                        vocab=4096)
+    bits, _ = synth.make_weights(m, 1)
+    names = [n for n, _ in synth.manifest(m)]
+    k = a.rows - 1
+    dec = ocrdec.Decoder(m.as_dict(), bits, names, max_k=3, max_batch=1, kv_capacity=256)
+    inp = synth.make_inputs(m, 101, 4, 4)
+    dec.prefill(0, torch.from_numpy(inp.visual).cuda(), torch.from_numpy(inp.prompt).cuda())
+    for _ in range(2):
+        dec.step(1, k)  # the last one leaves a k+1-row pass's rows and router partials
+    torch.cuda.synchronize()
+    assert dec.status() == 0
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream()
+    dec.reset_counters()
+    launch = lambda: dec.replay_moe_ffn(1, k, 1, 1)
+    if a.eager:
+        for i in range(3):
+            flush.fill_(i & 0xFF)
+            launch()
+        torch.cuda.synchronize()
+        print(json.dumps({"op": "moe", "eager_launches": 3, "status": dec.status()}))
+        return 0
+    launch()
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        launch()
+    times = []
+    for i in range(a.warmup + a.iters):
+        flush.fill_(i & 0xFF)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(s)
+        graph.replay()
+        e1.record(s)
+        torch.cuda.synchronize()
+        if i >= a.warmup:
+            times.append(e0.elapsed_time(e1))
+    touched, passes = dec.counters()
+    U = touched / max(1, passes)
+    ms = float(np.mean(times))
+    nbytes = (U + m.n_shared) * 3 * m.d_model * m.expert_ffn * 2 + 2 * a.rows * m.d_model * 4
+    print(json.dumps({"op": "moe", "rows": a.rows, "touched_routed": U, "mean_us": ms * 1e3,
+                      "min_us": min(times) * 1e3, "bytes": nbytes, "GBps": nbytes / (ms / 1e3) / 1e9,
+                      "status": dec.status()}))
+    dec.close()
+    return 0
 
 
 if __name__ == "__main__":
