@@ -247,17 +247,16 @@ OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* 
  * kernels appends one 24-byte record {uint64 t0_ns (%globaltimer, when the CTA
  * passed its dependency wait), uint32 ns to the end of phase 1, phase 2 and
  * phase 3 (= CTA end), uint16 kernel tag, uint16 SM id} to a device buffer of
- * 524,288 records; enabling clears it.  GEMV phases: activation prologue
- * (the expert gate/up routes the pass first, inside it), main loop,
- * epilogue/finish; attention: first K/V chunk landed, its softmax done, end
- * (after the cluster merge, the output projection and, in MoE layers, the
- * router partials).  ocrdec_read_trace copies
- * up to max_records records to host memory and sets *n to the number recorded
- * (synchronises `stream`).  Tags: 1 QKV, 4 expert gate/up (with the
- * routing), 5 expert down, 6 dense gate/up, 7 dense down, 8 verify LM head +
- * acceptance, 9 draft LM head, 10 draft input fc, 40 attention with the
- * output projection (41 for cluster rank 0), 42 verify setup, 43 draft setup,
- * 44 MoE combine. */
+ * 524,288 records; enabling clears it.  GEMV phases: activation prologue,
+ * main loop, epilogue/finish; MoE FFN (recorded by its epilogue warp): dependency wait
+ * returned, routing tables first needed, end; attention: first K/V chunk
+ * landed, its softmax done, end (after the cluster merge, the output
+ * projection and, in MoE layers, the router partials).  ocrdec_read_trace
+ * copies up to max_records records to host memory and sets *n to the number
+ * recorded (synchronises `stream`).  Tags: 1 QKV, 6 dense gate/up, 7 dense
+ * down, 8 verify LM head + acceptance, 9 draft LM head, 10 draft input fc,
+ * 11 MoE FFN (routing, experts, combine), 40 attention with the output
+ * projection (41 for cluster rank 0), 42 verify setup, 43 draft setup. */
 OCRDEC_API int ocrdec_set_trace(ocrdec_ctx* ctx, int enable, ocrdec_stream stream);
 OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_records, int32_t* n,
                                  ocrdec_stream stream);

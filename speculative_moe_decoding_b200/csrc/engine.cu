@@ -120,7 +120,7 @@ size_t align_up(size_t v) { return (v + 255) & ~(size_t)255; }
 
 struct Layout {
   size_t status, counters, moe_ctr, tile_ctr, slots, rows, hist, rope, split_part, kvk, kvv, dkvk, dkvv, x, xd, q, yp,
-      topk_ids, topk_gates, counts, offsets, rowlist, mats, n_mats, rpart, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
+      rpart, hbuf, hbuf_lo, ybuf, hdense, hdense_lo, fcin, fcin_lo,
       am_part, gtok, props,
       committed, ncommitted, hpend, total;
   int hist_ld, am_blocks;
@@ -154,13 +154,6 @@ Layout make_layout(const ocrdec_config& c, int am_blocks) {
   L.q = take(4 * R * d);
   L.yp = take(4 * H * kRmax * d);  // per-head output projections
   L.rpart = take(4 * R * kRouteParts * kRouteLd);
-  L.topk_ids = take(4 * R * K);
-  L.topk_gates = take(4 * R * K);
-  L.counts = take(4 * E);
-  L.offsets = take(4 * E);
-  L.rowlist = take(4 * R * K);
-  L.mats = take(4 * (E + S));
-  L.n_mats = take(4);
   L.hbuf = take(2 * R * nslot * f);
   L.hbuf_lo = take(2 * R * nslot * f);
   L.ybuf = take(4 * R * nslot * d);
@@ -195,7 +188,6 @@ cudaError_t prepare_kernels_now() {
                                        (int)attn_smem_bytes(kGemvMaxK, kAttnMaxDh, kMaxExperts));
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
   if (e == cudaSuccess) e = max_carveout(attention_kernel);
-  if (e == cudaSuccess) e = max_carveout(combine_kernel);
   if (e == cudaSuccess) e = max_carveout(verify_setup_kernel);
   if (e == cudaSuccess) e = max_carveout(prefill_setup_kernel);
   if (e == cudaSuccess)
@@ -318,7 +310,6 @@ GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* n
   GemvLaunch g;
   g.s.tag = tag;
   g.tm_w = m.map;
-  g.tm_sh = m.map;
   g.s.N = m.N;
   g.s.K = m.K;
   g.s.pair_half = pair_half;
@@ -1045,7 +1036,6 @@ int ocrdec_op_norm_gemv(const void* W, const float* x, const void* g, float eps,
   CK(cudaMemsetAsync(st, 0, part_off, s));  // status, counters, tile counters
   GemvLaunch gl;
   CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
-  gl.tm_sh = gl.tm_w;
   gl.s.N = N;
   gl.s.K = K;
   gl.s.rows_static = R;
@@ -1079,7 +1069,6 @@ int ocrdec_op_lm_argmax(const void* W, const float* x, const void* g, float eps,
   CK(cudaMemsetAsync(st, 0, 64, s));  // status, trace header (off), counter
   GemvLaunch gl;
   CK(encode_weight_map(W, K, N, 1, &gl.tm_w));
-  gl.tm_sh = gl.tm_w;
   gl.s.N = N;
   gl.s.K = K;
   gl.s.rows_static = R;

@@ -25,12 +25,9 @@
 // column depends on its own B column only.  That is what makes the
 // speculative path bit-identical to k = 0.
 //
-// Work items are (matrix, 32-row tile) pairs claimed by CTAs from a per-launch
-// counter.  Dense mode has one matrix; expert mode walks the list of touched
-// experts (shared experts first) so only the experts routed in this pass are
-// streamed.  Its routing tables live in shared memory: copied from memory, or
-// (expert gate/up) computed in every CTA from the attention kernel's router
-// partials.
+// Work items are 32-row tiles (or K-parts of them) claimed by CTAs from a
+// per-launch counter.  (The MoE experts have their own persistent kernel,
+// moe.cuh, built from the same tiles.)
 #pragma once
 
 #include <cuda.h>
@@ -64,19 +61,12 @@ struct GemvShape {
   int ns;               // 256-column slices
   int pair_half;        // 0: tile = 32 consecutive rows; else 16 rows + the 16 rows pair_half below
   int tiles_per_mat;
-  // expert mode (mats != nullptr)
-  const int* mats;      // mats[m] = routed expert id (< n_experts) or n_experts + shared index
-  const int* n_mats;
-  int n_experts, top_k;
-  const int* counts;    // rows routed to each expert
-  const int* offsets;   // start of each expert's entries in rowlist
-  const int* rowlist;   // entries r | (slot << 8)
   // rows of the pass
   const int* nrows;     // device row count, or nullptr to use rows_static
   int rows_static;
   int* status;
-  int* counter;         // last-block counter (argmax / routing epilogues)
-  // split-K (dense mode): each tile's K-slices are cut into kparts contiguous
+  int* counter;         // last-block counter (argmax epilogues)
+  // split-K: each tile's K-slices are cut into kparts contiguous
   // parts handled by separate work items; the last part of a tile to finish
   // adds the parts' partial sums in part order and runs the epilogue
   int kparts;           // 1 = no split
@@ -86,17 +76,6 @@ struct GemvShape {
   // dynamic work distribution: work[0] = next item to claim, work[1] = CTAs
   // done claiming; the last CTA resets both (zero between launches)
   int* work;
-  // expert mode: the routing tables (mats, n_mats, counts, offsets, rowlist)
-  // are copied into shared memory before any item is claimed.  With rpart set
-  // (expert gate/up), every CTA instead routes the pass itself from the
-  // attention kernel's router partials, and CTA 0 stores the tables, ids and
-  // gates for the kernels that follow.
-  const float* rpart;   // [rows][kRouteParts][kRouteLd]
-  int n_shared;
-  float rms_eps;
-  int* ids;             // [rows][top_k]
-  float* gates;         // [rows][top_k]
-  int* touched;         // optional: [0] += routed experts touched, [1] += 1
 };
 
 // Rows of one item: entry q = pass row | (output slot << 8).
@@ -149,42 +128,6 @@ __device__ __forceinline__ int stage_row(bool paired, int w, int i) {
 __device__ __forceinline__ int matrix_row(int r0, int r1, int srow) {
   return srow < kBoxRows ? r0 + srow : r1 + (srow - kBoxRows);
 }
-
-__device__ __forceinline__ void mat_info(const GemvShape& s, const RouteTables& rt, int m, int R, int* coord_e,
-                                         bool* shared, RowSet* rs) {
-  if (!s.mats) {
-    *coord_e = 0;
-    *shared = false;
-    if (rs) {
-      rs->n = R;
-#pragma unroll
-      for (int i = 0; i < kRmax; ++i) rs->e[i] = i;
-    }
-    return;
-  }
-  int e = rt.mats[m];
-  if (e < s.n_experts) {
-    *coord_e = e;
-    *shared = false;
-    if (rs) {
-      int n = rt.counts[e], off = rt.offsets[e];
-      n = n > kRmax ? kRmax : n;
-      rs->n = n;
-#pragma unroll
-      for (int i = 0; i < kRmax; ++i) rs->e[i] = i < n ? rt.rowlist[off + i] : 0;
-    }
-  } else {
-    int sh = e - s.n_experts;
-    *coord_e = sh;
-    *shared = true;
-    if (rs) {
-      rs->n = R;
-#pragma unroll
-      for (int i = 0; i < kRmax; ++i) rs->e[i] = i | ((s.top_k + sh) << 8);
-    }
-  }
-}
-
 
 // 4-D tensor-map load of one box: 4 chunks of 64 columns x 16 rows of matrix
 // `mat`, starting at column chunk c4 and row `row`; shared layout
@@ -377,41 +320,6 @@ struct SrcBf16 {
   template <int RG>
   __device__ static uint32_t lo_offset(int) { return (uint32_t)(RG * kXStride); }
   __device__ static uint32_t b_slice(int) { return 0; }
-};
-
-// The same rows, copied once per work item instead of once per stage: at an
-// item's first stage the producer copies the item's whole rows (high and low
-// parts, K + 8 elements apart) into one of two item buffers, so a stage
-// carries only weights.  Consumers release a buffer (x_empty barrier) after
-// the item's last stage.  For short rows (K <= 1024): the expert down
-// projections, whose per-stage copies made the producer thread the bottleneck.
-struct SrcBf16Item {
-  typedef SrcBf16::Params Params;
-  static constexpr bool kSmem = false;
-  static constexpr bool kStaged = true;   // activations arrive with the stages (second arrival)
-  static constexpr bool kItemX = true;
-  static constexpr int kMaxK = 1024;
-  __host__ __device__ static constexpr size_t buf_bytes(int K, int RG) { return (size_t)2 * RG * (K + 8) * 2; }
-  __host__ __device__ static constexpr size_t smem_bytes(int K, int RG) { return 2 * buf_bytes(K, RG); }
-  struct Pre {};
-  __device__ static void pre_wait(const Params&, int, int, Pre&) {}
-  template <int RG>
-  __device__ static void prologue(const Params&, int, int, unsigned char*, float*, int, const Pre&) {}
-  __device__ static uint32_t b_base(const unsigned char* xbuf, const unsigned char*, int K, int row, int lane) {
-    return smem_u32(xbuf) + (uint32_t)(row * (K + 8) + ((lane >> 3) & 1) * 8) * 2;
-  }
-  template <int RG>
-  __device__ static uint32_t lo_offset(int K) { return (uint32_t)(RG * (K + 8) * 2); }
-  __device__ static uint32_t b_slice(int slc) { return (uint32_t)slc * kSlice * 2; }
-};
-
-template <class Src>
-struct ItemX {
-  static constexpr bool value = false;
-};
-template <>
-struct ItemX<SrcBf16Item> {
-  static constexpr bool value = true;
 };
 
 // ---------------------------------------------------------------------------
@@ -683,7 +591,7 @@ template <class Src, int RG>
 constexpr int stage_stride() {
   // weights, then (staged sources) the slice rows, high and low; 1 KB-aligned
   // for the swizzle
-  return Src::kStaged && !ItemX<Src>::value ? (kStageBytes + 2 * RG * kXStride + 1023) / 1024 * 1024 : kStageBytes;
+  return Src::kStaged ? (kStageBytes + 2 * RG * kXStride + 1023) / 1024 * 1024 : kStageBytes;
 }
 
 // Dynamic shared memory of one CTA: 1 KB alignment slack, the ring, the
@@ -693,107 +601,15 @@ constexpr size_t gemv_smem_bytes(int K) {
   return 1024 + (size_t)kStages * stage_stride<Src, RG>() + Src::smem_bytes(K, RG) + kRedFloats * 4;
 }
 
-// Epilogues whose expert-mode launches may route the pass themselves.
-template <class Epi>
-struct EpiRoutes {
-  static constexpr bool value = false;
-};
-template <>
-struct EpiRoutes<EpiSwiGLU> {
-  static constexpr bool value = true;
-};
-
-// Expert mode: the routing tables of the pass from memory (written by an
-// earlier kernel) into shared memory; all loads are independent.
-__device__ __forceinline__ void load_tables(const GemvShape& s, int R, int tid, RouteTables& rt) {
-  const int E = s.n_experts;
-  if (tid == 0) rt.n_mats = *s.n_mats;
-  for (int i = tid; i < s.n_shared + E; i += kConsumers) rt.mats[i] = s.mats[i];
-  for (int e = tid; e < E; e += kConsumers) {
-    rt.counts[e] = s.counts[e];
-    rt.offsets[e] = s.offsets[e];
-  }
-  for (int i = tid; i < R * s.top_k; i += kConsumers) rt.rowlist[i] = s.rowlist[i];
-}
-
-// Expert gate/up: every CTA routes the pass.  The router logits of row r are
-// assembled from the attention kernel's partials in a fixed order:
-//   logit[r][e] = (sum_k dot[r][k][e]) * rsqrt((sum_k ss[r][k]) / d + eps)
-// - the RMSNorm scale applied after the row-block dot products of W_r with
-// g * x (the gain g folded in by the attention kernel).  Every CTA computes
-// the same tables; CTA 0 also stores them, with the ids and gates, for the
-// down projection and the combine.
-static __device__ __forceinline__ void route_in_cta(const GemvShape& s, int R, int tid, RouteTables& rt) {
-  __shared__ float s_lg[kRmax * kMaxExperts];
-  __shared__ int s_ids[kRmax * kMaxTopK];
-  __shared__ float s_gates[kRmax * kMaxTopK];
-  const int E = s.n_experts;
-  for (int idx = tid; idx < R * E; idx += kConsumers) {
-    const int r = idx / E, e = idx - r * E;
-    const float* pr = s.rpart + (size_t)r * kRouteParts * kRouteLd;
-    float dk[kRouteParts], sk[kRouteParts];
-#pragma unroll
-    for (int k = 0; k < kRouteParts; ++k) {
-      dk[k] = __ldcg(pr + k * kRouteLd + e);
-      sk[k] = __ldcg(pr + k * kRouteLd + kMaxExperts);
-    }
-    float dot = 0.f, ss = 0.f;
-#pragma unroll
-    for (int k = 0; k < kRouteParts; ++k) {
-      dot = __fadd_rn(dot, dk[k]);
-      ss = __fadd_rn(ss, sk[k]);
-    }
-    s_lg[idx] = __fmul_rn(dot, rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)s.K), s.rms_eps)));
-  }
-  named_sync(1, kConsumers);
-  RouteParams p{};
-  p.logits = s_lg;
-  p.E = E;
-  p.top_k = s.top_k;
-  p.S = s.n_shared;
-  p.ids = s_ids;
-  p.gates = s_gates;
-  p.counts = rt.counts;
-  p.offsets = rt.offsets;
-  p.rowlist = rt.rowlist;
-  p.mats = rt.mats;
-  p.n_mats = &rt.n_mats;
-  route_rows(p, R, tid, kConsumers, ConsumerBarrier{});
-  named_sync(1, kConsumers);
-  if (blockIdx.x == 0) {
-    const int K = s.top_k;
-    if (tid == 0) {
-      *const_cast<int*>(s.n_mats) = rt.n_mats;
-      if (s.touched) {
-        atomicAdd(&s.touched[0], rt.n_mats - s.n_shared);
-        atomicAdd(&s.touched[1], 1);
-      }
-    }
-    for (int i = tid; i < s.n_shared + E; i += kConsumers) const_cast<int*>(s.mats)[i] = rt.mats[i];
-    for (int e = tid; e < E; e += kConsumers) {
-      const_cast<int*>(s.counts)[e] = rt.counts[e];
-      const_cast<int*>(s.offsets)[e] = rt.offsets[e];
-    }
-    for (int i = tid; i < R * K; i += kConsumers) {
-      const_cast<int*>(s.rowlist)[i] = rt.rowlist[i];
-      s.ids[i] = s_ids[i];
-      s.gates[i] = s_gates[i];
-    }
-  }
-}
-
 template <int RG, class Src, class Epi>
 __global__ void __launch_bounds__(kGemvThreads, 2)
-gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_sh,
-            const GemvShape s, const typename Src::Params sp, const typename Epi::Params ep) {
+gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvShape s, const typename Src::Params sp,
+            const typename Epi::Params ep) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages], x_empty[2];
-  __shared__ int s_tag[kStages];               // item of the stage's slice (set with its first slice), -1 = end
-  __shared__ int s_rs[kStages][kRmax + 1];     // expert mode: the item's row set (n, entries), with its first slice
+  __shared__ __align__(8) uint64_t full_bar[kStages], empty_bar[kStages];
+  __shared__ int s_tag[kStages];  // item of the stage's slice (set with its first slice), -1 = end
   __shared__ float red_pro[kRmax * kNW];
   __shared__ int s_abort;
-  __shared__ RouteTables s_rt;                 // expert mode: the pass's routing tables
-  __shared__ __align__(8) uint64_t tab_bar;    // consumers -> producer: s_rt is ready
 
   const int tid = threadIdx.x;
   const int warp = tid >> 5, lane = tid & 31;
@@ -810,9 +626,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       mbar_init(&full_bar[i], Src::kStaged ? 2 : 1);
       mbar_init(&empty_bar[i], kNW);
     }
-    mbar_init(&x_empty[0], kNW);
-    mbar_init(&x_empty[1], kNW);
-    mbar_init(&tab_bar, 1);
     fence_mbar_init();
   }
   __syncthreads();
@@ -822,132 +635,81 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
     if (lane != 0) return;
     uint32_t it = 0;
     int R = 0;
-    RowSet prs;  // rows of the current item (expert mode / staged sources)
-    int prs_m = -1;
     const uint64_t wpol = l2_evict_first_policy();  // weights are read once per pass
     auto stage_wait = [&](int st) {
       // a wait that gives up records OCRDEC_ETIMEOUT and proceeds: control flow
       // stays uniform so the block always terminates
       if (it >= kStages) mbar_wait(&empty_bar[st], ((it / kStages) & 1) ^ 1, s.status);
     };
-    auto rows_of = [&](int m) {
-      if (m != prs_m) {
-        int ce;
-        bool sh;
-        mat_info(s, s_rt, m, R, &ce, &sh, &prs);
-        prs_m = m;
-      }
-    };
     // Stage = two weight boxes (one arrival with their transaction bytes) and,
-    // for a staged bf16 source, the item's activation slice rows (a second
-    // arrival, declared only after the dependency wait).
-    auto issue_w = [&](int item, int m, int t, int slc, bool first) {
-      int ce;
-      bool sh;
-      mat_info(s, s_rt, m, 0, &ce, &sh, nullptr);
-      const CUtensorMap* map = sh ? &tm_sh : &tm_w;
+    // for a staged bf16 source, the pass rows' slice (a second arrival,
+    // declared only after the dependency wait).
+    auto issue_w = [&](int item, int t, int slc, bool first) {
       int r0, r1;
       tile_boxes(s, t, &r0, &r1);
       const int st = it % kStages;
       stage_wait(st);
       s_tag[st] = first ? item : -2;
-      if (first && s.mats) {
-        rows_of(m);
-        s_rs[st][0] = prs.n;
-#pragma unroll
-        for (int q = 0; q < kRmax; ++q) s_rs[st][1 + q] = prs.e[q];
-      }
       mbar_arrive_expect_tx(&full_bar[st], kStageBytes);
       unsigned char* dst = stages + st * kStride;
-      tma_load_box(dst, map, slc * (kSlice / kChunk), r0, ce, &full_bar[st], wpol);
-      tma_load_box(dst + kBoxBytes, map, slc * (kSlice / kChunk), r1, ce, &full_bar[st], wpol);
+      tma_load_box(dst, &tm_w, slc * (kSlice / kChunk), r0, 0, &full_bar[st], wpol);
+      tma_load_box(dst + kBoxBytes, &tm_w, slc * (kSlice / kChunk), r1, 0, &full_bar[st], wpol);
       ++it;
     };
-    uint32_t xitems = 0;  // item buffers handed out (item-resident sources)
-    auto issue_x = [&](uint32_t j, int m, int slc, bool first) {
+    auto issue_x = [&](uint32_t j, int slc) {
       if (!Src::kStaged) return;
-      rows_of(m);
       const int st = j % kStages;
-      if (ItemX<Src>::value) {
-        if (!first) {  // the item's rows came with its first stage
-          mbar_arrive(&full_bar[st]);
-          return;
-        }
-        const int xb = xitems & 1;
-        const uint32_t use = xitems >> 1;
-        if (use > 0) mbar_wait(&x_empty[xb], (use - 1) & 1, s.status);  // consumers are done with it
-        ++xitems;
-        const int nq = min(prs.n, RG);
-        const int ld = s.K + 8;
-        unsigned char* xb_dst = xsm + xb * SrcBf16Item::buf_bytes(s.K, RG);
-        mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(2 * nq * s.K * 2));
-        const SrcBf16::Params& bp = reinterpret_cast<const SrcBf16::Params&>(sp);
-#pragma unroll
-        for (int q = 0; q < RG; ++q)
-          if (q < nq) {
-            const long long off = SrcBf16::row_off(bp, prs.r(q), prs.slot(q));
-            bulk_g2s(xb_dst + (size_t)q * ld * 2, bp.x + off, s.K * 2, &full_bar[st]);
-            bulk_g2s(xb_dst + (size_t)(RG + q) * ld * 2, bp.x_lo + off, s.K * 2, &full_bar[st]);
-          }
-        return;
-      }
       unsigned char* dst = stages + st * kStride + kStageBytes;
       const int cols = min(kSlice, s.K - slc * kSlice);
-      const int nq = min(prs.n, RG);
+      const int nq = min(R, RG);
       mbar_arrive_expect_tx(&full_bar[st], (uint32_t)(2 * nq * cols * 2));
       const SrcBf16::Params& bp = reinterpret_cast<const SrcBf16::Params&>(sp);
 #pragma unroll
       for (int q = 0; q < RG; ++q)
         if (q < nq) {
-          const long long off = SrcBf16::row_off(bp, prs.r(q), prs.slot(q)) + slc * kSlice;
+          const long long off = SrcBf16::row_off(bp, q, 0) + slc * kSlice;
           bulk_g2s(dst + q * kXStride, bp.x + off, cols * 2, &full_bar[st]);
           bulk_g2s(dst + (RG + q) * kXStride, bp.x_lo + off, cols * 2, &full_bar[st]);
         }
     };
     // items are claimed from the launch's work counter, so faster SMs take more
-    int total = s.mats ? 0 : s.tiles_per_mat * s.kparts;
-    // dense weights do not depend on earlier kernels: the stages of the CTA's
-    // first item are requested before the dependency wait (one item only, so
-    // that CTAs resident early do not take the work of those still arriving)
-    int pre_sl[kStages];
-    bool pre_first[kStages];
-    int npre = 0;
+    const int total = s.tiles_per_mat * s.kparts;
     int item = -1, sl = 0, sl_end = 0;
     auto claim = [&]() {
       item = atomicAdd(&s.work[0], 1);
       if (item < total) {
-        ItemPos ip = item_pos(s, item);
+        const ItemPos ip = item_pos(s, item);
         sl = ip.sl0;
         sl_end = ip.sl1;
       }
     };
+    // the weights do not depend on earlier kernels: the stages of the CTA's
+    // first item are requested before the dependency wait (one item only, so
+    // that CTAs resident early do not take the work of those still arriving)
+    int pre_sl[kStages];
+    int npre = 0;
+    claim();
     bool claimed = false;  // item/sl hold a claimed item not yet fully issued
-    if (!s.mats) {
-      claim();
-      if (item < total) {
-        const ItemPos ip = item_pos(s, item);
-        while (sl < sl_end && it < (uint32_t)kStages) {
-          pre_first[npre] = sl == ip.sl0;
-          pre_sl[npre++] = sl;
-          issue_w(item, 0, ip.t, sl, sl == ip.sl0);
-          ++sl;
-        }
-        claimed = sl < sl_end;
+    if (item < total) {
+      const ItemPos ip = item_pos(s, item);
+      while (sl < sl_end && it < (uint32_t)kStages) {
+        pre_sl[npre++] = sl;
+        issue_w(item, ip.t, sl, sl == ip.sl0);
+        ++sl;
       }
+      claimed = sl < sl_end;
     }
     pdl_wait();
     const bool ok = !status_bad(s.status);
     if (ok) {
       R = min(pass_rows(s), RG);
-      for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, 0, pre_sl[j], pre_first[j]);
-      // expert mode: the item list is known once the consumers have the tables
-      if (s.mats) total = mbar_wait(&tab_bar, 0, s.status) ? s_rt.n_mats * s.tiles_per_mat : 0;
+      for (int j = 0; j < npre; ++j) issue_x((uint32_t)j, pre_sl[j]);
       if (!claimed) claim();
       while (item < total) {
         const ItemPos ip = item_pos(s, item);
         const uint32_t j = it;
-        issue_w(item, ip.m, ip.t, sl, sl == ip.sl0);
-        issue_x(j, ip.m, sl, sl == ip.sl0);
+        issue_w(item, ip.t, sl, sl == ip.sl0);
+        issue_x(j, sl);
         if (++sl == sl_end) claim();
       }
     } else if (Src::kStaged) {
@@ -986,10 +748,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   }
   named_sync(1, kConsumers);
   if (s_abort) {
-    if (s.mats && tid == 0) {  // no items
-      s_rt.n_mats = 0;
-      mbar_arrive(&tab_bar);
-    }
     // consume the producer's stages up to its end marker so it can finish
     uint32_t it = 0;
     while (true) {
@@ -1007,17 +765,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
 
   const int R = min(pass_rows(s), RG);
   __shared__ int s_last_part;
-  if (s.mats) {
-    if constexpr (EpiRoutes<Epi>::value) {
-      if (s.rpart) route_in_cta(s, R, tid, s_rt);
-      else load_tables(s, R, tid, s_rt);
-    } else {
-      load_tables(s, R, tid, s_rt);
-    }
-    named_sync(1, kConsumers);
-    if (tid == 0) mbar_arrive(&tab_bar);  // releases the tables to the producer
-  }
-
   epi_init<Epi>(tid);
   Src::template prologue<RG>(sp, s.K, R, xsm, red_pro, tid, pre);
   if (!Src::kSmem) named_sync(1, kConsumers);
@@ -1030,17 +777,20 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
   const int a_row = (lane & 7) + ((lane >> 3) & 1) * 8;
   const uint32_t a_off = (uint32_t)(g * kBoxBytes + kq * (kBoxRows * 128) + a_row * 128);
   const int a_sw = a_row & 7, a_hi = lane >> 4;
-  // epilogue mapping: lane L = 8 i + q takes local row i, row-set entry q
+  // epilogue mapping: lane L = 8 i + q takes local row i, pass row q
   const int ep_i = lane >> 3, ep_q = lane & 7;
   const int ep_srow = stage_row(paired, warp, ep_i);
-
-  uint32_t it = 0;
-  int nitem = 0;
+  // the pass rows: entry q = row q
   RowSet rs;
   rs.n = R;
 #pragma unroll
   for (int q = 0; q < kRmax; ++q) rs.e[q] = q;
+  // B rows of this lane: pass row (lane & 7); columns past RG reuse row q % RG
+  const int bq = (lane & 7) % RG;
+  const uint32_t b_lo = Src::template lo_offset<RG>(s.K);
 
+  uint32_t it = 0;
+  int nitem = 0;
   while (true) {
     const int st0 = it % kStages;
     mbar_wait(&full_bar[st0], (it / kStages) & 1, s.status);
@@ -1052,15 +802,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       break;
     }
     const ItemPos ip = item_pos(s, item);
-    if (s.mats) {
-      rs.n = s_rs[st0][0];
-#pragma unroll
-      for (int q = 0; q < kRmax; ++q) rs.e[q] = s_rs[st0][1 + q];
-    }
-    // B rows of this lane: row-set entry (lane & 7); columns past RG reuse row q % RG
-    const int bq = (lane & 7) % RG;
-    const int brow = Src::kStaged ? bq : rs.r_sel(bq);
-    const uint32_t b_lo = Src::template lo_offset<RG>(s.K);
     float d[4] = {0.f, 0.f, 0.f, 0.f};
     for (int sl = ip.sl0; sl < ip.sl1; ++sl, ++it) {
       const int st = it % kStages;
@@ -1068,8 +809,7 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       if (sl * (kSlice / kChunk) + kq < nchunks) {
         const unsigned char* stg = stages + st * kStride;
         const uint32_t a_base = smem_u32(stg) + a_off;
-        const unsigned char* xsrc = ItemX<Src>::value ? xsm + (nitem & 1) * SrcBf16Item::buf_bytes(s.K, RG) : xsm;
-        const uint32_t b_addr = Src::b_base(xsrc, stg + kStageBytes, s.K, brow, lane) + Src::b_slice(sl) +
+        const uint32_t b_addr = Src::b_base(xsm, stg + kStageBytes, s.K, bq, lane) + Src::b_slice(sl) +
                                 (uint32_t)kq * kChunk * 2;
 #pragma unroll
         for (int k16 = 0; k16 < kChunk / 16; ++k16) {
@@ -1084,7 +824,6 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CU
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty_bar[st]);
     }
-    if (ItemX<Src>::value && lane == 0) mbar_arrive(&x_empty[nitem & 1]);  // the item's rows are no longer read
     // quarter partials -> shared, then every output adds its quarters in order
     float* rb = red + (nitem & 1) * (4 * kTile * 8);
     ++nitem;

@@ -17,7 +17,7 @@ int gemv_kparts(const GemvShape& s, int target_items) {
   // at least four slices long and only matrices too short to give every SM a
   // tile are split.
   constexpr int kMinSlicesPerPart = 4;
-  if (s.mats || s.tiles_per_mat >= 64 || s.ns < 2 * kMinSlicesPerPart) return 1;
+  if (s.tiles_per_mat >= 64 || s.ns < 2 * kMinSlicesPerPart) return 1;
   int want = (target_items + s.tiles_per_mat - 1) / s.tiles_per_mat;
   want = std::min(want, (s.ns + kMinSlicesPerPart - 1) / kMinSlicesPerPart);
   const int spp = (s.ns + want - 1) / want;  // slices per part
@@ -132,7 +132,6 @@ cudaError_t gemv_prepare() {
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmaxAccept>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<true>>();
-  if (e == cudaSuccess) e = configure_rg<SrcBf16Item, EpiStore<false>>();
   return e;
 }
 
@@ -149,8 +148,8 @@ static cudaError_t launch_one(const GemvLaunch& g, const typename Src::Params& s
     per_sm = 1;
   const int slots = std::min(per_sm, 2) * lc.num_sms;
   int grid = g.grid > 0 ? std::min(g.grid, slots) : slots;
-  if (!g.s.mats) grid = std::min(grid, g.s.tiles_per_mat * g.s.kparts);
-  return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.tm_sh, g.s, sp, ep);
+  grid = std::min(grid, g.s.tiles_per_mat * g.s.kparts);
+  return launch_ex(kern, dim3(grid), dim3(kGemvThreads), smem, lc, g.tm_w, g.s, sp, ep);
 }
 
 template <class Src, class Epi>
@@ -166,7 +165,7 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
   if (g.s.K % kChunk || (g.s.pair_half && (g.s.pair_half % kBoxRows || g.s.N % (2 * g.s.pair_half))))
     return cudaErrorInvalidValue;
   if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
-  if (g.s.kparts > 1 && (g.s.mats || !g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;
+  if (g.s.kparts > 1 && (!g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;
   if (!g.s.work) return cudaErrorInvalidValue;
   if (g.src == SrcKind::Norm) {
     switch (g.epi) {
@@ -180,10 +179,6 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
       }
       default: return cudaErrorInvalidValue;
     }
-  }
-  if (g.src == SrcKind::Bf16Item) {
-    if (g.s.K > SrcBf16Item::kMaxK || g.epi != EpiKind::Store) return cudaErrorInvalidValue;
-    return launch_rg<SrcBf16Item, EpiStore<false>>(g, g.bf, g.store, lc);
   }
   switch (g.epi) {
     case EpiKind::Store: return launch_rg<SrcBf16, EpiStore<false>>(g, g.bf, g.store, lc);

@@ -52,13 +52,12 @@ cudaError_t launch_cluster_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-enum class SrcKind { Norm, Bf16, Bf16Item };
+enum class SrcKind { Norm, Bf16 };
 enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, ArgmaxAccept };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.
 struct GemvLaunch {
-  CUtensorMap tm_w;   // routed experts / dense matrix
-  CUtensorMap tm_sh;  // shared experts (expert mode); unused otherwise
+  CUtensorMap tm_w;   // the matrix
   GemvShape s{};
   SrcKind src = SrcKind::Norm;
   EpiKind epi = EpiKind::Store;

@@ -61,7 +61,7 @@ cudaError_t moe_prepare() {
 
 cudaError_t launch_moe(const MoeLaunch& g, const int rows_bound, const LaunchCfg& lc) {
   const MoeParams& p = g.p;
-  if (p.d % 128 || p.d > kGemvMaxK || p.f % kChunk || p.f > SrcBf16Item::kMaxK || p.f % kBoxRows) return cudaErrorInvalidValue;
+  if (p.d % 128 || p.d > kGemvMaxK || p.f % kChunk || p.f > 1024 || p.f % kBoxRows) return cudaErrorInvalidValue;
   if (p.tiles_gu != p.f / kBoxRows || p.tiles_dn != p.d / kTile || p.tiles_dn > kMoeMaxTilesDn) return cudaErrorInvalidValue;
   if (p.E > kMaxExperts || p.S > kMaxShared || p.top_k > kMaxTopK || !p.ctr) return cudaErrorInvalidValue;
   if (rows_bound <= 1) return launch_rg<1>(g, lc);

@@ -1,53 +1,10 @@
 // The stand-alone kernels of the decode step (launched by the engine only):
-// pass setup, combine, acceptance, forced proposals, RoPE table.
+// pass setup, acceptance, forced proposals, RoPE table.
 #pragma once
 
 #include "step_kernels.cuh"
 
 namespace ocrdec {
-
-// The residual rows, the gates and the row count were written at least two
-// kernels back (attention, the expert gate/up's CTA 0, the pass setup), so
-// they are read before the dependency wait; only the expert outputs y (the
-// down projection, the kernel just before) and the status are read after it,
-// together.
-__global__ void __launch_bounds__(256) combine_kernel(const CombineParams p) {
-  constexpr int kSlots = kMaxTopK + kMaxShared;
-  const int R = min(__ldcg(p.nrows), kRmax);
-  const int nslot = p.top_k + p.S;
-  const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  const bool mine = idx < R * p.d;
-  const int r = mine ? idx / p.d : 0, n = mine ? idx - r * p.d : 0;
-  float xv = 0.f, g[kMaxTopK];
-#pragma unroll
-  for (int s = 0; s < kMaxTopK; ++s) g[s] = 0.f;
-  if (mine) {
-    xv = __ldcg(p.x + idx);
-#pragma unroll
-    for (int s = 0; s < kMaxTopK; ++s)
-      if (s < p.top_k) g[s] = __ldcg(p.gates + r * p.top_k + s);
-  }
-  pdl_wait();
-  TraceMarks tm;
-  if (threadIdx.x == 0) tm.t0 = gtimer();  // trace: after the dependency wait
-  const bool bad = status_bad(p.status);
-  float y[kSlots];
-  const float* yr = p.y + (long long)r * nslot * p.d + n;
-#pragma unroll
-  for (int s = 0; s < kSlots; ++s) y[s] = mine && s < nslot ? yr[(long long)s * p.d] : 0.f;
-  if (bad) return;
-  pdl_trigger();
-  if (mine) {
-    float t = 0.f;  // routed slots in order, then the shared ones
-#pragma unroll
-    for (int s = 0; s < kSlots; ++s) {
-      if (s < p.top_k) t = __fmaf_rn(g[s < kMaxTopK ? s : 0], y[s], t);
-      else if (s < nslot) t = __fadd_rn(t, y[s]);
-    }
-    p.x[idx] = __fadd_rn(xv, t);
-  }
-  if (threadIdx.x == 0) trace_end(p.status, 44, tm);
-}
 
 __global__ void rope_table_kernel(float2* tab, int cap, int Dh, double theta) {
   int half = Dh / 2;

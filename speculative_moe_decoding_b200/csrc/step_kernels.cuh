@@ -1,7 +1,7 @@
-// Small kernels of the decode step: the MoE combine, pass setup (embedding
-// gather, row metadata, draft inputs), greedy acceptance with commit and
-// rollback, the benchmark's forced-acceptance override, and the RoPE table.
-// (Routing is in route.cuh.)
+// Small kernels of the decode step: pass setup (embedding gather, row
+// metadata, draft inputs), greedy acceptance with commit and rollback, the
+// benchmark's forced-acceptance override, and the RoPE table.  (Routing is in
+// route.cuh, the MoE FFN in moe.cuh.)
 #pragma once
 
 #include "common.cuh"
@@ -34,19 +34,6 @@ constexpr int kMaxK = 3;  // draft tokens per step
 
 struct BlockSync {
   __device__ void operator()() const { __syncthreads(); }
-};
-
-
-
-// x[r][n] += sum_s gate[r][s] * y[r][s][n] (routed, ascending expert id)
-//            + sum_sh y[r][top_k + sh][n]   (shared)
-struct CombineParams {
-  float* x;
-  const float* y;
-  const float* gates;
-  const int* nrows;
-  int d, top_k, S;
-  int* status;
 };
 
 

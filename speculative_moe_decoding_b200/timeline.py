@@ -13,10 +13,9 @@ from typing import Dict, List
 
 import numpy as np
 
-TAGS = {1: "qkv", 4: "routing+expert_gate_up", 5: "expert_down", 6: "dense_gate_up", 7: "dense_down",
-        8: "lm_head_verify+accept", 9: "lm_head_draft", 10: "draft_fc", 40: "attention+o_proj(+router partials)",
-        41: "attention (cluster rank 0)", 42: "verify_setup", 43: "draft_setup", 44: "moe_combine",
-        11: "moe_ffn (routing+experts+combine)"}
+TAGS = {1: "qkv", 6: "dense_gate_up", 7: "dense_down", 8: "lm_head_verify+accept", 9: "lm_head_draft",
+        10: "draft_fc", 11: "moe_ffn (routing+experts+combine)", 40: "attention+o_proj(+router partials)",
+        41: "attention (cluster rank 0)", 42: "verify_setup", 43: "draft_setup"}
 
 
 def launches(rec: np.ndarray) -> List[dict]:
