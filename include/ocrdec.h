@@ -274,6 +274,23 @@ OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_re
 OCRDEC_API int ocrdec_replay_moe_ffn(ocrdec_ctx* ctx, int batch, int k, int first_layer, int n_layers,
                                      ocrdec_stream stream);
 
+/* Variant not on the pages: a cheaper draft argmax.  Every draft recursion
+ * ends with a full-vocabulary argmax over the LM head (V x d bf16, 331 MB at
+ * the full size); this call makes the draft read an e4m3 copy instead (half
+ * the bytes), with the activations as e4m3 high and low parts and the logits
+ * scaled back per row.  Verification keeps the bf16 head and greedy
+ * acceptance, so the committed tokens stay exactly those of plain greedy
+ * decoding (model page: verification is greedy); only which proposals get
+ * accepted can change.
+ * dev_buf: caller-owned device memory of ocrdec_draft_head_fp8_bytes(cfg)
+ * bytes, 256-byte aligned, kept alive while the variant is on; the call fills
+ * it on `stream` (row n of the head scaled by 448 / max_k |W[n][k]|, rounded
+ * to nearest even; then the V float32 inverse scales).  NULL switches back to
+ * the bf16 head.  Requires the weights (OCRDEC_ESTATE otherwise) and d_model a
+ * multiple of 128; OCRDEC_EINVAL for a short or misaligned buffer. */
+OCRDEC_API size_t ocrdec_draft_head_fp8_bytes(const ocrdec_config* cfg);
+OCRDEC_API int ocrdec_set_draft_head_fp8(ocrdec_ctx* ctx, void* dev_buf, size_t bytes, ocrdec_stream stream);
+
 /* Parity tap for the draft: when set, recursion j (1-based) of every draft
  * also writes its LM-head logits to dev_logits[j-1][slot][V] (float32,
  * max_k * max_batch * V entries).  NULL switches it off. */

@@ -242,6 +242,10 @@ struct ocrdec_ctx {
   float* dbg_logits = nullptr;
   float* dbg_draft_logits = nullptr;
   CUtensorMap kv_map[4];  // verifier K, V; draft K, V (encoded when the workspace is bound)
+  // the draft's e4m3 copy of the LM head (variant; nullptr: the bf16 head)
+  const unsigned char* head8 = nullptr;
+  const float* head8_inv = nullptr;  // [V] inverse row scales
+  CUtensorMap head8_map;
 
   template <class T>
   T* at(size_t off) const { return reinterpret_cast<T*>(ws + off); }
@@ -441,14 +445,24 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
 // final norm + LM head + argmax.  row_src selects x rows (nullptr: rows 0..);
 // nrows / rows_static the row count; tokens to tok[r * tok_stride].
 int lm_head(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const float* x, const bf16* norm, const int* row_src,
-            const int* nrows, int rows_static, int* tok, int tok_stride, float* logits, int which_counter) {
+            const int* nrows, int rows_static, int* tok, int tok_stride, float* logits, int which_counter,
+            bool fp8 = false) {
   const ocrdec_config& m = c->cfg;
   GemvLaunch g = dense_launch(c, c->lm_head, 0, nrows, rows_static, rmax, kTagLMDraft);
   g.s.counter = c->am_counter(which_counter);
   g.src = SrcKind::Norm;
+  if (fp8) {
+    // the e4m3 head: K counted in byte pairs, logits scaled back per row
+    g.tm_w = c->head8_map;
+    g.s.K = m.d_model / 2;
+    gemv_plan(g.s);
+    g.s.kparts = 1;
+    g.src = SrcKind::Norm8;
+  }
   g.norm = SrcNorm::Params{x, m.d_model, row_src, norm, m.rms_eps};
   g.epi = EpiKind::Argmax;
-  g.argmax = EpiArgmax::Params{tok, tok_stride, logits, c->at<float2>(c->L.am_part), nullptr};
+  g.argmax = EpiArgmax::Params{tok, tok_stride, logits, c->at<float2>(c->L.am_part), nullptr,
+                               fp8 ? c->head8_inv : nullptr};
   g.grid = std::min(g.s.tiles_per_mat, c->L.am_blocks);
   CK(c->gemv(g, lc));
   return OCRDEC_OK;
@@ -485,7 +499,8 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
   st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down);
   if (st) return st;
   float* dl = c->dbg_draft_logits ? c->dbg_draft_logits + (size_t)(j - 1) * m.max_batch * m.vocab : nullptr;
-  return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, dl, 1);
+  return lm_head(c, lc, m.max_batch, xd, w.final_norm, rows->last_row, &rows->n_last, 0, tok, tok_stride, dl, 1,
+                 c->head8 != nullptr);
 }
 
 int enqueue_draft(ocrdec_ctx* c, const LaunchCfg& lc, int B, int k, int* props) {
@@ -984,6 +999,36 @@ int ocrdec_replay_moe_ffn(ocrdec_ctx* c, int batch, int k, int first_layer, int 
     st = moe_ffn(c, lc, batch * (k + 1), c->layers[l], true);
     if (st) return st;
   }
+  return OCRDEC_OK;
+}
+
+size_t ocrdec_draft_head_fp8_bytes(const ocrdec_config* cfg) {
+  if (!config_ok(cfg)) return 0;
+  return align_up((size_t)cfg->vocab * cfg->d_model) + (size_t)cfg->vocab * sizeof(float);
+}
+
+int ocrdec_set_draft_head_fp8(ocrdec_ctx* c, void* buf, size_t bytes, ocrdec_stream stream) {
+  if (!c) return OCRDEC_EINVAL;
+  if (!buf) {
+    c->head8 = nullptr;
+    c->head8_inv = nullptr;
+    c->drop_graphs();
+    return OCRDEC_OK;
+  }
+  if (!c->have_weights) return OCRDEC_ESTATE;
+  const ocrdec_config& m = c->cfg;
+  if ((reinterpret_cast<uintptr_t>(buf) & 255) || bytes < ocrdec_draft_head_fp8_bytes(&m)) return OCRDEC_EINVAL;
+  if (m.d_model % (2 * kChunk)) return OCRDEC_EINVAL;  // whole 128-byte rows of e4m3 pairs
+  unsigned char* w8 = static_cast<unsigned char*>(buf);
+  float* inv = reinterpret_cast<float*>(w8 + align_up((size_t)m.vocab * m.d_model));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  quantize_rows_e4m3_kernel<<<(m.vocab + 7) / 8, 256, 0, s>>>(c->lm_head.p, m.vocab, m.d_model, w8, inv);
+  CK(cudaGetLastError());
+  // the e4m3 matrix read as [V][d/2] byte pairs: the bf16 tiles' geometry
+  CK(encode_weight_map(w8, m.d_model / 2, m.vocab, 1, &c->head8_map));
+  c->head8 = w8;
+  c->head8_inv = inv;
+  c->drop_graphs();
   return OCRDEC_OK;
 }
 

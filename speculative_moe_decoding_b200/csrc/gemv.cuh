@@ -31,6 +31,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp8.h>
 
 #include "common.cuh"
 #include "route.cuh"
@@ -159,6 +160,36 @@ __device__ __forceinline__ void mma_bf16(float (&d)[4], const uint32_t (&a)[4], 
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
 }
 
+// d += A (16x32, row) * B (32x8, col); e4m3 in, float32 accumulate.  The
+// 32-byte k-step spans the same bytes as a bf16 m16n8k16 step, so the same
+// swizzled tiles and ldmatrix addresses feed it.
+__device__ __forceinline__ void mma_e4m3(float (&d)[4], const uint32_t (&a)[4], const uint32_t (&b)[2]) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.f32.e4m3.e4m3.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// float <-> e4m3 (round to nearest even, saturating to +-448).
+__device__ __forceinline__ uint32_t f2e4m3(float v) {
+  return (uint32_t)__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3);
+}
+__device__ __forceinline__ float e4m32f(uint32_t b) {
+  return __half2float(__half(__nv_cvt_fp8_to_halfraw((__nv_fp8_storage_t)b, __NV_E4M3)));
+}
+
+// Four floats as high and low e4m3 parts, bytes in k order.
+__device__ __forceinline__ void split_e4m3x4(const float (&f)[4], uint32_t& hi, uint32_t& lo) {
+  hi = lo = 0u;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint32_t h = f2e4m3(f[i]);
+    hi |= h << (8 * i);
+    lo |= f2e4m3(__fsub_rn(f[i], e4m32f(h))) << (8 * i);
+  }
+}
+
 // Four floats as high and low bfloat16 parts (high = bf16(f), low = bf16(f - high)).
 __device__ __forceinline__ void split_bf16x4(float f0, float f1, float f2, float f3, uint2& hi, uint2& lo) {
   const bf16 h0 = f2bf(f0), h1 = f2bf(f1), h2 = f2bf(f2), h3 = f2bf(f3);
@@ -193,6 +224,7 @@ struct SrcNorm {
   };
   static constexpr bool kSmem = true;    // activations live in shared memory (prologue)
   static constexpr bool kStaged = false; // activations are not part of the weight stages
+  static constexpr bool kFp8 = false;    // bf16 weights and activation parts
   static constexpr int kG = 2;           // float4 groups per thread per row: K <= 2048
   __host__ __device__ static constexpr size_t smem_bytes(int K, int RG) { return (size_t)2 * RG * (K + 8) * 2; }
 
@@ -306,6 +338,7 @@ struct SrcBf16 {
   };
   static constexpr bool kSmem = false;
   static constexpr bool kStaged = true;
+  static constexpr bool kFp8 = false;
   __host__ __device__ static constexpr size_t smem_bytes(int, int) { return 0; }
   struct Pre {};
   __device__ static void pre_wait(const Params&, int, int, Pre&) {}
@@ -320,6 +353,91 @@ struct SrcBf16 {
   template <int RG>
   __device__ static uint32_t lo_offset(int) { return (uint32_t)(RG * kXStride); }
   __device__ static uint32_t b_slice(int) { return 0; }
+};
+
+// The same normalised rows as e4m3 high and low parts, for e4m3 weights (the
+// draft's quantised LM head).  Layout and addressing are those of SrcNorm with
+// K counted in byte pairs: the kernel's K is half the number of columns, and
+// a row of K pairs holds 2K e4m3 values in column order.
+struct SrcNorm8 {
+  typedef SrcNorm::Params Params;
+  static constexpr bool kSmem = true;
+  static constexpr bool kStaged = false;
+  static constexpr bool kFp8 = true;
+  static constexpr int kG = 2;  // float4 groups per thread per row: 2K <= 2048
+  __host__ __device__ static constexpr size_t smem_bytes(int K, int RG) { return SrcNorm::smem_bytes(K, RG); }
+  typedef SrcNorm::Pre Pre;
+  __device__ static void pre_wait(const Params& p, int K, int tid, Pre& pre) { SrcNorm::pre_wait(p, 2 * K, tid, pre); }
+
+  template <int RG>
+  __device__ static void prologue(const Params& p, int K, int R, unsigned char* xsm, float* red, int tid,
+                                  const Pre& pre) {
+    const int Kc = 2 * K, ng = Kc / 4, ld = (K + 8) * 2;  // columns, float4 groups, row bytes
+    unsigned char* xh = xsm;
+    unsigned char* xl = xsm + (size_t)RG * ld;
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int rb = 0; rb < R; rb += 4) {
+      float4 v[4][kG];
+      float a[4];
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = rb + rr;
+        a[rr] = 0.f;
+        const int src = r < R ? (p.row_src ? min(max(p.row_src[r], 0), kRmax - 1) : r) : 0;
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          const int m = tid + j * kConsumers;
+          v[rr][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+          if (r < R && m < ng) v[rr][j] = __ldcg(reinterpret_cast<const float4*>(p.x + (long long)src * p.ldx) + m);
+        }
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          a[rr] = __fmaf_rn(v[rr][j].x, v[rr][j].x, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].y, v[rr][j].y, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].z, v[rr][j].z, a[rr]);
+          a[rr] = __fmaf_rn(v[rr][j].w, v[rr][j].w, a[rr]);
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) a[rr] = __fadd_rn(a[rr], __shfl_xor_sync(0xffffffffu, a[rr], o));
+      if (lane == 0)
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) red[(rb + rr) * kNW + warp] = a[rr];
+      named_sync(1, kConsumers);
+#pragma unroll
+      for (int rr = 0; rr < 4; ++rr) {
+        const int r = rb + rr;
+        if (r >= R) break;
+        float ss = 0.f;
+#pragma unroll
+        for (int w = 0; w < kNW; ++w) ss = __fadd_rn(ss, red[r * kNW + w]);
+        const float sc = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)Kc), p.eps));
+#pragma unroll
+        for (int j = 0; j < kG; ++j) {
+          const int m = tid + j * kConsumers;
+          if (m < ng) {
+            const float f[4] = {__fmul_rn(__fmul_rn(v[rr][j].x, sc), pre.g[j].x),
+                                __fmul_rn(__fmul_rn(v[rr][j].y, sc), pre.g[j].y),
+                                __fmul_rn(__fmul_rn(v[rr][j].z, sc), pre.g[j].z),
+                                __fmul_rn(__fmul_rn(v[rr][j].w, sc), pre.g[j].w)};
+            uint32_t hi, lo;
+            split_e4m3x4(f, hi, lo);
+            *reinterpret_cast<uint32_t*>(xh + (size_t)r * ld + 4 * m) = hi;
+            *reinterpret_cast<uint32_t*>(xl + (size_t)r * ld + 4 * m) = lo;
+          }
+        }
+      }
+    }
+    named_sync(1, kConsumers);
+  }
+  __device__ static uint32_t b_base(const unsigned char* xsm, const unsigned char* sx, int K, int row, int lane) {
+    return SrcNorm::b_base(xsm, sx, K, row, lane);
+  }
+  template <int RG>
+  __device__ static uint32_t lo_offset(int K) { return SrcNorm::lo_offset<RG>(K); }
+  __device__ static uint32_t b_slice(int slc) { return SrcNorm::b_slice(slc); }
 };
 
 // ---------------------------------------------------------------------------
@@ -438,6 +556,7 @@ struct EpiArgmax {
     float* logits;      // optional [R][N]
     float2* partial;    // [gridDim][kRmax] (value, index as float bits)
     const int* row_dst; // pass row -> tok/logits row (nullptr: r)
+    const float* row_scale;  // optional [N]: each logit times this (quantised heads' inverse row scales)
   };
   __device__ static float* best_v() { __shared__ float v[kNW * kRmax]; return v; }
   __device__ static int* best_i() { __shared__ int v[kNW * kRmax]; return v; }
@@ -446,11 +565,12 @@ struct EpiArgmax {
                                int lane) {
     int nrow = o.n;
     bool valid = o.q < rs.n && nrow < s.N;
+    const float lv = p.row_scale && nrow < s.N ? __fmul_rn(o.v, __ldg(p.row_scale + nrow)) : o.v;
     if (p.logits && valid) {
       int r = rs.r_sel(o.q);
-      p.logits[(long long)(p.row_dst ? p.row_dst[r] : r) * s.N + nrow] = o.v;
+      p.logits[(long long)(p.row_dst ? p.row_dst[r] : r) * s.N + nrow] = lv;
     }
-    float bv = valid ? o.v : -INFINITY;
+    float bv = valid ? lv : -INFINITY;
     int bi = valid ? nrow : 0x7fffffff;
 #pragma unroll
     for (int m = 8; m <= 16; m <<= 1) {
@@ -817,8 +937,13 @@ gemv_kernel(const __grid_constant__ CUtensorMap tm_w, const GemvShape s, const t
           ldsm_x4(a_base + (uint32_t)((((2 * k16 + a_hi) ^ a_sw)) << 4), a);
           ldsm_x2(b_addr + k16 * 32, bh);
           ldsm_x2(b_addr + b_lo + k16 * 32, bl);
-          mma_bf16(d, a, bh);
-          mma_bf16(d, a, bl);
+          if constexpr (Src::kFp8) {
+            mma_e4m3(d, a, bh);
+            mma_e4m3(d, a, bl);
+          } else {
+            mma_bf16(d, a, bh);
+            mma_bf16(d, a, bl);
+          }
         }
       }
       __syncwarp();

@@ -132,6 +132,7 @@ cudaError_t gemv_prepare() {
   if (e == cudaSuccess) e = configure_rg<SrcNorm, EpiArgmaxAccept>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<false>>();
   if (e == cudaSuccess) e = configure_rg<SrcBf16, EpiStore<true>>();
+  if (e == cudaSuccess) e = configure_rg<SrcNorm8, EpiArgmax>();
   return e;
 }
 
@@ -167,6 +168,10 @@ cudaError_t launch_gemv(const GemvLaunch& g, const LaunchCfg& lc) {
   if (g.rows_bound > kRmax) return cudaErrorInvalidValue;
   if (g.s.kparts > 1 && (!g.s.part || !g.s.tile_counter)) return cudaErrorInvalidValue;
   if (!g.s.work) return cudaErrorInvalidValue;
+  if (g.src == SrcKind::Norm8) {
+    if (g.epi != EpiKind::Argmax) return cudaErrorInvalidValue;
+    return launch_rg<SrcNorm8, EpiArgmax>(g, g.norm, g.argmax, lc);
+  }
   if (g.src == SrcKind::Norm) {
     switch (g.epi) {
       case EpiKind::QKV: return launch_rg<SrcNorm, EpiQKV>(g, g.norm, g.qkv, lc);

@@ -52,7 +52,7 @@ cudaError_t launch_cluster_ex(void (*kernel)(KArgs...), dim3 grid, dim3 block, s
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
-enum class SrcKind { Norm, Bf16 };
+enum class SrcKind { Norm, Bf16, Norm8 };  // Norm8: e4m3 weights and activation parts
 enum class EpiKind { Store, StoreAdd, SwiGLU, QKV, Argmax, ArgmaxAccept };
 
 // One GEMV launch: shape + the parameters of the chosen source and epilogue.

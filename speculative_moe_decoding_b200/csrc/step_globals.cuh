@@ -6,6 +6,25 @@
 
 namespace ocrdec {
 
+// Row-wise e4m3 quantisation of a bfloat16 matrix [N][K] (the draft's copy of
+// the LM head): row n is scaled so that its largest magnitude maps to 448
+// (e4m3's largest finite value), rounded to nearest even, and inv[n] gets the
+// scale's inverse (all-zero rows: scale 1).  One warp per row.
+__global__ void __launch_bounds__(256) quantize_rows_e4m3_kernel(const bf16* W, int N, int K, unsigned char* W8,
+                                                                float* inv) {
+  const int lane = threadIdx.x & 31;
+  const int n = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (n >= N) return;
+  const bf16* w = W + (size_t)n * K;
+  float amax = 0.f;
+  for (int k = lane; k < K; k += 32) amax = fmaxf(amax, fabsf(bf2f(w[k])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float scale = amax > 0.f ? __fdiv_rn(448.f, amax) : 1.f;
+  for (int k = lane; k < K; k += 32) W8[(size_t)n * K + k] = (unsigned char)f2e4m3(__fmul_rn(bf2f(w[k]), scale));
+  if (lane == 0) inv[n] = amax > 0.f ? __fdiv_rn(amax, 448.f) : 1.f;
+}
+
 __global__ void rope_table_kernel(float2* tab, int cap, int Dh, double theta) {
   int half = Dh / 2;
   long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;

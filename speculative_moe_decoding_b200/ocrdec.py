@@ -68,6 +68,8 @@ ocrdec_step_kernel_count = _sig("ocrdec_step_kernel_count", _i32, _vp, _i32, _i3
 ocrdec_set_debug_taps = _sig("ocrdec_set_debug_taps", _i32, _vp, _vp, _vp)
 ocrdec_set_draft_taps = _sig("ocrdec_set_draft_taps", _i32, _vp, _vp)
 ocrdec_set_trace = _sig("ocrdec_set_trace", _i32, _vp, _i32, _vp)
+ocrdec_draft_head_fp8_bytes = _sig("ocrdec_draft_head_fp8_bytes", _sz, ctypes.POINTER(Config))
+ocrdec_set_draft_head_fp8 = _sig("ocrdec_set_draft_head_fp8", _i32, _vp, _vp, _sz, _vp)
 ocrdec_replay_moe_ffn = _sig("ocrdec_replay_moe_ffn", _i32, _vp, _i32, _i32, _i32, _i32, _vp)
 ocrdec_read_trace = _sig("ocrdec_read_trace", _i32, _vp, _vp, _i32, ctypes.POINTER(_i32), _vp)
 
@@ -274,6 +276,22 @@ class Decoder:
         (batch, k) pass's rows and routing."""
         check(ocrdec_replay_moe_ffn(self.ctx, batch, k, first_layer, n_layers, _stream(stream)),
               "ocrdec_replay_moe_ffn")
+
+    def set_draft_head_fp8(self, enable: bool = True, stream=None):
+        """Variant: the draft's argmax over an e4m3 copy of the LM head (verification unchanged).
+        Returns the (uint8) buffer holding the copy and its inverse row scales, or None."""
+        torch = self.torch
+        if not enable:
+            self._head8 = None
+            check(ocrdec_set_draft_head_fp8(self.ctx, None, 0, _stream(stream)), "ocrdec_set_draft_head_fp8")
+            return None
+        n = int(ocrdec_draft_head_fp8_bytes(ctypes.byref(self.cfg)))
+        buf = torch.empty(n + 256, dtype=torch.uint8, device=self.workspace.device)
+        off = (-buf.data_ptr()) % 256
+        self._head8 = buf[off:off + n]
+        check(ocrdec_set_draft_head_fp8(self.ctx, self._head8.data_ptr(), n, _stream(stream)),
+              "ocrdec_set_draft_head_fp8")
+        return self._head8
 
     def set_draft_taps(self, logits=None):
         self._dtaps = logits
