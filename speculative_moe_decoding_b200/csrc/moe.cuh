@@ -79,18 +79,24 @@ struct MoeParams {
 
 constexpr int kMoeThreads = kConsumers + 96;  // 8 MMA warps, the producer, epilogue and rows warps
 constexpr int kMoeProducerWarp = kNW, kMoeEpilogueWarp = kNW + 1, kMoeRowsWarp = kNW + 2;
-constexpr int kMoeRedSlots = 4;  // partial slots between the MMA warps and the epilogue warp
+constexpr int kMoeRedSlots = 2;  // partial slots between the MMA warps and the epilogue warp
 constexpr int kMoeQueue = 16;    // down items handed from the producer to the rows thread
 constexpr int kMoeRedSlotFloats = 4 * kTile * 8;
 
 __host__ __device__ constexpr size_t moe_xn_bytes(int d, int RG) { return (size_t)2 * RG * (d + 8) * 2; }
 __host__ __device__ constexpr size_t moe_xb_bytes(int f, int RG) { return (size_t)2 * RG * (f + 8) * 2; }
 // Dynamic shared memory: 1 KB alignment slack, the weight ring, the normalised
-// rows, two down-item row buffers and the partial slots.
+// rows, the down items' row buffer and the partial slots (which hold the
+// routing's logits and scratch before the first item).  Small enough for two
+// CTAs per SM at four stages and up to four rows: one SM's two CTAs stream
+// faster than one CTA with twice the ring (each CTA consumes its stages in
+// order, so the other covers its stalls).
 __host__ __device__ constexpr size_t moe_smem_bytes(int d, int f, int RG, int nst) {
-  return 1024 + (size_t)nst * kStageBytes + moe_xn_bytes(d, RG) + 2 * moe_xb_bytes(f, RG) +
+  return 1024 + (size_t)nst * kStageBytes + moe_xn_bytes(d, RG) + moe_xb_bytes(f, RG) +
          (size_t)kMoeRedSlots * kMoeRedSlotFloats * 4;
 }
+static_assert(kMoeRedSlots * kMoeRedSlotFloats * 4 >= kRmax * kMaxExperts * 4 + kRouteScratchBytes,
+              "the routing's logits and scratch fit in the partial slots");
 
 __device__ __forceinline__ int ld_acquire(const int* p) {
   int v;
@@ -181,9 +187,10 @@ __device__ __forceinline__ void moe_mat(const MoeParams& p, const RouteTables& r
 // Shared state of one CTA.
 struct MoeShared {
   uint64_t full_bar[kMoeMaxStages], empty_bar[kMoeMaxStages];  // weight ring
-  uint64_t x_full[2], x_empty[2];                              // down items' row buffers
+  uint64_t x_full, x_empty;                                    // the down items' row buffer
   uint64_t red_full[kMoeRedSlots], red_empty[kMoeRedSlots];    // MMA warps -> epilogue warp
   uint64_t tab_bar;                                            // routing tables ready (MMA warps -> others)
+  uint64_t xin_bar;                                            // the residual rows' copy landed
   int s_tag[kMoeMaxStages];            // per stage: item (first slice), -2 (other slices), -1 (end)
   int s_meta[kMoeMaxStages];           // per first stage: down << 31 | m << 16 | t
   int s_rs[kMoeMaxStages][kRmax + 1];  // the item's row set (n, entries), with its first slice
@@ -194,7 +201,6 @@ struct MoeShared {
   volatile int q_done;                 // the producer claims no more
   int s_irs[kMoeRedSlots][kRmax + 1];
   RouteTables rt;
-  float lg[kRmax * kMaxExperts];
   int ids[kRmax * kMaxTopK];
   float gates[kRmax * kMaxTopK];
   float ss[kRmax * kRouteParts];
@@ -214,7 +220,7 @@ __device__ __forceinline__ MoeItem moe_unmeta(int v) {
 }
 
 template <int RG>
-__global__ void __launch_bounds__(kMoeThreads, 1)
+__global__ void __launch_bounds__(kMoeThreads, RG <= 4 ? 2 : 1)
 moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CUtensorMap tm_sgu,
            const __grid_constant__ CUtensorMap tm_dn, const __grid_constant__ CUtensorMap tm_sdn,
            const MoeParams p) {
@@ -225,7 +231,13 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
   unsigned char* stages = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   unsigned char* xn = stages + (size_t)nst * kStageBytes;
   unsigned char* xb = xn + moe_xn_bytes(p.d, RG);
-  float* red = reinterpret_cast<float*>(xb + 2 * moe_xb_bytes(p.f, RG));
+  float* red = reinterpret_cast<float*>(xb + moe_xb_bytes(p.f, RG));
+  // routing scratch in the partial slots (free until the first item): logits
+  // [kRmax][kMaxExperts], probabilities, selected slots
+  float* lg = red;
+  float (*rt_p)[kMaxExperts] = reinterpret_cast<float (*)[kMaxExperts]>(red + kRmax * kMaxExperts);
+  unsigned char (*rt_slot)[kMaxExperts] =
+      reinterpret_cast<unsigned char (*)[kMaxExperts]>(red + 2 * kRmax * kMaxExperts);
   const int nslot = p.top_k + p.S;
   const int n_shared_items = p.S * p.tiles_gu;  // the items that do not depend on the routing
 
@@ -234,15 +246,14 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       mbar_init(&sh.full_bar[i], 1);  // the weights' transaction bytes
       mbar_init(&sh.empty_bar[i], kNW);
     }
-    mbar_init(&sh.x_full[0], 1);
-    mbar_init(&sh.x_full[1], 1);
-    mbar_init(&sh.x_empty[0], kNW);
-    mbar_init(&sh.x_empty[1], kNW);
+    mbar_init(&sh.x_full, 1);
+    mbar_init(&sh.x_empty, kNW);
     for (int i = 0; i < kMoeRedSlots; ++i) {
       mbar_init(&sh.red_full[i], kNW);
       mbar_init(&sh.red_empty[i], 1);
     }
     mbar_init(&sh.tab_bar, 1);
+    mbar_init(&sh.xin_bar, 1);
     sh.q_n = 0;
     sh.q_taken = 0;
     sh.q_done = 0;
@@ -380,21 +391,19 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       bool shm;
       RowSet rs;
       moe_mat(p, sh.rt, mi.m, R, &coord, &shm, &rs);
-      const int xbuf = xitems & 1;
-      const uint32_t xuse = xitems >> 1;
-      ++xitems;
-      if (xuse > 0) mbar_wait(&sh.x_empty[xbuf], (xuse - 1) & 1, p.status);  // the buffer's previous item is done
-      spin_geq(p.ctr + kMoeCtrGu + mi.m, p.tiles_gu, p.status);             // every gate/up tile of the matrix
+      const uint32_t xuse = xitems++;
+      spin_geq(p.ctr + kMoeCtrGu + mi.m, p.tiles_gu, p.status);       // every gate/up tile of the matrix
       fence_proxy_async_global();  // the rows were written through the generic proxy
+      if (xuse > 0) mbar_wait(&sh.x_empty, (xuse - 1) & 1, p.status);  // the previous down item is done
       const int nq = min(rs.n, RG);
-      unsigned char* xdst = xb + (size_t)xbuf * moe_xb_bytes(p.f, RG);
-      mbar_arrive_expect_tx(&sh.x_full[xbuf], (uint32_t)(2 * nq * p.f * 2));
+      unsigned char* xdst = xb;
+      mbar_arrive_expect_tx(&sh.x_full, (uint32_t)(2 * nq * p.f * 2));
 #pragma unroll
       for (int q = 0; q < RG; ++q)
         if (q < nq) {
           const long long off = (long long)((rs.e[q] & 0xff) * nslot + (rs.e[q] >> 8)) * p.f;
-          bulk_g2s(xdst + (size_t)q * (p.f + 8) * 2, p.h + off, p.f * 2, &sh.x_full[xbuf]);
-          bulk_g2s(xdst + (size_t)(RG + q) * (p.f + 8) * 2, p.h_lo + off, p.f * 2, &sh.x_full[xbuf]);
+          bulk_g2s(xdst + (size_t)q * (p.f + 8) * 2, p.h + off, p.f * 2, &sh.x_full);
+          bulk_g2s(xdst + (size_t)(RG + q) * (p.f + 8) * 2, p.h_lo + off, p.f * 2, &sh.x_full);
         }
     }
     return;
@@ -484,31 +493,44 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
         spin_geq(p.ctr + kMoeCtrRead, (int)gridDim.x, p.status);
       }
       __syncwarp();
-      constexpr int kSlots = kMaxTopK + kMaxShared;
-      // lane: columns lane of rows k (k < RG), four rows per round of loads
+      // lane: column lane of rows k (k < RG); four rows x eight slots per
+      // round of loads (one round for up to eight slots), the sum carried
+      // across rounds in slot order
 #pragma unroll
       for (int k0 = 0; k0 < RG; k0 += 4) {
-        float yv[4][kSlots], xo[4];
+        float t[4] = {0.f, 0.f, 0.f, 0.f}, xo[4];
+        const int nn = mi.t * kTile + lane;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int r = k0 + k, nn = mi.t * kTile + lane;
-          const bool ok = k0 + k < RG && r < R;
+          const int r = k0 + k;
+          xo[k] = k0 + k < RG && r < R ? __ldcg(p.x + (size_t)r * p.d + nn) : 0.f;
+        }
+        for (int s0 = 0; s0 < nslot; s0 += 8) {
+          float yv[4][8];
 #pragma unroll
-          for (int s = 0; s < kSlots; ++s)
-            yv[k][s] = ok && s < nslot ? __ldcg(p.y + ((size_t)r * nslot + s) * p.d + nn) : 0.f;
-          xo[k] = ok ? __ldcg(p.x + (size_t)r * p.d + nn) : 0.f;
+          for (int k = 0; k < 4; ++k) {
+            const int r = k0 + k;
+            const bool ok = k0 + k < RG && r < R;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+              yv[k][j] = ok && s0 + j < nslot ? __ldcg(p.y + ((size_t)r * nslot + s0 + j) * p.d + nn) : 0.f;
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = k0 + k;
+            if (k0 + k >= RG || r >= R) continue;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              const int sl = s0 + j;
+              if (sl < p.top_k) t[k] = __fmaf_rn(sh.gates[r * p.top_k + sl], yv[k][j], t[k]);
+              else if (sl < nslot) t[k] = __fadd_rn(t[k], yv[k][j]);
+            }
+          }
         }
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
-          const int r = k0 + k, nn = mi.t * kTile + lane;
-          if (k0 + k >= RG || r >= R) continue;
-          float t = 0.f;
-#pragma unroll
-          for (int s = 0; s < kSlots; ++s) {
-            if (s < p.top_k) t = __fmaf_rn(sh.gates[r * p.top_k + (s < kMaxTopK ? s : 0)], yv[k][s], t);
-            else if (s < nslot) t = __fadd_rn(t, yv[k][s]);
-          }
-          p.x[(size_t)r * p.d + nn] = __fadd_rn(xo[k], t);
+          const int r = k0 + k;
+          if (k0 + k < RG && r < R) p.x[(size_t)r * p.d + nn] = __fadd_rn(xo[k], t[k]);
         }
       }
     }
@@ -543,16 +565,14 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
   if (tid == 0) sh.abort_flag = status_bad(p.status);
   const int R = min(max(__ldcg(p.nrows), 0), RG);
   const int E = p.E;
-  // ---- one round of loads: residual rows, router dot products, sums of squares ----
-  float4 xv[RG][2];
-#pragma unroll
-  for (int r = 0; r < RG; ++r)
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int mq = tid + j * kConsumers;
-      xv[r][j] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (r < R && mq < p.d / 4) xv[r][j] = __ldcg(reinterpret_cast<const float4*>(p.x + (size_t)r * p.d) + mq);
-    }
+  // ---- one round of loads: the residual rows (bulk copies into the
+  // normalised-row buffer, as float32, until they are normalised), router dot
+  // products, sums of squares ----
+  float* xin = reinterpret_cast<float*>(xn);  // [R][d] float32 (fits: 4 RG d <= 4 RG (d + 8))
+  if (tid == 0) {
+    mbar_arrive_expect_tx(&sh.xin_bar, (uint32_t)(R * p.d * 4));
+    for (int r = 0; r < R; ++r) bulk_g2s(xin + (size_t)r * p.d, p.x + (size_t)r * p.d, p.d * 4, &sh.xin_bar);
+  }
   constexpr int kLgPer = kRmax * kMaxExperts / kConsumers;  // logits per thread (2)
   float dk[kLgPer][kRouteParts];
 #pragma unroll
@@ -587,7 +607,7 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       float s = sc[0];
 #pragma unroll
       for (int q = 1; q < RG; ++q) s = r == q ? sc[q] : s;
-      sh.lg[idx] = __fmul_rn(dot, s);
+      lg[idx] = __fmul_rn(dot, s);
     }
   }
   named_sync(1, kConsumers);
@@ -596,7 +616,9 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
   // waits for the tables before its first routed item) ----
   if (!abort_now) {
     RouteParams rp{};
-    rp.logits = sh.lg;
+    rp.logits = lg;
+    rp.s_p = rt_p;
+    rp.s_slot = rt_slot;
     rp.E = E;
     rp.top_k = p.top_k;
     rp.S = p.S;
@@ -619,8 +641,20 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       atomicAdd(&p.touched[1], 1);
     }
   }
-  // normalised rows as bfloat16 high / low parts (rows R..RG-1 zero)
+  // normalised rows as bfloat16 high / low parts (rows R..RG-1 zero), in
+  // place of the float32 rows: every thread reads its values, then writes
   {
+    mbar_wait(&sh.xin_bar, 0, p.status);
+    float4 xv[RG][2];
+#pragma unroll
+    for (int r = 0; r < RG; ++r)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int mq = tid + j * kConsumers;
+        xv[r][j] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (r < R && mq < p.d / 4) xv[r][j] = reinterpret_cast<const float4*>(xin + (size_t)r * p.d)[mq];
+      }
+    named_sync(1, kConsumers);
     bf16* xh = reinterpret_cast<bf16*>(xn);
     bf16* xl = xh + RG * (p.d + 8);
 #pragma unroll
@@ -678,15 +712,13 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       // B operand rows: a gate/up item reads the normalised pass row of its
       // row-set entry; a down item the entry's copied row
       const int bq = (lane & 7) % RG;
-      const int xbuf = ndown & 1;
       uint32_t b_base, b_lo;
       if (!mi.down) {
         b_base = smem_u32(xn) + (uint32_t)(rs.r_sel(bq) * (p.d + 8) + ((lane >> 3) & 1) * 8) * 2;
         b_lo = (uint32_t)(RG * (p.d + 8) * 2);
       } else {
-        mbar_wait(&sh.x_full[xbuf], (ndown >> 1) & 1, p.status);  // the item's rows are in
-        b_base = smem_u32(xb + (size_t)xbuf * moe_xb_bytes(p.f, RG)) +
-                 (uint32_t)(bq * (p.f + 8) + ((lane >> 3) & 1) * 8) * 2;
+        mbar_wait(&sh.x_full, ndown & 1, p.status);  // the item's rows are in
+        b_base = smem_u32(xb) + (uint32_t)(bq * (p.f + 8) + ((lane >> 3) & 1) * 8) * 2;
         b_lo = (uint32_t)(RG * (p.f + 8) * 2);
       }
       b_base += (uint32_t)kq * kChunk * 2;
@@ -726,7 +758,7 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       }
     }
     if (mi.down) {
-      if (lane == 0) mbar_arrive(&sh.x_empty[ndown & 1]);  // the item's rows are no longer read
+      if (lane == 0) mbar_arrive(&sh.x_empty);  // the item's rows are no longer read
       ++ndown;
     }
     if (abort_now) continue;  // nothing to post

@@ -33,20 +33,30 @@ cudaError_t launch_rg(const MoeLaunch& g, const LaunchCfg& lc) {
   MoeParams p = g.p;
   const int st = static_smem<RG>();
   if (st < 0) return cudaErrorInvalidDeviceFunction;
-  // the deepest weight ring that fits next to the rows and the item buffers
-  int nst = kMoeMaxStages;
-  while (nst > 2 && (int)moe_smem_bytes(p.d, p.f, RG, nst) + st > kSmemPerCta) --nst;
-  if ((int)moe_smem_bytes(p.d, p.f, RG, nst) + st > kSmemPerCta) return cudaErrorInvalidValue;
+  // two CTAs per SM with a ring of at least four stages if they fit (two
+  // in-order pipelines per SM stream faster than one with twice the ring),
+  // else one CTA with the deepest ring that fits
+  int nst = 0, per_sm = 0;
+  for (int want = 2; want >= 1 && !nst; --want)
+    for (int n = kMoeMaxStages; n >= (want == 2 ? 4 : 2); --n) {
+      int occ = 0;
+      const size_t smem = moe_smem_bytes(p.d, p.f, RG, n);
+      if ((int)smem + st > kSmemPerCta) continue;
+      if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, moe_kernel<RG>, kMoeThreads, smem) != cudaSuccess)
+        return cudaErrorInvalidConfiguration;
+      if (occ >= want) {
+        nst = n;
+        per_sm = want;
+        break;
+      }
+    }
+  if (!nst) return cudaErrorInvalidValue;
   p.nst = nst;
-  const size_t smem = moe_smem_bytes(p.d, p.f, RG, nst);
-  int per_sm = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, moe_kernel<RG>, kMoeThreads, smem) != cudaSuccess ||
-      per_sm < 1)
-    return cudaErrorInvalidConfiguration;
-  // one CTA per SM: every CTA of the grid is resident at once (the combine
-  // waits until all CTAs have read the residual)
-  const int grid = lc.num_sms;
-  return launch_ex(moe_kernel<RG>, dim3(grid), dim3(kMoeThreads), smem, lc, g.tm_gu, g.tm_sgu, g.tm_dn, g.tm_sdn, p);
+  // every CTA of the grid is resident at once (the combines wait until all
+  // CTAs have read the residual)
+  const int grid = per_sm * lc.num_sms;
+  return launch_ex(moe_kernel<RG>, dim3(grid), dim3(kMoeThreads), moe_smem_bytes(p.d, p.f, RG, nst), lc, g.tm_gu,
+                   g.tm_sgu, g.tm_dn, g.tm_sdn, p);
 }
 
 }  // namespace

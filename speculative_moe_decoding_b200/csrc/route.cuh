@@ -42,14 +42,20 @@ struct RouteParams {
   int* n_mats;
   int* touched;         // optional: [0] += routed experts touched, [1] += 1
   int* status;
+  // shared-memory scratch: [kRmax][kMaxExperts] probabilities (16-byte
+  // aligned) and [kRmax][kMaxExperts] selected slots
+  float (*s_p)[kMaxExperts];
+  unsigned char (*s_slot)[kMaxExperts];
 };
+// Bytes of the scratch route_rows needs.
+constexpr int kRouteScratchBytes = kRmax * kMaxExperts * (4 + 1);
 
 // Routing of the R rows by nthreads (>= 32 * R) cooperating threads; sync()
 // is a barrier over exactly those threads.
 template <class Sync>
 __device__ void route_rows(const RouteParams& p, int R, int tid, int nthreads, Sync sync) {
-  __shared__ __align__(16) float s_p[kRmax][kMaxExperts];  // softmax probabilities, -1 past E
-  __shared__ unsigned char s_slot[kRmax][kMaxExperts];      // slot of a selected expert, 0xff otherwise
+  float (*s_p)[kMaxExperts] = p.s_p;                // softmax probabilities, -1 past E
+  unsigned char (*s_slot)[kMaxExperts] = p.s_slot;  // slot of a selected expert, 0xff otherwise
   const int lane = tid & 31, warp = tid >> 5;
   const int E = p.E, K = p.top_k;
   // warp r: softmax of row r (fixed-order sums), top-k by rank and the slots
