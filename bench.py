@@ -201,9 +201,11 @@ def reference_arm(args, dims):
 
 # ---- our arm --------------------------------------------------------------------
 
-def profiled_traffic(name):
+def profiled_traffic(name, algorithmic_bytes=None):
     """DRAM bytes per launch recorded in a profiles/ summary, if the kernel
-    sources it lists still hash to the recorded value (else None)."""
+    sources it lists still hash to the recorded value (else None).  With
+    algorithmic_bytes, a capture of a smaller case is scaled: its traffic per
+    algorithmic byte times this launch's algorithmic bytes."""
     import hashlib
     path = os.path.join(ROOT, "profiles", name)
     if not os.path.exists(path):
@@ -219,8 +221,11 @@ def profiled_traffic(name):
             h.update(open(os.path.join(ROOT, f), "rb").read())
         if h.hexdigest() != fields["source_sha256"]:
             return None
-        return int(fields["traffic_bytes_per_launch"])
-    except (KeyError, OSError, ValueError):
+        traffic = int(fields["traffic_bytes_per_launch"])
+        if algorithmic_bytes is not None:
+            return traffic / int(fields["algorithmic_bytes_per_launch"]) * algorithmic_bytes
+        return traffic
+    except (KeyError, OSError, ValueError, ZeroDivisionError):
         return None
 
 
@@ -560,7 +565,7 @@ def main():
             cpu["variants"] = oracle_variants(dims, k, bits)
 
     if rank == 0:
-        moe_traffic = profiled_traffic("moe_ffn_full_spec_k3.md")
+        moe_traffic = profiled_traffic("moe_ffn_full_spec_k3.md", moe_bytes)
         line = {
             "metric": "accepted tokens/sec (speculative decode step, batch 1)",
             "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
