@@ -106,7 +106,8 @@ typedef struct {
  * experts, top-6, vocabulary 129,280, RoPE theta = 10^6; the head layout and
  * FFN widths are free parameters of the config.
  * Validates the config (positive sizes, n_heads*head_dim == d_model, head_dim
- * 64 or 128, n_heads <= 16, d_model <= 2048 and a multiple of 128, the FFN
+ * 64 or 128, n_heads <= 16, d_model <= 1280 (each attention CTA keeps its
+ * 3 * head_dim / 8 rows of W_qkv in shared memory) and a multiple of 128, the FFN
  * widths multiples of 64,
  * vocab a multiple of 8, top_k <= min(n_experts, 8), n_experts <= 64,
  * n_shared <= 8, max_k <= 3, kv_capacity <= 8192).
@@ -249,14 +250,16 @@ OCRDEC_API int ocrdec_set_debug_taps(ocrdec_ctx* ctx, float* dev_hidden, float* 
  * phase 3 (= CTA end), uint16 kernel tag, uint16 SM id} to a device buffer of
  * 524,288 records; enabling clears it.  GEMV phases: activation prologue,
  * main loop, epilogue/finish; MoE FFN (recorded by its epilogue warp): dependency wait
- * returned, routing tables first needed, end; attention: first K/V chunk
- * landed, its softmax done, end (after the cluster merge, the output
+ * returned, routing tables first needed, end; attention block: q and the new
+ * K/V rows broadcast in the cluster (RMSNorm + QKV projection + RoPE done),
+ * the first K/V group's softmax done, end (after the cluster merge, the output
  * projection and, in MoE layers, the router partials).  ocrdec_read_trace
  * copies up to max_records records to host memory and sets *n to the number
- * recorded (synchronises `stream`).  Tags: 1 QKV, 6 dense gate/up, 7 dense
+ * recorded (synchronises `stream`).  Tags: 1 QKV (draft KV append of
+ * prefill pairs), 6 dense gate/up, 7 dense
  * down, 8 verify LM head + acceptance, 9 draft LM head, 10 draft input fc,
- * 11 MoE FFN (routing, experts, combine), 40 attention with the output
- * projection (41 for cluster rank 0), 42 verify setup, 43 draft setup. */
+ * 11 MoE FFN (routing, experts, combine), 40 attention block (RMSNorm,
+ * QKV + RoPE + KV append, attention, output projection; 41 for cluster rank 0), 42 verify setup, 43 draft setup. */
 OCRDEC_API int ocrdec_set_trace(ocrdec_ctx* ctx, int enable, ocrdec_stream stream);
 OCRDEC_API int ocrdec_read_trace(ocrdec_ctx* ctx, void* host_records, int max_records, int32_t* n,
                                  ocrdec_stream stream);

@@ -1,15 +1,28 @@
-// Decode attention over a contiguous per-slot KV cache, split over a
-// thread-block cluster, with both contractions on the tensor cores.
+// The attention block of one layer for the pass rows, split over a
+// thread-block cluster per (slot, head), with every contraction on the tensor
+// cores: RMSNorm -> QKV projection -> RoPE -> causal attention over the slot's
+// KV cache -> output projection -> residual add (-> router partials).
 //
-// For pass row r (slot b, position pos_r) and head h:
-//   out[r][h] = softmax_j(q_r . k_j / sqrt(Dh)) v_j over positions j = 0..pos_r
-// (causal: rows of one pass see each other's keys up to their own position).
+// QKV projection.  CTA k of the cluster of head h holds 3 * Dh/8 rows of
+// W_qkv: for each of q, k, v, the head's dims k*Dh/16 + j and their rotation
+// partners Dh/2 + k*Dh/16 + j (j < Dh/16; RoPE rotates dim i with dim
+// i + Dh/2), copied into shared memory before the dependency wait.  Each warp
+// loads its eighth of the reduction width of the pass rows straight into MMA
+// B fragments, the rows' RMSNorm scale comes from the warps' sums of squares,
+// and the scaled rows (bfloat16 high and low parts) multiply the W_qkv rows;
+// the warps' partial sums are added in warp order.  Rotated q goes to every
+// CTA of the cluster through distributed shared memory; the new K and V rows
+// go to the cache and, the same way, to every CTA.
 //
-// The position axis is cut into fixed kAttnChunk-position chunks.  The
-// kAttnSplit CTAs of one cluster serve one (slot, head); CTA k takes chunks
-// k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time (a group):
+// Attention.  For pass row r (position pos_r) and head h:
+//   out[r][h] = softmax_j(q_r . k_j / sqrt(Dh)) v_j over positions j = 0..pos_r.
+// The position axis is cut into fixed kAttnChunk-position chunks; CTA k takes
+// chunks k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time (a
+// group):
 //   * TMA brings each chunk's K and V rows into shared memory (5-D tensor map
-//     over the cache, 128-byte swizzle, no multicast);
+//     over the cache, 128-byte swizzle, no multicast); the pass's own rows are
+//     then written over their positions from the broadcast K and V rows, so
+//     every chunk can be requested before the dependency wait;
 //   * scores S[j][r] = K[j] . q_r as m16n8k16 MMAs (positions x rows, the up
 //     to 8 pass rows are the 8 MMA columns); q is split into bfloat16 high and
 //     low parts, so the products carry float32-level precision;
@@ -18,26 +31,22 @@
 //     P again split into bfloat16 high and low parts; each warp owns 16 dims.
 // The CTAs then merge their (M, L, O) states through distributed shared
 // memory in rank order, each CTA producing Dh / kAttnSplit output dims of the
-// head and storing them (as bf16 high and low parts) into every CTA of the
-// cluster.
+// head and storing them (as bf16 high and low parts) into every CTA.
 //
-// The output projection is folded in: CTA k multiplies the head's output by
-// its block of W_o (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; the
-// block arrives by TMA before the dependency wait) and writes the partial sums
-// per head; the last of the H heads to finish a row block adds the partials
-// in head order to the residual stream.  In MoE layers that last arriver also
-// writes the block's router partials (route.cuh): the dot products of its
-// columns of W_r with g * x (g the FFN RMSNorm gains, x the new residual, as
-// bf16 high and low parts, on the tensor cores) and the block's sum of
-// squares of x; the expert gate/up GEMV finishes the router logits from them.
-// Which CTA takes a chunk and the order of every sum depend only on positions
-// (an MMA column depends on its own row's data only; positions a row does not
-// see carry p = 0 exactly), so a row's result does not depend on the other
-// rows of the pass.
+// Output projection.  CTA k multiplies the head's output by its block of W_o
+// (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; brought by TMA into
+// the space the W_qkv rows held) and writes the partial sums per head; the
+// last of the H heads to finish a row block adds the partials in head order
+// to the residual stream.  In MoE layers that last arriver also writes the
+// block's router partials (route.cuh): the dot products of its columns of W_r
+// with g * x (g the FFN RMSNorm gains, x the new residual, as bf16 high and
+// low parts, on the tensor cores) and the block's sum of squares of x; the MoE
+// kernel finishes the router logits from them.
 //
-// Chunks that lie wholly below the pass's first new position are not written
-// by the kernel before this one (which writes the pass rows' keys and values),
-// so their copies are issued before the dependency wait.
+// Which CTA takes a chunk and the order of every sum depend only on the model
+// width and positions (an MMA column depends on its own row's data only;
+// positions a row does not see carry p = 0 exactly), so a row's result does
+// not depend on the other rows of the pass.
 #pragma once
 
 #include <cuda.h>
@@ -49,22 +58,37 @@ namespace ocrdec {
 
 constexpr int kAttnChunk = 64;
 constexpr int kAttnSplit = 8;    // CTAs per (slot, head): one cluster
-constexpr int kAttnBufs = 3;     // K/V chunks per group (ring)
+constexpr int kAttnBufs = 2;     // K/V chunks per group (ring)
 constexpr int kTagAttention = 40;
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
 constexpr int kAttnRows = 8;     // rows of one slot in a pass (MMA columns)
 constexpr int kAttnMaxDh = 128;
 constexpr int kAttnMaxHeads = 16;  // heads summed by the fused output projection
+constexpr int kAttnMaxD = 1280;    // model width: the CTA's W_qkv rows stay in shared memory
+constexpr int kAttnMaxKs = kAttnMaxD / 16 / kAttnWarps;  // k16 steps of the QKV projection per warp
+constexpr int kAttnQTiles = 3;   // 16-row MMA tiles of a CTA's W_qkv rows (Dh 128: 3, Dh 64: 2)
 constexpr int kAttnQLd = kAttnMaxDh + 8;                // bf16 q row (+16 B: conflict-free ldmatrix)
 constexpr int kAttnPLd = kAttnBufs * kAttnChunk + 8;    // bf16 P row
 constexpr int kAttnChunkBytes = kAttnChunk * kAttnMaxDh * 2;  // K (or V) of one chunk: [half][pos][128 B]
-
-// K and V of every chunk in the ring, plus 1 KB of alignment slack (the
-// 128-byte swizzle repeats every 1 KB).
-// Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
-// every 1 KB), the K/V ring, and the CTA's W_o block (d / kAttnSplit rows x Dh).
 static_assert(kAttnSplit == kRouteParts, "router partials: one per attention row block");
+
+// Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
+// every 1 KB), the K/V ring, region B, and the router block.  Region B first
+// holds the CTA's W_qkv rows (16-row tiles, rows padded by 16 bytes), then
+// the W_o block (d / kAttnSplit rows x Dh, swizzled), the scores, P and the
+// QKV projection's per-warp partial sums.
+constexpr int attn_qkv_tiles(int Dh) { return (3 * (Dh / 16) + 7) / 8; }
+constexpr size_t attn_qkv_bytes(int d, int Dh) { return (size_t)attn_qkv_tiles(Dh) * 16 * (d + 8) * 2; }
+constexpr size_t attn_sc_bytes() { return (size_t)kAttnRows * kAttnBufs * kAttnChunk * 4; }
+constexpr size_t attn_p_bytes() { return (size_t)2 * kAttnRows * kAttnPLd * 2; }
+constexpr size_t attn_red_bytes() { return (size_t)kAttnWarps * kAttnQTiles * 32 * 4 * 4; }
+constexpr size_t attn_wo_bytes(int d, int Dh) { return (size_t)(d / kAttnSplit) * Dh * 2; }
+constexpr size_t attn_regionb_bytes(int d, int Dh) {
+  return attn_qkv_bytes(d, Dh) > attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_red_bytes()
+             ? attn_qkv_bytes(d, Dh)
+             : attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_red_bytes();
+}
 
 // Router block of a CTA (MoE layers): W_r rows (E rounded up to 16, zero
 // padded) x the CTA's d / kAttnSplit columns, rows padded by 16 bytes, then the
@@ -74,11 +98,10 @@ constexpr size_t attn_router_bytes(int d, int E) {
 }
 
 constexpr size_t attn_smem_bytes(int d, int Dh, int E) {
-  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + (size_t)(d / kAttnSplit) * Dh * 2 + attn_router_bytes(d, E);
+  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + attn_regionb_bytes(d, Dh) + attn_router_bytes(d, E);
 }
 
 struct AttnParams {
-  const float* q;          // [R][H*Dh]
   int layer;               // cache layer index (map coordinate slot * n_layers + layer)
   int n_layers;            // layers in the cache (1 for the draft cache)
   int cap, H, Dh;          // Dh 64 or 128
@@ -86,10 +109,19 @@ struct AttnParams {
   const int* slot_row0;    // [B] first pass row of each slot
   const int* slot_nrows;   // [B] rows of each slot in this pass
   const int* row_pos;      // [R]
+  int rows_pre_wait;       // 1: the pass rows were written two or more kernels back (read before the wait)
   float* x;                // residual rows [R][d] (+= the projected attention output)
   float* yp;               // [H][kRmax][d] per-head partial projections
   int* cnt;                // [B][kAttnSplit] arrivals per row block, zero between launches
   int d;                   // model width (= H * Dh), a multiple of 16 * kAttnSplit
+  // QKV projection
+  const bf16* wqkv;        // [3d][d]: q rows, k rows, v rows (head-major within each)
+  const bf16* g_attn;      // attention RMSNorm gains [d]
+  float eps;
+  const float2* rope;      // [cap][Dh/2] (cos, sin) of position * theta^(-2i/Dh)
+  bf16* kc;                // K cache of this layer, slot 0: [H][cap][Dh] per slot
+  bf16* vc;
+  long long slot_stride;   // elements between slots in the cache arrays
   // MoE layers: the router partials of the updated residual rows (see route.cuh)
   const bf16* wr;          // W_r [E][d], or nullptr (dense FFN layer)
   const bf16* g_ffn;       // FFN RMSNorm gains [d]
@@ -106,6 +138,28 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Split cluster barrier: every thread arrives early (no ordering) and waits
+// right before its first access to another CTA's shared memory, which is then
+// guaranteed to have started.
+__device__ __forceinline__ void cluster_arrive_relaxed() {
+  asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Orders this thread's generic shared-memory writes before later TMA
+// (async-proxy) writes to the same addresses.
+__device__ __forceinline__ void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// Bulk copy of weights (read once per pass): evict-first in L2.
+__device__ __forceinline__ void bulk_g2s_weights(void* dst, const void* src, uint32_t bytes, uint64_t* bar,
+                                                 uint64_t pol) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::
+          "r"(smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar)), "l"(pol)
+      : "memory");
 }
 
 // Generic address of `p` in the shared memory of the cluster's CTA `rank`;
@@ -170,64 +224,108 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                  const __grid_constant__ CUtensorMap tm_wo, const AttnParams p) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  __shared__ __align__(8) uint64_t bar[kAttnBufs], wo_bar;
+  __shared__ __align__(8) uint64_t bar[kAttnBufs], qkv_bar, wo_bar, r_bar;
   __shared__ __align__(16) bf16 s_head[2][kAttnRows][kAttnQLd];  // the head's merged output, high / low parts
+  __shared__ __align__(16) bf16 s_q[2][kAttnRows][kAttnQLd];     // rotated q, high / low parts
+  __shared__ __align__(16) bf16 s_kn[2][kAttnRows][kAttnMaxDh];  // the pass rows' new K (0) and V (1)
+  __shared__ float s_ss[kAttnWarps][kAttnRows];                   // per-warp sums of squares of the rows
   __shared__ int s_last;
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
-  __shared__ __align__(16) bf16 s_q[2][kAttnRows][kAttnQLd];   // q high / low parts
-  __shared__ __align__(16) bf16 s_p[2][kAttnRows][kAttnPLd];   // P high / low parts
-  __shared__ float sc[kAttnRows][kAttnBufs * kAttnChunk];      // scores
   __shared__ float s_M[kAttnRows], s_L[kAttnRows], s_corr[kAttnRows];
   __shared__ float s_O[kAttnRows][kAttnMaxDh];
 
   const int k = (int)cluster_rank();
   const int h = blockIdx.y, b = blockIdx.z;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int Dh = p.Dh;
+  const int Dh = p.Dh, d = p.d;
   unsigned char* ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t ring_s = smem_u32(ring);
-  unsigned char* wo_s = ring + (size_t)kAttnBufs * 2 * kAttnChunkBytes;  // [Dh/64][nb rows][128 B]
-  const int nb = p.d / kAttnSplit;  // W_o rows of this CTA
+  unsigned char* regb = ring + (size_t)kAttnBufs * 2 * kAttnChunkBytes;
+  // region B while projecting: the CTA's W_qkv rows [tile][16][d + 8]
+  bf16* s_w = reinterpret_cast<bf16*>(regb);
+  const int ldq = d + 8;
+  // region B afterwards: the W_o block [Dh/64][nb rows][128 B], scores, P, the projection's partial sums
+  unsigned char* wo_s = regb;
+  const size_t wob = attn_wo_bytes(d, Dh);
+  float(*sc)[kAttnBufs * kAttnChunk] = reinterpret_cast<float(*)[kAttnBufs * kAttnChunk]>(regb + wob);
+  bf16(*s_p)[kAttnRows][kAttnPLd] = reinterpret_cast<bf16(*)[kAttnRows][kAttnPLd]>(regb + wob + attn_sc_bytes());
+  float* red = reinterpret_cast<float*>(regb + wob + attn_sc_bytes() + attn_p_bytes());
+  const int nb = d / kAttnSplit;  // W_o rows of this CTA
   const int E16 = p.wr ? (p.E + 15) / 16 * 16 : 0;
   const int ldw = nb + 8;
-  bf16* s_wr = reinterpret_cast<bf16*>(wo_s + (size_t)nb * Dh * 2);  // [E16][ldw]
-  bf16* s_gr = s_wr + (size_t)E16 * ldw;                                // [nb]
+  bf16* s_wr = reinterpret_cast<bf16*>(regb + attn_regionb_bytes(d, Dh));  // [E16][ldw]
+  bf16* s_gr = s_wr + (size_t)E16 * ldw;                                    // [nb]
+  const int P = Dh / 16;                  // dims of each of q, k, v per CTA and half
+  const int nt = attn_qkv_tiles(Dh);      // 16-row tiles of W_qkv rows
+  const int ks = d / 16 / kAttnWarps;     // k16 steps of the projection per warp
 
   if (tid == 0) {
     for (int i = 0; i < kAttnBufs; ++i) mbar_init(&bar[i], 1);
+    mbar_init(&qkv_bar, 1);
     mbar_init(&wo_bar, 1);
+    mbar_init(&r_bar, 1);
     fence_mbar_init();
-    // the W_o block (and the router block) are weights: requested before anything else
-    mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2 + (p.wr ? (p.E + 1) * nb * 2 : 0)));
-    tma_load_wo(wo_s, &tm_wo, k * nb, h * (Dh / 64), &wo_bar);
-    if (p.wr) {
-      for (int e = 0; e < p.E; ++e)
-        bulk_g2s(s_wr + (size_t)e * ldw, p.wr + (size_t)e * p.d + k * nb, nb * 2, &wo_bar);
-      bulk_g2s(s_gr, p.g_ffn + k * nb, nb * 2, &wo_bar);
-    }
-  }
-  for (int i = p.E * ldw + tid; i < E16 * ldw; i += kAttnThreads) s_wr[i] = f2bf(0.f);  // padding rows
-  // pass rows and positions are written by the pass's setup kernel, which
-  // finished before the kernel this one follows
-  const int r0 = p.slot_row0[b];
-  const int nr = max(0, min(p.slot_nrows[b], kAttnRows));
-  if (tid < kAttnRows) {
-    s_pos[tid] = tid < nr ? p.row_pos[r0 + tid] : -1;  // -1: sees nothing
-    s_M[tid] = -INFINITY;
-    s_L[tid] = 0.f;
   }
   __syncthreads();
-  int minpos = 0x7fffffff, maxpos = -1;
-  for (int i = 0; i < nr; ++i) {
-    minpos = min(minpos, s_pos[i]);
-    maxpos = max(maxpos, s_pos[i]);
+  const uint64_t wpol = l2_evict_first_policy();
+  // Weights first.  Tile t, row i of the W_qkv block is list entry
+  // li = 8t + (i & 7): matrix m = li / P (q, k, v), j = li % P, head dim
+  // (i >> 3) * Dh/2 + k*P + j; rows i and i + 8 of a tile are a RoPE pair.
+  if (warp == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(&qkv_bar, (uint32_t)(6 * P * d * 2));
+    __syncwarp();
+    for (int row = lane; row < nt * 16; row += 32) {
+      const int t = row >> 4, i = row & 15, li = t * 8 + (i & 7);
+      if (li < 3 * P) {
+        const int m = li / P, j = li - m * P;
+        const int dim = (i >> 3) * (Dh / 2) + k * P + j;
+        bulk_g2s_weights(s_w + (size_t)row * ldq, p.wqkv + ((size_t)m * d + h * Dh + dim) * d, (uint32_t)(d * 2),
+                         &qkv_bar, wpol);
+      }
+    }
+  } else if (warp == 1 && p.wr) {
+    if (lane == 0) mbar_arrive_expect_tx(&r_bar, (uint32_t)((p.E + 1) * nb * 2));
+    __syncwarp();
+    for (int e = lane; e < p.E; e += 32)
+      bulk_g2s_weights(s_wr + (size_t)e * ldw, p.wr + (size_t)e * d + k * nb, (uint32_t)(nb * 2), &r_bar, wpol);
+    if (lane == 0) bulk_g2s(s_gr, p.g_ffn + k * nb, (uint32_t)(nb * 2), &r_bar);
   }
-  maxpos = min(maxpos, p.cap - 1);
-  const int nch = maxpos >= 0 ? maxpos / kAttnChunk + 1 : 0;  // chunks of the slot
-  const int n_my = nch > k ? (nch - 1 - k) / kAttnSplit + 1 : 0;  // this CTA's chunks
-  const int plane = b * p.n_layers + p.layer;
+  for (int i = p.E * ldw + tid; i < E16 * ldw; i += kAttnThreads) s_wr[i] = f2bf(0.f);  // padding rows
+  for (int row = 3 * P + (tid >> 6); row < nt * 8; row += kAttnThreads / 64)          // padding entries (Dh 64)
+    for (int c = tid & 63; c < d; c += 64) {
+      s_w[(size_t)((row >> 3) * 16 + (row & 7)) * ldq + c] = f2bf(0.f);
+      s_w[(size_t)((row >> 3) * 16 + (row & 7) + 8) * ldq + c] = f2bf(0.f);
+    }
+  // the attention RMSNorm gains of this lane's B-fragment columns (see below)
+  uint32_t gq[kAttnMaxKs][2];
+#pragma unroll
+  for (int s = 0; s < kAttnMaxKs; ++s)
+    if (s < ks) {
+      const int kk = (warp * ks + s) * 16 + (lane & 3) * 2;
+      gq[s][0] = __ldg(reinterpret_cast<const unsigned int*>(p.g_attn + kk));
+      gq[s][1] = __ldg(reinterpret_cast<const unsigned int*>(p.g_attn + kk + 8));
+    }
+  cluster_arrive_relaxed();
 
+  // pass rows: the slot's rows r0 .. r0 + nr - 1 at positions s_pos
+  int r0 = 0, nr = 0, maxpos = -1, n_my = 0;
+  const int plane = b * p.n_layers + p.layer;
+  auto setup_rows = [&]() {
+    r0 = p.slot_row0[b];
+    nr = max(0, min(p.slot_nrows[b], kAttnRows));
+    if (tid < kAttnRows) {
+      s_pos[tid] = tid < nr ? p.row_pos[r0 + tid] : -1;  // -1: sees nothing
+      s_M[tid] = -INFINITY;
+      s_L[tid] = 0.f;
+    }
+    __syncthreads();
+    maxpos = -1;
+    for (int i = 0; i < nr; ++i) maxpos = max(maxpos, s_pos[i]);
+    maxpos = min(maxpos, p.cap - 1);
+    const int nch = maxpos >= 0 ? maxpos / kAttnChunk + 1 : 0;  // chunks of the slot
+    n_my = nch > k ? (nch - 1 - k) / kAttnSplit + 1 : 0;        // this CTA's chunks
+  };
   // chunk i of this CTA: position p0, valid positions npos, ring buffer i % kAttnBufs
   auto chunk_p0 = [&](int i) { return (k + i * kAttnSplit) * kAttnChunk; };
   auto chunk_npos = [&](int i) { return min(kAttnChunk, maxpos + 1 - chunk_p0(i)); };
@@ -238,64 +336,215 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     tma_load_kv(kd, &tm_k, chunk_p0(i), h, plane, &bar[buf]);
     tma_load_kv(kd + kAttnChunkBytes, &tm_v, chunk_p0(i), h, plane, &bar[buf]);
   };
-  auto old_chunk = [&](int i) { return chunk_p0(i) + kAttnChunk <= minpos; };
-  const int n_first = min(n_my, kAttnBufs);
-  if (tid == 0)
-    for (int i = 0; i < n_first; ++i)
-      if (old_chunk(i)) issue(i);
+  // The cache rows this pass writes are written over in shared memory once
+  // their chunk lands, so every chunk may be requested before the wait.
+  int n_issued = 0;
+  if (p.rows_pre_wait) {
+    setup_rows();
+    n_issued = min(n_my, kAttnBufs);
+    if (tid == 0)
+      for (int i = 0; i < n_issued; ++i) issue(i);
+  }
 
   pdl_wait();
-  TraceMarks tm;  // trace: wait returned, first group landed, its softmax done
-  float qv[kAttnRows];
-#pragma unroll
-  for (int i = 0; i < kAttnRows; ++i)
-    qv[i] = (i < nr && tid < Dh) ? p.q[(long long)(r0 + i) * p.H * Dh + h * Dh + tid] : 0.f;
+  TraceMarks tm;  // trace: wait returned, q/k/v broadcast, first group's softmax done
   if (tid == 0) {
     tm.t0 = gtimer();
-    const int ab = status_bad(p.status);
-    s_abort = ab;
-    if (!ab)
-      for (int i = 0; i < n_first; ++i)
-        if (!old_chunk(i)) issue(i);
+    s_abort = status_bad(p.status);
   }
-  if (tid < kAttnMaxDh)
-#pragma unroll
-    for (int i = 0; i < kAttnRows; ++i) {  // q = hi + lo, both bfloat16; zeros past nr and Dh
-      const bf16 hi = f2bf(qv[i]);
-      s_q[0][i][tid] = hi;
-      s_q[1][i][tid] = f2bf(__fsub_rn(qv[i], bf2f(hi)));
-    }
   __syncthreads();
-  const bool work = !s_abort && nr > 0;
+  const bool abort = s_abort != 0;
+  if (!p.rows_pre_wait) {
+    setup_rows();
+    if (!abort) {
+      n_issued = min(n_my, kAttnBufs);
+      if (tid == 0)
+        for (int i = 0; i < n_issued; ++i) issue(i);
+    }
+  }
+  const bool work = !abort && nr > 0;
   pdl_trigger();
 
-  // PV accumulators: warp w owns dims [16w, 16w + 16) (MMA m) for all 8 rows
-  // (MMA n): o0 (dim 16w + lane/4, row 2(lane%4)), o1 (row + 1), o2/o3 (dim + 8)
-  float o[4] = {0.f, 0.f, 0.f, 0.f};
-  const bool pv_warp = warp * 16 < Dh;
   // fragment lane roles
   const int fr_row = (lane & 7) + ((lane >> 3) & 1) * 8;   // ldmatrix.x4 row within a 16-row tile
   const int fr_hi = lane >> 4;                             // second 16-byte unit for lanes 16..31
   const int b_n = lane & 7, b_k8 = ((lane >> 3) & 1) * 8;  // ldmatrix.x2: MMA column and k offset
 
+  // ---- QKV projection: warp w takes k16 steps [w*ks, (w+1)*ks) of the rows ----
+  if (work) {
+    // B fragments straight from the residual rows: lane -> pass row lane / 4,
+    // columns (lane % 4) * 2 + {0, 1, 8, 9} of each k16 step
+    const int n = lane >> 2;
+    float xv[kAttnMaxKs][4];
+    const float* xr = p.x + (long long)(r0 + n) * d;
+#pragma unroll
+    for (int s = 0; s < kAttnMaxKs; ++s) {
+      xv[s][0] = xv[s][1] = xv[s][2] = xv[s][3] = 0.f;
+      if (s < ks && n < nr) {
+        const int kk = (warp * ks + s) * 16 + (lane & 3) * 2;
+        const float2 u = __ldcg(reinterpret_cast<const float2*>(xr + kk));
+        const float2 v = __ldcg(reinterpret_cast<const float2*>(xr + kk + 8));
+        xv[s][0] = u.x;
+        xv[s][1] = u.y;
+        xv[s][2] = v.x;
+        xv[s][3] = v.y;
+      }
+    }
+    // the row's sum of squares: lane order, then its 4 lanes, then warps in order
+    float a = 0.f;
+#pragma unroll
+    for (int s = 0; s < kAttnMaxKs; ++s)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a = __fmaf_rn(xv[s][e], xv[s][e], a);
+    a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 1));
+    a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, 2));
+    if ((lane & 3) == 0) s_ss[warp][n] = a;
+    __syncthreads();
+    float ss = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) ss = __fadd_rn(ss, s_ss[w][n]);
+    const float rs = rsqrtf(__fadd_rn(__fdiv_rn(ss, (float)d), p.eps));
+    uint32_t bh[kAttnMaxKs][2], bl[kAttnMaxKs][2];
+#pragma unroll
+    for (int s = 0; s < kAttnMaxKs; ++s) {
+      float f[4];
+      f[0] = __fmul_rn(__fmul_rn(xv[s][0], rs), bf_lo(gq[s][0]));
+      f[1] = __fmul_rn(__fmul_rn(xv[s][1], rs), bf_hi(gq[s][0]));
+      f[2] = __fmul_rn(__fmul_rn(xv[s][2], rs), bf_lo(gq[s][1]));
+      f[3] = __fmul_rn(__fmul_rn(xv[s][3], rs), bf_hi(gq[s][1]));
+      bh[s][0] = pack2(f[0], f[1]);
+      bh[s][1] = pack2(f[2], f[3]);
+      bl[s][0] = pack2(__fsub_rn(f[0], bf_lo(bh[s][0])), __fsub_rn(f[1], bf_hi(bh[s][0])));
+      bl[s][1] = pack2(__fsub_rn(f[2], bf_lo(bh[s][1])), __fsub_rn(f[3], bf_hi(bh[s][1])));
+    }
+    mbar_wait(&qkv_bar, 0, p.status);
+    float acc[kAttnQTiles][4];
+#pragma unroll
+    for (int t = 0; t < kAttnQTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
+#pragma unroll
+    for (int s = 0; s < kAttnMaxKs; ++s)
+      if (s < ks) {
+        const int k0 = (warp * ks + s) * 16;
+#pragma unroll
+        for (int t = 0; t < kAttnQTiles; ++t)
+          if (t < nt) {
+            uint32_t af[4];
+            attn_ldsm_x4(smem_u32(s_w + (size_t)(t * 16 + fr_row) * ldq + k0 + fr_hi * 8), af);
+            attn_mma(acc[t], af, bh[s]);
+            attn_mma(acc[t], af, bl[s]);
+          }
+      }
+    __syncthreads();  // region B: the W_qkv rows are read
+    if (tid == 0) {
+      // the W_o block is a weight: requested as soon as its space is free
+      mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2));
+      tma_load_wo(wo_s, &tm_wo, k * nb, h * (Dh / 64), &wo_bar);
+    }
+#pragma unroll
+    for (int t = 0; t < kAttnQTiles; ++t)
+      if (t < nt)
+        *reinterpret_cast<float4*>(red + ((warp * kAttnQTiles + t) * 32 + lane) * 4) =
+            make_float4(acc[t][0], acc[t][1], acc[t][2], acc[t][3]);
+  }
+  __syncthreads();
+  cluster_wait();  // every CTA of the cluster runs: remote stores may start
+  if (work && tid < nt * 64) {
+    // output pair (tile t, rows i and i + 8, pass row r): warps' partials in order
+    const int t = tid >> 6, L = (tid >> 1) & 31, par = tid & 1;
+    float va = 0.f, vb = 0.f;
+#pragma unroll
+    for (int w = 0; w < kAttnWarps; ++w) {
+      va = __fadd_rn(va, red[((w * kAttnQTiles + t) * 32 + L) * 4 + par]);
+      vb = __fadd_rn(vb, red[((w * kAttnQTiles + t) * 32 + L) * 4 + 2 + par]);
+    }
+    const int i = L >> 2, r = (L & 3) * 2 + par, li = t * 8 + i;
+    if (li < 3 * P) {
+      const int m = li / P, j = li - m * P;
+      const int dl = k * P + j, dp = dl + Dh / 2;
+      const int pos = s_pos[r];
+      const bool real = r < nr && pos >= 0 && pos < p.cap;
+      if (m < 2 && real) {  // RoPE: (dl, dp) turn by pos * theta^(-2 dl / Dh)
+        const float2 cs = p.rope[(long long)pos * (Dh / 2) + dl];
+        const float a2 = __fsub_rn(__fmul_rn(va, cs.x), __fmul_rn(vb, cs.y));
+        const float b2 = __fadd_rn(__fmul_rn(vb, cs.x), __fmul_rn(va, cs.y));
+        va = a2;
+        vb = b2;
+      }
+      if (m == 0) {
+        const bf16 ha = f2bf(va), hb = f2bf(vb);
+        const bf16 la = f2bf(__fsub_rn(va, bf2f(ha))), lb = f2bf(__fsub_rn(vb, bf2f(hb)));
+#pragma unroll
+        for (int q = 0; q < kAttnSplit; ++q) {
+          *const_cast<bf16*>(cluster_map(&s_q[0][r][dl], q)) = ha;
+          *const_cast<bf16*>(cluster_map(&s_q[1][r][dl], q)) = la;
+          *const_cast<bf16*>(cluster_map(&s_q[0][r][dp], q)) = hb;
+          *const_cast<bf16*>(cluster_map(&s_q[1][r][dp], q)) = lb;
+        }
+      } else {
+        const bf16 ka = f2bf(va), kb = f2bf(vb);
+        if (real) {
+          bf16* c = (m == 1 ? p.kc : p.vc) + (long long)b * p.slot_stride + ((long long)h * p.cap + pos) * Dh;
+          c[dl] = ka;
+          c[dp] = kb;
+        }
+#pragma unroll
+        for (int q = 0; q < kAttnSplit; ++q) {
+          *const_cast<bf16*>(cluster_map(&s_kn[m - 1][r][dl], q)) = ka;
+          *const_cast<bf16*>(cluster_map(&s_kn[m - 1][r][dp], q)) = kb;
+        }
+      }
+    }
+  }
+  cluster_sync_all();  // q and the new K / V rows are in every CTA
+  if (tid == 0) tm.t1 = gtimer();
+
+  // PV accumulators: warp w owns dims [16w, 16w + 16) (MMA m) for all 8 rows
+  // (MMA n): o0 (dim 16w + lane/4, row 2(lane%4)), o1 (row + 1), o2/o3 (dim + 8)
+  float o[4] = {0.f, 0.f, 0.f, 0.f};
+  const bool pv_warp = warp * 16 < Dh;
+
   for (int i0 = 0, grp = 0; work && i0 < n_my; i0 += kAttnBufs, ++grp) {
     const int ni = min(kAttnBufs, n_my - i0);
     for (int ii = 0; ii < ni; ++ii)
       mbar_wait(&bar[ii], grp & 1, p.status);  // gives up with OCRDEC_ETIMEOUT; control flow stays uniform
-    if (tid == 0 && grp == 0) tm.t1 = gtimer();
+
+    // ---- the pass's own rows over their positions in the landed chunks ----
+    auto local_chunk = [&](int pr) {  // group buffer of position pr, or -1
+      if (pr < 0 || pr > maxpos) return -1;
+      const int c = pr / kAttnChunk;
+      if (c % kAttnSplit != k) return -1;
+      const int ii = c / kAttnSplit - i0;
+      return ii >= 0 && ii < ni ? ii : -1;
+    };
+    bool patch = false;
+    for (int r = 0; r < nr; ++r) patch |= local_chunk(s_pos[r]) >= 0;
+    if (patch) {
+      for (int idx = tid; idx < nr * Dh; idx += kAttnThreads) {
+        const int r = idx / Dh, dd = idx - r * Dh;
+        const int pr = s_pos[r], ii = local_chunk(pr);
+        if (ii < 0) continue;
+        const int pp = pr % kAttnChunk;
+        const size_t off = (size_t)ii * 2 * kAttnChunkBytes + (dd >> 6) * kAttnChunk * 128 + pp * 128 +
+                           ((((dd & 63) >> 3) ^ (pp & 7)) << 4) + (dd & 7) * 2;
+        *reinterpret_cast<bf16*>(ring + off) = s_kn[0][r][dd];
+        *reinterpret_cast<bf16*>(ring + off + kAttnChunkBytes) = s_kn[1][r][dd];
+      }
+      fence_proxy_async_smem();  // the buffer is refilled by TMA later
+      __syncthreads();
+    }
 
     // ---- scores: 16-position tiles t = warp, warp + 8, ... of the group ----
     for (int t = warp; t < ni * (kAttnChunk / 16); t += kAttnWarps) {
       const int ii = t / (kAttnChunk / 16), pt = (t % (kAttnChunk / 16)) * 16;
       const uint32_t kb = ring_s + (uint32_t)(ii * 2 * kAttnChunkBytes);
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      float dacc[4] = {0.f, 0.f, 0.f, 0.f};
       for (int s = 0; s < Dh / 16; ++s) {
-        uint32_t a[4], bh[2], bl[2];
-        attn_ldsm_x4(kv_addr(kb, s >> 2, pt + fr_row, (s & 3) * 2 + fr_hi), a);
+        uint32_t af[4], bh[2], bl[2];
+        attn_ldsm_x4(kv_addr(kb, s >> 2, pt + fr_row, (s & 3) * 2 + fr_hi), af);
         attn_ldsm_x2(smem_u32(&s_q[0][b_n][s * 16 + b_k8]), bh);
         attn_ldsm_x2(smem_u32(&s_q[1][b_n][s * 16 + b_k8]), bl);
-        attn_mma(d, a, bh);
-        attn_mma(d, a, bl);
+        attn_mma(dacc, af, bh);
+        attn_mma(dacc, af, bl);
       }
       const int p0 = chunk_p0(i0 + ii), npos = chunk_npos(i0 + ii);
 #pragma unroll
@@ -303,7 +552,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int j = pt + (lane >> 2) + (e >> 1) * 8;  // position in the chunk
         const int r = 2 * (lane & 3) + (e & 1);         // row
         const bool valid = j < npos && p0 + j <= s_pos[r];
-        sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(d[e], p.scale) : -INFINITY;
+        sc[r][ii * kAttnChunk + j] = valid ? __fmul_rn(dacc[e], p.scale) : -INFINITY;
       }
     }
     __syncthreads();
@@ -365,13 +614,13 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
           // dims 0-7, 24-31 pos 8-15 dims 8-15
           const int pos = s * 16 + (lane & 7) + (lane >> 4) * 8;
           const int u = u0 + ((lane >> 3) & 1);
-          uint32_t a[4], bh[2], bl[2];
-          attn_ldsm_x4_t(kv_addr(vb, hf, pos, u), a);
+          uint32_t af[4], bh[2], bl[2];
+          attn_ldsm_x4_t(kv_addr(vb, hf, pos, u), af);
           const int pc = ii * kAttnChunk + s * 16 + b_k8;
           attn_ldsm_x2(smem_u32(&s_p[0][b_n][pc]), bh);
           attn_ldsm_x2(smem_u32(&s_p[1][b_n][pc]), bl);
-          attn_mma(o, a, bh);
-          attn_mma(o, a, bl);
+          attn_mma(o, af, bh);
+          attn_mma(o, af, bl);
         }
       }
     }
@@ -389,10 +638,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       s_O[c0][dm + 8] = o[2];
       s_O[c0 + 1][dm + 8] = o[3];
     }
-  } else if (s_abort && tid == 0) {
-    // copies issued before the dependency wait land before the CTA exits
-    for (int i = 0; i < n_first; ++i)
-      if (old_chunk(i)) mbar_wait(&bar[i], 0, p.status);
+  } else if (tid == 0) {
+    // copies issued before the wait land before the CTA exits
+    mbar_wait(&qkv_bar, 0, p.status);
+    for (int i = 0; i < n_issued; ++i) mbar_wait(&bar[i], 0, p.status);
   }
   cluster_sync_all();  // every CTA's state is visible to the cluster
 
@@ -402,14 +651,14 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   if (work) {
     const int dpr = Dh / kAttnSplit;
     if (tid < nr * dpr) {
-      const int r = tid / dpr, d = k * dpr + (tid - r * dpr);
+      const int r = tid / dpr, dm = k * dpr + (tid - r * dpr);
       // all remote loads are issued before any is used
       float Mk[kAttnSplit], Lk[kAttnSplit], Ok[kAttnSplit];
 #pragma unroll
       for (int q = 0; q < kAttnSplit; ++q) {
         Mk[q] = *cluster_map(&s_M[r], q);
         Lk[q] = *cluster_map(&s_L[r], q);
-        Ok[q] = *cluster_map(&s_O[r][d], q);
+        Ok[q] = *cluster_map(&s_O[r][dm], q);
       }
       float Mg = -INFINITY;
 #pragma unroll
@@ -425,15 +674,15 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const bf16 hi = f2bf(ov), lo = f2bf(__fsub_rn(ov, bf2f(hi)));
 #pragma unroll
       for (int q = 0; q < kAttnSplit; ++q) {
-        *const_cast<bf16*>(cluster_map(&s_head[0][r][d], q)) = hi;
-        *const_cast<bf16*>(cluster_map(&s_head[1][r][d], q)) = lo;
+        *const_cast<bf16*>(cluster_map(&s_head[0][r][dm], q)) = hi;
+        *const_cast<bf16*>(cluster_map(&s_head[1][r][dm], q)) = lo;
       }
     } else if (tid < kAttnRows * dpr) {  // rows past nr: zeros (MMA columns stay finite)
-      const int r = tid / dpr, d = k * dpr + (tid - r * dpr);
+      const int r = tid / dpr, dm = k * dpr + (tid - r * dpr);
 #pragma unroll
       for (int q = 0; q < kAttnSplit; ++q) {
-        *const_cast<bf16*>(cluster_map(&s_head[0][r][d], q)) = f2bf(0.f);
-        *const_cast<bf16*>(cluster_map(&s_head[1][r][d], q)) = f2bf(0.f);
+        *const_cast<bf16*>(cluster_map(&s_head[0][r][dm], q)) = f2bf(0.f);
+        *const_cast<bf16*>(cluster_map(&s_head[1][r][dm], q)) = f2bf(0.f);
       }
     }
   }
@@ -447,19 +696,19 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     for (int t = warp; t < nb / 16; t += kAttnWarps) {
       float d4[4] = {0.f, 0.f, 0.f, 0.f};
       for (int s = 0; s < Dh / 16; ++s) {
-        uint32_t a[4], bh[2], bl[2];
+        uint32_t af[4], bh[2], bl[2];
         const int row = t * 16 + fr_row, u = (s & 3) * 2 + fr_hi;
-        attn_ldsm_x4(wb + (uint32_t)((s >> 2) * nb * 128 + row * 128 + ((u ^ (row & 7)) << 4)), a);
+        attn_ldsm_x4(wb + (uint32_t)((s >> 2) * nb * 128 + row * 128 + ((u ^ (row & 7)) << 4)), af);
         attn_ldsm_x2(smem_u32(&s_head[0][b_n][s * 16 + b_k8]), bh);
         attn_ldsm_x2(smem_u32(&s_head[1][b_n][s * 16 + b_k8]), bl);
-        attn_mma(d4, a, bh);
-        attn_mma(d4, a, bl);
+        attn_mma(d4, af, bh);
+        attn_mma(d4, af, bl);
       }
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        const int n = k * nb + t * 16 + (lane >> 2) + (e >> 1) * 8;
+        const int nn = k * nb + t * 16 + (lane >> 2) + (e >> 1) * 8;
         const int r = 2 * (lane & 3) + (e & 1);
-        if (r < nr) p.yp[((long long)h * kAttnRows + r0 + r) * p.d + n] = d4[e];
+        if (r < nr) p.yp[((long long)h * kAttnRows + r0 + r) * d + nn] = d4[e];
       }
     }
     // the last head to finish this row block adds the heads' partials in
@@ -473,8 +722,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int idx = tid + i * kAttnThreads;
       xv[i] = 0.f;
       if (idx < nr * nb) {
-        const int r = idx / nb, n = k * nb + (idx - r * nb);
-        xv[i] = __ldcg(p.x + (long long)(r0 + r) * p.d + n);
+        const int r = idx / nb, nn = k * nb + (idx - r * nb);
+        xv[i] = __ldcg(p.x + (long long)(r0 + r) * d + nn);
       }
     }
     __threadfence();
@@ -491,20 +740,20 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       for (int i = 0; i < kPer; ++i) {
         const int idx = tid + i * kAttnThreads;
         if (idx >= kAttnRows * nb) break;
-        const int r = idx / nb, nl = idx - r * nb, n = k * nb + nl;
+        const int r = idx / nb, nl = idx - r * nb, nn = k * nb + nl;
         float xn = 0.f;
         if (r < nr) {
-          const float* yr = p.yp + (long long)(r0 + r) * p.d + n;
+          const float* yr = p.yp + (long long)(r0 + r) * d + nn;
           float y[kAttnMaxHeads];
 #pragma unroll
           for (int hh = 0; hh < kAttnMaxHeads; ++hh)
-            if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * p.d);
+            if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * d);
           float v = 0.f;
 #pragma unroll
           for (int hh = 0; hh < kAttnMaxHeads; ++hh)
             if (hh < p.H) v = __fadd_rn(v, y[hh]);
           xn = __fadd_rn(xv[i], v);
-          p.x[(long long)(r0 + r) * p.d + n] = xn;
+          p.x[(long long)(r0 + r) * d + nn] = xn;
         }
         if (p.wr) {
           const float u = __fmul_rn(xn, bf2f(s_gr[nl]));
@@ -516,26 +765,27 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       }
       if (tid == 0) p.cnt[b * kAttnSplit + k] = 0;
       if (p.wr) {
+        mbar_wait(&r_bar, 0, p.status);
         __syncthreads();
         float* rp = p.rpart + (size_t)r0 * kRouteParts * kRouteLd + k * kRouteLd;
         // each row's sum of squares over the block (warp w: row w, fixed order)
         if (warp < nr) {
-          float a = 0.f;
-          for (int nl = lane; nl < nb; nl += 32) a = __fmaf_rn(sx[warp * nb + nl], sx[warp * nb + nl], a);
+          float s2 = 0.f;
+          for (int nl = lane; nl < nb; nl += 32) s2 = __fmaf_rn(sx[warp * nb + nl], sx[warp * nb + nl], s2);
 #pragma unroll
-          for (int off = 16; off > 0; off >>= 1) a = __fadd_rn(a, __shfl_xor_sync(0xffffffffu, a, off));
-          if (lane == 0) rp[(size_t)warp * kRouteParts * kRouteLd + kMaxExperts] = a;
+          for (int off = 16; off > 0; off >>= 1) s2 = __fadd_rn(s2, __shfl_xor_sync(0xffffffffu, s2, off));
+          if (lane == 0) rp[(size_t)warp * kRouteParts * kRouteLd + kMaxExperts] = s2;
         }
         // dot products of the block's W_r columns with u (experts x rows MMAs)
         for (int t = warp; t < E16 / 16; t += kAttnWarps) {
           float d4[4] = {0.f, 0.f, 0.f, 0.f};
           for (int s = 0; s < nb / 16; ++s) {
-            uint32_t a[4], bh[2], bl[2];
-            attn_ldsm_x4(smem_u32(s_wr + (size_t)(t * 16 + fr_row) * ldw + s * 16 + fr_hi * 8), a);
+            uint32_t af[4], bh[2], bl[2];
+            attn_ldsm_x4(smem_u32(s_wr + (size_t)(t * 16 + fr_row) * ldw + s * 16 + fr_hi * 8), af);
             attn_ldsm_x2(smem_u32(su + b_n * ldw + s * 16 + b_k8), bh);
             attn_ldsm_x2(smem_u32(su + (kAttnRows + b_n) * ldw + s * 16 + b_k8), bl);
-            attn_mma(d4, a, bh);
-            attn_mma(d4, a, bl);
+            attn_mma(d4, af, bh);
+            attn_mma(d4, af, bl);
           }
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
@@ -546,9 +796,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         }
       }
     }
-  } else if (tid == 0) {
-    mbar_wait(&wo_bar, 0, p.status);  // the W_o copy lands before the CTA exits
   }
+  // the router block's copy lands before the CTA exits
+  if (tid == 0 && p.wr) mbar_wait(&r_bar, 0, p.status);
   if (tid == 0 && work && n_my > 0) trace_end(p.status, k == 0 ? kTagAttention + 1 : kTagAttention, tm);
 }
 

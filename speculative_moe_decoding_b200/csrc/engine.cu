@@ -109,6 +109,7 @@ bool config_ok(const ocrdec_config* c) {
   if (c->max_k < 0 || c->max_k > 3) return false;
   if (c->max_batch > kRmax || c->max_batch * (c->max_k + 1) > kRmax) return false;
   if (c->d_model > kGemvMaxK) return false;  // shared-memory copy of the normalised rows
+  if (c->d_model > kAttnMaxD) return false;  // the attention block's W_qkv rows stay in shared memory
   // attention's fused output projection: d / 8 rows of W_o per CTA, whole 16-row MMA tiles, one TMA box
   if (c->d_model % (16 * kAttnSplit) || c->d_model / kAttnSplit > 256 || c->n_heads > kAttnMaxHeads) return false;
   if (c->kv_capacity > 8192) return false;  // documented limit of the C ABI
@@ -185,7 +186,7 @@ cudaError_t max_carveout(K kernel) {
 
 cudaError_t prepare_kernels_now() {
   cudaError_t e = cudaFuncSetAttribute(attention_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)attn_smem_bytes(kGemvMaxK, kAttnMaxDh, kMaxExperts));
+                                       (int)attn_smem_bytes(kAttnMaxD, kAttnMaxDh, kMaxExperts));
   // one shared-memory carveout for every kernel (no SM reconfiguration between launches)
   if (e == cudaSuccess) e = max_carveout(attention_kernel);
   if (e == cudaSuccess) e = max_carveout(verify_setup_kernel);
@@ -328,22 +329,17 @@ GemvLaunch dense_launch(ocrdec_ctx* c, const Mat& m, int pair_half, const int* n
   return g;
 }
 
-// router / ffn_norm: a MoE layer's router and FFN norm gains (the attention
-// kernel then also writes the router partials), or nullptr.
-int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* attn_norm, const Mat& wqkv,
-                   const Mat& wo, const BlockIO& io, const bf16* router = nullptr, const bf16* ffn_norm = nullptr) {
+// The attention block: RMSNorm, QKV + RoPE + KV append, attention, output
+// projection and residual add in one clustered launch.  router / ffn_norm: a
+// MoE layer's router and FFN norm gains (the kernel then also writes the router
+// partials), or nullptr.  rows_pre_wait: the pass rows were written two or
+// more kernels back, so the kernel may read them before its dependency wait.
+int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, const bf16* attn_norm, const Mat& wqkv, const Mat& wo,
+                   const BlockIO& io, bool rows_pre_wait, const bf16* router = nullptr,
+                   const bf16* ffn_norm = nullptr) {
   const ocrdec_config& m = c->cfg;
   PassRows* rows = c->rows();
-  GemvLaunch g = dense_launch(c, wqkv, m.head_dim / 2, &rows->n, 0, rmax, kTagQKV);
-  g.src = SrcKind::Norm;
-  g.norm = SrcNorm::Params{io.x, m.d_model, nullptr, attn_norm, m.rms_eps};
-  g.epi = EpiKind::QKV;
-  g.qkv = EpiQKV::Params{c->at<float>(c->L.q), io.kc, io.vc, io.slot_stride, m.kv_capacity, m.n_heads,
-                         m.head_dim, c->at<float2>(c->L.rope), rows->slot, rows->pos};
-  CK(c->gemv(g, lc));
-
   AttnParams a{};
-  a.q = c->at<float>(c->L.q);
   a.layer = io.layer;
   a.n_layers = io.n_layers;
   a.cap = m.kv_capacity;
@@ -353,16 +349,23 @@ int qkv_attn_oproj(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, const bf16* att
   a.slot_row0 = rows->slot_row0;
   a.slot_nrows = rows->slot_nrows;
   a.row_pos = rows->pos;
+  a.rows_pre_wait = rows_pre_wait ? 1 : 0;
   a.x = io.x;
   a.yp = c->at<float>(c->L.yp);
   a.cnt = c->attn_counters();
   a.d = m.d_model;
+  a.wqkv = wqkv.p;
+  a.g_attn = attn_norm;
+  a.eps = m.rms_eps;
+  a.rope = c->at<float2>(c->L.rope);
+  a.kc = io.kc;
+  a.vc = io.vc;
+  a.slot_stride = io.slot_stride;
   a.wr = router;
   a.g_ffn = ffn_norm;
   a.rpart = c->at<float>(c->L.rpart);
   a.E = m.n_experts;
   a.status = c->status();
-  // attention and the output projection (x += attn . W_o^T) in one launch
   CK(launch_cluster_ex(attention_kernel, dim3(kAttnSplit, m.n_heads, m.max_batch), dim3(kAttnThreads),
                        attn_smem_bytes(m.d_model, m.head_dim, router ? m.n_experts : 0), lc, kAttnSplit, *io.tk,
                        *io.tv, wo.map_attn, a));
@@ -430,7 +433,8 @@ int verifier_layers(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool count) {
     const LayerW& w = c->layers[l];
     BlockIO io{c->at<float>(c->L.x), c->at<bf16>(c->L.kvk) + l * layer_elems, c->at<bf16>(c->L.kvv) + l * layer_elems,
                layer_elems * m.n_layers, &c->kv_map[0], &c->kv_map[1], l, m.n_layers};
-    int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io, w.dense ? nullptr : w.router.p,
+    // layer 0 follows the pass's setup kernel: its rows are read after the wait
+    int st = qkv_attn_oproj(c, lc, w.attn_norm, w.wqkv, w.wo, io, l > 0, w.dense ? nullptr : w.router.p,
                             w.ffn_norm);
     if (st) return st;
     st = w.dense ? dense_ffn(c, lc, rmax, io.x, w.ffn_norm, w.w_gu, w.w_down) : moe_ffn(c, lc, rmax, w, count);
@@ -494,7 +498,7 @@ int draft_block(ocrdec_ctx* c, const LaunchCfg& lc, int rmax, bool kv_only, int*
     CK(c->gemv(g, lc));
     return OCRDEC_OK;
   }
-  int st = qkv_attn_oproj(c, lc, rmax, w.attn_norm, w.wqkv, w.wo, io);
+  int st = qkv_attn_oproj(c, lc, w.attn_norm, w.wqkv, w.wo, io, true);  // draft setup, fc, then this
   if (st) return st;
   st = dense_ffn(c, lc, rmax, xd, w.ffn_norm, w.w_gu, w.w_down);
   if (st) return st;

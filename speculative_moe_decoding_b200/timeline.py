@@ -14,7 +14,7 @@ from typing import Dict, List
 import numpy as np
 
 TAGS = {1: "qkv", 6: "dense_gate_up", 7: "dense_down", 8: "lm_head_verify+accept", 9: "lm_head_draft",
-        10: "draft_fc", 11: "moe_ffn (routing+experts+combine)", 40: "attention+o_proj(+router partials)",
+        10: "draft_fc", 11: "moe_ffn (routing+experts+combine)", 40: "norm+qkv+rope+attention+o_proj(+router partials)",
         41: "attention (cluster rank 0)", 42: "verify_setup", 43: "draft_setup"}
 
 

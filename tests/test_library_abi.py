@@ -69,6 +69,7 @@ def test_config_validation(lib):
         dict(good, n_shared=9),            # shared experts beyond the routing tables
         dict(good, top_k=0),               # sizes must be positive
         dict(good, d_model=2176, n_heads=17),  # d_model beyond 2048 (and > 16 heads)
+        dict(good, d_model=1536, n_heads=12, head_dim=128),  # W_qkv rows of an attention CTA beyond shared memory
         dict(good, n_dense_first=3),       # more dense layers than layers
         dict(good, n_dense_first=1, dense_ffn=100),  # dense width a multiple of 64
         dict(good, expert_ffn=96, shared_ffn=96),    # expert width a multiple of 64
