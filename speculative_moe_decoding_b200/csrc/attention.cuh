@@ -29,9 +29,10 @@
 //   * an online softmax per row (running max M, sum L) over the group;
 //   * O[d][r] += V[j][d] P[r][j] as MMAs on V transposed (ldmatrix .trans),
 //     P again split into bfloat16 high and low parts; each warp owns 16 dims.
-// The CTAs then merge their (M, L, O) states through distributed shared
-// memory in rank order, each CTA producing Dh / kAttnSplit output dims of the
-// head and storing them (as bf16 high and low parts) into every CTA.
+// Each CTA then stores its (M, L) and the O of dims [k, k+1) * Dh/kAttnSplit
+// into CTA k (distributed shared memory); CTA k merges the eight states of its
+// dims in rank order and stores them (bf16 high and low parts) into the head
+// output of every CTA of the cluster.
 //
 // Output projection.  CTA k multiplies the head's output by its block of W_o
 // (rows [k, k+1) * d/kAttnSplit, the head's Dh columns; brought by TMA into
@@ -76,18 +77,25 @@ static_assert(kAttnSplit == kRouteParts, "router partials: one per attention row
 // Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
 // every 1 KB), the K/V ring, region B, and the router block.  Region B first
 // holds the CTA's W_qkv rows (16-row tiles, rows padded by 16 bytes), then
-// the W_o block (d / kAttnSplit rows x Dh, swizzled), the scores, P and the
-// QKV projection's per-warp partial sums.
+// the W_o block (d / kAttnSplit rows x Dh, swizzled), the scores, P, and
+// either the QKV projection's per-warp partial sums or (later) the merge's
+// receive buffer.
 constexpr int attn_qkv_tiles(int Dh) { return (3 * (Dh / 16) + 7) / 8; }
 constexpr size_t attn_qkv_bytes(int d, int Dh) { return (size_t)attn_qkv_tiles(Dh) * 16 * (d + 8) * 2; }
 constexpr size_t attn_sc_bytes() { return (size_t)kAttnRows * kAttnBufs * kAttnChunk * 4; }
 constexpr size_t attn_p_bytes() { return (size_t)2 * kAttnRows * kAttnPLd * 2; }
 constexpr size_t attn_red_bytes() { return (size_t)kAttnWarps * kAttnQTiles * 32 * 4 * 4; }
 constexpr size_t attn_wo_bytes(int d, int Dh) { return (size_t)(d / kAttnSplit) * Dh * 2; }
+// the merge's receive buffer: every CTA's (M, L) of every row and O of the
+// receiving CTA's Dh / kAttnSplit dims
+constexpr size_t attn_recv_bytes(int Dh) { return (size_t)kAttnSplit * kAttnRows * (2 + Dh / kAttnSplit) * 4; }
+constexpr size_t attn_tail_bytes(int Dh) {
+  return attn_red_bytes() > attn_recv_bytes(Dh) ? attn_red_bytes() : attn_recv_bytes(Dh);
+}
 constexpr size_t attn_regionb_bytes(int d, int Dh) {
-  return attn_qkv_bytes(d, Dh) > attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_red_bytes()
+  return attn_qkv_bytes(d, Dh) > attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_tail_bytes(Dh)
              ? attn_qkv_bytes(d, Dh)
-             : attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_red_bytes();
+             : attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_tail_bytes(Dh);
 }
 
 // Router block of a CTA (MoE layers): W_r rows (E rounded up to 16, zero
@@ -147,6 +155,15 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
   asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
+
+// Arrival count with acquire-release semantics at GPU scope: after a CTA
+// barrier it publishes the CTA's earlier writes, and the CTA that sees the
+// final count (followed by a CTA barrier) observes every arriver's writes.
+__device__ __forceinline__ int attn_arrive_acq_rel(int* p) {
+  int old;
+  asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(p) : "memory");
+  return old;
+}
 
 // Orders this thread's generic shared-memory writes before later TMA
 // (async-proxy) writes to the same addresses.
@@ -233,7 +250,6 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __shared__ int s_abort;
   __shared__ int s_pos[kAttnRows];
   __shared__ float s_M[kAttnRows], s_L[kAttnRows], s_corr[kAttnRows];
-  __shared__ float s_O[kAttnRows][kAttnMaxDh];
 
   const int k = (int)cluster_rank();
   const int h = blockIdx.y, b = blockIdx.z;
@@ -251,6 +267,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   float(*sc)[kAttnBufs * kAttnChunk] = reinterpret_cast<float(*)[kAttnBufs * kAttnChunk]>(regb + wob);
   bf16(*s_p)[kAttnRows][kAttnPLd] = reinterpret_cast<bf16(*)[kAttnRows][kAttnPLd]>(regb + wob + attn_sc_bytes());
   float* red = reinterpret_cast<float*>(regb + wob + attn_sc_bytes() + attn_p_bytes());
+  // merge receive buffer (same place as red, used after every CTA's projection):
+  // [source CTA][row] (M, L), then [source CTA][row][Dh / kAttnSplit] O of this CTA's dims
+  float* rcv_ml = red;
+  float* rcv_o = red + kAttnSplit * kAttnRows * 2;
+  const int dpr = Dh / kAttnSplit;  // merged dims per CTA
   const int nb = d / kAttnSplit;  // W_o rows of this CTA
   const int E16 = p.wr ? (p.E + 15) / 16 * 16 : 0;
   const int ldw = nb + 8;
@@ -284,12 +305,6 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
                          &qkv_bar, wpol);
       }
     }
-  } else if (warp == 1 && p.wr) {
-    if (lane == 0) mbar_arrive_expect_tx(&r_bar, (uint32_t)((p.E + 1) * nb * 2));
-    __syncwarp();
-    for (int e = lane; e < p.E; e += 32)
-      bulk_g2s_weights(s_wr + (size_t)e * ldw, p.wr + (size_t)e * d + k * nb, (uint32_t)(nb * 2), &r_bar, wpol);
-    if (lane == 0) bulk_g2s(s_gr, p.g_ffn + k * nb, (uint32_t)(nb * 2), &r_bar);
   }
   for (int i = p.E * ldw + tid; i < E16 * ldw; i += kAttnThreads) s_wr[i] = f2bf(0.f);  // padding rows
   for (int row = 3 * P + (tid >> 6); row < nt * 8; row += kAttnThreads / 64)          // padding entries (Dh 64)
@@ -338,12 +353,30 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   };
   // The cache rows this pass writes are written over in shared memory once
   // their chunk lands, so every chunk may be requested before the wait.
+  // the RoPE (cos, sin) of this thread's projection output (see below)
+  float2 rcs = make_float2(1.f, 0.f);
+  auto load_rope = [&]() {
+    if (tid < nt * 64) {
+      const int t = tid >> 6, L = (tid >> 1) & 31, r = (L & 3) * 2 + (tid & 1), li = t * 8 + (L >> 2);
+      const int pos = s_pos[r];
+      if (li < 2 * P && r < nr && pos >= 0 && pos < p.cap) rcs = p.rope[(long long)pos * (Dh / 2) + k * P + li % P];
+    }
+  };
+  // The first group's chunks are requested once the W_qkv rows have landed
+  // (they are needed only after the projection, and the two would share the
+  // SM's bandwidth while the kernel before this one still streams).
   int n_issued = 0;
   if (p.rows_pre_wait) {
     setup_rows();
-    n_issued = min(n_my, kAttnBufs);
-    if (tid == 0)
-      for (int i = 0; i < n_issued; ++i) issue(i);
+    load_rope();
+  }
+  // the router block is needed last: requested after everything else
+  if (warp == 0 && p.wr) {
+    if (lane == 0) mbar_arrive_expect_tx(&r_bar, (uint32_t)((p.E + 1) * nb * 2));
+    __syncwarp();
+    for (int e = lane; e < p.E; e += 32)
+      bulk_g2s_weights(s_wr + (size_t)e * ldw, p.wr + (size_t)e * d + k * nb, (uint32_t)(nb * 2), &r_bar, wpol);
+    if (lane == 0) bulk_g2s(s_gr, p.g_ffn + k * nb, (uint32_t)(nb * 2), &r_bar);
   }
 
   pdl_wait();
@@ -356,13 +389,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const bool abort = s_abort != 0;
   if (!p.rows_pre_wait) {
     setup_rows();
-    if (!abort) {
-      n_issued = min(n_my, kAttnBufs);
-      if (tid == 0)
-        for (int i = 0; i < n_issued; ++i) issue(i);
-    }
+    load_rope();
   }
   const bool work = !abort && nr > 0;
+  if (work) n_issued = min(n_my, kAttnBufs);
   pdl_trigger();
 
   // fragment lane roles
@@ -418,6 +448,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       bl[s][1] = pack2(__fsub_rn(f[2], bf_lo(bh[s][1])), __fsub_rn(f[3], bf_hi(bh[s][1])));
     }
     mbar_wait(&qkv_bar, 0, p.status);
+    if (tid == 0)
+      for (int i = 0; i < n_issued; ++i) issue(i);
     float acc[kAttnQTiles][4];
 #pragma unroll
     for (int t = 0; t < kAttnQTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -463,10 +495,9 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       const int dl = k * P + j, dp = dl + Dh / 2;
       const int pos = s_pos[r];
       const bool real = r < nr && pos >= 0 && pos < p.cap;
-      if (m < 2 && real) {  // RoPE: (dl, dp) turn by pos * theta^(-2 dl / Dh)
-        const float2 cs = p.rope[(long long)pos * (Dh / 2) + dl];
-        const float a2 = __fsub_rn(__fmul_rn(va, cs.x), __fmul_rn(vb, cs.y));
-        const float b2 = __fadd_rn(__fmul_rn(vb, cs.x), __fmul_rn(va, cs.y));
+      if (m < 2 && real) {  // RoPE: (dl, dp) turn by pos * theta^(-2 dl / Dh); rcs was loaded early
+        const float a2 = __fsub_rn(__fmul_rn(va, rcs.x), __fmul_rn(vb, rcs.y));
+        const float b2 = __fadd_rn(__fmul_rn(vb, rcs.x), __fmul_rn(va, rcs.y));
         va = a2;
         vb = b2;
       }
@@ -629,61 +660,56 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       for (int ii = 0; ii < kAttnBufs && i0 + kAttnBufs + ii < n_my; ++ii) issue(i0 + kAttnBufs + ii);
   }
 
-  // ---- this CTA's state: every warp holds the final O of its 16 dims ----
+  // ---- this CTA's state: (M, L) to every CTA, the O of dims
+  // [q*dpr, (q+1)*dpr) to CTA q (warp w holds dims [16w, 16w + 16)) ----
   if (work) {
     if (pv_warp) {
-      const int dm = warp * 16 + (lane >> 2), c0 = 2 * (lane & 3);
-      s_O[c0][dm] = o[0];
-      s_O[c0 + 1][dm] = o[1];
-      s_O[c0][dm + 8] = o[2];
-      s_O[c0 + 1][dm + 8] = o[3];
+      const int c0 = 2 * (lane & 3);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int dm = warp * 16 + (lane >> 2) + (e >> 1) * 8, r = c0 + (e & 1);
+        const int q = dm / dpr;
+        if (r < nr)
+          *const_cast<float*>(cluster_map(rcv_o + ((size_t)k * kAttnRows + r) * dpr + (dm - q * dpr), q)) = o[e];
+      }
+    }
+    if (tid < kAttnRows * kAttnSplit) {
+      const int r = tid & (kAttnRows - 1), q = tid / kAttnRows;
+      float* dst = const_cast<float*>(cluster_map(rcv_ml + (k * kAttnRows + r) * 2, q));
+      dst[0] = s_M[r];
+      dst[1] = s_L[r];
     }
   } else if (tid == 0) {
-    // copies issued before the wait land before the CTA exits
-    mbar_wait(&qkv_bar, 0, p.status);
-    for (int i = 0; i < n_issued; ++i) mbar_wait(&bar[i], 0, p.status);
+    mbar_wait(&qkv_bar, 0, p.status);  // the W_qkv copies land before the CTA exits
   }
-  cluster_sync_all();  // every CTA's state is visible to the cluster
+  cluster_sync_all();  // CTA k holds every CTA's state of its dims
 
   // ---- merge: CTA k forms dims [k*dpr, (k+1)*dpr) of every row, combining
   // the CTAs' states in rank order, and stores them (bf16) into the head
   // output of every CTA of the cluster ----
-  if (work) {
-    const int dpr = Dh / kAttnSplit;
-    if (tid < nr * dpr) {
-      const int r = tid / dpr, dm = k * dpr + (tid - r * dpr);
-      // all remote loads are issued before any is used
-      float Mk[kAttnSplit], Lk[kAttnSplit], Ok[kAttnSplit];
-#pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) {
-        Mk[q] = *cluster_map(&s_M[r], q);
-        Lk[q] = *cluster_map(&s_L[r], q);
-        Ok[q] = *cluster_map(&s_O[r][dm], q);
-      }
+  if (work && tid < kAttnRows * dpr) {
+    const int r = tid / dpr, dl = tid - r * dpr, dm = k * dpr + dl;
+    bf16 hi = f2bf(0.f), lo = f2bf(0.f);  // rows past nr: zeros (MMA columns stay finite)
+    if (r < nr) {
       float Mg = -INFINITY;
 #pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) Mg = fmaxf(Mg, Mk[q]);
+      for (int q = 0; q < kAttnSplit; ++q) Mg = fmaxf(Mg, rcv_ml[(q * kAttnRows + r) * 2]);
       float L = 0.f, O = 0.f;
 #pragma unroll
       for (int q = 0; q < kAttnSplit; ++q) {
-        const float f = Mk[q] == -INFINITY ? 0.f : expf(__fsub_rn(Mk[q], Mg));
-        L = __fmaf_rn(Lk[q], f, L);
-        O = __fmaf_rn(Ok[q], f, O);
+        const float Mq = rcv_ml[(q * kAttnRows + r) * 2];
+        const float f = Mq == -INFINITY ? 0.f : expf(__fsub_rn(Mq, Mg));
+        L = __fmaf_rn(rcv_ml[(q * kAttnRows + r) * 2 + 1], f, L);
+        O = __fmaf_rn(rcv_o[((size_t)q * kAttnRows + r) * dpr + dl], f, O);
       }
       const float ov = __fdiv_rn(O, L);
-      const bf16 hi = f2bf(ov), lo = f2bf(__fsub_rn(ov, bf2f(hi)));
+      hi = f2bf(ov);
+      lo = f2bf(__fsub_rn(ov, bf2f(hi)));
+    }
 #pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) {
-        *const_cast<bf16*>(cluster_map(&s_head[0][r][dm], q)) = hi;
-        *const_cast<bf16*>(cluster_map(&s_head[1][r][dm], q)) = lo;
-      }
-    } else if (tid < kAttnRows * dpr) {  // rows past nr: zeros (MMA columns stay finite)
-      const int r = tid / dpr, dm = k * dpr + (tid - r * dpr);
-#pragma unroll
-      for (int q = 0; q < kAttnSplit; ++q) {
-        *const_cast<bf16*>(cluster_map(&s_head[0][r][dm], q)) = f2bf(0.f);
-        *const_cast<bf16*>(cluster_map(&s_head[1][r][dm], q)) = f2bf(0.f);
-      }
+    for (int q = 0; q < kAttnSplit; ++q) {
+      *const_cast<bf16*>(cluster_map(&s_head[0][r][dm], q)) = hi;
+      *const_cast<bf16*>(cluster_map(&s_head[1][r][dm], q)) = lo;
     }
   }
   cluster_sync_all();  // every CTA holds the whole head output; no remote access follows
@@ -715,52 +741,65 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // head order to the residual stream.  The block's residual values are
     // read first (no kernel writes them meanwhile), so the tail after the
     // arrival count is one round of loads.
-    constexpr int kPer = kAttnRows * 256 / kAttnThreads;  // elements per thread: nr * nb <= 8 * 256
-    float xv[kPer];
+    // Float4 groups of the block: row r, columns k*nb + 4c .. 4c+3 (nb / 4
+    // groups per row; at most 4 rows fit one pass of the CTA's threads).
+    constexpr int kG4 = (kAttnRows * (kAttnMaxD / kAttnSplit) / 4 + kAttnThreads - 1) / kAttnThreads;
+    const int n4 = nb / 4;
+    float4 xv[kG4];
 #pragma unroll
-    for (int i = 0; i < kPer; ++i) {
-      const int idx = tid + i * kAttnThreads;
-      xv[i] = 0.f;
-      if (idx < nr * nb) {
-        const int r = idx / nb, nn = k * nb + (idx - r * nb);
-        xv[i] = __ldcg(p.x + (long long)(r0 + r) * d + nn);
+    for (int i = 0; i < kG4; ++i) {
+      const int g = tid + i * kAttnThreads;
+      xv[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (g < nr * n4) {
+        const int r = g / n4, c = (g - r * n4) * 4;
+        xv[i] = __ldcg(reinterpret_cast<const float4*>(p.x + (long long)(r0 + r) * d + k * nb + c));
       }
     }
-    __threadfence();
     __syncthreads();
-    if (tid == 0) s_last = atomicAdd(&p.cnt[b * kAttnSplit + k], 1) == p.H - 1;
+    if (tid == 0) s_last = attn_arrive_acq_rel(&p.cnt[b * kAttnSplit + k]) == p.H - 1;
     __syncthreads();
     if (s_last) {
-      __threadfence();
       // MoE layers: u = g * x (new residual) as bf16 high and low parts and
       // x itself go to the (now free) K/V ring for the router partials
       bf16* su = reinterpret_cast<bf16*>(ring);                                    // [2][kAttnRows][ldw]
       float* sx = reinterpret_cast<float*>(ring + (size_t)2 * kAttnRows * ldw * 2);  // [kAttnRows][nb]
 #pragma unroll
-      for (int i = 0; i < kPer; ++i) {
-        const int idx = tid + i * kAttnThreads;
-        if (idx >= kAttnRows * nb) break;
-        const int r = idx / nb, nl = idx - r * nb, nn = k * nb + nl;
-        float xn = 0.f;
+      for (int i = 0; i < kG4; ++i) {
+        const int g = tid + i * kAttnThreads;
+        if (g >= kAttnRows * n4) break;
+        const int r = g / n4, c = (g - r * n4) * 4;
+        float4 xn = make_float4(0.f, 0.f, 0.f, 0.f);
         if (r < nr) {
-          const float* yr = p.yp + (long long)(r0 + r) * d + nn;
-          float y[kAttnMaxHeads];
+          // the heads' partials of the group (all loads in flight), added in head order
+          const float* yr = p.yp + (long long)(r0 + r) * d + k * nb + c;
+          float4 y[kAttnMaxHeads];
 #pragma unroll
           for (int hh = 0; hh < kAttnMaxHeads; ++hh)
-            if (hh < p.H) y[hh] = __ldcg(yr + (long long)hh * kAttnRows * d);
-          float v = 0.f;
+            if (hh < p.H) y[hh] = __ldcg(reinterpret_cast<const float4*>(yr + (long long)hh * kAttnRows * d));
+          float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
           for (int hh = 0; hh < kAttnMaxHeads; ++hh)
-            if (hh < p.H) v = __fadd_rn(v, y[hh]);
-          xn = __fadd_rn(xv[i], v);
-          p.x[(long long)(r0 + r) * d + nn] = xn;
+            if (hh < p.H) {
+              v.x = __fadd_rn(v.x, y[hh].x);
+              v.y = __fadd_rn(v.y, y[hh].y);
+              v.z = __fadd_rn(v.z, y[hh].z);
+              v.w = __fadd_rn(v.w, y[hh].w);
+            }
+          xn = make_float4(__fadd_rn(xv[i].x, v.x), __fadd_rn(xv[i].y, v.y), __fadd_rn(xv[i].z, v.z),
+                           __fadd_rn(xv[i].w, v.w));
+          *reinterpret_cast<float4*>(p.x + (long long)(r0 + r) * d + k * nb + c) = xn;
         }
         if (p.wr) {
-          const float u = __fmul_rn(xn, bf2f(s_gr[nl]));
-          const bf16 hi = f2bf(u);
-          su[r * ldw + nl] = hi;
-          su[(kAttnRows + r) * ldw + nl] = f2bf(__fsub_rn(u, bf2f(hi)));
-          sx[r * nb + nl] = xn;
+          const float xe[4] = {xn.x, xn.y, xn.z, xn.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int nl = c + e;
+            const float u = __fmul_rn(xe[e], bf2f(s_gr[nl]));
+            const bf16 hi = f2bf(u);
+            su[r * ldw + nl] = hi;
+            su[(kAttnRows + r) * ldw + nl] = f2bf(__fsub_rn(u, bf2f(hi)));
+            sx[r * nb + nl] = xe[e];
+          }
         }
       }
       if (tid == 0) p.cnt[b * kAttnSplit + k] = 0;
