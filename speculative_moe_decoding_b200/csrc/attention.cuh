@@ -245,6 +245,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   __shared__ __align__(16) bf16 s_head[2][kAttnRows][kAttnQLd];  // the head's merged output, high / low parts
   __shared__ __align__(16) bf16 s_q[2][kAttnRows][kAttnQLd];     // rotated q, high / low parts
   __shared__ __align__(16) bf16 s_kn[2][kAttnRows][kAttnMaxDh];  // the pass rows' new K (0) and V (1)
+  __shared__ __align__(16) bf16 s_stage[4][kAttnRows][16];        // this CTA's q high, q low, K, V dims
   __shared__ float s_ss[kAttnWarps][kAttnRows];                   // per-warp sums of squares of the rows
   __shared__ int s_last;
   __shared__ int s_abort;
@@ -491,38 +492,54 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     }
     const int i = L >> 2, r = (L & 3) * 2 + par, li = t * 8 + i;
     if (li < 3 * P) {
-      const int m = li / P, j = li - m * P;
-      const int dl = k * P + j, dp = dl + Dh / 2;
+      const int m = li / P, j = li - m * P;  // dims k*P + j and Dh/2 + k*P + j
       const int pos = s_pos[r];
       const bool real = r < nr && pos >= 0 && pos < p.cap;
-      if (m < 2 && real) {  // RoPE: (dl, dp) turn by pos * theta^(-2 dl / Dh); rcs was loaded early
+      if (m < 2 && real) {  // RoPE: the pair turns by pos * theta^(-2 (k*P + j) / Dh); rcs was loaded early
         const float a2 = __fsub_rn(__fmul_rn(va, rcs.x), __fmul_rn(vb, rcs.y));
         const float b2 = __fadd_rn(__fmul_rn(vb, rcs.x), __fmul_rn(va, rcs.y));
         va = a2;
         vb = b2;
       }
+      // staged as runs of P contiguous dims (low dims, then their partners)
       if (m == 0) {
         const bf16 ha = f2bf(va), hb = f2bf(vb);
-        const bf16 la = f2bf(__fsub_rn(va, bf2f(ha))), lb = f2bf(__fsub_rn(vb, bf2f(hb)));
-#pragma unroll
-        for (int q = 0; q < kAttnSplit; ++q) {
-          *const_cast<bf16*>(cluster_map(&s_q[0][r][dl], q)) = ha;
-          *const_cast<bf16*>(cluster_map(&s_q[1][r][dl], q)) = la;
-          *const_cast<bf16*>(cluster_map(&s_q[0][r][dp], q)) = hb;
-          *const_cast<bf16*>(cluster_map(&s_q[1][r][dp], q)) = lb;
-        }
+        s_stage[0][r][j] = ha;
+        s_stage[0][r][P + j] = hb;
+        s_stage[1][r][j] = f2bf(__fsub_rn(va, bf2f(ha)));
+        s_stage[1][r][P + j] = f2bf(__fsub_rn(vb, bf2f(hb)));
       } else {
-        const bf16 ka = f2bf(va), kb = f2bf(vb);
-        if (real) {
-          bf16* c = (m == 1 ? p.kc : p.vc) + (long long)b * p.slot_stride + ((long long)h * p.cap + pos) * Dh;
-          c[dl] = ka;
-          c[dp] = kb;
-        }
-#pragma unroll
-        for (int q = 0; q < kAttnSplit; ++q) {
-          *const_cast<bf16*>(cluster_map(&s_kn[m - 1][r][dl], q)) = ka;
-          *const_cast<bf16*>(cluster_map(&s_kn[m - 1][r][dp], q)) = kb;
-        }
+        s_stage[1 + m][r][j] = f2bf(va);
+        s_stage[1 + m][r][P + j] = f2bf(vb);
+      }
+    }
+  }
+  __syncthreads();
+  if (work) {
+    // q (high, low), K and V runs to every CTA of the cluster, one P-dim run
+    // per store: [destination][part][row][run]
+    for (int w = tid; w < kAttnSplit * 4 * kAttnRows * 2; w += kAttnThreads) {
+      const int q = w >> 6, part = (w >> 4) & 3, r = (w >> 1) & 7, run = w & 1;
+      const int col = run * (Dh / 2) + k * P;
+      bf16* dst = part < 2 ? &s_q[part][r][col] : &s_kn[part - 2][r][col];
+      const bf16* src = &s_stage[part][r][run * P];
+      if (P == 8)
+        *reinterpret_cast<uint4*>(const_cast<bf16*>(cluster_map(dst, q))) = *reinterpret_cast<const uint4*>(src);
+      else
+        *reinterpret_cast<uint2*>(const_cast<bf16*>(cluster_map(dst, q))) = *reinterpret_cast<const uint2*>(src);
+    }
+    // the new K and V rows of the real pass rows to the cache
+    if (tid < kAttnRows * 4) {
+      const int r = tid >> 2, kv = (tid >> 1) & 1, run = tid & 1;
+      const int pos = s_pos[r];
+      if (r < nr && pos >= 0 && pos < p.cap) {
+        bf16* c = (kv ? p.vc : p.kc) + (long long)b * p.slot_stride + ((long long)h * p.cap + pos) * Dh +
+                  run * (Dh / 2) + k * P;
+        const bf16* src = &s_stage[2 + kv][r][run * P];
+        if (P == 8)
+          *reinterpret_cast<uint4*>(c) = *reinterpret_cast<const uint4*>(src);
+        else
+          *reinterpret_cast<uint2*>(c) = *reinterpret_cast<const uint2*>(src);
       }
     }
   }

@@ -130,7 +130,7 @@ struct Layout {
 Layout make_layout(const ocrdec_config& c, int am_blocks) {
   Layout L{};
   const size_t R = kRmax, B = c.max_batch, cap = c.kv_capacity, d = c.d_model, H = c.n_heads, Dh = c.head_dim;
-  const size_t E = c.n_experts, K = c.top_k, S = c.n_shared, f = c.expert_ffn;
+  const size_t K = c.top_k, S = c.n_shared, f = c.expert_ffn;
   const size_t F = std::max(c.dense_ffn, c.draft_ffn);
   const size_t nslot = K + S;
   L.hist_ld = c.kv_capacity + 8;
