@@ -31,9 +31,10 @@
 //     activations' bf16 high and low parts, fp32 accumulation) and post their
 //     column-quarter partials to a small queue; they do no global round trips;
 //   * the epilogue warp adds the quarter partials in order, applies SwiGLU /
-//     stores and publishes each tile with a GPU-scope release; the down tile
-//     of the last matrix waits for the tile's other matrices and adds all the
-//     experts' outputs to the residual in a fixed order.
+//     stores and publishes each tile with a GPU-scope release; the last of
+//     the matrices to finish an output tile (an acq_rel count per tile) adds
+//     all the experts' outputs of that tile to the residual in a fixed order,
+//     so no CTA waits for another's down tile.
 // The residual's RMSNorm scale comes from the attention kernel's per-block
 // sums of squares (the same ones the router logits use), so the prologue is
 // one round of loads (router partials, residual rows).
@@ -480,19 +481,18 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
         n_mats = sh.rt.n_mats;
         if (lane == 0) tm.t1 = gtimer();
       }
-      if (mi.m < n_mats - 1) {
-        if (lane == 0) red_release_add(p.ctr + kMoeCtrDn + mi.t, 1);  // publish the tile's outputs
-        continue;
-      }
-      // the last matrix's tile: once the other matrices' tiles are in, add
-      // x[r][n] += sum gate * y (routed slots in order) + sum y (shared).
-      // Every CTA must have read x first (it normalises it).  All loads are
-      // issued together, this tile's own outputs included.
+      // publish the tile's outputs; the last of the matrices to finish this
+      // output tile adds x[r][n] += sum gate * y (routed slots in order) +
+      // sum y (shared).  Every CTA must have read x first (it normalises it).
+      // All loads are issued together, this tile's own outputs included.
+      int last = 0;
       if (lane == 0) {
-        spin_geq(p.ctr + kMoeCtrDn + mi.t, n_mats - 1, p.status);
-        spin_geq(p.ctr + kMoeCtrRead, (int)gridDim.x, p.status);
+        last = atom_acq_rel_add(p.ctr + kMoeCtrDn + mi.t, 1) == n_mats - 1;
+        if (last) spin_geq(p.ctr + kMoeCtrRead, (int)gridDim.x, p.status);
       }
+      last = __shfl_sync(0xffffffffu, last, 0);
       __syncwarp();
+      if (!last) continue;
       // lane: column lane of rows k (k < RG); four rows x eight slots per
       // round of loads (one round for up to eight slots), the sum carried
       // across rounds in slot order
