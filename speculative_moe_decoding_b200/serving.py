@@ -11,10 +11,13 @@ Once the queue is empty a finished slot is re-prefilled with its own request
 again (its further tokens are discarded), so no slot decodes past the KV
 capacity while the others finish.
 
-The decoder needs ``prefill(slot, visual, prompt)``, ``step(batch, k)``,
-``stats(slot)`` (fields n_context, n_generated) and
-``history(slot, start, n)``; ``speculative_moe_decoding_b200.ocrdec.Decoder``
-has them."""
+The decoder needs ``prefill(slot, visual, prompt)``, ``step(batch, k)``
+(returning the step's committed tokens and their count per slot, as
+``speculative_moe_decoding_b200.ocrdec.Decoder`` does) and
+``history(slot, start, n)``.  The loop counts each slot's tokens on the host:
+one after the prefill (its first token), then the step's counts, read with
+one device-to-host copy per step.  A request whose target is already met after
+its prefill (n_generate <= 1) is collected without a step."""
 from __future__ import annotations
 
 from dataclasses import dataclass, field
@@ -59,35 +62,52 @@ def serve(dec, requests: Sequence[Request], batch: int, k: int, max_steps: Optio
         return res
     slot_req: List[Optional[Request]] = [None] * batch
     live = [False] * batch  # the slot's request still needs tokens
+    gen = [0] * batch       # tokens the slot's request has produced
 
     def fill(slot: int, req: Request, counts: bool):
         dec.prefill(slot, req.visual, req.prompt)
         slot_req[slot] = req
         live[slot] = counts
+        gen[slot] = 1  # the prefill's first token
+
+    def collect(slot: int) -> None:
+        """Records a finished request and gives the slot its next one."""
+        req = slot_req[slot]
+        n_ctx = int(req.visual.shape[0]) + int(req.prompt.shape[0])
+        toks = dec.history(slot, n_ctx, req.n_generate)
+        res.outputs[req.rid] = np.asarray(toks.cpu() if hasattr(toks, "cpu") else toks).copy()
+        res.useful_tokens += req.n_generate
+        if queue:
+            fill(slot, queue.pop(0), True)
+        else:
+            fill(slot, req, False)  # idle slot: start over, stay within capacity
+
+    def harvest() -> None:
+        # a refilled slot may be done at once (n_generate <= 1): loop until none is
+        done = True
+        while done:
+            done = False
+            for s in range(batch):
+                if live[s] and gen[s] >= slot_req[s].n_generate:
+                    collect(s)
+                    done = True
+                elif not live[s] and gen[s] >= slot_req[s].n_generate:
+                    fill(s, slot_req[s], False)
 
     for s in range(batch):
         if queue:
             fill(s, queue.pop(0), True)
         else:  # fewer requests than slots: idle slots repeat the first request
             fill(s, requests[0], False)
+    harvest()
     while any(live):
         if max_steps is not None and res.steps >= max_steps:
             raise RuntimeError(f"requests unfinished after {max_steps} steps")
-        dec.step(batch, k)
+        _, n_committed = dec.step(batch, k)
+        counts = np.asarray(n_committed.cpu() if hasattr(n_committed, "cpu") else n_committed).reshape(-1)
         res.steps += 1
         res.slot_steps += sum(live)
         for s in range(batch):
-            req = slot_req[s]
-            st = dec.stats(s)
-            if not live[s] or st.n_generated < req.n_generate:
-                if not live[s] and st.n_generated >= req.n_generate:
-                    fill(s, req, False)  # idle slot: start over, stay within capacity
-                continue
-            toks = dec.history(s, st.n_context, req.n_generate)
-            res.outputs[req.rid] = np.asarray(toks.cpu() if hasattr(toks, "cpu") else toks).copy()
-            res.useful_tokens += req.n_generate
-            if queue:
-                fill(s, queue.pop(0), True)
-            else:
-                fill(s, req, False)
+            gen[s] += int(counts[s])
+        harvest()
     return res

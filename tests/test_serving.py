@@ -20,6 +20,7 @@ class ScriptedDecoder:
         self.rng = np.random.default_rng(seed)
         self.slots = {}
         self.prefills = 0
+        self.steps = 0
 
     @staticmethod
     def token(key: int, i: int) -> int:
@@ -32,6 +33,7 @@ class ScriptedDecoder:
         self.prefills += 1
 
     def step(self, batch, k):
+        counts = np.zeros(batch, np.int32)
         for s in range(batch):
             st = self.slots[s]
             # the pass writes K/V at kv .. kv + k (the library's capacity check)
@@ -40,6 +42,9 @@ class ScriptedDecoder:
             for _ in range(m):
                 st.toks.append(self.token(st.key, len(st.toks)))
             st.kv += m
+            counts[s] = m
+        self.steps += 1
+        return None, counts
 
     def stats(self, slot):
         st = self.slots[slot]
@@ -70,6 +75,15 @@ def test_every_request_gets_exactly_its_tokens(batch, k):
     assert dec.prefills >= len(reqs)
 
 
+def test_single_token_requests_are_collected_without_a_step():
+    reqs = _requests([1, 1, 1])
+    dec = ScriptedDecoder(cap=serving.required_capacity(reqs, 1))
+    res = serving.serve(dec, reqs, 2, 1, max_steps=10)
+    assert res.steps == 0 and dec.steps == 0
+    for r in reqs:
+        assert list(res.outputs[r.rid]) == [ScriptedDecoder.token(100 + r.rid, 0)]
+
+
 def test_fewer_requests_than_slots_and_empty_queue():
     reqs = _requests([4, 6])
     dec = ScriptedDecoder(cap=serving.required_capacity(reqs, 2))
@@ -92,9 +106,11 @@ class OracleSlots:
         self.st[slot] = O.prefill(self.orc, visual, list(prompt))
 
     def step(self, batch, k):
+        counts = np.zeros(batch, np.int32)
         for s in range(batch):
             props = O.draft_propose(self.orc, self.st[s], k) if k > 0 else []
-            O.verify_commit(self.orc, self.st[s], props)
+            counts[s] = len(O.verify_commit(self.orc, self.st[s], props))
+        return None, counts
 
     def stats(self, slot):
         st = self.st[slot]
