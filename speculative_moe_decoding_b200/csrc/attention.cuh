@@ -18,7 +18,8 @@
 //   out[r][h] = softmax_j(q_r . k_j / sqrt(Dh)) v_j over positions j = 0..pos_r.
 // The position axis is cut into fixed kAttnChunk-position chunks; CTA k takes
 // chunks k, k + kAttnSplit, ... in increasing order, kAttnBufs at a time (a
-// group):
+// group; two buffers are the kernel's own, the third reuses the space the
+// W_qkv rows held):
 //   * TMA brings each chunk's K and V rows into shared memory (5-D tensor map
 //     over the cache, 128-byte swizzle, no multicast); the pass's own rows are
 //     then written over their positions from the broadcast K and V rows, so
@@ -59,7 +60,8 @@ namespace ocrdec {
 
 constexpr int kAttnChunk = 64;
 constexpr int kAttnSplit = 8;    // CTAs per (slot, head): one cluster
-constexpr int kAttnBufs = 2;     // K/V chunks per group (ring)
+constexpr int kAttnBufs = 3;     // K/V chunks per group
+constexpr int kAttnRingBufs = 2; // of them in the dedicated ring; the third in region B once the W_qkv rows are read
 constexpr int kTagAttention = 40;
 constexpr int kAttnThreads = 256;
 constexpr int kAttnWarps = kAttnThreads / 32;
@@ -75,11 +77,11 @@ constexpr int kAttnChunkBytes = kAttnChunk * kAttnMaxDh * 2;  // K (or V) of one
 static_assert(kAttnSplit == kRouteParts, "router partials: one per attention row block");
 
 // Dynamic shared memory: 1 KB alignment slack (the 128-byte swizzle repeats
-// every 1 KB), the K/V ring, region B, and the router block.  Region B first
-// holds the CTA's W_qkv rows (16-row tiles, rows padded by 16 bytes), then
-// the W_o block (d / kAttnSplit rows x Dh, swizzled), the scores, P, and
+// every 1 KB), two K/V chunk buffers, region B, and the router block.  Region
+// B first holds the CTA's W_qkv rows (16-row tiles, rows padded by 16 bytes),
+// then the W_o block (d / kAttnSplit rows x Dh, swizzled), the scores, P,
 // either the QKV projection's per-warp partial sums or (later) the merge's
-// receive buffer.
+// receive buffer, and the third K/V chunk buffer.
 constexpr int attn_qkv_tiles(int Dh) { return (3 * (Dh / 16) + 7) / 8; }
 constexpr size_t attn_qkv_bytes(int d, int Dh) { return (size_t)attn_qkv_tiles(Dh) * 16 * (d + 8) * 2; }
 constexpr size_t attn_sc_bytes() { return (size_t)kAttnRows * kAttnBufs * kAttnChunk * 4; }
@@ -92,10 +94,13 @@ constexpr size_t attn_recv_bytes(int Dh) { return (size_t)kAttnSplit * kAttnRows
 constexpr size_t attn_tail_bytes(int Dh) {
   return attn_red_bytes() > attn_recv_bytes(Dh) ? attn_red_bytes() : attn_recv_bytes(Dh);
 }
+// offset in region B of the third K/V chunk buffer (1 KB aligned: the swizzle)
+constexpr size_t attn_buf2_off(int d, int Dh) {
+  return (attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_tail_bytes(Dh) + 1023) / 1024 * 1024;
+}
 constexpr size_t attn_regionb_bytes(int d, int Dh) {
-  return attn_qkv_bytes(d, Dh) > attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_tail_bytes(Dh)
-             ? attn_qkv_bytes(d, Dh)
-             : attn_wo_bytes(d, Dh) + attn_sc_bytes() + attn_p_bytes() + attn_tail_bytes(Dh);
+  return attn_qkv_bytes(d, Dh) > attn_buf2_off(d, Dh) + 2 * kAttnChunkBytes ? attn_qkv_bytes(d, Dh)
+                                                                           : attn_buf2_off(d, Dh) + 2 * kAttnChunkBytes;
 }
 
 // Router block of a CTA (MoE layers): W_r rows (E rounded up to 16, zero
@@ -106,7 +111,7 @@ constexpr size_t attn_router_bytes(int d, int E) {
 }
 
 constexpr size_t attn_smem_bytes(int d, int Dh, int E) {
-  return 1024 + (size_t)kAttnBufs * 2 * kAttnChunkBytes + attn_regionb_bytes(d, Dh) + attn_router_bytes(d, E);
+  return 1024 + (size_t)kAttnRingBufs * 2 * kAttnChunkBytes + attn_regionb_bytes(d, Dh) + attn_router_bytes(d, E);
 }
 
 struct AttnParams {
@@ -258,7 +263,11 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   const int Dh = p.Dh, d = p.d;
   unsigned char* ring = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t ring_s = smem_u32(ring);
-  unsigned char* regb = ring + (size_t)kAttnBufs * 2 * kAttnChunkBytes;
+  unsigned char* regb = ring + (size_t)kAttnRingBufs * 2 * kAttnChunkBytes;
+  // K/V chunk buffer b (K then V): two in the ring, the third in region B
+  auto kvbuf = [&](int b) {
+    return b < kAttnRingBufs ? ring + (size_t)b * 2 * kAttnChunkBytes : regb + attn_buf2_off(d, Dh);
+  };
   // region B while projecting: the CTA's W_qkv rows [tile][16][d + 8]
   bf16* s_w = reinterpret_cast<bf16*>(regb);
   const int ldq = d + 8;
@@ -347,7 +356,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
   auto chunk_npos = [&](int i) { return min(kAttnChunk, maxpos + 1 - chunk_p0(i)); };
   auto issue = [&](int i) {
     const int buf = i % kAttnBufs;
-    unsigned char* kd = ring + (size_t)buf * 2 * kAttnChunkBytes;
+    unsigned char* kd = kvbuf(buf);
     mbar_arrive_expect_tx(&bar[buf], (uint32_t)(2 * kAttnChunk * Dh * 2));
     tma_load_kv(kd, &tm_k, chunk_p0(i), h, plane, &bar[buf]);
     tma_load_kv(kd + kAttnChunkBytes, &tm_v, chunk_p0(i), h, plane, &bar[buf]);
@@ -449,8 +458,8 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       bl[s][1] = pack2(__fsub_rn(f[2], bf_lo(bh[s][1])), __fsub_rn(f[3], bf_hi(bh[s][1])));
     }
     mbar_wait(&qkv_bar, 0, p.status);
-    if (tid == 0)
-      for (int i = 0; i < n_issued; ++i) issue(i);
+    if (tid == 0)  // the ring's chunks now; the third (region B) once the W_qkv rows are read
+      for (int i = 0; i < n_issued && i < kAttnRingBufs; ++i) issue(i);
     float acc[kAttnQTiles][4];
 #pragma unroll
     for (int t = 0; t < kAttnQTiles; ++t) acc[t][0] = acc[t][1] = acc[t][2] = acc[t][3] = 0.f;
@@ -472,6 +481,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       // the W_o block is a weight: requested as soon as its space is free
       mbar_arrive_expect_tx(&wo_bar, (uint32_t)(nb * Dh * 2));
       tma_load_wo(wo_s, &tm_wo, k * nb, h * (Dh / 64), &wo_bar);
+      for (int i = kAttnRingBufs; i < n_issued; ++i) issue(i);
     }
 #pragma unroll
     for (int t = 0; t < kAttnQTiles; ++t)
@@ -572,10 +582,10 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
         const int pr = s_pos[r], ii = local_chunk(pr);
         if (ii < 0) continue;
         const int pp = pr % kAttnChunk;
-        const size_t off = (size_t)ii * 2 * kAttnChunkBytes + (dd >> 6) * kAttnChunk * 128 + pp * 128 +
-                           ((((dd & 63) >> 3) ^ (pp & 7)) << 4) + (dd & 7) * 2;
-        *reinterpret_cast<bf16*>(ring + off) = s_kn[0][r][dd];
-        *reinterpret_cast<bf16*>(ring + off + kAttnChunkBytes) = s_kn[1][r][dd];
+        const size_t off = (dd >> 6) * kAttnChunk * 128 + pp * 128 + ((((dd & 63) >> 3) ^ (pp & 7)) << 4) +
+                           (dd & 7) * 2;
+        *reinterpret_cast<bf16*>(kvbuf(ii) + off) = s_kn[0][r][dd];
+        *reinterpret_cast<bf16*>(kvbuf(ii) + off + kAttnChunkBytes) = s_kn[1][r][dd];
       }
       fence_proxy_async_smem();  // the buffer is refilled by TMA later
       __syncthreads();
@@ -584,7 +594,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
     // ---- scores: 16-position tiles t = warp, warp + 8, ... of the group ----
     for (int t = warp; t < ni * (kAttnChunk / 16); t += kAttnWarps) {
       const int ii = t / (kAttnChunk / 16), pt = (t % (kAttnChunk / 16)) * 16;
-      const uint32_t kb = ring_s + (uint32_t)(ii * 2 * kAttnChunkBytes);
+      const uint32_t kb = smem_u32(kvbuf(ii));
       float dacc[4] = {0.f, 0.f, 0.f, 0.f};
       for (int s = 0; s < Dh / 16; ++s) {
         uint32_t af[4], bh[2], bl[2];
@@ -654,7 +664,7 @@ attention_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant
       o[3] = __fmul_rn(o[3], cr1);
       const int hf = (warp * 16) / 64, u0 = ((warp * 16) % 64) / 8;
       for (int ii = 0; ii < ni; ++ii) {
-        const uint32_t vb = ring_s + (uint32_t)(ii * 2 * kAttnChunkBytes + kAttnChunkBytes);
+        const uint32_t vb = smem_u32(kvbuf(ii)) + (uint32_t)kAttnChunkBytes;
 #pragma unroll
         for (int s = 0; s < kAttnChunk / 16; ++s) {
           // A = V^T (16 dims x 16 positions) from the stored [pos][dim] tile:

@@ -265,6 +265,12 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
   if (warp == kMoeProducerWarp) {
     // ================= producer (one thread): weights and row copies =================
     if (lane != 0) return;
+    // the four tensor maps' descriptors into the TMA unit's cache up front (the
+    // items alternate between them)
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_gu)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_sgu)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_dn)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tm_sdn)) : "memory");
     const uint64_t wpol = l2_evict_first_policy();
     int st = 0;
     uint32_t ph = 0, it = 0;  // ring slot, its phase parity, stages issued
