@@ -111,11 +111,14 @@ class ClockSampler:
 ORACLE_SAMPLE = dict(n_visual=32, n_prompt=8, n_ref=16)
 
 
-def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.0, threads=None):
+def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.0, threads=None,
+                      timed_steps=None, warm_steps: int = 0):
     """Times the oracle's speculative decode (forced acceptance, draft running;
     k = 0: plain greedy decode) on a bounded sample: the decode of the first
     n_ref tokens after a short context, repeated (each repetition from a fresh
-    prefill, not timed) until about budget_s of timed decode has run.
+    prefill, not timed) until about budget_s of timed decode has run - or,
+    with timed_steps, until exactly warm_steps untimed and then timed_steps
+    timed decode steps have run.
     threads limits the BLAS threads of the timed part (None: all cores).
     Returns (tokens/s, description, threads, steps, seconds)."""
     from contextlib import nullcontext
@@ -140,15 +143,20 @@ def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.
         threadpoolctl = None
     limiter = threadpoolctl.threadpool_limits(threads) if (threads and threadpoolctl) else nullcontext()
     dt = 0.0
-    steps = toks = reps = 0
+    steps = toks = reps = warm = 0
+
+    def more():
+        return steps < timed_steps if timed_steps is not None else dt < budget_s
+
     used = 1
     with limiter:
         if threadpoolctl:
             used = max((i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()), default=1)
-        while dt < budget_s:
+        while more():
             st = O.prefill(orc, inp.visual, inp.prompt)
-            t0 = time.perf_counter()
-            while st.n_generated < ORACLE_SAMPLE["n_ref"] - k - 1:
+            while st.n_generated < ORACLE_SAMPLE["n_ref"] - k - 1 and more():
+                timed = warm >= warm_steps
+                t0 = time.perf_counter()
                 before = st.n_generated
                 if k > 0:
                     O.draft_propose(orc, st, k)  # the draft runs; the forced stream decides
@@ -156,9 +164,12 @@ def run_oracle_sample(dims: synth.ModelDims, k: int, bits, budget_s: float = 20.
                 else:
                     props = []
                 O.verify_commit(orc, st, props)
-                toks += st.n_generated - before
-                steps += 1
-            dt += time.perf_counter() - t0
+                if timed:
+                    dt += time.perf_counter() - t0
+                    toks += st.n_generated - before
+                    steps += 1
+                else:
+                    warm += 1
             reps += 1
     mode = f"spec decode k={k}, forced acceptance, draft running" if k > 0 else "greedy decode (k=0)"
     desc = (f"oracle {mode}; context {C} rows "
@@ -186,10 +197,11 @@ def reference_arm(args, dims):
     if rank != 0:
         return 0
     bits, _ = synth.make_weights(dims, synth.WORKLOADS["full_spec"].weight_seed)
-    tps, desc, threads, steps, dt = run_oracle_sample(dims, args.k, bits,
-                                                      budget_s=min(60.0, 20.0 * max(1, args.steps) / 50))
+    # W untimed, then exactly K timed oracle steps of the bounded sample
+    tps, desc, threads, steps, dt = run_oracle_sample(dims, args.k, bits, timed_steps=max(1, args.steps),
+                                                      warm_steps=max(0, args.warmup))
     line = {"impl": "reference", "metric": "accepted tokens/sec (speculative decode step, batch 1)",
-            "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": 0,
+            "value": tps, "unit": "tokens/s", "n_gpus": args.gpus, "steps": steps, "warmup": max(0, args.warmup),
             "ms_per_step": 1000 * dt / max(1, steps), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f32", "data": "synthetic",
             "config": {"workload": "full_spec", "k": args.k, "batch": 1, "sample": desc},
