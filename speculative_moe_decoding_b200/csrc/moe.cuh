@@ -10,10 +10,10 @@
 //   experts' gate/up tiles (the experts touched by the pass, ascending id),
 //   then the down tiles (32 output rows) of the same matrices in the same
 //   order.
-// CTA c takes item c first, then claims items from a counter (one claim in
-// flight while the current item is issued): the TMA stream of some SMs runs
-// slower than others from launch to launch, and claiming lets the fast ones
-// take more.  The shared items do not depend on the routing: every CTA whose
+// CTA c takes item c first, then claims items from a counter, each once the
+// previous item's stages are requested: the TMA stream of some SMs runs slower
+// than others from launch to launch, and claiming lets the fast ones take
+// more.  The shared items do not depend on the routing: every CTA whose
 // first item is one of them requests its weights before the dependency wait.
 //
 // Warp roles:
@@ -339,18 +339,19 @@ moe_kernel(const __grid_constant__ CUtensorMap tm_gu, const __grid_constant__ CU
       }
     };
     if (!abort_p) {
-      // items: the first one (unless already issued), then claims, the next
-      // claim in flight while the current item is issued
-      int next = (int)gridDim.x + atomicAdd(p.ctr + kMoeCtrClaim, 1);
+      // items: the first one (unless already issued), then claims.  The next
+      // item is claimed once the current one's stages are all requested: the
+      // ring still holds them while the claim returns, and a CTA never holds
+      // an item it has not started when the items run out (the kernel ends
+      // with the slowest CTA)
       if (!pre) {
         need_total();
         if (first < total) issue_item(first, moe_item(p, n_mats, first));
       }
       while (true) {
-        const int cur = next;
+        const int cur = (int)gridDim.x + atomicAdd(p.ctr + kMoeCtrClaim, 1);
         if (cur >= n_shared_items) need_total();
         if (total >= 0 && cur >= total) break;
-        next = (int)gridDim.x + atomicAdd(p.ctr + kMoeCtrClaim, 1);
         issue_item(cur, moe_item(p, n_mats, cur));
       }
     }
