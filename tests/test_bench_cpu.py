@@ -23,3 +23,27 @@ def test_step_bytes_dense_set():
     assert union0 == dep0 == 694_026_240
     union1, _ = bench.step_bytes(m, 0, 1.0, 0.0)
     assert union1 - union0 == 11 * 6_881_280
+
+
+def test_oracle_sample_exact_steps():
+    # the reference arm: W untimed steps, then exactly K timed ones
+    bits, _ = synth.make_weights(synth.TINY, synth.WORKLOADS["tiny"].weight_seed, workers=1)
+    tps, desc, used, steps, dt = bench.run_oracle_sample(synth.TINY, 3, bits, timed_steps=7, warm_steps=2)
+    assert steps == 7 and tps > 0 and dt > 0
+
+
+def test_profiled_traffic_hash_and_scaling(tmp_path, monkeypatch):
+    import hashlib
+    src = tmp_path / "kernel.cuh"
+    src.write_text("// kernel source\n")
+    digest = hashlib.sha256(src.read_bytes()).hexdigest()
+    (tmp_path / "profiles").mkdir()
+    prof = tmp_path / "profiles" / "k.md"
+    prof.write_text("# capture\n\n    traffic_bytes_per_launch: 1030\n    algorithmic_bytes_per_launch: 1000\n"
+                    f"    source_sha256: {digest}\n    source_files: kernel.cuh\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.profiled_traffic("k.md") == 1030
+    assert abs(bench.profiled_traffic("k.md", 5000) - 5150) < 1e-9  # the ratio, scaled to this launch
+    assert bench.profiled_traffic("missing.md") is None
+    src.write_text("// kernel source, changed\n")
+    assert bench.profiled_traffic("k.md") is None  # counters of an older kernel are not reported
